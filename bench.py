@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid compressed / sparse / sliding attention forward pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl reference]
+
+One step = one pass of the whole forward path over one batch of the workload:
+block_merge of K, V (and indexer keys for CSA) -> indexer scores + exact top-K
+(CSA) -> hybrid attention.  Default workload: the HCA+SWA batch (B=2, L=8192,
+16 query / 16 KV heads, d=128, m=128, W=128).  Inputs are synthetic, seeded and
+resident in HBM before the timed region; L2 is flushed (a 256 MiB write)
+between timed steps, outside the per-step CUDA events.  Rank 0 prints one JSON
+line.  With N > 1 (torchrun) every rank runs an independent replica of the
+workload (the path shards by sequence with no exchange): weak scaling, value =
+all ranks' query tokens / max-over-ranks time.
+
+--impl reference times the CPU oracle (fp64 C, OpenMP) on a bounded sample of
+the same workload on the host cores; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "query-tokens/s"
+DEFAULT_CONFIG = 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+# ----------------------------------------------------------------- work counts
+def n_visible(t, m, W, Nc):
+    a = t - W + 1
+    return 0 if a <= 0 else min(a // m, Nc)
+
+
+def algorithmic_counts(w):
+    """Per step: attention keys and FLOP, indexer FLOP, unique bytes per stage."""
+    if w.is_decode:
+        t = w.L - 1
+        nv = n_visible(t, w.m, w.W, w.Nc)
+        sel = min(w.topk, nv)
+        keys_per_tok = sel + min(w.W, t + 1)
+        attn_keys = w.B * keys_per_tok
+        idx_pairs = w.B * nv
+    else:
+        t = np.arange(w.L, dtype=np.int64)
+        nv = np.clip((t - w.W + 1) // w.m, 0, w.Nc)
+        nv[t - w.W + 1 <= 0] = 0
+        sel = np.minimum(nv, w.topk) if w.topk else nv
+        win = np.minimum(w.W, t + 1)
+        attn_keys = int(w.B * (sel + win).sum())
+        idx_pairs = int(w.B * nv.sum()) if w.topk else 0
+    attn_flop = 4 * w.d * w.Hq * attn_keys
+    idx_flop = 2 * w.Hi * w.di * idx_pairs
+    bf = 2
+    B, Lq, Hq, Hkv, d, Nc = w.B, w.Lq, w.Hq, w.Hkv, w.d, w.Nc
+    q_o = 2 * B * Lq * Hq * d * bf
+    if w.is_decode:
+        # unique bytes: q/o, the selected compressed rows, the raw window rows, the indexer keys
+        attn_bytes = q_o + (w.B * keys_per_tok) * Hkv * d * bf * 2 + w.B * w.topk * 4
+        compress_bytes = 0
+        idx_bytes = B * nv * w.di * bf + B * w.Hi * w.di * bf + B * w.topk * 4
+    else:
+        attn_bytes = q_o + 2 * B * w.L * Hkv * d * bf + 2 * B * Nc * Hkv * d * bf
+        if w.topk:
+            attn_bytes += B * Lq * w.topk * 4
+        compress_bytes = 2 * B * w.L * Hkv * d * bf + 2 * B * Nc * Hkv * d * bf
+        if w.topk:
+            compress_bytes += B * w.L * w.di * bf + B * Nc * w.di * bf
+        idx_bytes = (B * Lq * (w.Hi * w.di * bf + w.Hi * 4) + B * Nc * w.di * bf +
+                     B * Lq * w.topk * 4) if w.topk else 0
+    return dict(attn_keys=attn_keys, attn_flop=attn_flop, idx_flop=idx_flop, attn_bytes=attn_bytes,
+                compress_bytes=compress_bytes, idx_bytes=idx_bytes)
+
+
+# ----------------------------------------------------------------- GPU arm
+def problem_for(hb, w, inp):
+    if w.is_decode:
+        return hb.problem(B=w.B, Lq=1, Lkv=w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
+                          topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc, q_pos=inp["q_pos"],
+                          kv_pos0=inp["kv_pos0"])
+    return hb.problem(B=w.B, Lq=w.L, Lkv=w.L, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
+                      topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc)
+
+
+class Step:
+    """One forward pass as the three C-ABI stages on one stream, with CUDA
+    events between the stages (the same kernels hyb_fused_fwd launches)."""
+
+    def __init__(self, hb, w, inp):
+        self.hb, self.w, self.inp = hb, w, inp
+        self.p = problem_for(hb, w, inp)
+        dev = inp["q"].device
+        if w.is_decode:
+            self.kc, self.vc, self.kic = inp["kc"], inp["vc"], inp["kic"]
+        else:
+            self.kc = torch.empty((w.B, w.Nc, w.Hkv, w.d), dtype=torch.bfloat16, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            self.kic = (torch.empty((w.B, w.Nc, w.di), dtype=torch.bfloat16, device=dev)
+                        if w.topk else None)
+        self.idx = (torch.empty((w.B, w.Lq, w.topk), dtype=torch.int32, device=dev)
+                    if w.topk else None)
+        self.o = torch.empty((w.B, w.Lq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        need = hb.hyb_workspace_size(self.p)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        self.launches = 0
+
+    def run(self, stream):
+        hb, w, inp, ev = self.hb, self.w, self.inp, self.ev
+        launches = 0
+        ev[0].record(stream)
+        if not w.is_decode:
+            hb.hyb_hca_compress(inp["k"], inp["wk"], w.m, out=self.kc, stream=stream)
+            hb.hyb_hca_compress(inp["v"], inp["wv"], w.m, out=self.vc, stream=stream)
+            launches += 2
+            if w.topk:
+                hb.hyb_hca_compress(inp["ki"], inp["wib"], w.m, out=self.kic, stream=stream)
+                launches += 1
+        ev[1].record(stream)
+        if w.topk:
+            hb.hyb_csa_index_topk(self.p, inp["qi"], inp["wi"], self.kic, idx=self.idx, ws=self.ws,
+                                  stream=stream)
+            launches += 2
+        ev[2].record(stream)
+        hb.hyb_attn_fwd(self.p, inp["q"], self.kc, self.vc, self.idx,
+                        inp["k_raw"] if w.is_decode else inp["k"],
+                        inp["v_raw"] if w.is_decode else inp["v"], o=self.o, stream=stream)
+        launches += 1
+        ev[3].record(stream)
+        self.launches = launches
+
+    def times_ms(self):
+        e = self.ev
+        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                e[2].elapsed_time(e[3]))
+
+
+def sample_clocks_start():
+    try:
+        return subprocess.Popen(
+            ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+             "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "100",
+             "-i", str(torch.cuda.current_device())],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    except Exception:
+        return None
+
+
+def sample_clocks_stop(proc):
+    if proc is None:
+        return None
+    proc.terminate()
+    try:
+        out, _ = proc.communicate(timeout=5)
+    except Exception:
+        proc.kill()
+        return None
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in out.strip().splitlines():
+        f = [x.strip() for x in line.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1]))
+            mx = max(mx, float(f[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, f[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def kernel_traffic(kernel: str, config_no: int):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        ent = tab[f"{kernel}@{config_no}"]
+        src = os.path.join(ROOT, "compressed_sparse_sliding_b200", "csrc", ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return int(ent["bytes_per_launch"]) if h == ent["source_sha"] else None
+    except Exception:
+        return None
+
+
+def run_gpu(args, rank, world):
+    import compressed_sparse_sliding_b200 as hb
+    w = WORKLOADS[args.config]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(w, device=dev, seed=20260 + w.no + 1000 * rank)
+    if not w.is_decode:
+        inp["k_raw"], inp["v_raw"] = inp["k"], inp["v"]
+    stream = torch.cuda.current_stream()
+    step = Step(hb, w, inp)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    counts = algorithmic_counts(w)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.run(stream)
+    torch.cuda.synchronize()
+    st = hb.hyb_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {hb.hyb_error_string(st)}")
+
+    clk = sample_clocks_start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    tot, comp, idx, att = [], [], [], []
+    launches = 0
+    for _ in range(args.steps):
+        flush.fill_(1)  # L2 flush, outside the step's events
+        step.run(stream)
+        torch.cuda.synchronize()
+        a, b, c, d = step.times_ms()
+        tot.append(a); comp.append(b); idx.append(c); att.append(d)
+        launches += step.launches
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sample_clocks_stop(clk)
+    st = hb.hyb_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {hb.hyb_error_string(st)}")
+
+    total_ms = float(sum(tot))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.B * w.Lq * world
+    value = tokens / (ms_per_step / 1e3)
+
+    # ---- end to end through the fused C-ABI call with host buffers ----
+    host = {k: v.cpu().pin_memory() for k, v in inp.items()
+            if k in ("q", "k", "v", "wk", "wv", "qi", "wi", "ki", "wib", "kc", "vc", "kic",
+                     "k_raw", "v_raw", "q_pos", "kv_pos0")}
+    if not w.is_decode:
+        host.pop("k_raw", None)
+        host.pop("v_raw", None)
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        if not w.is_decode:
+            dev_in["k_raw"], dev_in["v_raw"] = dev_in["k"], dev_in["v"]
+        p = problem_for(hb, w, dev_in)
+        res = hb.hyb_fused_fwd(p, dev_in["q"], dev_in["k_raw"], dev_in["v_raw"], wk=dev_in.get("wk"),
+                               wv=dev_in.get("wv"), qi=dev_in.get("qi"), wi=dev_in.get("wi"),
+                               ki_raw=dev_in.get("ki"), wib=dev_in.get("wib"), kc=dev_in.get("kc"),
+                               vc=dev_in.get("vc"), kic=dev_in.get("kic"), o=step.o, ws=step.ws,
+                               stream=stream)
+        o_host.copy_(res["o"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(2, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peaks = load_peaks()
+    att_ms = statistics.mean(att)
+    hbm_bound = w.is_decode or w.no == 2
+    if hbm_bound:
+        achieved = counts["attn_bytes"] / (att_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4)}
+    else:
+        achieved = counts["attn_flop"] / (att_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4)}
+    roof["kernel"] = "hybrid_attn_kernel"
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = kernel_traffic("hybrid_attn_kernel", w.no)
+    stages = {"compress_ms": round(statistics.mean(comp), 4),
+              "index_topk_ms": round(statistics.mean(idx), 4),
+              "attention_ms": round(att_ms, 4)}
+    if counts["compress_bytes"] and statistics.mean(comp) > 0:
+        stages["compress_GBps"] = round(counts["compress_bytes"] / (statistics.mean(comp) / 1e3) / 1e9, 1)
+    if w.topk and statistics.mean(idx) > 0:
+        stages["index_topk_TFLOPs"] = round(counts["idx_flop"] / (statistics.mean(idx) / 1e3) / 1e12, 2)
+    stages["attention_TFLOPs"] = round(counts["attn_flop"] / (att_ms / 1e3) / 1e12, 1)
+    stages["attention_GBps"] = round(counts["attn_bytes"] / (att_ms / 1e3) / 1e9, 1)
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "query-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 inputs, N(0,1) block weights, U(0,1) head weights)",
+        "config": {"workload": w.name, "desc": w.describe(), "global_batch": w.B * world,
+                   "seq_len": w.L, "parallelism": f"replicas{world}",
+                   "l2": "flushed between steps (256 MiB write)"},
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "query-tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "stages": stages,
+        "clocks": clocks,
+    }
+    return res
+
+
+# ----------------------------------------------------------------- CPU oracle
+def run_oracle(w, budget_s=12.0, rows_hint=None):
+    """Times the oracle on a bounded sample of the workload.  Compression of
+    the whole batch is timed once and charged per query token; indexer, top-K
+    and attention are timed on a sample of query rows."""
+    import oracle
+    inp = make_inputs(w, device="cpu")
+    cores = os.cpu_count()
+    bits = {k: oracle.bf16_bits(v) for k, v in inp.items() if v.dtype == torch.bfloat16}
+    t0 = time.perf_counter()
+    if w.is_decode:
+        kc, vc, kic = bits["kc"], bits["vc"], bits["kic"]
+        t_comp = 0.0
+    else:
+        _, kc = oracle.block_merge(bits["k"], inp["wk"].numpy(), w.m)
+        _, vc = oracle.block_merge(bits["v"], inp["wv"].numpy(), w.m)
+        kic = None
+        if w.topk:
+            _, kic = oracle.block_merge(bits["ki"][:, :, None, :], inp["wib"].numpy(), w.m)
+            kic = kic[:, :, 0, :]
+        t_comp = time.perf_counter() - t0
+    total_rows = w.B * w.Lq
+
+    def rows_work(rows):
+        t1 = time.perf_counter()
+        qp = inp["q_pos"].numpy() if w.is_decode else None
+        idx = None
+        if w.topk:
+            sc, nv = oracle.index_scores(bits["qi"], inp["wi"].numpy(), kic, w.m, w.W, q_pos=qp,
+                                         rows=rows)
+            sel = oracle.topk(sc, nv, w.topk)
+            idx = np.full((total_rows, w.topk), -1, np.int32)
+            idx[rows] = sel
+            idx = idx.reshape(w.B, w.Lq, w.topk)
+        if w.is_decode:
+            oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k_raw"], bits["v_raw"], w.m, w.W,
+                                    q_pos=qp, kv_pos0=inp["kv_pos0"].numpy(), rows=rows)
+        else:
+            oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k"], bits["v"], w.m, w.W,
+                                    rows=rows)
+        return time.perf_counter() - t1
+
+    rng = np.random.default_rng(0)
+    n = 8 if rows_hint is None else rows_hint
+    while True:
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        dt = rows_work(rows)
+        if dt > budget_s / 4 or n >= total_rows:
+            break
+        n = min(total_rows, int(n * max(2.0, (budget_s / 2) / max(dt, 1e-3))))
+    per_row = t_comp / total_rows + dt / len(rows)
+    return {"value": round(1.0 / per_row, 3), "unit": "query-tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": (f"{len(rows)} of {total_rows} query rows (indexer, top-K, attention) + "
+                       f"compression of the whole batch ({t_comp:.2f} s) charged per token")}
+
+
+def run_reference_arm(args):
+    w = WORKLOADS[args.config]
+    per_step = []
+    base = None
+    for _ in range(args.warmup):
+        run_oracle(w, budget_s=2.0, rows_hint=4)
+    for _ in range(args.steps):
+        base = run_oracle(w, budget_s=6.0, rows_hint=8)
+        per_step.append(1.0 / base["value"])
+    value = 1.0 / statistics.mean(per_step)
+    cpu = dict(base)
+    cpu["value"] = round(value, 3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "query-tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * statistics.mean(per_step) * w.B * w.Lq, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": w.name, "desc": w.describe(), "global_batch": w.B, "seq_len": w.L,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(value, 3), "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference_arm(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    try:
+        res = run_gpu(args, rank, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config])
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+"""B200 (sm_100a) hybrid compressed / sparse / sliding-window attention.
+
+Thin ctypes binding over ``libhybattn.so`` (C ABI in ``include/hybattn.h``).
+Every step of the forward pass runs in the library's CUDA kernels; this module
+only marshals arguments: it takes device tensors, passes their data pointers
+and the current CUDA stream, and allocates outputs with torch.  There is no
+CPU or PyTorch fallback: importing fails loudly when the library is missing.
+
+Entry points (same names as the C ABI):
+  hyb_hca_compress     block_merge of raw K / V / indexer keys
+  hyb_csa_index_topk   lightning-indexer scores + exact per-query top-K
+  hyb_attn_fwd         one softmax over compressed (selected / all visible)
+                       keys and the raw sliding window
+  hyb_fused_fwd        the three stages on one stream
+  hyb_workspace_size, hyb_get_device_status, hyb_error_string
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhybattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_sliding_b200.build` "
+        "(nvcc, sm_100a). There is no fallback implementation.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+HYB_OK = 0
+HYB_ERR_INVALID_ARG = -1
+HYB_ERR_UNSUPPORTED = -2
+HYB_ERR_WORKSPACE = -3
+HYB_ERR_CUDA = -4
+HYB_ERR_DEVICE_TIMEOUT = -5
+HYB_ERR_DEVICE_BOUNDS = -6
+
+
+class HybProblem(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("Lq", ctypes.c_int), ("Lkv", ctypes.c_int),
+        ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("d", ctypes.c_int),
+        ("m", ctypes.c_int), ("W", ctypes.c_int), ("topk", ctypes.c_int),
+        ("Hi", ctypes.c_int), ("di", ctypes.c_int), ("Nc", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("q_pos", ctypes.c_void_p), ("kv_pos0", ctypes.c_void_p),
+    ]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_PP = ctypes.POINTER(HybProblem)
+_lib.hyb_workspace_size.argtypes = [_PP]
+_lib.hyb_workspace_size.restype = ctypes.c_size_t
+_lib.hyb_hca_compress.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
+_lib.hyb_hca_compress.restype = _I
+_lib.hyb_csa_index_topk.argtypes = [_PP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.hyb_csa_index_topk.restype = _I
+_lib.hyb_attn_fwd.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+_lib.hyb_attn_fwd.restype = _I
+_lib.hyb_fused_fwd.argtypes = [_PP] + [_P] * 16 + [ctypes.c_size_t, _P]
+_lib.hyb_fused_fwd.restype = _I
+_lib.hyb_get_device_status.argtypes = [_P]
+_lib.hyb_get_device_status.restype = _I
+_lib.hyb_error_string.argtypes = [_I]
+_lib.hyb_error_string.restype = ctypes.c_char_p
+
+
+class HybError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {hyb_error_string(status)} ({status})")
+
+
+def hyb_error_string(status: int) -> str:
+    return _lib.hyb_error_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != HYB_OK:
+        raise HybError(status, where)
+
+
+def problem(B, Lq, Lkv, Hq, Hkv, d, m, W, topk=0, Hi=0, di=0, Nc=0, scale=0.0, q_pos=None,
+            kv_pos0=None) -> HybProblem:
+    """Builds the C problem struct; q_pos / kv_pos0 are int32 device tensors or None."""
+    p = HybProblem(B, Lq, Lkv, Hq, Hkv, d, m, W, topk, Hi, di, Nc, float(scale), None, None)
+    p.q_pos = None if q_pos is None else q_pos.data_ptr()
+    p.kv_pos0 = None if kv_pos0 is None else kv_pos0.data_ptr()
+    p._keep = (q_pos, kv_pos0)
+    return p
+
+
+def hyb_workspace_size(p: HybProblem) -> int:
+    return int(_lib.hyb_workspace_size(ctypes.byref(p)))
+
+
+def hyb_hca_compress(x: torch.Tensor, w: torch.Tensor, m: int, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """x [B, L, H, dx] (or [B, L, dx]) bf16, w [m, dx] fp32 -> [B, L//m, H, dx] bf16."""
+    squeeze = x.dim() == 3
+    xv = x.unsqueeze(2) if squeeze else x
+    B, L, H, dx = xv.shape
+    if out is None:
+        out = torch.empty((B, L // m, H, dx), dtype=torch.bfloat16, device=x.device)
+    st = _lib.hyb_hca_compress(_ptr(xv), B, L, H, dx, m, _ptr(w), _ptr(out), _stream(stream))
+    _check(st, "hyb_hca_compress")
+    return out.squeeze(2) if squeeze and out.dim() == 4 else out
+
+
+def hyb_csa_index_topk(p: HybProblem, qi, wi, kic, idx=None, sel_scores=None, ws=None,
+                       stream=None):
+    """Top-K entry indices [B, Lq, topk] int32 (ascending, -1 padded)."""
+    if idx is None:
+        idx = torch.empty((p.B, p.Lq, p.topk), dtype=torch.int32, device=qi.device)
+    need = hyb_workspace_size(p)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=qi.device)
+    st = _lib.hyb_csa_index_topk(ctypes.byref(p), _ptr(qi), _ptr(wi), _ptr(kic), _ptr(idx),
+                                 _ptr(sel_scores), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "hyb_csa_index_topk")
+    return idx
+
+
+def hyb_attn_fwd(p: HybProblem, q, kc, vc, idx, k_raw, v_raw, o=None, lse=None, stream=None):
+    """o [B, Lq, Hq, d] bf16 (and lse [B, Hq, Lq] fp32 when given)."""
+    if o is None:
+        o = torch.empty((p.B, p.Lq, p.Hq, p.d), dtype=torch.bfloat16, device=q.device)
+    st = _lib.hyb_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(kc), _ptr(vc), _ptr(idx), _ptr(k_raw),
+                           _ptr(v_raw), _ptr(o), _ptr(lse), _stream(stream))
+    _check(st, "hyb_attn_fwd")
+    return o
+
+
+def hyb_fused_fwd(p: HybProblem, q, k_raw, v_raw, wk=None, wv=None, qi=None, wi=None, ki_raw=None,
+                  wib=None, kc=None, vc=None, kic=None, idx=None, o=None, lse=None, ws=None,
+                  stream=None):
+    """Whole forward pass.  Returns dict(o, kc, vc, kic, idx)."""
+    dev = q.device
+    if kc is None:
+        kc = torch.empty((p.B, p.Nc, p.Hkv, p.d), dtype=torch.bfloat16, device=dev)
+        vc = torch.empty_like(kc)
+    if p.topk > 0:
+        if kic is None:
+            kic = torch.empty((p.B, p.Nc, p.di), dtype=torch.bfloat16, device=dev)
+        if idx is None:
+            idx = torch.empty((p.B, p.Lq, p.topk), dtype=torch.int32, device=dev)
+    if o is None:
+        o = torch.empty((p.B, p.Lq, p.Hq, p.d), dtype=torch.bfloat16, device=dev)
+    need = hyb_workspace_size(p)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    st = _lib.hyb_fused_fwd(ctypes.byref(p), _ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(wk), _ptr(wv),
+                            _ptr(qi), _ptr(wi), _ptr(ki_raw), _ptr(wib), _ptr(kc), _ptr(vc),
+                            _ptr(kic), _ptr(idx), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                            _stream(stream))
+    _check(st, "hyb_fused_fwd")
+    return dict(o=o, kc=kc, vc=vc, kic=kic, idx=idx)
+
+
+def hyb_get_device_status(stream=None) -> int:
+    return int(_lib.hyb_get_device_status(_stream(stream)))

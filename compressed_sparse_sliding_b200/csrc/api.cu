@@ -1,0 +1,216 @@
+// api.cu -- the C ABI declared in include/hybattn.h: argument validation on
+// the host, workspace carve-up and kernel launches on the caller's stream.
+#include <math.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace hyb {
+
+
+
+cudaError_t launch_block_merge(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                               void *out, cudaStream_t stream, int num_sms);
+cudaError_t launch_index_scores_simt(const void *qi, const float *wi, const void *kic, float *scores,
+                                     int B, int Lq, int Hi, int di, int Nc, int m, int W,
+                                     const int32_t *q_pos, cudaStream_t stream);
+cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m, int W, int K,
+                              const int32_t *q_pos, int32_t *idx, float *sel_scores,
+                              cudaStream_t stream);
+cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, int Nc, int m, int W,
+                               int topk, float scale, const int32_t *q_pos, const int32_t *kv_pos0,
+                               const void *q, const void *kc, const void *vc, const int32_t *idx,
+                               const void *kr, const void *vr, void *o, float *lse,
+                               cudaStream_t stream);
+
+static int num_sms_current()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+static bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+static hyb_status cuda_status(cudaError_t e)
+{
+    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
+// Largest shared-memory footprint of one top-K row (keys) + static tables.
+static constexpr size_t kTopkSmemLimit = 227 * 1024 - 20 * 1024;
+
+static hyb_status check_problem(const hyb_problem *p, bool need_indexer)
+{
+    if (!p)
+        return HYB_ERR_INVALID_ARG;
+    if (p->B <= 0 || p->Lq <= 0 || p->Lkv < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->m <= 0 ||
+        p->W < 0 || p->Nc < 0)
+        return HYB_ERR_INVALID_ARG;
+    if (p->Hq % p->Hkv != 0)
+        return HYB_ERR_INVALID_ARG;
+    if (p->d != 64 && p->d != 128)
+        return HYB_ERR_UNSUPPORTED;
+    if (p->topk > 0) {
+        if (p->Hq / p->Hkv > 64 || p->topk > 2048)
+            return HYB_ERR_UNSUPPORTED;
+    }
+    if (need_indexer) {
+        if (p->topk <= 0 || p->Hi <= 0 || p->di <= 0)
+            return HYB_ERR_INVALID_ARG;
+        if (p->di != 32 && p->di != 64)
+            return HYB_ERR_UNSUPPORTED;
+        if (p->Hi > 16 || (size_t)p->Nc * 4 > kTopkSmemLimit)
+            return HYB_ERR_UNSUPPORTED;
+    }
+    if (p->Lkv >= (1 << 30) || p->Lq >= (1 << 30) || p->Nc >= (1 << 30))
+        return HYB_ERR_UNSUPPORTED;
+    return HYB_OK;
+}
+
+static float softmax_scale(const hyb_problem *p)
+{
+    return p->scale != 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+}
+
+}  // namespace hyb
+
+using namespace hyb;
+
+extern "C" {
+
+size_t hyb_workspace_size(const hyb_problem *p)
+{
+    if (!p || p->topk <= 0)
+        return 0;
+    size_t scores = (size_t)p->B * p->Lq * p->Nc * sizeof(float);
+    return (scores + 255) & ~(size_t)255;
+}
+
+hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                            void *out, cudaStream_t stream)
+{
+    if (!x || !w || !out || B <= 0 || L < 0 || H <= 0 || dx <= 0 || m <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (dx % 8 != 0 || !aligned16(x) || !aligned16(out) || !aligned16(w))
+        return HYB_ERR_INVALID_ARG;
+    if (m > 256 || (size_t)m * dx > 32768)
+        return HYB_ERR_UNSUPPORTED;
+    return cuda_status(launch_block_merge(x, B, L, H, dx, m, w, out, stream, num_sms_current()));
+}
+
+hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float *wi, const void *kic,
+                              int32_t *idx, float *sel_scores, void *ws, size_t ws_bytes,
+                              cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, true);
+    if (st != HYB_OK)
+        return st;
+    if (!qi || !wi || !kic || !idx || !aligned16(qi) || !aligned16(kic))
+        return HYB_ERR_INVALID_ARG;
+    const size_t need = hyb_workspace_size(p);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return HYB_ERR_WORKSPACE;
+    float *scores = static_cast<float *>(ws);
+    cudaError_t e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
+                                             p->m, p->W, p->q_pos, stream);
+    if (e != cudaSuccess)
+        return HYB_ERR_CUDA;
+    e = launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos, idx, sel_scores,
+                          stream);
+    return cuda_status(e);
+}
+
+hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                        const int32_t *idx, const void *k_raw, const void *v_raw, void *o, float *lse,
+                        cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, false);
+    if (st != HYB_OK)
+        return st;
+    if (!q || !o || !k_raw || !v_raw)
+        return HYB_ERR_INVALID_ARG;
+    if (p->Nc > 0 && (!kc || !vc))
+        return HYB_ERR_INVALID_ARG;
+    if (idx && p->topk <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o) || !aligned16(k_raw) || !aligned16(v_raw) ||
+        (kc && !aligned16(kc)) || (vc && !aligned16(vc)))
+        return HYB_ERR_INVALID_ARG;
+    if (p->Lkv <= 0 && p->W > 0)
+        return HYB_ERR_INVALID_ARG;
+    const int Lkv = p->Lkv > 0 ? p->Lkv : 1;
+    cudaError_t e = launch_hybrid_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->d, p->Nc, p->m, p->W,
+                                       p->topk, softmax_scale(p), p->q_pos, p->kv_pos0, q, kc, vc, idx,
+                                       k_raw, v_raw, o, lse, stream);
+    return cuda_status(e);
+}
+
+hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw, const void *v_raw,
+                         const float *wk, const float *wv, const void *qi, const float *wi,
+                         const void *ki_raw, const float *wib, void *kc, void *vc, void *kic,
+                         int32_t *idx, void *o, float *lse, void *ws, size_t ws_bytes,
+                         cudaStream_t stream)
+{
+    const bool csa = p && p->topk > 0;
+    hyb_status st = check_problem(p, csa);
+    if (st != HYB_OK)
+        return st;
+    if (!kc || !vc || (csa && (!kic || !idx || !qi || !wi)))
+        return HYB_ERR_INVALID_ARG;
+    if (wk) {  // prefill: build the compressed caches from the raw rows
+        if (!wv || (csa && (!ki_raw || !wib)))
+            return HYB_ERR_INVALID_ARG;
+        if (p->Nc != p->Lkv / p->m)
+            return HYB_ERR_INVALID_ARG;
+        st = hyb_hca_compress(k_raw, p->B, p->Lkv, p->Hkv, p->d, p->m, wk, kc, stream);
+        if (st != HYB_OK)
+            return st;
+        st = hyb_hca_compress(v_raw, p->B, p->Lkv, p->Hkv, p->d, p->m, wv, vc, stream);
+        if (st != HYB_OK)
+            return st;
+        if (csa) {
+            st = hyb_hca_compress(ki_raw, p->B, p->Lkv, 1, p->di, p->m, wib, kic, stream);
+            if (st != HYB_OK)
+                return st;
+        }
+    }
+    if (csa) {
+        st = hyb_csa_index_topk(p, qi, wi, kic, idx, nullptr, ws, ws_bytes, stream);
+        if (st != HYB_OK)
+            return st;
+    }
+    return hyb_attn_fwd(p, q, kc, vc, csa ? idx : nullptr, k_raw, v_raw, o, lse, stream);
+}
+
+hyb_status hyb_get_device_status(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    return (hyb_status)v;
+}
+
+const char *hyb_error_string(hyb_status s)
+{
+    switch (s) {
+    case HYB_OK: return "ok";
+    case HYB_ERR_INVALID_ARG: return "invalid argument";
+    case HYB_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case HYB_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case HYB_ERR_CUDA: return "CUDA runtime error";
+    case HYB_ERR_DEVICE_TIMEOUT: return "device wait exceeded its bound";
+    case HYB_ERR_DEVICE_BOUNDS: return "device met an out-of-range index";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

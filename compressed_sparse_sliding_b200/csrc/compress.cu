@@ -1,0 +1,191 @@
+// compress.cu -- stage 1, block_merge (CSDN DeepSeek-V4 CSA/HCA code page,
+// section 1): one compressed entry per block of m tokens, the weighted sum of
+// the block's tokens with per-channel softmax weights over the m positions.
+//
+// Memory-bound streaming kernel.  Every thread owns 8 consecutive channels of
+// one (b, j) block row and reads 16-byte vectors; a warp covers 512
+// contiguous bytes of a token row, so each load instruction is fully
+// coalesced.  When there are too few (b, j, channel-octet) items to fill the
+// GPU (few, long blocks such as m = 128), the m positions are split over S
+// thread groups of the CTA and their partial sums are reduced in shared
+// memory.  CTAs are persistent: the [m, dx] weights are staged into shared
+// memory with 16-byte loads and turned into softmax weights once per CTA, then
+// reused for every block the CTA processes.
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads)
+block_merge_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
+                   __nv_bfloat16 *__restrict__ out, int B, int L, int H, int dx, int m, int S)
+{
+    extern __shared__ __align__(16) float sm_merge[];
+    float *P = sm_merge;                        // [m][dx]
+    float *part = sm_merge + (size_t)m * dx;    // [S-1][items_per_cta][8]
+    const int tid = threadIdx.x;
+
+    // ---- stage the [m, dx] weights with 16-byte loads, then softmax over the
+    //      m positions separately for every channel, in place ----
+    {
+        const float4 *w4 = reinterpret_cast<const float4 *>(w);
+        float4 *P4 = reinterpret_cast<float4 *>(P);
+        for (int i = tid; i < m * dx / 4; i += kMergeThreads)
+            P4[i] = __ldg(w4 + i);
+    }
+    __syncthreads();
+    {
+        int G = 1;  // threads per channel (power of two)
+        while (G * 2 * dx <= kMergeThreads && G * 2 <= m)
+            G *= 2;
+        const int cpr = kMergeThreads / G;  // channels per round
+        const int g = tid % G;
+        for (int c = tid / G; c < dx + (cpr - (dx % cpr)) % cpr; c += cpr) {
+            const bool live = c < dx;
+            float mx = -INFINITY;
+            if (live)
+                for (int i = g; i < m; i += G)
+                    mx = fmaxf(mx, P[(size_t)i * dx + c]);
+            for (int off = 1; off < G; off <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            float den = 0.f;
+            if (live)
+                for (int i = g; i < m; i += G) {
+                    float e = expf(P[(size_t)i * dx + c] - mx);
+                    P[(size_t)i * dx + c] = e;
+                    den += e;
+                }
+            for (int off = 1; off < G; off <<= 1)
+                den += __shfl_xor_sync(0xffffffffu, den, off);
+            if (live) {
+                float inv = 1.f / den;
+                for (int i = g; i < m; i += G)
+                    P[(size_t)i * dx + c] *= inv;
+            }
+        }
+    }
+    __syncthreads();
+
+    const int Nc = L / m;
+    const int E8 = H * dx / 8;                 // 16-byte octets per token row
+    const long long items = (long long)B * Nc * E8;
+    const int ipc = kMergeThreads / S;         // items per CTA tile
+    const int s = tid / ipc;                   // position split owned by this thread
+    const int li = tid % ipc;
+    const long long ntiles = (items + ipc - 1) / ipc;
+    const size_t row_elems = (size_t)H * dx;
+
+    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const long long item = tile * ipc + li;
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            acc[k] = 0.f;
+        const bool live = item < items;
+        if (live) {
+            const long long unit = item / E8;
+            const int e8 = (int)(item % E8);
+            const int b = (int)(unit / Nc);
+            const int j = (int)(unit % Nc);
+            const int c0 = (e8 * 8) % dx;
+            const __nv_bfloat16 *src =
+                x + ((size_t)b * L + (size_t)j * m) * row_elems + (size_t)e8 * 8;
+            int i = s;
+            // eight independent 16-byte loads in flight per thread
+            for (; i + 7 * S < m; i += 8 * S) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    v[u] = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)(i + u * S) * row_elems));
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float *pw = P + (size_t)(i + u * S) * dx + c0;
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        float2 f = __bfloat1622float2(h2[k]);
+                        acc[2 * k] = fmaf(pw[2 * k], f.x, acc[2 * k]);
+                        acc[2 * k + 1] = fmaf(pw[2 * k + 1], f.y, acc[2 * k + 1]);
+                    }
+                }
+            }
+            for (; i < m; i += S) {
+                uint4 v = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)i * row_elems));
+                const float *pw = P + (size_t)i * dx + c0;
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float2 f = __bfloat1622float2(h2[k]);
+                    acc[2 * k] = fmaf(pw[2 * k], f.x, acc[2 * k]);
+                    acc[2 * k + 1] = fmaf(pw[2 * k + 1], f.y, acc[2 * k + 1]);
+                }
+            }
+        }
+        if (S > 1) {
+            if (s > 0) {
+                float4 *dst = reinterpret_cast<float4 *>(part + ((size_t)(s - 1) * ipc + li) * 8);
+                dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+            __syncthreads();
+            if (s == 0) {
+                for (int q = 1; q < S; ++q) {
+                    const float4 *srcp =
+                        reinterpret_cast<const float4 *>(part + ((size_t)(q - 1) * ipc + li) * 8);
+                    float4 a = srcp[0], bq = srcp[1];
+                    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+                    acc[4] += bq.x; acc[5] += bq.y; acc[6] += bq.z; acc[7] += bq.w;
+                }
+            }
+            __syncthreads();
+        }
+        if (s == 0 && live) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            *reinterpret_cast<uint4 *>(out + (size_t)item * 8) = o;
+        }
+    }
+}
+
+// Launch helper: picks the position split S and a persistent grid.
+cudaError_t launch_block_merge(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                               void *out, cudaStream_t stream, int num_sms)
+{
+    const int Nc = L / m;
+    const long long items = (long long)B * Nc * (H * dx / 8);
+    if (items == 0)
+        return cudaSuccess;
+    // split the m positions over S thread groups only while every thread keeps
+    // at least 8 loads and the grid is short of ~1024 threads per SM
+    int S = 1;
+    const long long target = (long long)num_sms * 1024;
+    while (S * 2 <= m / 8 && S * 2 <= 32 && items * S < target)
+        S *= 2;
+    const size_t smem = sizeof(float) * ((size_t)m * dx + (size_t)(S - 1) * (kMergeThreads / S) * 8);
+    cudaError_t e = cudaFuncSetAttribute(block_merge_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_merge_kernel, kMergeThreads,
+                                                      smem);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        per_sm = 1;
+    const int ipc = kMergeThreads / S;
+    const long long ntiles = (items + ipc - 1) / ipc;
+    long long grid = (long long)num_sms * per_sm;
+    if (grid > ntiles)
+        grid = ntiles;
+    block_merge_kernel<<<(unsigned)grid, kMergeThreads, smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(x), w, static_cast<__nv_bfloat16 *>(out), B, L, H, dx,
+        m, S);
+    return cudaGetLastError();
+}
+
+}  // namespace hyb

@@ -1,0 +1,369 @@
+// index_topk.cu -- stage 2 of CSA ("deepseek-v4" blog, section 1, CSA: a
+// lightning indexer picks the top-K compressed entries for the current
+// query).  Score: I[t, s] = sum_h wi[t, h] * relu(qi[t, h, :] . kic[s, :]),
+// kept in fp32, over the entries visible to t; then an exact top-K with ties
+// resolved toward the lower entry index, written in ascending index order.
+//
+// Two kernels:
+//   index_scores_simt  CUDA-core scores for a tile of query rows x keys into a
+//                      workspace row per query (only the visible prefix);
+//                      used for decode (one query row per sequence, the
+//                      kic stream from HBM is the bound) and small shapes.
+//   topk_radix         one CTA per query row: order-preserving uint32 keys in
+//                      shared memory, a 12 + 10 + 10-bit radix select of the
+//                      K-th largest key, then an index-order emission that
+//                      takes every key above the threshold and the lowest-
+//                      index keys equal to it.
+#include "common.cuh"
+
+namespace hyb {
+
+// Number of compressed entries visible to a query at absolute position t:
+// j is visible iff (j + 1) * m - 1 < t - W + 1.
+__device__ __forceinline__ int visible_entries(long long t, int m, int W, int Nc)
+{
+    long long a = t - W + 1;
+    if (a <= 0)
+        return 0;
+    long long n = a / m;
+    return n < Nc ? (int)n : Nc;
+}
+
+// ------------------------------------------------------------------------
+// Scores on CUDA cores.  CTA tile: kRows query rows x kKeys entries.  The
+// key tile and the query tile are staged in shared memory as fp32 (rows of
+// the key tile padded by one float so that 16 different keys read by a warp
+// fall in distinct banks).
+// ------------------------------------------------------------------------
+constexpr int kScRows = 16;
+constexpr int kScKeys = 128;
+constexpr int kScThreads = 256;
+
+__global__ void __launch_bounds__(kScThreads)
+index_scores_simt(const __nv_bfloat16 *__restrict__ qi, const float *__restrict__ wi,
+                  const __nv_bfloat16 *__restrict__ kic, float *__restrict__ scores, int B, int Lq,
+                  int Hi, int di, int Nc, int m, int W, const int32_t *__restrict__ q_pos)
+{
+    extern __shared__ __align__(16) float sm_sc[];
+    const int ldk = di + 1;
+    float *sk = sm_sc;                                 // [kScKeys][di + 1]
+    float *sq = sk + kScKeys * ldk;                    // [kScRows][Hi][di]
+    float *sw = sq + kScRows * Hi * di;                // [kScRows][Hi]
+    int *snv = reinterpret_cast<int *>(sw + kScRows * Hi);  // [kScRows]
+
+    const int b = blockIdx.z;
+    const int r0 = blockIdx.y * kScRows;
+    const int k0 = blockIdx.x * kScKeys;
+    const int tid = threadIdx.x;
+
+    if (tid < kScRows) {
+        int t = r0 + tid;
+        int nv = 0;
+        if (t < Lq) {
+            long long pos = q_pos ? q_pos[(size_t)b * Lq + t] : t;
+            nv = visible_entries(pos, m, W, Nc);
+        }
+        snv[tid] = nv;
+    }
+    __syncthreads();
+    int nv_max = 0;
+#pragma unroll 1
+    for (int r = 0; r < kScRows; ++r)
+        nv_max = max(nv_max, snv[r]);
+    if (k0 >= nv_max)
+        return;  // no row of this tile sees any entry of this key tile
+
+    // stage keys (bf16 -> fp32), 8 channels per thread step
+    const int kd8 = di / 8;
+    for (int e = tid; e < kScKeys * kd8; e += kScThreads) {
+        int kk = e / kd8, c8 = e % kd8;
+        int s = k0 + kk;
+        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (s < Nc) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(kic + ((size_t)b * Nc + s) * di + c8 * 8));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float2 f = __bfloat1622float2(h2[q]);
+                v[2 * q] = f.x;
+                v[2 * q + 1] = f.y;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            sk[kk * ldk + c8 * 8 + q] = v[q];
+    }
+    const int qd8 = Hi * di / 8;
+    for (int e = tid; e < kScRows * qd8; e += kScThreads) {
+        int r = e / qd8, c8 = e % qd8;
+        int t = r0 + r;
+        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (t < Lq) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi + ((size_t)b * Lq + t) * Hi * di + c8 * 8));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float2 f = __bfloat1622float2(h2[q]);
+                v[2 * q] = f.x;
+                v[2 * q + 1] = f.y;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            sq[r * Hi * di + c8 * 8 + q] = v[q];
+    }
+    for (int e = tid; e < kScRows * Hi; e += kScThreads) {
+        int r = e / Hi, h = e % Hi;
+        int t = r0 + r;
+        sw[e] = t < Lq ? wi[((size_t)b * Lq + t) * Hi + h] : 0.f;
+    }
+    __syncthreads();
+
+    // thread -> (row, key lane); each thread scores kScKeys / 16 keys of one row
+    const int r = tid / 16;
+    const int kl = tid % 16;
+    const int t = r0 + r;
+    if (t >= Lq)
+        return;
+    const int nv = snv[r];
+    float *out = scores + ((size_t)b * Lq + t) * Nc;
+    for (int kk = kl; kk < kScKeys; kk += 16) {
+        const int s = k0 + kk;
+        if (s >= nv)
+            break;
+        float I = 0.f;
+        for (int h = 0; h < Hi; ++h) {
+            const float *qv = sq + (r * Hi + h) * di;
+            const float *kv = sk + kk * ldk;
+            float dot = 0.f;
+            for (int c = 0; c < di; ++c)
+                dot = fmaf(qv[c], kv[c], dot);
+            I = fmaf(sw[r * Hi + h], fmaxf(dot, 0.f), I);
+        }
+        out[s] = I;
+    }
+}
+
+cudaError_t launch_index_scores_simt(const void *qi, const float *wi, const void *kic, float *scores,
+                                     int B, int Lq, int Hi, int di, int Nc, int m, int W,
+                                     const int32_t *q_pos, cudaStream_t stream)
+{
+    const size_t smem = sizeof(float) * ((size_t)kScKeys * (di + 1) + (size_t)kScRows * Hi * di +
+                                         (size_t)kScRows * Hi) +
+                        sizeof(int) * kScRows;
+    cudaError_t e = cudaFuncSetAttribute(index_scores_simt,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid((Nc + kScKeys - 1) / kScKeys, (Lq + kScRows - 1) / kScRows, B);
+    index_scores_simt<<<grid, kScThreads, smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(qi), wi, static_cast<const __nv_bfloat16 *>(kic), scores,
+        B, Lq, Hi, di, Nc, m, W, q_pos);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------
+// Exact top-K by radix select.
+// ------------------------------------------------------------------------
+constexpr int kTkThreads = 512;
+constexpr int kTkWarps = kTkThreads / 32;
+
+// Larger float -> larger unsigned key; -0.0 is folded onto +0.0 first so that
+// equal scores give equal keys.
+__device__ __forceinline__ uint32_t order_key(float f)
+{
+    uint32_t u = __float_as_uint(f + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix sum (in thread order) of one value per thread.
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off)
+            x += y;
+    }
+    if (lane == 31)
+        warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int w = lane < kTkWarps ? warp_tot[lane] : 0;
+        int inc = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off)
+                inc += y;
+        }
+        if (lane < kTkWarps)
+            warp_tot[lane] = inc - w;  // exclusive warp offsets
+        if (lane == kTkWarps - 1)
+            *total = inc;
+    }
+    __syncthreads();
+    int r = warp_tot[wid] + x - v;
+    __syncthreads();
+    return r;
+}
+
+// Histogram the digit (key >> shift) & (NB - 1) of the keys whose bits under
+// `pmask` equal `prefix`; then find the digit holding the `need`-th largest
+// such key.  Returns that digit; *above receives the number of matching keys
+// with a larger digit.
+template <int BITS>
+__device__ int radix_pass(const uint32_t *keys, int n, uint32_t prefix, uint32_t pmask, int shift,
+                          int need, int *hist, int *warp_tot, int *scratch, int *above)
+{
+    constexpr int NB = 1 << BITS;
+    for (int i = threadIdx.x; i < NB; i += kTkThreads)
+        hist[i] = 0;
+    __syncthreads();
+    const int n_round = (n + kTkThreads - 1) / kTkThreads * kTkThreads;
+    for (int i = threadIdx.x; i < n_round; i += kTkThreads) {
+        uint32_t k = i < n ? keys[i] : 0u;
+        bool match = i < n && (k & pmask) == prefix;
+        unsigned active = __ballot_sync(0xffffffffu, match);
+        if (match) {
+            int dg = (int)((k >> shift) & (NB - 1));
+            unsigned peers = __match_any_sync(active, dg);
+            if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31))
+                atomicAdd(&hist[dg], __popc(peers));
+        }
+    }
+    __syncthreads();
+    // thread t owns PER consecutive bins counted down from the top digit
+    constexpr int PER = (NB + kTkThreads - 1) / kTkThreads;
+    int mine = 0;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        int bin = NB - 1 - ((int)threadIdx.x * PER + q);
+        if (bin >= 0)
+            mine += hist[bin];
+    }
+    const int ex = block_excl_scan(mine, warp_tot, scratch);  // keys in higher runs
+    if (ex < need && ex + mine >= need) {
+        int acc = ex;
+        for (int q = 0; q < PER; ++q) {
+            int bin = NB - 1 - ((int)threadIdx.x * PER + q);
+            int c = hist[bin];
+            if (acc + c >= need) {
+                scratch[1] = bin;
+                scratch[2] = acc;
+                break;
+            }
+            acc += c;
+        }
+    }
+    __syncthreads();
+    const int dg = scratch[1];
+    *above = scratch[2];
+    __syncthreads();
+    return dg;
+}
+
+__global__ void __launch_bounds__(kTkThreads)
+topk_radix(const float *__restrict__ scores, int B, int Lq, int Nc, int m, int W, int K,
+           const int32_t *__restrict__ q_pos, int32_t *__restrict__ idx_out,
+           float *__restrict__ sel_scores)
+{
+    extern __shared__ __align__(16) uint32_t sm_tk[];
+    __shared__ int hist[4096];
+    __shared__ int warp_tot[32];
+    __shared__ int scratch[4];
+
+    const int row = blockIdx.x;  // b * Lq + t
+    const int b = row / Lq;
+    const int t = row % Lq;
+    const long long pos = q_pos ? q_pos[row] : t;
+    const int n = visible_entries(pos, m, W, Nc);
+    const int keff = n < K ? n : K;
+    const float *src = scores + (size_t)row * Nc;
+    int32_t *dst = idx_out + (size_t)row * K;
+    float *dsc = sel_scores ? sel_scores + (size_t)row * K : nullptr;
+    (void)b;
+
+    if (keff == n) {  // every visible entry is selected
+        for (int i = threadIdx.x; i < K; i += kTkThreads) {
+            dst[i] = i < n ? i : -1;
+            if (dsc)
+                dsc[i] = i < n ? src[i] : -INFINITY;
+        }
+        return;
+    }
+
+    uint32_t *keys = sm_tk;
+    for (int i = threadIdx.x; i < n; i += kTkThreads)
+        keys[i] = order_key(src[i]);
+    __syncthreads();
+
+    int need = keff, above;
+    uint32_t prefix = 0, pmask = 0;
+    int dg = radix_pass<12>(keys, n, prefix, pmask, 20, need, hist, warp_tot, scratch, &above);
+    need -= above;
+    prefix |= (uint32_t)dg << 20;
+    pmask |= 0xFFFu << 20;
+    dg = radix_pass<10>(keys, n, prefix, pmask, 10, need, hist, warp_tot, scratch, &above);
+    need -= above;
+    prefix |= (uint32_t)dg << 10;
+    pmask |= 0x3FFu << 10;
+    dg = radix_pass<10>(keys, n, prefix, pmask, 0, need, hist, warp_tot, scratch, &above);
+    need -= above;
+    const uint32_t T = prefix | (uint32_t)dg;  // key of the K-th largest score
+    // select: every key > T, plus the `need` lowest-index keys == T
+
+    // contiguous chunk per thread (odd length: conflict-free shared reads)
+    int C = (n + kTkThreads - 1) / kTkThreads;
+    C |= 1;
+    const int i0 = threadIdx.x * C;
+    const int i1 = min(n, i0 + C);
+    int gt = 0, eq = 0;
+    for (int i = i0; i < i1; ++i) {
+        uint32_t k = keys[i];
+        gt += k > T;
+        eq += k == T;
+    }
+    int eq_before = block_excl_scan(eq, warp_tot, scratch);
+    int take_eq = min(eq, max(0, need - eq_before));
+    int sel = gt + take_eq;
+    int out_base = block_excl_scan(sel, warp_tot, scratch);
+    int e_seen = 0;
+    for (int i = i0; i < i1; ++i) {
+        uint32_t k = keys[i];
+        bool pick = k > T;
+        if (k == T) {
+            pick = e_seen < take_eq;
+            ++e_seen;
+        }
+        if (pick) {
+            dst[out_base] = i;
+            if (dsc)
+                dsc[out_base] = src[i];
+            ++out_base;
+        }
+    }
+    for (int i = keff + threadIdx.x; i < K; i += kTkThreads) {
+        dst[i] = -1;
+        if (dsc)
+            dsc[i] = -INFINITY;
+    }
+}
+
+cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m, int W, int K,
+                              const int32_t *q_pos, int32_t *idx, float *sel_scores,
+                              cudaStream_t stream)
+{
+    const size_t smem = sizeof(uint32_t) * (size_t)Nc;
+    cudaError_t e = cudaFuncSetAttribute(topk_radix, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    topk_radix<<<B * Lq, kTkThreads, smem, stream>>>(scores, B, Lq, Nc, m, W, K, q_pos, idx,
+                                                     sel_scores);
+    return cudaGetLastError();
+}
+
+}  // namespace hyb

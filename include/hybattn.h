@@ -1,0 +1,144 @@
+/*
+ * hybattn.h -- C ABI of the B200 (sm_100a) library for the forward pass of
+ * DeepSeek-V4-style hybrid attention: compressed sparse attention (CSA),
+ * heavily compressed attention (HCA) and a raw sliding window (SWA) under one
+ * softmax.
+ *
+ * Sources of the operations (web pages on DeepSeek-V4 hybrid attention):
+ *   "deepseek-v4" blog (s1mplewind), section 1 "hybrid attn": CSA (4:1
+ *     compression, lightning indexer, top-K per query, sparse attention), HCA
+ *     (m = 128, dense attention over the compressed history) and SWA (raw KV of
+ *     the latest 128 tokens plus the compressed history, fed to one attention).
+ *   CSDN "DeepSeek-V4 CSA / HCA mechanism" code page, section 1 (block_merge:
+ *     per-channel softmax of a [m, d] weight over the block positions, then a
+ *     weighted sum) and section 2 (block_compress).
+ *   CS336 lecture notes, "Attention Heads variants" (MQA / GQA head sharing)
+ *     and "Attention Alternatives" (FlashAttention; DSA lightning indexer).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *     and contiguous in the stated shape.  bf16 tensors are passed as void*.
+ *   - Every call is asynchronous on `stream`.  Argument errors are detected on
+ *     the host and returned before anything is launched.  Errors found by a
+ *     kernel (an index out of range, a wait that timed out) are recorded in a
+ *     per-device status word that hyb_get_device_status() reads and clears.
+ *   - The library never allocates device memory.  Scratch space comes from
+ *     the caller's workspace, sized by hyb_workspace_size().
+ *   - Supported shapes: head dim d in {64, 128}; indexer dim di in {32, 64};
+ *     Hq % Hkv == 0; sparse (top-K) attention needs Hq / Hkv <= 64 and
+ *     topk <= 2048; block size 1 <= m <= 256 with m * dx <= 32768.
+ *   - Visibility: compressed entry j (raw positions j*m .. j*m+m-1) is visible
+ *     to a query at position t iff (j + 1) * m - 1 < t - W + 1, i.e. it lies
+ *     entirely before the query's raw window [max(0, t-W+1), t].
+ */
+#ifndef HYBATTN_H
+#define HYBATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hyb_status {
+    HYB_OK = 0,
+    HYB_ERR_INVALID_ARG = -1,     /* null pointer, bad size, inconsistent shape   */
+    HYB_ERR_UNSUPPORTED = -2,     /* a valid shape this build does not implement  */
+    HYB_ERR_WORKSPACE = -3,       /* workspace missing or smaller than required   */
+    HYB_ERR_CUDA = -4,            /* a CUDA runtime call failed                   */
+    HYB_ERR_DEVICE_TIMEOUT = -5,  /* a kernel wait exceeded its bound (device)    */
+    HYB_ERR_DEVICE_BOUNDS = -6    /* a kernel met an out-of-range index (device)  */
+} hyb_status;
+
+/* Problem description shared by the indexer, the attention and the fused
+ * entry point.  Prefill: Lq == Lkv == L, q_pos == NULL, kv_pos0 == NULL.
+ * Decode: Lq == 1, q_pos[b] = absolute position of the query, raw rows are the
+ * last Lkv tokens with kv_pos0[b] = position of raw row 0, and the compressed
+ * caches hold Nc entries per sequence. */
+typedef struct hyb_problem {
+    int B;          /* sequences                                              */
+    int Lq;         /* query tokens per sequence                              */
+    int Lkv;        /* raw K/V rows per sequence                              */
+    int Hq;         /* query heads                                            */
+    int Hkv;        /* KV heads; query head h uses KV head h / (Hq / Hkv)     */
+    int d;          /* head dim (64 or 128)                                   */
+    int m;          /* compression block size (CSA 4, HCA 128)                */
+    int W;          /* sliding-window length in tokens (0 disables the window)*/
+    int topk;       /* K of the per-query top-K; <= 0 selects HCA (dense)     */
+    int Hi;         /* indexer heads (CSA only)                               */
+    int di;         /* indexer dim (CSA only)                                 */
+    int Nc;         /* compressed entries per sequence (cache capacity)       */
+    float scale;    /* softmax scale; 0 means 1/sqrt(d)                       */
+    const int32_t *q_pos;    /* [B, Lq] absolute query positions, or NULL (t) */
+    const int32_t *kv_pos0;  /* [B] position of raw row 0, or NULL (0)        */
+} hyb_problem;
+
+/* Bytes of device workspace hyb_csa_index_topk / hyb_fused_fwd need for `p`
+ * (0 for HCA).  The workspace must be 256-byte aligned. */
+size_t hyb_workspace_size(const hyb_problem *p);
+
+/* Stage 1, block_merge (CSDN code page, section 1):
+ *   out[b, j, h, c] = sum_{i<m} P[i, c] * x[b, j*m + i, h, c],
+ *   P[i, c] = exp(w[i, c]) / sum_{i'} exp(w[i', c]),  j < floor(L / m).
+ * x: [B, L, H, dx] bf16; w: [m, dx] fp32; out: [B, floor(L/m), H, dx] bf16
+ * (fp32 accumulation, rounded to nearest even).  A trailing partial block is
+ * ignored.  Used for the K and V caches (d) and the indexer keys (di, H = 1). */
+hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m,
+                            const float *w, void *out, cudaStream_t stream);
+
+/* Stage 2, lightning indexer + exact per-query top-K (deepseek-v4 blog,
+ * section 1, CSA; formula: ReLU-weighted head sum):
+ *   I[t, s] = sum_h wi[t, h] * max(0, qi[t, h, :] . kic[s, :])   (fp32)
+ * over the entries s visible to query t, then the K largest, ties to the
+ * lower s.  idx[b, t, :] receives the chosen entries in ascending order, -1
+ * padded when fewer than K are visible.  sel_scores (nullable) receives the
+ * fp32 score of each idx slot (-inf for padding).
+ * qi: [B, Lq, Hi, di] bf16; wi: [B, Lq, Hi] fp32; kic: [B, Nc, di] bf16;
+ * idx: [B, Lq, topk] int32; ws: workspace of >= hyb_workspace_size(p) bytes. */
+hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float *wi,
+                              const void *kic, int32_t *idx, float *sel_scores,
+                              void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Stage 3, hybrid attention (deepseek-v4 blog, section 1, SWA): for every
+ * (b, t, h) one softmax over
+ *   compressed keys  idx[b, t, :] entries that are >= 0 and visible (CSA), or
+ *                    every visible entry when idx == NULL (HCA), and
+ *   raw keys         positions max(0, t-W+1) .. t (rows p - kv_pos0[b]),
+ *   o = sum softmax(scale * q . k) v,  lse = log sum exp(scale * q . k).
+ * q: [B, Lq, Hq, d]; kc, vc: [B, Nc, Hkv, d]; k_raw, v_raw: [B, Lkv, Hkv, d],
+ * all bf16; idx: [B, Lq, topk] int32 (distinct entries) or NULL;
+ * o: [B, Lq, Hq, d] bf16; lse: [B, Hq, Lq] fp32 (nullable).  An empty key set
+ * gives o = 0 and lse = -inf.  idx entries >= Nc are skipped and flagged as
+ * HYB_ERR_DEVICE_BOUNDS. */
+hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                        const int32_t *idx, const void *k_raw, const void *v_raw, void *o,
+                        float *lse, cudaStream_t stream);
+
+/* The whole forward pass on one stream:
+ *   prefill (wk != NULL): kc = block_merge(k_raw, wk), vc = block_merge(v_raw, wv)
+ *     and, for CSA, kic = block_merge(ki_raw, wib); Nc must equal Lkv / m.
+ *   decode (wk == NULL): kc, vc, kic are read as ready caches of Nc entries.
+ *   CSA (topk > 0): idx = top-K of the indexer scores (stage 2).
+ *   then o, lse = hybrid attention (stage 3).
+ * ki_raw: [B, Lkv, di] bf16; wk, wv: [m, d] fp32; wib: [m, di] fp32;
+ * kc, vc: [B, Nc, Hkv, d]; kic: [B, Nc, di]; idx: [B, Lq, topk] (CSA only).
+ * ws must hold hyb_workspace_size(p) bytes. */
+hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
+                         const void *v_raw, const float *wk, const float *wv, const void *qi,
+                         const float *wi, const void *ki_raw, const float *wib, void *kc,
+                         void *vc, void *kic, int32_t *idx, void *o, float *lse, void *ws,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device (HYB_OK, HYB_ERR_DEVICE_TIMEOUT or HYB_ERR_DEVICE_BOUNDS). */
+hyb_status hyb_get_device_status(cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *hyb_error_string(hyb_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYBATTN_H */

@@ -1,0 +1,61 @@
+"""The C-ABI library loads and exports every entry point of include/hybattn.h,
+and host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hybattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from compressed_sparse_sliding_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyb_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert {"hyb_hca_compress", "hyb_csa_index_topk", "hyb_attn_fwd", "hyb_fused_fwd",
+            "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_error_strings(lib):
+    lib.hyb_error_string.restype = ctypes.c_char_p
+    for code in range(-6, 1):
+        assert lib.hyb_error_string(code)
+    assert lib.hyb_error_string(0) == b"ok"
+
+
+def test_host_side_argument_checks(lib):
+    import compressed_sparse_sliding_b200 as hb
+    # null inputs are rejected before any launch
+    st = hb._lib.hyb_hca_compress(None, 1, 8, 1, 64, 4, None, None, None)
+    assert st == hb.HYB_ERR_INVALID_ARG
+    p = hb.problem(B=1, Lq=16, Lkv=16, Hq=4, Hkv=3, d=64, m=4, W=8)
+    assert hb._lib.hyb_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, None,
+                                None) == hb.HYB_ERR_INVALID_ARG
+    p = hb.problem(B=1, Lq=16, Lkv=16, Hq=4, Hkv=1, d=96, m=4, W=8)
+    assert hb._lib.hyb_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, None,
+                                None) == hb.HYB_ERR_UNSUPPORTED
+    # workspace: scores of every (query row, entry) pair, fp32, 256-byte rounded
+    p = hb.problem(B=2, Lq=100, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=2, di=32, Nc=25)
+    assert hb.hyb_workspace_size(p) == (2 * 100 * 25 * 4 + 255) // 256 * 256
+    p.topk = 0
+    assert hb.hyb_workspace_size(p) == 0
+    # missing workspace is reported as such
+    p = hb.problem(B=1, Lq=8, Lkv=8, Hq=4, Hkv=1, d=64, m=4, W=8, topk=4, Hi=2, di=32, Nc=2)
+    buf = ctypes.c_void_p(256)
+    st = hb._lib.hyb_csa_index_topk(ctypes.byref(p), buf, buf, buf, buf, None, None, 0, None)
+    assert st == hb.HYB_ERR_WORKSPACE
