@@ -4,3 +4,4 @@
 #include "index_topk.cu"
 #include "attn.cu"
 #include "api.cu"
+#include "noalloc.cu"

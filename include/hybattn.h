@@ -101,6 +101,29 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
                               const void *kic, int32_t *idx, float *sel_scores,
                               void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Bytes of the fixed device scratch behind hyb_csa_index_topk_noalloc. */
+#define HYB_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* Stage 2 without a workspace (the pages have no counterpart: this is a
+ * service of the library, not a step of the method).  Same inputs, outputs
+ * and results as hyb_csa_index_topk, but the score rows live in a fixed
+ * 8 MiB device array inside the library, so the call allocates nothing and
+ * needs no workspace.  Meant for callers that may not allocate device memory
+ * themselves: an engine whose memory planner owns every buffer, or a decode
+ * loop where cudaMalloc / cudaFree would synchronise the device.
+ *   - B * Lq * Nc * 4 bytes must fit in HYB_NOALLOC_SCRATCH_BYTES, otherwise
+ *     the call returns HYB_ERR_UNSUPPORTED and launches nothing (the decode
+ *     shape 64 x 16384 entries uses 4 MiB).
+ *   - Every GPU that loads the library holds the array until the process
+ *     exits.  The first call on a device looks up the array's address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels overlap on the GPU (for
+ *     example on different streams) race and must be serialised by the
+ *     caller.  Nothing in it needs clearing between calls. */
+hyb_status hyb_csa_index_topk_noalloc(const hyb_problem *p, const void *qi, const float *wi,
+                                      const void *kic, int32_t *idx, float *sel_scores,
+                                      cudaStream_t stream);
+
 /* Stage 3, hybrid attention (deepseek-v4 blog, section 1, SWA): for every
  * (b, t, h) one softmax over
  *   compressed keys  idx[b, t, :] entries that are >= 0 and visible (CSA), or
