@@ -2,6 +2,7 @@
 // the host, workspace carve-up and kernel launches on the caller's stream.
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 
@@ -14,9 +15,19 @@ cudaError_t launch_block_merge(const void *x, int B, int L, int H, int dx, int m
 cudaError_t launch_index_scores_simt(const void *qi, const float *wi, const void *kic, float *scores,
                                      int B, int Lq, int Hi, int di, int Nc, int m, int W,
                                      const int32_t *q_pos, cudaStream_t stream);
+cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *kic, float *scores,
+                                   int B, int Lq, int Hi, int di, int Nc, int m, int W,
+                                   const int32_t *q_pos, cudaStream_t stream);
 cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m, int W, int K,
                               const int32_t *q_pos, int32_t *idx, float *sel_scores,
                               cudaStream_t stream);
+cudaError_t launch_hca_attn(int B, int L, int Lkv, int Hq, int Hkv, int d, int Nc, int m, int W,
+                            float scale, const void *q, const void *kc, const void *vc, const void *kr,
+                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms);
+cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int m, int W, int topk,
+                            float scale, const int32_t *q_pos, const int32_t *kv_pos0, const void *q,
+                            const void *kc, const void *vc, const int32_t *idx, const void *kr,
+                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms);
 cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, int Nc, int m, int W,
                                int topk, float scale, const int32_t *q_pos, const int32_t *kv_pos0,
                                const void *q, const void *kc, const void *vc, const int32_t *idx,
@@ -36,9 +47,15 @@ static bool aligned16(const void *p)
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// With HYB_VERBOSE set in the environment, failed CUDA calls are reported on stderr.
 static hyb_status cuda_status(cudaError_t e)
 {
-    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+    if (e == cudaSuccess)
+        return HYB_OK;
+    static const bool verbose = getenv("HYB_VERBOSE") != nullptr;
+    if (verbose)
+        fprintf(stderr, "hybattn: CUDA error %d: %s\n", (int)e, cudaGetErrorString(e));
+    return HYB_ERR_CUDA;
 }
 
 // Largest shared-memory footprint of one top-K row (keys) + static tables.
@@ -116,8 +133,12 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return HYB_ERR_WORKSPACE;
     float *scores = static_cast<float *>(ws);
-    cudaError_t e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
-                                             p->m, p->W, p->q_pos, stream);
+    // tensor cores for prefill-sized query tiles, CUDA cores otherwise
+    cudaError_t e = launch_index_scores_tc(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
+                                           p->m, p->W, p->q_pos, stream);
+    if (e == cudaErrorNotSupported)
+        e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc, p->m,
+                                     p->W, p->q_pos, stream);
     if (e != cudaSuccess)
         return HYB_ERR_CUDA;
     e = launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos, idx, sel_scores,
@@ -144,6 +165,18 @@ hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, con
     if (p->Lkv <= 0 && p->W > 0)
         return HYB_ERR_INVALID_ARG;
     const int Lkv = p->Lkv > 0 ? p->Lkv : 1;
+    if (!idx && !p->q_pos && !p->kv_pos0 && p->Lq == p->Lkv) {
+        // prefill HCA: persistent two-tile kernel
+        return cuda_status(launch_hca_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->d, p->Nc, p->m, p->W,
+                                           softmax_scale(p), q, kc, vc, k_raw, v_raw, o, lse, stream,
+                                           num_sms_current()));
+    }
+    if (idx && p->d == 128 && p->Nc > 0) {
+        // CSA: per-token selections, transposed tcgen05 kernel
+        return cuda_status(launch_csa_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->Nc, p->m, p->W,
+                                           p->topk, softmax_scale(p), p->q_pos, p->kv_pos0, q, kc, vc,
+                                           idx, k_raw, v_raw, o, lse, stream, num_sms_current()));
+    }
     cudaError_t e = launch_hybrid_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->d, p->Nc, p->m, p->W,
                                        p->topk, softmax_scale(p), p->q_pos, p->kv_pos0, q, kc, vc, idx,
                                        k_raw, v_raw, o, lse, stream);

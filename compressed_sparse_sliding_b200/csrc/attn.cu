@@ -75,19 +75,6 @@ __device__ __forceinline__ int n_visible(long long t, int m, int W, int Nc)
     return n < Nc ? (int)n : Nc;
 }
 
-// Bounded wait used while unwinding: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t addr = smem_u32(bar);
-    uint64_t t0 = global_ns();
-    while (!mbar_try_wait(addr, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) {
-            set_error(HYB_ERR_DEVICE_TIMEOUT);
-            return;
-        }
-    }
-}
-
 template <int D, bool SPARSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 hybrid_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
@@ -523,44 +510,6 @@ hybrid_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// 4-D map over a [N3][N2][N1][d] bf16 tensor with a (64, box1, box2, 1) box and
-// 128-byte swizzle.  Out-of-range elements read as zero.
-static bool make_map(CUtensorMap *map, const void *base, int d, int n1, int n2, int n3, int box1,
-                     int box2)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn)
-        return false;
-    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
-    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * n1,
-                             (cuuint64_t)d * 2 * n1 * n2};
-    cuuint32_t box[4] = {64, (cuuint32_t)box1, (cuuint32_t)box2, 1};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
-                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int D, bool SPARSE>
 static cudaError_t launch_attn_t(const AttnParams &p, const void *q, cudaStream_t stream)
 {

@@ -1,0 +1,725 @@
+// attn_sparse.cu -- stage 3 for CSA ("deepseek-v4" blog, section 1, CSA and
+// SWA): every query token attends to its own top-K compressed entries plus
+// the raw window, with all query heads of a KV group (MQA / GQA, CS336
+// "Attention Heads variants") sharing those keys.
+//
+// Because each token has its own key set, query rows of different tokens
+// cannot share a key tile.  The kernel therefore computes the transposed
+// products with the keys in the MMA's M dimension:
+//     S^T [128 keys x NH heads]  = K_tile [128 x d] . Q^T        (tcgen05, TMEM)
+//     O^T [d x NH]              += V_tile^T [d x 128] . P^T       (V as MN-major A)
+// where NH is the group's head count padded to 16, 32 or 64.  No MMA row is
+// padding for the 32- and 64-head groups of the CSA workloads.
+//
+// Softmax: thread = key (TMEM lane), holding that key's NH scores.  A per-head
+// reference max lives in shared memory; it is moved (with a block-wide max
+// reduction, and a rescale of O^T and of the partial sums) only when some key
+// exceeds it by more than 2^8, i.e. on the first tile of a token and rarely
+// after.  Partial row sums stay per thread and are reduced once per token.
+// P^T is written to shared memory in the 32/64/128-byte swizzle matching NH.
+//
+// Gathers: two producer warps copy the selected compressed rows and the
+// window rows with 16-byte cp.async (16 lanes per 256-byte row, so every warp
+// instruction moves two whole rows) straight into the 128-byte-swizzled tile
+// layout; each thread then arms the stage's mbarrier with an asynchronous
+// arrive that fires when its copies land, so the producers never block on a
+// copy.  Unselected, invisible or out-of-range slots are zero-filled and
+// masked.  The token's selection list is staged once in shared memory.
+// Roles (224 threads): warps 0-3 softmax + epilogue, warps 4-5 producer,
+// warp 6 MMA; work items (b, t, KV head) go round-robin to persistent CTAs.
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kSpThreads = 224;
+constexpr int kSpBN = 128;     // keys per tile (the M of S^T)
+constexpr int kSpKS = 3;       // K ring depth
+constexpr int kSpVS = 2;       // V ring depth
+constexpr int kSpD = 128;      // head dim handled by this kernel
+
+struct SparseParams {
+    int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
+    long long n_items;
+    float scale_log2;
+    const int32_t *q_pos, *kv_pos0, *idx;
+    const __nv_bfloat16 *kc, *vc, *kr, *vr;   // [B, rows, Hkv, 128]
+    __nv_bfloat16 *o;
+    float *lse;
+};
+
+template <int NH>
+struct SparseSmem {
+    static constexpr int Q_BYTES = NH * kSpD * 2;
+    static constexpr int KV_BYTES = kSpBN * kSpD * 2;
+    static constexpr int P_BYTES = kSpBN * NH * 2;
+    static constexpr int OFF_Q = 0;                                // 2 buffers
+    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+    static constexpr int OFF_V = OFF_K + kSpKS * KV_BYTES;
+    static constexpr int OFF_P = OFF_V + kSpVS * KV_BYTES;
+    static constexpr int OFF_RED = OFF_P + ((P_BYTES + 1023) & ~1023);  // [4][NH] floats
+    static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;             // [NH] floats
+    static constexpr int OFF_BAR = OFF_MREF + NH * 4;
+    static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
+    static constexpr int OFF_IDX = OFF_MISC + 16 * 4;               // producer's selection list
+    static constexpr int BASE_BYTES = OFF_IDX;                      // + topk * 4
+};
+
+enum {
+    SB_QF = 0, SB_QE = 2, SB_KF = 4, SB_KE = 7, SB_VF = 10, SB_VE = 12, SB_SF = 14, SB_PF = 16,
+    SB_OD = 17, SB_OE = 18, SB_DONE = 20
+};
+
+struct SparseTok {
+    int b, t, kvh;
+    long long pos, kv0;
+    int nct, nrt, rlo, rhi;
+};
+
+__device__ __forceinline__ SparseTok sparse_tok(const SparseParams &p, long long w)
+{
+    SparseTok k;
+    k.kvh = (int)(w % p.Hkv);
+    const long long bt = w / p.Hkv;
+    k.b = (int)(bt / p.Lq);
+    k.t = (int)(bt % p.Lq);
+    k.pos = p.q_pos ? p.q_pos[bt] : k.t;
+    k.kv0 = p.kv_pos0 ? p.kv_pos0[k.b] : 0;
+    k.nct = (p.topk + kSpBN - 1) / kSpBN;
+    long long lo = k.pos - p.W + 1;
+    if (lo < 0)
+        lo = 0;
+    lo -= k.kv0;
+    if (lo < 0)
+        lo = 0;
+    long long hi = k.pos - k.kv0;
+    if (hi > p.Lkv - 1)
+        hi = p.Lkv - 1;
+    k.rlo = (int)lo;
+    k.rhi = (int)hi;
+    k.nrt = (p.W > 0 && hi >= lo) ? (int)((hi - lo + kSpBN) / kSpBN) : 0;
+    return k;
+}
+
+// Selection entry of key slot c of tile i (compressed tiles only; -1 past topk
+// and for raw tiles).  Loads are issued a tile ahead of their use.
+__device__ __forceinline__ int slot_entry(const SparseParams &p, const SparseTok &k, int i, int c)
+{
+    if (i >= k.nct)
+        return -1;
+    const int s = i * kSpBN + c;
+    return s < p.topk ? __ldg(p.idx + ((size_t)k.b * p.Lq + k.t) * p.topk + s) : -1;
+}
+
+// Row of the flattened [B * rows * Hkv, d] view holding key slot c of tile i
+// (j: its selection entry), and whether the slot is a real key of the token.
+__device__ __forceinline__ bool slot_row(const SparseParams &p, const SparseTok &k, int i, int c, int j,
+                                         int *row)
+{
+    if (i < k.nct) {
+        const bool ok = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < k.pos - p.W + 1);
+        *row = ((k.b * p.Nc + (ok ? j : 0)) * p.Hkv) + k.kvh;
+        return ok;
+    }
+    const int r = k.rlo + (i - k.nct) * kSpBN + c;
+    const bool ok = r <= k.rhi;
+    *row = ((k.b * p.Lkv + (ok ? r : 0)) * p.Hkv) + k.kvh;
+    return ok;
+}
+
+// Arrive on `bar` once every cp.async issued so far by this thread has landed
+// (the pending count is raised first, so a regular arrive must follow).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier among the 64 producer threads (named barrier 2).
+__device__ __forceinline__ void prod_sync()
+{
+    asm volatile("bar.sync 2, 64;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// OR-reduction of a predicate over the 128 softmax threads (named barrier 1).
+__device__ __forceinline__ bool sm_any(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void sm_sync()
+{
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Shared-memory descriptor with a selectable swizzle (layout 2: 128 B, 4: 64 B, 6: 32 B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N])
+{
+    static_assert(N % 16 == 0, "");
+#pragma unroll
+    for (int c = 0; c < N; c += 16) {
+        uint32_t r[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+              "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+              "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr + c));
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            v[c + q] = __uint_as_float(r[q]);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float (&v)[N])
+{
+#pragma unroll
+    for (int c = 0; c < N; c += 16) {
+        uint32_t r[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            r[q] = __float_as_uint(v[c + q]);
+        tmem_st16(taddr + c, r);
+    }
+}
+
+template <int NH>
+__global__ void __launch_bounds__(kSpThreads, 1)
+csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_vr, const SparseParams p)
+{
+    using SM = SparseSmem<NH>;
+    constexpr int RB = NH * 2;                                  // bytes of one P^T row
+    constexpr uint32_t PLAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
+    constexpr int PCH = RB / 16;                                // 16-byte chunks per row
+    extern __shared__ __align__(1024) uint8_t sp_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sp_smem_raw) + 1023) &
+                                                ~(uintptr_t)1023);
+    uint8_t *sQ = smem + SM::OFF_Q;
+    uint8_t *sK = smem + SM::OFF_K;
+    uint8_t *sV = smem + SM::OFF_V;
+    uint8_t *sP = smem + SM::OFF_P;
+    float *sRed = reinterpret_cast<float *>(smem + SM::OFF_RED);
+    float *sMref = reinterpret_cast<float *>(smem + SM::OFF_MREF);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
+    int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
+    int *sIdx = reinterpret_cast<int *>(smem + SM::OFF_IDX);
+    volatile int *abort_flag = misc + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[SB_QF + s], 1);
+            mbar_init(&bar[SB_QE + s], 1);
+            mbar_init(&bar[SB_SF + s], 1);
+            mbar_init(&bar[SB_OE + s], 128);
+        }
+        for (int s = 0; s < kSpKS; ++s) {
+            mbar_init(&bar[SB_KF + s], 64);
+            mbar_init(&bar[SB_KE + s], 1);
+        }
+        for (int s = 0; s < kSpVS; ++s) {
+            mbar_init(&bar[SB_VF + s], 64);
+            mbar_init(&bar[SB_VE + s], 1);
+        }
+        mbar_init(&bar[SB_PF], 128);
+        mbar_init(&bar[SB_OD], 1);
+        mbar_init(&bar[SB_DONE], 1);
+        mbar_fence_init();
+        misc[1] = 0;
+    }
+    if (warp == 6)
+        tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+    // TMEM columns: S^T buffers at 0 and NH, O^T buffers at 2NH and 3NH
+    const uint32_t TM_S0 = 0, TM_O0 = 2 * NH;
+
+    if (warp == 4 || warp == 5) {
+        // ================================ producer ================================
+        // 64 threads: 16 lanes per 256-byte row, two rows per warp instruction
+        const int pt = threadIdx.x - 128;
+        const int c8 = pt & 15;                 // 16-byte chunk of the row
+        const uint32_t dchunk = (uint32_t)(c8 >> 3) * kSpBN * 128;
+        uint32_t kc = 0, vc = 0, nq = 0;
+        bool ok = true;
+        for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+            const SparseTok k = sparse_tok(p, w);
+            const int qb = nq & 1;
+            if (nq >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_QE + qb], ((nq >> 1) - 1) & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
+            if (pt == 0) {
+                mbar_arrive_expect_tx(&bar[SB_QF + qb], SM::Q_BYTES);
+                const int qrow = (int)(((long long)k.b * p.Lq + k.t) * p.Hq) + k.kvh * p.g;
+                for (int cb = 0; cb < 2; ++cb)
+                    tma_load_2d(sQ + qb * SM::Q_BYTES + cb * NH * 128, &tm_q, &bar[SB_QF + qb], cb * 64,
+                                qrow);
+            }
+            // the token's selection list, staged once (producer-private)
+            prod_sync();
+            const int32_t *irow = p.idx + ((size_t)k.b * p.Lq + k.t) * p.topk;
+            for (int q = pt; q < p.topk; q += 64)
+                sIdx[q] = __ldg(irow + q);
+            prod_sync();
+            const int nt = k.nct + k.nrt;
+            for (int i = 0; i < nt && ok; ++i) {
+                const bool comp = i < k.nct;
+                const __nv_bfloat16 *bk = comp ? p.kc : p.kr;
+                const __nv_bfloat16 *bv = comp ? p.vc : p.vr;
+                // source rows of this thread's 32 slots (row r = 4u + pt / 16)
+                uint32_t src[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int r = u * 4 + (pt >> 4);
+                    int row;
+                    bool v;
+                    if (comp) {
+                        const int sidx = i * kSpBN + r;
+                        const int j = sidx < p.topk ? sIdx[sidx] : -1;
+                        v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < k.pos - p.W + 1);
+                        if (j >= p.Nc && c8 == 0)
+                            set_error(HYB_ERR_DEVICE_BOUNDS);
+                        row = (k.b * p.Nc + (v ? j : 0)) * p.Hkv + k.kvh;
+                    } else {
+                        const int rr = k.rlo + (i - k.nct) * kSpBN + r;
+                        v = rr <= k.rhi;
+                        row = (k.b * p.Lkv + (v ? rr : 0)) * p.Hkv + k.kvh;
+                    }
+                    src[u] = v ? (uint32_t)row : 0xFFFFFFFFu;
+                }
+                const uint32_t ks = kc % kSpKS;
+                if (kc >= kSpKS &&
+                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_KE + ks], ((kc / kSpKS) - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                {
+                    const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int r = u * 4 + (pt >> 4);
+                        const bool v = src[u] != 0xFFFFFFFFu;
+                        cp_async_16(dst + sw128_offset(r, c8 & 7),
+                                    bk + (size_t)(v ? src[u] : 0) * kSpD + c8 * 8, v ? 16u : 0u);
+                    }
+                    cp_async_mbar_arrive(&bar[SB_KF + ks]);
+                    mbar_arrive(&bar[SB_KF + ks]);
+                }
+                ++kc;
+                const uint32_t vs = vc % kSpVS;
+                if (vc >= kSpVS &&
+                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_VE + vs], ((vc / kSpVS) - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                {
+                    const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int r = u * 4 + (pt >> 4);
+                        const bool v = src[u] != 0xFFFFFFFFu;
+                        cp_async_16(dst + sw128_offset(r, c8 & 7),
+                                    bv + (size_t)(v ? src[u] : 0) * kSpD + c8 * 8, v ? 16u : 0u);
+                    }
+                    cp_async_mbar_arrive(&bar[SB_VF + vs]);
+                    mbar_arrive(&bar[SB_VF + vs]);
+                }
+                ++vc;
+            }
+        }
+        // unwinding: every copy issued by this thread has landed
+        cp_async_wait_group<0>();
+        if (pt == 0) {
+            for (uint32_t q = (nq > 2 ? nq - 2 : 0); q < nq; ++q)
+                drain_wait(&bar[SB_QF + (q & 1)], (q >> 1) & 1);
+        }
+    } else if (warp == 6) {
+        // ================================ MMA issue ================================
+        if (lane == 0) {
+            const uint32_t idesc_qk = idesc_bf16(kSpBN, NH, false, false);
+            const uint32_t idesc_pv = idesc_bf16(kSpD, NH, true, true);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+            uint32_t kc = 0, vc = 0, nq = 0, gt = 0, pcnt = 0;
+            bool ok = true;
+            for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+                const SparseTok k = sparse_tok(p, w);
+                const int nt = k.nct + k.nrt;
+                const int qb = nq & 1, ob = nq & 1;
+                if (!mbar_wait(&bar[SB_QF + qb], (nq >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                auto issue_pv = [&](bool first) -> bool {
+                    const uint32_t vs = vc % kSpVS;
+                    if (!mbar_wait(&bar[SB_PF], pcnt & 1, abort_flag) ||
+                        !mbar_wait(&bar[SB_VF + vs], (vc / kSpVS) & 1, abort_flag))
+                        return false;
+                    ++pcnt;
+                    if (first && nq >= 2 &&
+                        !mbar_wait(&bar[SB_OE + ob], ((nq >> 1) - 1) & 1, abort_flag))
+                        return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kSpBN / 16; ++kk) {
+                        const uint64_t da = smem_desc(aV + vs * SM::KV_BYTES + kk * 16 * 128,
+                                                      kSpBN * 128, 1024, 2);
+                        const uint64_t db = smem_desc(aP + kk * 16 * RB, 16, 8 * RB, PLAYOUT);
+                        mma_bf16_ss(tmem + TM_O0 + ob * NH, da, db, idesc_pv,
+                                    (first && kk == 0) ? 0u : 1u);
+                    }
+                    mma_commit(&bar[SB_OD]);
+                    mma_commit(&bar[SB_VE + vs]);
+                    ++vc;
+                    return true;
+                };
+                for (int i = 0; i < nt; ++i, ++gt) {
+                    const uint32_t ks = kc % kSpKS;
+                    if (!mbar_wait(&bar[SB_KF + ks], (kc / kSpKS) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kSpD / 16; ++kk) {
+                        const uint64_t da = sw128_desc(aK + ks * SM::KV_BYTES + (kk >> 2) * kSpBN * 128 +
+                                                           (kk & 3) * 32, 16, 1024);
+                        const uint64_t db = sw128_desc(aQ + qb * SM::Q_BYTES + (kk >> 2) * NH * 128 +
+                                                           (kk & 3) * 32, 16, 1024);
+                        mma_bf16_ss(tmem + TM_S0 + (gt & 1) * NH, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bar[SB_SF + (gt & 1)]);
+                    mma_commit(&bar[SB_KE + ks]);
+                    ++kc;
+                    if (i == nt - 1)
+                        mma_commit(&bar[SB_QE + qb]);
+                    if (i > 0 && !issue_pv(i == 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok)
+                    break;
+                if (nt == 0) {
+                    mma_commit(&bar[SB_QE + qb]);
+                } else if (!issue_pv(nt == 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            mma_commit(&bar[SB_DONE]);
+            drain_wait(&bar[SB_DONE], 0);
+        }
+    } else {
+        // ========================== softmax + epilogue ==========================
+        const int quad = warp;                       // warps 0-3
+        const int r = quad * 32 + lane;              // key lane (S^T) / d lane (O^T)
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        uint32_t nq = 0, gt = 0;
+        bool ok = true;
+        const uint32_t prow = smem_u32(sP) + r * RB;
+        for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+            const SparseTok k = sparse_tok(p, w);
+            const int nt = k.nct + k.nrt;
+            const int ob = nq & 1;
+            float lpart[NH];
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+                lpart[h] = 0.f;
+            if (threadIdx.x < NH)
+                sMref[threadIdx.x] = -INFINITY;
+            sm_sync();
+            int jnext = slot_entry(p, k, 0, r);
+            for (int i = 0; i < nt; ++i, ++gt) {
+                int row_unused;
+                const bool valid = slot_row(p, k, i, r, jnext, &row_unused);
+                jnext = slot_entry(p, k, i + 1, r);  // next tile, in flight
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + (gt & 1)], (gt >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float s[NH];
+                tmem_ld_cols<NH>(tl + TM_S0 + (gt & 1) * NH, s);
+                tmem_ld_wait();
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
+                bool exceed = false;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    exceed |= s[h] > sMref[h] + 8.f;
+                if (sm_any(exceed)) {
+                    // block-wide max per head over this tile
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        float v = s[h];
+#pragma unroll
+                        for (int off = 16; off; off >>= 1)
+                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                        if (lane == 0)
+                            sRed[quad * NH + h] = v;
+                    }
+                    sm_sync();
+                    // new reference: the tile max where it exceeds the old one by
+                    // more than 2^8; every thread derives the same factors
+                    bool moved = false;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]),
+                                                fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
+                        const float old = sMref[h];
+                        const float nw = tmx > old + 8.f ? tmx : old;
+                        const float a = (nw == old) ? 1.f : (old == -INFINITY ? 0.f : ex2_approx(old - nw));
+                        moved |= a != 1.f;
+                        lpart[h] *= a;
+                    }
+                    if (i > 0 && moved) {
+                        // O^T holds every earlier PV of this token: wait for the
+                        // last one, then scale column h by its factor
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < NH; c += 16) {
+                            float ov[16];
+                            tmem_ld_cols<16>(tl + TM_O0 + ob * NH + c, ov);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                const int h = c + q;
+                                const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]),
+                                                        fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
+                                const float old = sMref[h];
+                                const float nw = tmx > old + 8.f ? tmx : old;
+                                ov[q] *= (nw == old) ? 1.f : (old == -INFINITY ? 0.f : ex2_approx(old - nw));
+                            }
+                            tmem_st_cols<16>(tl + TM_O0 + ob * NH + c, ov);
+                        }
+                        tmem_st_wait();
+                    }
+                    sm_sync();  // every thread has read the old reference
+                    if (threadIdx.x < NH) {
+                        const int h = threadIdx.x;
+                        const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]), fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
+                        const float old = sMref[h];
+                        sMref[h] = tmx > old + 8.f ? tmx : old;
+                    }
+                    sm_sync();
+                }
+                // P^T row of this key: exp2(s - mref), 0 for masked keys
+                uint32_t pk[NH / 2];
+#pragma unroll
+                for (int h = 0; h < NH; h += 2) {
+                    const float m0 = sMref[h], m1 = sMref[h + 1];
+                    const float e0 = (m0 == -INFINITY) ? 0.f : ex2_approx(s[h] - m0);
+                    const float e1 = (m1 == -INFINITY) ? 0.f : ex2_approx(s[h + 1] - m1);
+                    lpart[h] += e0;
+                    lpart[h + 1] += e1;
+                    pk[h >> 1] = pack_bf16x2(e0, e1);
+                }
+                // the P^T buffer is free once PV of the previous tile completed
+                if (gt > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int c = 0; c < PCH; ++c) {
+                    uint32_t phys;
+                    if (RB == 128)
+                        phys = c ^ (r & 7);
+                    else if (RB == 64)
+                        phys = c ^ ((r >> 1) & 3);
+                    else
+                        phys = c ^ ((r >> 2) & 1);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + phys * 16),
+                                 "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar[SB_PF]);
+            }
+            if (!ok)
+                break;
+            // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                float v = lpart[h];
+#pragma unroll
+                for (int off = 16; off; off >>= 1)
+                    v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0)
+                    sRed[quad * NH + h] = v;
+            }
+            bool have_o = nt > 0;
+            if (have_o) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            sm_sync();
+            float ov[NH];
+            if (have_o) {
+                tmem_ld_cols<NH>(tl + TM_O0 + ob * NH, ov);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    ov[h] = 0.f;
+            }
+            const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                if (h < p.g) {
+                    const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
+                    const float v = l > 0.f ? ov[h] / l : 0.f;
+                    p.o[obase + (size_t)h * kSpD + r] = __float2bfloat16_rn(v);
+                }
+            }
+            if (p.lse && r < p.g) {
+                const int h = r;
+                const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
+                p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + h) * p.Lq + k.t] =
+                    l > 0.f ? (sMref[h] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            }
+            sm_sync();  // sRed / sMref are reused by the next token
+            tc_fence_before();
+            mbar_arrive(&bar[SB_OE + ob]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 6) {
+        tc_fence_after();
+        tmem_dealloc((uint32_t)misc[0], 256);
+    }
+}
+
+// 2-D map over a [rows, 128] bf16 view with a (64, box_rows) box, 128-byte swizzle.
+static bool make_map_2d(CUtensorMap *map, const void *base, long long rows, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kSpD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kSpD * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int NH>
+static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void *kc, const void *vc,
+                                const void *kr, const void *vr, cudaStream_t stream, int num_sms)
+{
+    using SM = SparseSmem<NH>;
+    CUtensorMap mq, mkc, mvc, mkr, mvr;
+    bool ok = make_map_2d(&mq, q, (long long)p.B * p.Lq * p.Hq, NH);
+    ok &= make_map_2d(&mkc, kc, (long long)p.B * p.Nc * p.Hkv, 1);
+    ok &= make_map_2d(&mvc, vc, (long long)p.B * p.Nc * p.Hkv, 1);
+    ok &= make_map_2d(&mkr, kr, (long long)p.B * p.Lkv * p.Hkv, 1);
+    ok &= make_map_2d(&mvr, vr, (long long)p.B * p.Lkv * p.Hkv, 1);
+    if (!ok)
+        return cudaErrorInvalidValue;
+    size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.topk * 4;
+    auto kern = csa_attn_kernel<NH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSpThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        return cudaErrorLaunchOutOfResources;
+    long long grid = (long long)num_sms * per_sm;
+    if (grid > p.n_items)
+        grid = p.n_items;
+    if (grid < 1)
+        return cudaSuccess;
+    kern<<<(unsigned)grid, kSpThreads, smem, stream>>>(mq, mkc, mvc, mkr, mvr, p);
+    return cudaGetLastError();
+}
+
+// CSA attention with per-token selections, head dim 128, Hq / Hkv <= 64.
+cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int m, int W, int topk,
+                            float scale, const int32_t *q_pos, const int32_t *kv_pos0, const void *q,
+                            const void *kc, const void *vc, const int32_t *idx, const void *kr,
+                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms)
+{
+    SparseParams p;
+    p.B = B;
+    p.Lq = Lq;
+    p.Lkv = Lkv;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.g = Hq / Hkv;
+    p.Nc = Nc;
+    p.m = m;
+    p.W = W;
+    p.topk = topk;
+    p.NH = p.g <= 16 ? 16 : (p.g <= 32 ? 32 : 64);
+    p.n_items = (long long)B * Lq * Hkv;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.q_pos = q_pos;
+    p.kv_pos0 = kv_pos0;
+    p.idx = idx;
+    p.kc = static_cast<const __nv_bfloat16 *>(kc);
+    p.vc = static_cast<const __nv_bfloat16 *>(vc);
+    p.kr = static_cast<const __nv_bfloat16 *>(kr);
+    p.vr = static_cast<const __nv_bfloat16 *>(vr);
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    if (p.NH == 16)
+        return launch_csa_t<16>(p, q, kc, vc, kr, vr, stream, num_sms);
+    if (p.NH == 32)
+        return launch_csa_t<32>(p, q, kc, vc, kr, vr, stream, num_sms);
+    return launch_csa_t<64>(p, q, kc, vc, kr, vr, stream, num_sms);
+}
+
+}  // namespace hyb

@@ -2,6 +2,9 @@
 // status word and every kernel in one module without relocatable device code).
 #include "compress.cu"
 #include "index_topk.cu"
+#include "index_tc.cu"
 #include "attn.cu"
+#include "attn_dense.cu"
+#include "attn_sparse.cu"
 #include "api.cu"
 #include "noalloc.cu"

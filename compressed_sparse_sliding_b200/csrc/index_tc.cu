@@ -1,0 +1,274 @@
+// index_tc.cu -- lightning-indexer scores on tcgen05 for prefill ("deepseek-v4"
+// blog, section 1, CSA; score = ReLU-weighted head sum, fp32):
+//     I[t, s] = sum_h wi[t, h] * max(0, qi[t, h, :] . kic[s, :])
+// A CTA owns 128 query tokens and a run of 64-entry key tiles.  For every key
+// tile one MMA per indexer head writes D_h[128 tokens x 64 keys] (fp32) into
+// TMEM (two buffers of Hi x 64 columns); the epilogue thread of a token reads
+// the Hi accumulators of its row, forms the weighted ReLU sum and stores the
+// visible part of the tile into the token's score row.  Queries (one TMA box
+// per head) stay in shared memory; key tiles stream through a 4-stage ring.
+// Roles (256 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 4-7
+// epilogue (TMEM lane quadrants 0-3); warps 2-3 idle.
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kIxThreads = 256;
+constexpr int kIxBM = 128;        // query tokens per CTA
+constexpr int kIxBN = 64;         // keys per tile
+constexpr int kIxStages = 4;
+constexpr int kIxDi = 64;         // indexer dim handled here
+constexpr int kIxChunkTiles = 32; // key tiles per CTA (2048 entries)
+
+struct IndexParams {
+    int B, Lq, Hi, Nc, m, W;
+    int n_ttiles, n_chunks;       // token tiles, key chunks per token tile
+    const int32_t *q_pos;
+    const float *wi;              // [B, Lq, Hi]
+    float *scores;                // [B * Lq, Nc]
+};
+
+template <int HI>
+struct IxSmem {
+    static constexpr int Q_BYTES = kIxBM * kIxDi * 2;     // one head
+    static constexpr int K_BYTES = kIxBN * kIxDi * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = HI * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_K + kIxStages * K_BYTES;
+    static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+    static constexpr int BYTES = OFF_MISC + 16 * 4;
+};
+
+template <int HI>
+__global__ void __launch_bounds__(kIxThreads, 1)
+index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const IndexParams p)
+{
+    using SM = IxSmem<HI>;
+    extern __shared__ __align__(1024) uint8_t ix_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(ix_smem_raw) + 1023) &
+                                                ~(uintptr_t)1023);
+    uint8_t *sQ = smem + SM::OFF_Q;
+    uint8_t *sK = smem + SM::OFF_K;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
+    int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
+    volatile int *abort_flag = misc + 1;
+    // bars: 0 Q full, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // heavy token tiles first
+    const int ttile = p.n_ttiles - 1 - (int)(blockIdx.x / p.n_chunks);
+    const int chunk = (int)(blockIdx.x % p.n_chunks);
+    const int b = blockIdx.y;
+    const int t0 = ttile * kIxBM;
+    const int t_last = min(t0 + kIxBM - 1, p.Lq - 1);
+    auto pos_of = [&](int t) -> long long { return p.q_pos ? p.q_pos[(size_t)b * p.Lq + t] : t; };
+    long long pmax = -1;
+    // positions may be arbitrary; the tile covers up to the largest one
+    if (p.q_pos) {
+        for (int t = t0; t <= t_last; ++t)
+            pmax = max(pmax, pos_of(t));
+    } else {
+        pmax = t_last;
+    }
+    int nvmax = 0;
+    {
+        long long a = pmax - p.W + 1;
+        if (a > 0)
+            nvmax = (int)min((long long)p.Nc, a / p.m);
+    }
+    const int ntiles_all = (nvmax + kIxBN - 1) / kIxBN;
+    const int j0 = chunk * kIxChunkTiles;
+    const int j1 = min(ntiles_all, j0 + kIxChunkTiles);
+    const int nt = j1 - j0;
+    if (nt <= 0)
+        return;  // uniform across the CTA: nothing to score here
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        for (int s = 0; s < kIxStages; ++s) {
+            mbar_init(&bar[1 + s], 1);
+            mbar_init(&bar[5 + s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[9 + s], 1);
+            mbar_init(&bar[11 + s], 128);
+        }
+        mbar_init(&bar[13], 1);
+        mbar_fence_init();
+        misc[1] = 0;
+    }
+    if (warp == 1)
+        tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[0], HI * SM::Q_BYTES);
+            for (int h = 0; h < HI; ++h)
+                tma_load_4d(sQ + h * SM::Q_BYTES, &tm_q, &bar[0], 0, h, t0, b);
+            int issued = 0;
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % kIxStages;
+                if (i >= kIxStages && !mbar_wait(&bar[5 + s], ((i / kIxStages) - 1) & 1, abort_flag))
+                    break;
+                mbar_arrive_expect_tx(&bar[1 + s], SM::K_BYTES);
+                tma_load_4d(sK + s * SM::K_BYTES, &tm_k, &bar[1 + s], 0, 0, (j0 + i) * kIxBN, b);
+                ++issued;
+            }
+            drain_wait(&bar[0], 0);
+            for (int i = max(0, issued - kIxStages); i < issued; ++i)
+                drain_wait(&bar[1 + i % kIxStages], (i / kIxStages) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kIxBM, kIxBN, false, false);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+            bool ok = mbar_wait(&bar[0], 0, abort_flag);
+            for (int i = 0; ok && i < nt; ++i) {
+                const int s = i % kIxStages, db = i & 1;
+                if (!mbar_wait(&bar[1 + s], (i / kIxStages) & 1, abort_flag))
+                    break;
+                if (i >= 2 && !mbar_wait(&bar[11 + db], ((i >> 1) - 1) & 1, abort_flag))
+                    break;
+                tc_fence_after();
+                for (int h = 0; h < HI; ++h) {
+#pragma unroll
+                    for (int kk = 0; kk < kIxDi / 16; ++kk) {
+                        const uint64_t da = sw128_desc(aQ + h * SM::Q_BYTES + kk * 32, 16, 1024);
+                        const uint64_t dbk = sw128_desc(aK + s * SM::K_BYTES + kk * 32, 16, 1024);
+                        mma_bf16_ss(tmem + (db * HI + h) * kIxBN, da, dbk, idesc, kk > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(&bar[9 + db]);
+                mma_commit(&bar[5 + s]);
+            }
+            mma_commit(&bar[13]);
+            drain_wait(&bar[13], 0);
+        }
+    } else if (warp >= 4) {
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int t = t0 + row;
+        const bool valid = t < p.Lq;
+        int nv = 0;
+        float wv[HI];
+        if (valid) {
+            const long long a = pos_of(t) - p.W + 1;
+            nv = a > 0 ? (int)min((long long)p.Nc, a / p.m) : 0;
+#pragma unroll
+            for (int h = 0; h < HI; ++h)
+                wv[h] = p.wi[((size_t)b * p.Lq + t) * HI + h];
+        } else {
+#pragma unroll
+            for (int h = 0; h < HI; ++h)
+                wv[h] = 0.f;
+        }
+        float *srow = p.scores + ((size_t)b * p.Lq + (valid ? t : 0)) * p.Nc;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        for (int i = 0; i < nt; ++i) {
+            const int db = i & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (i >> 1) & 1, abort_flag)))
+                break;
+            tc_fence_after();
+            const int s0 = (j0 + i) * kIxBN;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                // the Hi accumulators of this row's 32 keys, one wait
+                float d[HI][32];
+#pragma unroll
+                for (int h = 0; h < HI; ++h)
+                    tmem_ld32(tl + (db * HI + h) * kIxBN + half * 32, d[h]);
+                tmem_ld_wait();
+                float acc[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    float a = wv[0] * fmaxf(d[0][q], 0.f);
+#pragma unroll
+                    for (int h = 1; h < HI; ++h)
+                        a = fmaf(wv[h], fmaxf(d[h][q], 0.f), a);
+                    acc[q] = a;
+                }
+                const int sb = s0 + half * 32;
+                if (valid && sb < nv) {
+                    if (sb + 32 <= nv && (p.Nc & 3) == 0) {
+#pragma unroll
+                        for (int q = 0; q < 32; q += 4)
+                            *reinterpret_cast<float4 *>(srow + sb + q) =
+                                make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+                    } else {
+                        for (int q = 0; q < 32 && sb + q < nv; ++q)
+                            srow[sb + q] = acc[q];
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bar[11 + db]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc((uint32_t)misc[0], 512);
+    }
+}
+
+template <int HI>
+static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const void *kic,
+                                     cudaStream_t stream)
+{
+    using SM = IxSmem<HI>;
+    CUtensorMap mq, mk;
+    // qi [B, Lq, Hi, 64] as (64, Hi, Lq, B) with a (64, 1, 128, 1) box
+    bool ok = make_map(&mq, qi, kIxDi, HI, p.Lq, p.B, 1, kIxBM);
+    // kic [B, Nc, 64] as (64, 1, Nc, B) with a (64, 1, 64, 1) box
+    ok &= make_map(&mk, kic, kIxDi, 1, p.Nc, p.B, 1, kIxBN);
+    if (!ok)
+        return cudaErrorInvalidValue;
+    size_t smem = 1024 + SM::BYTES;
+    if (smem < 120 * 1024)
+        smem = 120 * 1024;  // one CTA per SM: each holds all 512 TMEM columns
+    auto kern = index_scores_tc<HI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid(p.n_ttiles * p.n_chunks, p.B);
+    kern<<<grid, kIxThreads, smem, stream>>>(mq, mk, p);
+    return cudaGetLastError();
+}
+
+// Prefill indexer scores on tensor cores (di = 64, Hi <= 4).  Returns
+// cudaErrorNotSupported for other shapes (the caller uses the CUDA-core path).
+cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *kic, float *scores,
+                                   int B, int Lq, int Hi, int di, int Nc, int m, int W,
+                                   const int32_t *q_pos, cudaStream_t stream)
+{
+    if (di != kIxDi || Hi < 1 || Hi > 4 || Lq < 64)
+        return cudaErrorNotSupported;
+    IndexParams p;
+    p.B = B;
+    p.Lq = Lq;
+    p.Hi = Hi;
+    p.Nc = Nc;
+    p.m = m;
+    p.W = W;
+    p.n_ttiles = (Lq + kIxBM - 1) / kIxBM;
+    p.n_chunks = (Nc + kIxBN * kIxChunkTiles - 1) / (kIxBN * kIxChunkTiles);
+    if (p.n_chunks < 1)
+        p.n_chunks = 1;
+    p.q_pos = q_pos;
+    p.wi = wi;
+    p.scores = scores;
+    switch (Hi) {
+    case 1: return launch_index_tc_t<1>(p, qi, kic, stream);
+    case 2: return launch_index_tc_t<2>(p, qi, kic, stream);
+    case 3: return launch_index_tc_t<3>(p, qi, kic, stream);
+    default: return launch_index_tc_t<4>(p, qi, kic, stream);
+    }
+}
+
+}  // namespace hyb
