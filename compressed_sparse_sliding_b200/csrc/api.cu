@@ -89,6 +89,23 @@ static hyb_status check_problem(const hyb_problem *p, bool need_indexer)
     return HYB_OK;
 }
 
+// Stage 2 into a caller-chosen score buffer of B * Lq * Nc floats: tensor
+// cores where the shape allows, CUDA cores otherwise, then the exact top-K.
+static cudaError_t index_topk_into(const hyb_problem *p, const void *qi, const float *wi,
+                                   const void *kic, int32_t *idx, float *sel_scores, float *scores,
+                                   cudaStream_t stream)
+{
+    cudaError_t e = launch_index_scores_tc(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
+                                           p->m, p->W, p->q_pos, stream);
+    if (e == cudaErrorNotSupported)
+        e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc, p->m,
+                                     p->W, p->q_pos, stream);
+    if (e != cudaSuccess)
+        return e;
+    return launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos, idx,
+                             sel_scores, stream);
+}
+
 static float softmax_scale(const hyb_problem *p)
 {
     return p->scale != 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
@@ -132,18 +149,8 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
     const size_t need = hyb_workspace_size(p);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return HYB_ERR_WORKSPACE;
-    float *scores = static_cast<float *>(ws);
-    // tensor cores for prefill-sized query tiles, CUDA cores otherwise
-    cudaError_t e = launch_index_scores_tc(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
-                                           p->m, p->W, p->q_pos, stream);
-    if (e == cudaErrorNotSupported)
-        e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc, p->m,
-                                     p->W, p->q_pos, stream);
-    if (e != cudaSuccess)
-        return HYB_ERR_CUDA;
-    e = launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos, idx, sel_scores,
-                          stream);
-    return cuda_status(e);
+    return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, static_cast<float *>(ws),
+                                       stream));
 }
 
 hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,

@@ -60,7 +60,8 @@ struct SparseSmem {
     static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;             // [NH] floats
     static constexpr int OFF_BAR = OFF_MREF + NH * 4;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
-    static constexpr int OFF_IDX = OFF_MISC + 16 * 4;               // producer's selection list
+    static constexpr int OFF_VAL = OFF_MISC + 16 * 4;               // [kSpVS][128] slot validity
+    static constexpr int OFF_IDX = OFF_VAL + kSpVS * kSpBN;         // producer's selection list
     static constexpr int BASE_BYTES = OFF_IDX;                      // + topk * 4
 };
 
@@ -98,32 +99,6 @@ __device__ __forceinline__ SparseTok sparse_tok(const SparseParams &p, long long
     k.rhi = (int)hi;
     k.nrt = (p.W > 0 && hi >= lo) ? (int)((hi - lo + kSpBN) / kSpBN) : 0;
     return k;
-}
-
-// Selection entry of key slot c of tile i (compressed tiles only; -1 past topk
-// and for raw tiles).  Loads are issued a tile ahead of their use.
-__device__ __forceinline__ int slot_entry(const SparseParams &p, const SparseTok &k, int i, int c)
-{
-    if (i >= k.nct)
-        return -1;
-    const int s = i * kSpBN + c;
-    return s < p.topk ? __ldg(p.idx + ((size_t)k.b * p.Lq + k.t) * p.topk + s) : -1;
-}
-
-// Row of the flattened [B * rows * Hkv, d] view holding key slot c of tile i
-// (j: its selection entry), and whether the slot is a real key of the token.
-__device__ __forceinline__ bool slot_row(const SparseParams &p, const SparseTok &k, int i, int c, int j,
-                                         int *row)
-{
-    if (i < k.nct) {
-        const bool ok = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < k.pos - p.W + 1);
-        *row = ((k.b * p.Nc + (ok ? j : 0)) * p.Hkv) + k.kvh;
-        return ok;
-    }
-    const int r = k.rlo + (i - k.nct) * kSpBN + c;
-    const bool ok = r <= k.rhi;
-    *row = ((k.b * p.Lkv + (ok ? r : 0)) * p.Hkv) + k.kvh;
-    return ok;
 }
 
 // Arrive on `bar` once every cp.async issued so far by this thread has landed
@@ -235,6 +210,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     int *sIdx = reinterpret_cast<int *>(smem + SM::OFF_IDX);
+    uint8_t *sVal = smem + SM::OFF_VAL;
     volatile int *abort_flag = misc + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -261,6 +237,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_fence_init();
         misc[1] = 0;
     }
+    if (threadIdx.x < NH)
+        sMref[threadIdx.x] = -INFINITY;
     if (warp == 6)
         tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 256);
     tc_fence_before();
@@ -348,6 +326,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     !__all_sync(0xffffffffu, mbar_wait(&bar[SB_VE + vs], ((vc / kSpVS) - 1) & 1, abort_flag))) {
                     ok = false;
                     break;
+                }
+                if (c8 == 0) {
+                    // which slots are real keys, published with the V stage (the
+                    // softmax reads them after waiting on it)
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        sVal[vs * kSpBN + u * 4 + (pt >> 4)] = src[u] != 0xFFFFFFFFu ? 1 : 0;
                 }
                 {
                     const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
@@ -462,18 +447,16 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int h = 0; h < NH; ++h)
                 lpart[h] = 0.f;
-            if (threadIdx.x < NH)
-                sMref[threadIdx.x] = -INFINITY;
-            sm_sync();
-            int jnext = slot_entry(p, k, 0, r);
+            // No global memory access inside this loop: a CTA barrier (the
+            // votes below) waits for every outstanding access of its threads.
             for (int i = 0; i < nt; ++i, ++gt) {
-                int row_unused;
-                const bool valid = slot_row(p, k, i, r, jnext, &row_unused);
-                jnext = slot_entry(p, k, i + 1, r);  // next tile, in flight
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + (gt & 1)], (gt >> 1) & 1, abort_flag))) {
+                const int vs = gt % kSpVS;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + (gt & 1)], (gt >> 1) & 1, abort_flag) &&
+                                                 mbar_wait(&bar[SB_VF + vs], (gt / kSpVS) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
+                const bool valid = sVal[vs * kSpBN + r] != 0;
                 tc_fence_after();
                 float s[NH];
                 tmem_ld_cols<NH>(tl + TM_S0 + (gt & 1) * NH, s);
@@ -599,6 +582,21 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
             }
             sm_sync();
+            float inv[NH];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
+                inv[h] = l > 0.f ? 1.f / l : 0.f;
+            }
+            float lse_v = -INFINITY;
+            if (r < NH) {
+                const float l = sRed[r] + sRed[NH + r] + sRed[2 * NH + r] + sRed[3 * NH + r];
+                lse_v = l > 0.f ? (sMref[r] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            }
+            sm_sync();  // everyone has read sRed / sMref of this token
+            if (threadIdx.x < NH)
+                sMref[threadIdx.x] = -INFINITY;
+            sm_sync();  // the next token starts from a cleared reference
             float ov[NH];
             if (have_o) {
                 tmem_ld_cols<NH>(tl + TM_O0 + ob * NH, ov);
@@ -608,22 +606,14 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int h = 0; h < NH; ++h)
                     ov[h] = 0.f;
             }
+            // global stores only after the last barrier of the token
             const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                if (h < p.g) {
-                    const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
-                    const float v = l > 0.f ? ov[h] / l : 0.f;
-                    p.o[obase + (size_t)h * kSpD + r] = __float2bfloat16_rn(v);
-                }
-            }
-            if (p.lse && r < p.g) {
-                const int h = r;
-                const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
-                p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + h) * p.Lq + k.t] =
-                    l > 0.f ? (sMref[h] + log2f(l)) * 0.6931471805599453f : -INFINITY;
-            }
-            sm_sync();  // sRed / sMref are reused by the next token
+            for (int h = 0; h < NH; ++h)
+                if (h < p.g)
+                    p.o[obase + (size_t)h * kSpD + r] = __float2bfloat16_rn(ov[h] * inv[h]);
+            if (p.lse && r < p.g)
+                p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + r) * p.Lq + k.t] = lse_v;
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
         }

@@ -8,8 +8,8 @@
 // coalesced.  When there are too few (b, j, channel-octet) items to fill the
 // GPU (few, long blocks such as m = 128), the m positions are split over S
 // thread groups of the CTA and their partial sums are reduced in shared
-// memory.  CTAs are persistent: the [m, dx] weights are staged into shared
-// memory with 16-byte loads and turned into softmax weights once per CTA, then
+// memory.  CTAs are persistent: the [m, dx] weights arrive in shared memory
+// by one bulk copy and are turned into softmax weights once per CTA, then
 // reused for every block the CTA processes.
 #include "common.cuh"
 
@@ -24,16 +24,29 @@ block_merge_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict_
     extern __shared__ __align__(16) float sm_merge[];
     float *P = sm_merge;                        // [m][dx]
     float *part = sm_merge + (size_t)m * dx;    // [S-1][items_per_cta][8]
+    __shared__ __align__(8) uint64_t wbar;
+    __shared__ int wabort;
     const int tid = threadIdx.x;
 
-    // ---- stage the [m, dx] weights with 16-byte loads, then softmax over the
+    // ---- stage the [m, dx] weights with one bulk copy, then softmax over the
     //      m positions separately for every channel, in place ----
-    {
-        const float4 *w4 = reinterpret_cast<const float4 *>(w);
-        float4 *P4 = reinterpret_cast<float4 *>(P);
-        for (int i = tid; i < m * dx / 4; i += kMergeThreads)
-            P4[i] = __ldg(w4 + i);
+    if (tid == 0) {
+        wabort = 0;
+        mbar_init(&wbar, 1);
+        mbar_fence_init();
     }
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t bytes = (uint32_t)(m * dx) * 4u;
+        mbar_arrive_expect_tx(&wbar, bytes);
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                smem_u32(P)),
+            "l"(w), "r"(bytes), "r"(smem_u32(&wbar))
+            : "memory");
+    }
+    if (!mbar_wait(&wbar, 0, &wabort))
+        return;  // recorded as a device timeout; the copy was issued by thread 0 only
     __syncthreads();
     {
         int G = 1;  // threads per channel (power of two)

@@ -241,13 +241,215 @@ static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// Decode form: few query rows per sequence.  Keys go in the MMA's M
+// dimension (128 per tile) and the query row's indexer heads, padded to 16,
+// in N: D[128 keys x 16] = K_tile . Q^T.  The epilogue thread of a key forms
+// sum_h w[h] relu(D[key][h]) and stores one fp32 score; the kernel streams the
+// indexer-key cache once (HBM bound).  One CTA per (query row, run of tiles).
+// Roles (192 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 2-5
+// epilogue (warp w reads TMEM lane quadrant w % 4).
+// ------------------------------------------------------------------------
+constexpr int kDcThreads = 192;
+constexpr int kDcBM = 128;       // keys per tile
+constexpr int kDcN = 16;         // padded indexer heads
+constexpr int kDcStages = 4;
+constexpr int kDcChunk = 16;     // key tiles per CTA
+
+struct DecIndexParams {
+    int B, Lq, Hi, Nc, m, W, n_chunks;
+    const int32_t *q_pos;
+    const float *wi;
+    float *scores;
+};
+
+__global__ void __launch_bounds__(kDcThreads, 1)
+index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const DecIndexParams p)
+{
+    constexpr int Q_BYTES = kDcN * kIxDi * 2;      // 2 KB
+    constexpr int K_BYTES = kDcBM * kIxDi * 2;     // 16 KB
+    extern __shared__ __align__(1024) uint8_t dc_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dc_smem_raw) + 1023) &
+                                                ~(uintptr_t)1023);
+    uint8_t *sK = smem;                              // stages, 1024-aligned
+    uint8_t *sQ = smem + kDcStages * K_BYTES;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sQ + Q_BYTES);
+    int *misc = reinterpret_cast<int *>(bar + 16);
+    volatile int *abort_flag = misc + 1;
+    // bars: 0 Q, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int row = blockIdx.x / p.n_chunks;          // b * Lq + t
+    const int chunk = blockIdx.x % p.n_chunks;
+    const int b = row / p.Lq, t = row % p.Lq;
+    const long long pos = p.q_pos ? p.q_pos[row] : t;
+    int nv = 0;
+    {
+        const long long a = pos - p.W + 1;
+        if (a > 0)
+            nv = (int)min((long long)p.Nc, a / p.m);
+    }
+    const int j0 = chunk * kDcChunk;
+    const int j1 = min((nv + kDcBM - 1) / kDcBM, j0 + kDcChunk);
+    const int nt = j1 - j0;
+    if (nt <= 0)
+        return;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 16; ++i)
+            mbar_init(&bar[i], (i == 11 || i == 12) ? 128 : 1);
+        mbar_fence_init();
+        misc[1] = 0;
+    }
+    if (warp == 1)
+        tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 32);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[0], Q_BYTES);
+            // rows row*Hi .. row*Hi+15 of the [B*Lq*Hi, 64] view; rows past this
+            // query's heads only feed unused columns
+            tma_load_2d_box(sQ, &tm_q, &bar[0], 0, row * p.Hi);
+            int issued = 0;
+            for (int i = 0; i < nt; ++i) {
+                const int s = i % kDcStages;
+                if (i >= kDcStages && !mbar_wait(&bar[5 + s], ((i / kDcStages) - 1) & 1, abort_flag))
+                    break;
+                mbar_arrive_expect_tx(&bar[1 + s], K_BYTES);
+                tma_load_4d(sK + s * K_BYTES, &tm_k, &bar[1 + s], 0, 0, (j0 + i) * kDcBM, b);
+                ++issued;
+            }
+            drain_wait(&bar[0], 0);
+            for (int i = max(0, issued - kDcStages); i < issued; ++i)
+                drain_wait(&bar[1 + i % kDcStages], (i / kDcStages) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kDcBM, kDcN, false, false);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+            bool ok = mbar_wait(&bar[0], 0, abort_flag);
+            for (int i = 0; ok && i < nt; ++i) {
+                const int s = i % kDcStages, db = i & 1;
+                if (!mbar_wait(&bar[1 + s], (i / kDcStages) & 1, abort_flag))
+                    break;
+                if (i >= 2 && !mbar_wait(&bar[11 + db], ((i >> 1) - 1) & 1, abort_flag))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kIxDi / 16; ++kk)
+                    mma_bf16_ss(tmem + db * kDcN, sw128_desc(aK + s * K_BYTES + kk * 32, 16, 1024),
+                                sw128_desc(aQ + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                mma_commit(&bar[9 + db]);
+                mma_commit(&bar[5 + s]);
+            }
+            mma_commit(&bar[13]);
+            drain_wait(&bar[13], 0);
+        }
+    } else {
+        const int quad = warp & 3;
+        const int key = quad * 32 + lane;
+        float wv[kDcN];
+#pragma unroll
+        for (int h = 0; h < kDcN; ++h)
+            wv[h] = h < p.Hi ? p.wi[(size_t)row * p.Hi + h] : 0.f;
+        float *srow = p.scores + (size_t)row * p.Nc;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        for (int i = 0; i < nt; ++i) {
+            const int db = i & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (i >> 1) & 1, abort_flag)))
+                break;
+            tc_fence_after();
+            uint32_t d[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]),
+                  "=r"(d[6]), "=r"(d[7]), "=r"(d[8]), "=r"(d[9]), "=r"(d[10]), "=r"(d[11]),
+                  "=r"(d[12]), "=r"(d[13]), "=r"(d[14]), "=r"(d[15])
+                : "r"(tl + db * kDcN));
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&bar[11 + db]);
+            float I = 0.f;
+#pragma unroll
+            for (int h = 0; h < kDcN; ++h)
+                if (h < p.Hi)
+                    I = fmaf(wv[h], fmaxf(__uint_as_float(d[h]), 0.f), I);
+            const int sidx = (j0 + i) * kDcBM + key;
+            if (sidx < nv)
+                srow[sidx] = I;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc((uint32_t)misc[0], 32);
+    }
+}
+
+static cudaError_t launch_index_dec(const void *qi, const float *wi, const void *kic, float *scores,
+                                    int B, int Lq, int Hi, int Nc, int m, int W, const int32_t *q_pos,
+                                    cudaStream_t stream)
+{
+    CUtensorMap mq, mk;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return cudaErrorInvalidValue;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)kIxDi, (cuuint64_t)B * Lq * Hi};
+        cuuint64_t strides[1] = {(cuuint64_t)kIxDi * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)kDcN};
+        cuuint32_t es[2] = {1, 1};
+        if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(qi), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    if (!make_map(&mk, kic, kIxDi, 1, Nc, B, 1, kDcBM))
+        return cudaErrorInvalidValue;
+    DecIndexParams p;
+    p.B = B;
+    p.Lq = Lq;
+    p.Hi = Hi;
+    p.Nc = Nc;
+    p.m = m;
+    p.W = W;
+    p.n_chunks = (Nc + kDcBM * kDcChunk - 1) / (kDcBM * kDcChunk);
+    if (p.n_chunks < 1)
+        p.n_chunks = 1;
+    p.q_pos = q_pos;
+    p.wi = wi;
+    p.scores = scores;
+    const size_t smem = 1024 + kDcStages * kDcBM * kIxDi * 2 + kDcN * kIxDi * 2 + 16 * 8 + 16 * 4;
+    cudaError_t e = cudaFuncSetAttribute(index_scores_dec, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    index_scores_dec<<<(unsigned)(B * Lq * p.n_chunks), kDcThreads, smem, stream>>>(mq, mk, p);
+    return cudaGetLastError();
+}
+
 // Prefill indexer scores on tensor cores (di = 64, Hi <= 4).  Returns
 // cudaErrorNotSupported for other shapes (the caller uses the CUDA-core path).
 cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *kic, float *scores,
                                    int B, int Lq, int Hi, int di, int Nc, int m, int W,
                                    const int32_t *q_pos, cudaStream_t stream)
 {
-    if (di != kIxDi || Hi < 1 || Hi > 4 || Lq < 64)
+    if (di != kIxDi || Hi < 1)
+        return cudaErrorNotSupported;
+    if (Lq < 64) {
+        // decode: one tile of keys per MMA, the query's heads in N
+        if (Hi > kDcN)
+            return cudaErrorNotSupported;
+        return launch_index_dec(qi, wi, kic, scores, B, Lq, Hi, Nc, m, W, q_pos, stream);
+    }
+    if (Hi > 4)
         return cudaErrorNotSupported;
     IndexParams p;
     p.B = B;

@@ -66,11 +66,6 @@ extern "C" hyb_status hyb_csa_index_topk_noalloc(const hyb_problem *p, const voi
     st = noalloc_scratch(&scores);
     if (st != HYB_OK)
         return st;
-    cudaError_t e = launch_index_scores_simt(qi, wi, kic, scores, p->B, p->Lq, p->Hi, p->di, p->Nc,
-                                             p->m, p->W, p->q_pos, stream);
-    if (e != cudaSuccess)
-        return HYB_ERR_CUDA;
-    e = launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos, idx, sel_scores,
-                          stream);
-    return e == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+    // the same kernels as hyb_csa_index_topk, on the fixed scratch
+    return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, scores, stream));
 }
