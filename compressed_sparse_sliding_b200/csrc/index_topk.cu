@@ -530,16 +530,9 @@ cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m,
                               const int32_t *q_pos, int32_t *idx, float *sel_scores,
                               cudaStream_t stream)
 {
-    // rows of up to 16384 entries: keys in registers
-    if (Nc <= 256 * kRgPer) {
-        topk_regs<256><<<B * Lq, 256, 0, stream>>>(scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores);
-        return cudaGetLastError();
-    }
-    if (Nc <= 512 * kRgPer) {
-        topk_regs<512><<<B * Lq, 512, 0, stream>>>(scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores);
-        return cudaGetLastError();
-    }
-    if (Nc <= 1024 * kRgPer) {
+    // Rows of 8193..16384 entries: keys in registers (measured faster there);
+    // shorter rows: the shared-memory radix select (measured faster there).
+    if (Nc > 512 * kRgPer && Nc <= 1024 * kRgPer) {
         topk_regs<1024><<<B * Lq, 1024, 0, stream>>>(scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores);
         return cudaGetLastError();
     }
