@@ -164,6 +164,186 @@ block_merge_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict_
     }
 }
 
+// ---------------------------------------------------------------------------
+// Register-weight form.  With S chosen so that each thread owns at most 8
+// positions (NPOS = m / S) and a fixed octet of channels (items per tile times
+// 8 is a multiple of dx), the thread's NPOS x 8 softmax weights live in
+// registers: the main loop is only 16-byte global loads and FMAs.  The
+// per-channel max and sum over the m positions are combined across the S
+// position groups through a small shared table (2 x S x dx floats).
+// ---------------------------------------------------------------------------
+template <int NPOS>
+__global__ void __launch_bounds__(kMergeThreads)
+block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
+                 __nv_bfloat16 *__restrict__ out, int B, int L, int H, int dx, int m, int S)
+{
+    extern __shared__ __align__(16) float sm_rg[];
+    float *red = sm_rg;                         // [S][dx] partial max, then partial sums
+    float *part = sm_rg + (size_t)S * dx;       // [2][S / groups per warp][ipc][8] partial sums
+    const int tid = threadIdx.x;
+    const int ipc = kMergeThreads / S;
+    const int s = tid / ipc;
+    const int li = tid % ipc;
+    const int c0 = (li * 8) % dx;               // fixed channel octet of this thread
+    const bool owner = li < dx / 8;             // one thread per (s, channel octet) writes
+
+    // ---- this thread's weights: positions s, s + S, ... (NPOS of them) ----
+    float P[NPOS][8];
+#pragma unroll
+    for (int k = 0; k < NPOS; ++k) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(w + (size_t)(s + k * S) * dx + c0));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(w + (size_t)(s + k * S) * dx + c0 + 4));
+        P[k][0] = a.x; P[k][1] = a.y; P[k][2] = a.z; P[k][3] = a.w;
+        P[k][4] = b.x; P[k][5] = b.y; P[k][6] = b.z; P[k][7] = b.w;
+    }
+    float mx[8], den[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float v = P[0][q];
+#pragma unroll
+        for (int k = 1; k < NPOS; ++k)
+            v = fmaxf(v, P[k][q]);
+        mx[q] = v;
+    }
+    if (owner)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            red[s * dx + c0 + q] = mx[q];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float v = red[c0 + q];
+        for (int g = 1; g < S; ++g)
+            v = fmaxf(v, red[g * dx + c0 + q]);
+        mx[q] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < NPOS; ++k) {
+            P[k][q] = expf(P[k][q] - mx[q]);
+            acc += P[k][q];
+        }
+        den[q] = acc;
+    }
+    if (owner)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            red[s * dx + c0 + q] = den[q];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float v = 0.f;
+        for (int g = 0; g < S; ++g)
+            v += red[g * dx + c0 + q];
+        const float inv = 1.f / v;
+#pragma unroll
+        for (int k = 0; k < NPOS; ++k)
+            P[k][q] *= inv;
+    }
+
+    // ---- stream the blocks ----
+    const int Nc = L / m;
+    const int E8 = H * dx / 8;
+    const long long items = (long long)B * Nc * E8;
+    const long long ntiles = (items + ipc - 1) / ipc;
+    const size_t row_elems = (size_t)H * dx;
+    const int gw = ipc < 32 ? 32 / ipc : 1;     // position groups per warp
+    const int np = S / gw;                      // partial sets after the warp fold
+    int parity = 0;
+    for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const long long item = tile * ipc + li;
+        const bool live = item < items;
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            acc[q] = 0.f;
+        if (live) {
+            const long long unit = item / E8;
+            const int e8 = (int)(item % E8);
+            const int b = (int)(unit / Nc);
+            const int j = (int)(unit % Nc);
+            const __nv_bfloat16 *src =
+                x + ((size_t)b * L + (size_t)j * m + s) * row_elems + (size_t)e8 * 8;
+            uint4 v[NPOS];
+#pragma unroll
+            for (int k = 0; k < NPOS; ++k)
+                v[k] = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)k * S * row_elems));
+#pragma unroll
+            for (int k = 0; k < NPOS; ++k) {
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v[k]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(h2[q]);
+                    acc[2 * q] = fmaf(P[k][2 * q], f.x, acc[2 * q]);
+                    acc[2 * q + 1] = fmaf(P[k][2 * q + 1], f.y, acc[2 * q + 1]);
+                }
+            }
+        }
+        if (S > 1) {
+            // fold the position groups that share a warp, then the per-warp
+            // partial sets through the table (double-buffered: one barrier)
+            for (int off = ipc; off < 32; off <<= 1)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
+            float *pt = part + (size_t)(parity & 1) * np * ipc * 8;
+            if ((tid & 31) < ipc) {
+                float4 *dst = reinterpret_cast<float4 *>(pt + ((size_t)(s / gw) * ipc + li) * 8);
+                dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+            __syncthreads();
+            for (int e = tid; e < ipc * 8; e += kMergeThreads) {
+                float v = 0.f;
+                for (int g = 0; g < np; ++g)
+                    v += pt[(size_t)g * ipc * 8 + e];
+                const long long item2 = tile * ipc + (e >> 3);
+                if (item2 < items)
+                    out[(size_t)item2 * 8 + (e & 7)] = __float2bfloat16_rn(v);
+            }
+            ++parity;
+        } else if (live) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            *reinterpret_cast<uint4 *>(out + (size_t)item * 8) = o;
+        }
+    }
+}
+
+template <int NPOS>
+static cudaError_t launch_merge_regs(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                                     void *out, int S, long long items, cudaStream_t stream,
+                                     int num_sms)
+{
+    const int ipc = kMergeThreads / S;
+    const size_t smem = sizeof(float) * ((size_t)S * dx + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0));
+    cudaError_t e = cudaFuncSetAttribute(block_merge_regs<NPOS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_merge_regs<NPOS>, kMergeThreads,
+                                                      smem);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        per_sm = 1;
+    const long long ntiles = (items + ipc - 1) / ipc;
+    long long grid = (long long)num_sms * per_sm;
+    if (grid > ntiles)
+        grid = ntiles;
+    block_merge_regs<NPOS><<<(unsigned)grid, kMergeThreads, smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(x), w, static_cast<__nv_bfloat16 *>(out), B, L, H, dx, m,
+        S);
+    return cudaGetLastError();
+}
+
 // Launch helper: picks the position split S and a persistent grid.
 cudaError_t launch_block_merge(const void *x, int B, int L, int H, int dx, int m, const float *w,
                                void *out, cudaStream_t stream, int num_sms)
@@ -172,6 +352,25 @@ cudaError_t launch_block_merge(const void *x, int B, int L, int H, int dx, int m
     const long long items = (long long)B * Nc * (H * dx / 8);
     if (items == 0)
         return cudaSuccess;
+    {
+        // register-weight form: at most 8 positions per thread, fixed channel octet
+        int Sr = 1;
+        while (Sr * 8 < m && Sr < 32)
+            Sr *= 2;
+        while (Sr < 32 && m % (Sr * 2) == 0 && m / (Sr * 2) >= 4 &&
+               ((kMergeThreads / (Sr * 2)) * 8) % dx == 0 && items * Sr < (long long)num_sms * 2048)
+            Sr *= 2;  // more position groups while the grid is short of work
+        const int ipc = kMergeThreads / Sr;
+        if (m % Sr == 0 && m / Sr <= 8 && (ipc * 8) % dx == 0 && dx <= 256) {
+            switch (m / Sr) {
+            case 1: return launch_merge_regs<1>(x, B, L, H, dx, m, w, out, Sr, items, stream, num_sms);
+            case 2: return launch_merge_regs<2>(x, B, L, H, dx, m, w, out, Sr, items, stream, num_sms);
+            case 4: return launch_merge_regs<4>(x, B, L, H, dx, m, w, out, Sr, items, stream, num_sms);
+            case 8: return launch_merge_regs<8>(x, B, L, H, dx, m, w, out, Sr, items, stream, num_sms);
+            default: break;
+            }
+        }
+    }
     // split the m positions over S thread groups only while every thread keeps
     // at least 8 loads and the grid is short of ~1024 threads per SM
     int S = 1;

@@ -31,6 +31,11 @@ def _randn_bf16(g, shape, scale=1.0):
     (1, 513, 1, 32, 4),
     (1, 64, 2, 64, 1),
     (3, 130, 1, 64, 3),
+    (1, 300, 3, 64, 8),
+    (2, 257, 2, 128, 16),
+    (1, 1100, 5, 64, 64),
+    (1, 700, 2, 256, 128),
+    (2, 99, 4, 128, 2),
 ])
 def test_block_merge_matches_oracle(hb, B, L, H, dx, m):
     g = torch.Generator().manual_seed(B * 1000 + L + m)
