@@ -35,7 +35,6 @@
 namespace hyb {
 
 constexpr int kSpBN = 128;     // keys per tile (the M of S^T)
-constexpr int kSpKS = 3;       // K ring depth
 constexpr int kSpVS = 2;       // V ring depth
 constexpr int kSpD = 128;      // head dim handled by this kernel
 
@@ -54,13 +53,16 @@ struct SparseSmem {
     static constexpr int Q_BYTES = NH * kSpD * 2;
     static constexpr int KV_BYTES = kSpBN * kSpD * 2;
     static constexpr int P_BYTES = kSpBN * NH * 2;
+    static constexpr int P_STRIDE = (P_BYTES + 1023) & ~1023;
+    static constexpr int KS = NH == 64 ? 2 : 3;                    // K ring depth
     static constexpr int OFF_Q = 0;                                // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + kSpKS * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + kSpVS * KV_BYTES;
-    static constexpr int OFF_RED = OFF_P + ((P_BYTES + 1023) & ~1023);  // [4][NH] floats
-    static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;             // [NH] floats
-    static constexpr int OFF_BAR = OFF_MREF + NH * 4;
+    static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
+    static constexpr int OFF_P = OFF_V + kSpVS * KV_BYTES;         // 2 buffers
+    static constexpr int OFF_RED = OFF_P + 2 * P_STRIDE;           // [NH][4] floats
+    static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;          // [2][NH] floats
+    static constexpr int OFF_INV = OFF_MREF + 2 * NH * 4;          // [NH] floats
+    static constexpr int OFF_BAR = OFF_INV + NH * 4;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
     static constexpr int OFF_VAL = OFF_MISC + 16 * 4;               // [kSpVS][128] slot validity
     static constexpr int OFF_IDX = OFF_VAL + kSpVS * kSpBN;         // producer's selection list
@@ -69,7 +71,7 @@ struct SparseSmem {
 
 enum {
     SB_QF = 0, SB_QE = 2, SB_KF = 4, SB_KE = 7, SB_VF = 10, SB_VE = 12, SB_SF = 14, SB_PF = 16,
-    SB_OD = 17, SB_OE = 18, SB_DONE = 20
+    SB_OD = 18, SB_OE = 20, SB_DONE = 22
 };
 
 struct SparseTok {
@@ -146,6 +148,61 @@ __device__ __forceinline__ void sm_sync()
     asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
+// Per-head totals over the 32 lanes of a warp by recursive halving: at each
+// step a lane keeps one half of its values (the upper half where its lane
+// bit is set), receives the partner's copy of that half and combines.  NH
+// values cost NH - 1 shuffles (plus one per remaining lane bit for NH < 32).
+// Afterwards lane l holds in v[0 .. SpHeads<NH>::VPL) the warp totals of the
+// heads SpHeads<NH>::head(l, e).
+template <int NH>
+struct SpHeads {
+    static constexpr int VPL = NH >= 32 ? NH / 32 : 1;     // values per lane
+    static constexpr int LPH = NH >= 32 ? 1 : 32 / NH;     // lanes per head
+    __device__ static int head(int lane, int e) { return NH >= 32 ? lane * VPL + e : lane / LPH; }
+};
+
+template <bool MAX, int N, int OFF, int NH>
+__device__ __forceinline__ void halve_heads(float (&v)[NH], int lane)
+{
+    if constexpr (OFF >= 1) {
+        if constexpr (N > 1) {
+            constexpr int H = N / 2;
+            const bool up = (lane & OFF) != 0;
+#pragma unroll
+            for (int j = 0; j < H; ++j) {
+                const float send = up ? v[j] : v[j + H];
+                const float keep = up ? v[j + H] : v[j];
+                const float got = __shfl_xor_sync(0xffffffffu, send, OFF);
+                v[j] = MAX ? fmaxf(keep, got) : keep + got;
+            }
+            halve_heads<MAX, H, OFF / 2>(v, lane);
+        } else {
+            const float got = __shfl_xor_sync(0xffffffffu, v[0], OFF);
+            v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+            halve_heads<MAX, 1, OFF / 2>(v, lane);
+        }
+    }
+}
+
+template <int NH, bool MAX>
+__device__ __forceinline__ void warp_reduce_heads(float (&v)[NH], int lane)
+{
+    halve_heads<MAX, NH, 16>(v, lane);
+}
+
+// New reference for one head: moves only when the tile max exceeds the old
+// one by more than 2^8.
+__device__ __forceinline__ float sp_new_ref(float4 q4, float old)
+{
+    const float tmx = fmaxf(fmaxf(q4.x, q4.y), fmaxf(q4.z, q4.w));
+    return tmx > old + 8.f ? tmx : old;
+}
+
+__device__ __forceinline__ float sp_factor(float old, float nw)
+{
+    return nw == old ? 1.f : (old == -INFINITY ? 0.f : ex2_approx(old - nw));
+}
+
 // Shared-memory descriptor with a selectable swizzle (layout 2: 128 B, 4: 64 B, 6: 32 B).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
 {
@@ -207,6 +264,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_vr, const SparseParams p)
 {
     using SM = SparseSmem<NH>;
+    constexpr int KS = SM::KS;
     constexpr int RB = NH * 2;                                  // bytes of one P^T row
     constexpr uint32_t PLAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
     constexpr int PCH = RB / 16;                                // 16-byte chunks per row
@@ -219,6 +277,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t *sP = smem + SM::OFF_P;
     float *sRed = reinterpret_cast<float *>(smem + SM::OFF_RED);
     float *sMref = reinterpret_cast<float *>(smem + SM::OFF_MREF);
+    float *sInv = reinterpret_cast<float *>(smem + SM::OFF_INV);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     int *sIdx = reinterpret_cast<int *>(smem + SM::OFF_IDX);
@@ -234,8 +293,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bar[SB_QE + s], 1);
             mbar_init(&bar[SB_SF + s], 1);
             mbar_init(&bar[SB_OE + s], 128);
+            mbar_init(&bar[SB_PF + s], 128);
+            mbar_init(&bar[SB_OD + s], 1);
         }
-        for (int s = 0; s < kSpKS; ++s) {
+        for (int s = 0; s < KS; ++s) {
             mbar_init(&bar[SB_KF + s], 32 * SpRoles<NH>::PW);
             mbar_init(&bar[SB_KE + s], 1);
         }
@@ -243,13 +304,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bar[SB_VF + s], 32 * SpRoles<NH>::PW);
             mbar_init(&bar[SB_VE + s], 1);
         }
-        mbar_init(&bar[SB_PF], 128);
-        mbar_init(&bar[SB_OD], 1);
         mbar_init(&bar[SB_DONE], 1);
         mbar_fence_init();
         misc[1] = 0;
     }
-    if (threadIdx.x < NH)
+    if (threadIdx.x < 2 * NH)
         sMref[threadIdx.x] = -INFINITY;
     if (warp == SpRoles<NH>::MMA_WARP)
         tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 256);
@@ -319,9 +378,9 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         src[u] = rr <= k.rhi ? (k.b * p.Lkv + rr) * p.Hkv + k.kvh : -1;
                     }
                 }
-                const uint32_t ks = kc % kSpKS;
-                if (kc >= kSpKS &&
-                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_KE + ks], ((kc / kSpKS) - 1) & 1, abort_flag))) {
+                const uint32_t ks = kc % KS;
+                if (kc >= KS &&
+                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_KE + ks], ((kc / KS) - 1) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -390,10 +449,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 auto issue_pv = [&](bool first) -> bool {
                     const uint32_t vs = vc % kSpVS;
-                    if (!mbar_wait(&bar[SB_PF], pcnt & 1, abort_flag) ||
+                    const uint32_t pb = pcnt & 1;
+                    if (!mbar_wait(&bar[SB_PF + pb], (pcnt >> 1) & 1, abort_flag) ||
                         !mbar_wait(&bar[SB_VF + vs], (vc / kSpVS) & 1, abort_flag))
                         return false;
-                    ++pcnt;
                     if (first && nq >= 2 &&
                         !mbar_wait(&bar[SB_OE + ob], ((nq >> 1) - 1) & 1, abort_flag))
                         return false;
@@ -402,18 +461,20 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int kk = 0; kk < kSpBN / 16; ++kk) {
                         const uint64_t da = smem_desc(aV + vs * SM::KV_BYTES + kk * 16 * 128,
                                                       kSpBN * 128, 1024, 2);
-                        const uint64_t db = smem_desc(aP + kk * 16 * RB, 16, 8 * RB, PLAYOUT);
+                        const uint64_t db = smem_desc(aP + pb * SM::P_STRIDE + kk * 16 * RB, 16, 8 * RB,
+                                                      PLAYOUT);
                         mma_bf16_ss(tmem + TM_O0 + ob * NH, da, db, idesc_pv,
                                     (first && kk == 0) ? 0u : 1u);
                     }
-                    mma_commit(&bar[SB_OD]);
+                    mma_commit(&bar[SB_OD + pb]);
                     mma_commit(&bar[SB_VE + vs]);
                     ++vc;
+                    ++pcnt;
                     return true;
                 };
                 for (int i = 0; i < nt; ++i, ++gt) {
-                    const uint32_t ks = kc % kSpKS;
-                    if (!mbar_wait(&bar[SB_KF + ks], (kc / kSpKS) & 1, abort_flag)) {
+                    const uint32_t ks = kc % KS;
+                    if (!mbar_wait(&bar[SB_KF + ks], (kc / KS) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -450,12 +511,18 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ========================== softmax + epilogue ==========================
+        // The reference maxima live in shared memory in two buffers, sMref[mb]
+        // current; a move writes the other buffer and flips mb after a barrier,
+        // so readers of the old values never race the writers.
+        using HD = SpHeads<NH>;
         const int quad = warp;                       // warps 0-3
         const int r = quad * 32 + lane;              // key lane (S^T) / d lane (O^T)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        uint32_t nq = 0, gt = 0;
+        const bool head_owner = (lane % HD::LPH) == 0;
+        uint32_t nq = 0, gt = 0, mb = 0;
         bool ok = true;
         const uint32_t prow = smem_u32(sP) + r * RB;
+        const float4 *red4 = reinterpret_cast<const float4 *>(sRed);
         for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
             const SparseTok k = sparse_tok(p, w);
             const int nt = k.nct + k.nrt;
@@ -468,7 +535,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // votes below) waits for every outstanding access of its threads.
             for (int i = 0; i < nt; ++i, ++gt) {
                 const int vs = gt % kSpVS;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + (gt & 1)], (gt >> 1) & 1, abort_flag) &&
+                const uint32_t sb = gt & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag) &&
                                                  mbar_wait(&bar[SB_VF + vs], (gt / kSpVS) & 1, abort_flag))) {
                     ok = false;
                     break;
@@ -476,44 +544,49 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const bool valid = sVal[vs * kSpBN + r] != 0;
                 tc_fence_after();
                 float s[NH];
-                tmem_ld_cols<NH>(tl + TM_S0 + (gt & 1) * NH, s);
+                tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, s);
                 tmem_ld_wait();
 #pragma unroll
                 for (int h = 0; h < NH; ++h)
                     s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
-                bool exceed = false;
+                bool need = i == 0;   // the first tile of a token always sets the reference
+                if (!need) {
+                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH);
+                    bool exceed = false;
 #pragma unroll
-                for (int h = 0; h < NH; ++h)
-                    exceed |= s[h] > sMref[h] + 8.f;
-                if (sm_any(exceed)) {
-                    // block-wide max per head over this tile
+                    for (int h = 0; h < NH; h += 4) {
+                        const float4 mr = m4[h >> 2];
+                        exceed |= (s[h] > mr.x + 8.f) | (s[h + 1] > mr.y + 8.f) | (s[h + 2] > mr.z + 8.f) |
+                                  (s[h + 3] > mr.w + 8.f);
+                    }
+                    need = sm_any(exceed);
+                }
+                if (need) {
+                    // per-head max over the tile: warp halving, then the four
+                    // warps' values through sRed [head][warp]
+                    warp_reduce_heads<NH, true>(s, lane);
+                    if (head_owner) {
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        float v = s[h];
-#pragma unroll
-                        for (int off = 16; off; off >>= 1)
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                        if (lane == 0)
-                            sRed[quad * NH + h] = v;
+                        for (int e = 0; e < HD::VPL; ++e)
+                            sRed[HD::head(lane, e) * 4 + quad] = s[e];
                     }
                     sm_sync();
-                    // new reference: the tile max where it exceeds the old one by
-                    // more than 2^8; every thread derives the same factors
+                    const float *mold = sMref + mb * NH;
                     bool moved = false;
+                    if (i > 0) {
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]),
-                                                fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
-                        const float old = sMref[h];
-                        const float nw = tmx > old + 8.f ? tmx : old;
-                        const float a = (nw == old) ? 1.f : (old == -INFINITY ? 0.f : ex2_approx(old - nw));
-                        moved |= a != 1.f;
-                        lpart[h] *= a;
+                        for (int h = 0; h < NH; ++h) {
+                            const float old = mold[h];
+                            const float a = sp_factor(old, sp_new_ref(red4[h], old));
+                            moved |= a != 1.f;
+                            lpart[h] *= a;
+                        }
                     }
-                    if (i > 0 && moved) {
+                    if (moved) {
                         // O^T holds every earlier PV of this token: wait for the
                         // last one, then scale column h by its factor
-                        if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)],
+                                                               ((gt - 1) >> 1) & 1, abort_flag))) {
                             ok = false;
                             break;
                         }
@@ -525,42 +598,50 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             tmem_ld_wait();
 #pragma unroll
                             for (int q = 0; q < 16; ++q) {
-                                const int h = c + q;
-                                const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]),
-                                                        fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
-                                const float old = sMref[h];
-                                const float nw = tmx > old + 8.f ? tmx : old;
-                                ov[q] *= (nw == old) ? 1.f : (old == -INFINITY ? 0.f : ex2_approx(old - nw));
+                                const float old = mold[c + q];
+                                ov[q] *= sp_factor(old, sp_new_ref(red4[c + q], old));
                             }
                             tmem_st_cols<16>(tl + TM_O0 + ob * NH + c, ov);
                         }
                         tmem_st_wait();
                     }
-                    sm_sync();  // every thread has read the old reference
-                    if (threadIdx.x < NH) {
-                        const int h = threadIdx.x;
-                        const float tmx = fmaxf(fmaxf(sRed[h], sRed[NH + h]), fmaxf(sRed[2 * NH + h], sRed[3 * NH + h]));
-                        const float old = sMref[h];
-                        sMref[h] = tmx > old + 8.f ? tmx : old;
-                    }
+                    if (threadIdx.x < NH)
+                        sMref[(mb ^ 1) * NH + threadIdx.x] =
+                            sp_new_ref(red4[threadIdx.x], mold[threadIdx.x]);
                     sm_sync();
+                    mb ^= 1;
+                    // the halving consumed the scores: load them again
+                    tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, s);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
                 }
                 // P^T row of this key: exp2(s - mref), 0 for masked keys
                 uint32_t pk[NH / 2];
+                {
+                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH);
 #pragma unroll
-                for (int h = 0; h < NH; h += 2) {
-                    const float m0 = sMref[h], m1 = sMref[h + 1];
-                    const float e0 = (m0 == -INFINITY) ? 0.f : ex2_approx(s[h] - m0);
-                    const float e1 = (m1 == -INFINITY) ? 0.f : ex2_approx(s[h + 1] - m1);
-                    lpart[h] += e0;
-                    lpart[h + 1] += e1;
-                    pk[h >> 1] = pack_bf16x2(e0, e1);
+                    for (int h = 0; h < NH; h += 4) {
+                        const float4 mr = m4[h >> 2];
+                        const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
+                        float e[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            e[q] = (mm[q] == -INFINITY) ? 0.f : ex2_approx(s[h + q] - mm[q]);
+                            lpart[h + q] += e[q];
+                        }
+                        pk[h >> 1] = pack_bf16x2(e[0], e[1]);
+                        pk[(h >> 1) + 1] = pack_bf16x2(e[2], e[3]);
+                    }
                 }
-                // the P^T buffer is free once PV of the previous tile completed
-                if (gt > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                // P^T buffer sb is free once the PV of tile gt - 2 completed
+                if (gt >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1,
+                                                                  abort_flag))) {
                     ok = false;
                     break;
                 }
+                const uint32_t prow_b = prow + sb * SM::P_STRIDE;
 #pragma unroll
                 for (int c = 0; c < PCH; ++c) {
                     uint32_t phys;
@@ -570,50 +651,43 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         phys = c ^ ((r >> 1) & 3);
                     else
                         phys = c ^ ((r >> 2) & 1);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + phys * 16),
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_b + phys * 16),
                                  "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                                  : "memory");
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&bar[SB_PF]);
+                mbar_arrive(&bar[SB_PF + sb]);
             }
             if (!ok)
                 break;
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
+            warp_reduce_heads<NH, false>(lpart, lane);
+            if (head_owner) {
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                float v = lpart[h];
-#pragma unroll
-                for (int off = 16; off; off >>= 1)
-                    v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0)
-                    sRed[quad * NH + h] = v;
+                for (int e = 0; e < HD::VPL; ++e)
+                    sRed[HD::head(lane, e) * 4 + quad] = lpart[e];
             }
-            bool have_o = nt > 0;
+            const bool have_o = nt > 0;
             if (have_o) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD], (gt - 1) & 1, abort_flag))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1,
+                                                       abort_flag))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
             }
             sm_sync();
-            float inv[NH];
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                const float l = sRed[h] + sRed[NH + h] + sRed[2 * NH + h] + sRed[3 * NH + h];
-                inv[h] = l > 0.f ? 1.f / l : 0.f;
-            }
             float lse_v = -INFINITY;
             if (r < NH) {
-                const float l = sRed[r] + sRed[NH + r] + sRed[2 * NH + r] + sRed[3 * NH + r];
-                lse_v = l > 0.f ? (sMref[r] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                const float4 q4 = red4[r];
+                const float l = (q4.x + q4.y) + (q4.z + q4.w);
+                sInv[r] = l > 0.f ? 1.f / l : 0.f;
+                lse_v = l > 0.f ? (sMref[mb * NH + r] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                sMref[(mb ^ 1) * NH + r] = -INFINITY;   // the next token's reference
             }
-            sm_sync();  // everyone has read sRed / sMref of this token
-            if (threadIdx.x < NH)
-                sMref[threadIdx.x] = -INFINITY;
-            sm_sync();  // the next token starts from a cleared reference
+            sm_sync();  // sRed / sMref read, sInv written, next reference cleared
+            mb ^= 1;
             float ov[NH];
             if (have_o) {
                 tmem_ld_cols<NH>(tl + TM_O0 + ob * NH, ov);
@@ -625,10 +699,16 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             // global stores only after the last barrier of the token
             const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+            const float4 *inv4 = reinterpret_cast<const float4 *>(sInv);
 #pragma unroll
-            for (int h = 0; h < NH; ++h)
-                if (h < p.g)
-                    p.o[obase + (size_t)h * kSpD + r] = __float2bfloat16_rn(ov[h] * inv[h]);
+            for (int h = 0; h < NH; h += 4) {
+                const float4 iv = inv4[h >> 2];
+                const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (h + q < p.g)
+                        p.o[obase + (size_t)(h + q) * kSpD + r] = __float2bfloat16_rn(ov[h + q] * ivs[q]);
+            }
             if (p.lse && r < p.g)
                 p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + r) * p.Lq + k.t] = lse_v;
             tc_fence_before();
