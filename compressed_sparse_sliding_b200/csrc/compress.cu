@@ -16,6 +16,7 @@
 namespace hyb {
 
 constexpr int kMergeThreads = 256;
+constexpr int kMergeStages = 3;   // cp.async ring depth of the register-weight kernel
 
 __global__ void __launch_bounds__(kMergeThreads)
 block_merge_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
@@ -245,6 +246,10 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
     }
 
     // ---- stream the blocks ----
+    // Every thread copies its own NPOS 16-byte pieces of a tile into private
+    // slots of a kMergeStages-deep shared ring with cp.async, kMergeStages - 1
+    // tiles ahead of the one it reduces; a thread only ever reads the slots it
+    // filled, so the ring needs no barrier (cp.async.wait_group orders it).
     const int Nc = L / m;
     const int E8 = H * dx / 8;
     const long long items = (long long)B * Nc * E8;
@@ -252,8 +257,32 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
     const size_t row_elems = (size_t)H * dx;
     const int gw = ipc < 32 ? 32 / ipc : 1;     // position groups per warp
     const int np = S / gw;                      // partial sets after the warp fold
-    int parity = 0;
+    const uint32_t ring = smem_u32(part + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0));
+    auto slot = [&](int stage, int k) -> uint32_t {
+        return ring + (uint32_t)(((stage * NPOS + k) * kMergeThreads + tid) * 16);
+    };
+    auto issue = [&](long long tile, int stage) {
+        const long long item = tile * ipc + li;
+        if (tile < ntiles && item < items) {
+            const long long unit = item / E8;
+            const int e8 = (int)(item % E8);
+            const int b = (int)(unit / Nc);
+            const int j = (int)(unit % Nc);
+            const __nv_bfloat16 *src =
+                x + ((size_t)b * L + (size_t)j * m + s) * row_elems + (size_t)e8 * 8;
+#pragma unroll
+            for (int k = 0; k < NPOS; ++k)
+                cp_async_16(slot(stage, k), src + (size_t)k * S * row_elems, 16u);
+        }
+        cp_async_commit();   // one group per tile, empty past the end
+    };
+#pragma unroll
+    for (int d = 0; d < kMergeStages - 1; ++d)
+        issue((long long)blockIdx.x + (long long)d * gridDim.x, d);
+    int parity = 0, stage = 0;
     for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        issue(tile + (long long)(kMergeStages - 1) * gridDim.x, (stage + kMergeStages - 1) % kMergeStages);
+        cp_async_wait_group<kMergeStages - 1>();   // this tile's copies have landed
         const long long item = tile * ipc + li;
         const bool live = item < items;
         float acc[8];
@@ -261,16 +290,12 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
         for (int q = 0; q < 8; ++q)
             acc[q] = 0.f;
         if (live) {
-            const long long unit = item / E8;
-            const int e8 = (int)(item % E8);
-            const int b = (int)(unit / Nc);
-            const int j = (int)(unit % Nc);
-            const __nv_bfloat16 *src =
-                x + ((size_t)b * L + (size_t)j * m + s) * row_elems + (size_t)e8 * 8;
             uint4 v[NPOS];
 #pragma unroll
             for (int k = 0; k < NPOS; ++k)
-                v[k] = __ldg(reinterpret_cast<const uint4 *>(src + (size_t)k * S * row_elems));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v[k].x), "=r"(v[k].y), "=r"(v[k].z), "=r"(v[k].w)
+                             : "r"(slot(stage, k)));
 #pragma unroll
             for (int k = 0; k < NPOS; ++k) {
                 const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v[k]);
@@ -313,7 +338,9 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
             o.w = pack_bf16x2(acc[6], acc[7]);
             *reinterpret_cast<uint4 *>(out + (size_t)item * 8) = o;
         }
+        stage = stage + 1 == kMergeStages ? 0 : stage + 1;
     }
+    cp_async_wait_group<0>();
 }
 
 template <int NPOS>
@@ -322,7 +349,8 @@ static cudaError_t launch_merge_regs(const void *x, int B, int L, int H, int dx,
                                      int num_sms)
 {
     const int ipc = kMergeThreads / S;
-    const size_t smem = sizeof(float) * ((size_t)S * dx + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0));
+    const size_t smem = sizeof(float) * ((size_t)S * dx + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0)) +
+                        (size_t)kMergeStages * NPOS * kMergeThreads * 16;
     cudaError_t e = cudaFuncSetAttribute(block_merge_regs<NPOS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)

@@ -49,11 +49,16 @@ def test_block_merge_matches_oracle(hb, B, L, H, dx, m):
 
 
 # ------------------------------------------------------------ indexer + top-K
-def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None):
+def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, pool=0):
     g = torch.Generator().manual_seed(seed)
     qi = _randn_bf16(g, (B, Lq, Hi, di))
     wi = torch.rand((B, Lq, Hi), generator=g)
     kic = _randn_bf16(g, (B, Nc, di))
+    if pool:
+        # entries drawn from `pool` distinct rows: every score value repeats,
+        # so the K-th score is an exact tie broken toward the lower index
+        pick = torch.randint(0, pool, (B, Nc), generator=g)
+        kic = torch.stack([kic[b, pick[b]] for b in range(B)])
     qp = None if q_pos is None else torch.as_tensor(q_pos, dtype=torch.int32).reshape(B, Lq)
     p = hb.problem(B=B, Lq=Lq, Lkv=max(W, 1), Hq=4, Hkv=1, d=64, m=m, W=W, topk=K, Hi=Hi, di=di,
                    Nc=Nc, q_pos=None if qp is None else qp.cuda())
@@ -102,6 +107,33 @@ def test_index_topk_large_rows_sampled(hb):
     # entries per row as in the long CSA prefill (up to 8160 visible), sampled rows
     rows = list(range(0, 32768, 997)) + [32767, 520, 521]
     _index_case(hb, 1, 32768, 4, 64, 8192, 4, 128, 512, seed=5, rows=rows)
+
+
+@pytest.mark.parametrize("Nc,pool", [(3001, 16), (8192, 7), (12000, 16), (16384, 0), (20000, 16)])
+def test_index_topk_exact_ties_and_row_lengths(hb, Nc, pool):
+    # one query per sequence near the end of the cache, rows of every length
+    # class of the selection kernels; pooled keys make the threshold a tie
+    B, m, W, K = 3, 4, 128, 300
+    L = Nc * m + W
+    pos = [[L - 1], [L // 2], [L - 1 - 7 * m]]
+    exact = _index_case(hb, B, 1, 4, 64, Nc, m, W, K, q_pos=pos, seed=Nc + pool, pool=pool)
+    if pool:
+        assert exact.all()   # exact ties are compared index for index
+
+
+@pytest.mark.parametrize("Nc,pool", [(3000, 0), (3000, 16), (8192, 0), (12000, 16)])
+def test_index_topk_many_rows(hb, Nc, pool):
+    # 1500 query rows at spread positions: the narrow per-row selection CTAs
+    B, Lq, m, W, K = 3, 500, 4, 128, 300
+    L = Nc * m + W
+    rng = np.random.default_rng(Nc)
+    pos = rng.integers(0, L, size=(B, Lq)).astype(np.int32)
+    pos[0, :4] = [L - 1, W + K * m + 3, W + K * m - 5, 0]
+    rows = [0, 1, 2, 3] + sorted(rng.choice(B * Lq, size=40, replace=False).tolist())
+    exact = _index_case(hb, B, Lq, 4, 64, Nc, m, W, K, q_pos=pos, seed=Nc + 7 * pool, pool=pool,
+                        rows=rows)
+    if pool:
+        assert exact.all()
 
 
 # ----------------------------------------------------------------- attention
