@@ -163,7 +163,57 @@ class Step:
                 e[2].elapsed_time(e[3]))
 
 
+class ClockSampler:
+    """SM clock and clock-event reasons of this process's GPU, polled through
+    NVML from a background thread while the timed region runs (nvidia-smi's
+    loop is far coarser than a timed region of a few milliseconds)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+        bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.sm, self.mask = [], 0
+        self.stop_ev = threading.Event()
+        self.th = threading.Thread(target=self._run, daemon=True)
+        self.th.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                self.mask |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                return
+            time.sleep(0.0002)
+
+    def stop(self):
+        self.stop_ev.set()
+        self.th.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        if not self.sm:
+            return None
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(n for bit, n in self.REASONS.items() if self.mask & bit),
+                "samples": len(self.sm), "source": "nvml"}
+
+
 def sample_clocks_start():
+    try:
+        return ClockSampler()
+    except Exception:
+        pass
     try:
         return subprocess.Popen(
             ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
@@ -179,6 +229,8 @@ def sample_clocks_start():
 def sample_clocks_stop(proc):
     if proc is None:
         return None
+    if isinstance(proc, ClockSampler):
+        return proc.stop()
     proc.terminate()
     try:
         out, _ = proc.communicate(timeout=5)
@@ -202,7 +254,7 @@ def sample_clocks_stop(proc):
     if not sm:
         return None
     return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-            "samples": len(sm)}
+            "samples": len(sm), "source": "nvidia-smi"}
 
 
 def attention_kernel(w):
@@ -259,7 +311,8 @@ def run_gpu(args, rank, world):
         raise RuntimeError(f"device status after warm-up: {hb.hyb_error_string(st)}")
 
     clk = sample_clocks_start()
-    time.sleep(0.3)
+    if not isinstance(clk, ClockSampler):
+        time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()

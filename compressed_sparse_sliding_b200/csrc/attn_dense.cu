@@ -12,12 +12,16 @@
 // Items are ordered longest first (late tokens see more compressed entries)
 // and handed out round-robin to one CTA per SM.
 //
-// Roles (320 threads):
+// Roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + epilogue of tile A, warps 4-7 of tile B: one thread
-//               per TMEM lane (= query row), the row's 128 scores in registers.
+//               per TMEM lane (= query row).  These two warpgroups raise their
+//               register budget to 208 (setmaxnreg) so that a row's 128 scores
+//               stay in registers from one TMEM load through max, exp2 and
+//               the P write.
 //   warp 8      TMA producer: Q_A, Q_B once per item, K and V tiles through
 //               separate two-stage rings (128-byte swizzle, no multicast).
 //   warp 9      TMEM allocation; lane 0 issues every tcgen05.mma.
+//   warps 10-11 idle; the third warpgroup gives registers back (88 each).
 // TMEM (512 columns): S_A, S_B (128 fp32 columns each), O_A, O_B (D each).
 // After the softmax pass P (bf16 pairs) overwrites the first 64 columns of S
 // and feeds O += P V directly from TMEM, so shared memory only holds Q and
@@ -29,7 +33,9 @@
 
 namespace hyb {
 
-constexpr int kDnThreads = 320;
+constexpr int kDnThreads = 384;
+constexpr int kDnSoftmaxRegs = 208;   // 2 x 128 x 208 + 128 x 88 = 384 x 168 (the launch budget)
+constexpr int kDnOtherRegs = 88;
 constexpr int kDnBM = 128;
 constexpr int kDnBN = 128;
 constexpr int kDnKStages = 2;
@@ -188,8 +194,8 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = (uint32_t)misc[0];
     constexpr uint32_t TM_S[2] = {0, kDnBN};
     constexpr uint32_t TM_O[2] = {2 * kDnBN, 2 * kDnBN + 128};
-
     if (warp == 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDnOtherRegs));
         // ================================ producer ================================
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
@@ -247,6 +253,7 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 drain_wait(&bar[DB_VF + c % kDnVStages], (c / kDnVStages) & 1);
         }
     } else if (warp == 9) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDnOtherRegs));
         // ================================ MMA issue ================================
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16(kDnBM, kDnBN, false, false);
@@ -354,7 +361,10 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mma_commit(&bar[DB_DONE]);
             drain_wait(&bar[DB_DONE], 0);
         }
+    } else if (warp >= 10) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDnOtherRegs));
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDnSoftmaxRegs));
         // ========================== softmax + epilogue ==========================
         const int x = warp >> 2;            // 0: tile A, 1: tile B
         const int quad = warp & 3;
@@ -396,20 +406,21 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 ++scnt;
                 tc_fence_after();
-                // pass 1: all 128 scores in flight (one wait), masked row max
-                // over eight independent 3-input max chains
+                // all 128 scores in flight (one wait); masked columns become -inf,
+                // so they drop out of the max and give exp2 = 0 below
+                float sv[kDnBN];
+#pragma unroll
+                for (int c = 0; c < kDnBN / 32; ++c)
+                    tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
+                tmem_ld_wait();
+                if (!full) {
+#pragma unroll
+                    for (int c = 0; c < kDnBN; ++c)
+                        sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
+                }
+                // row max over eight independent 3-input max chains
                 float tmax;
                 {
-                    float sv[kDnBN];
-#pragma unroll
-                    for (int c = 0; c < kDnBN / 32; ++c)
-                        tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
-                    tmem_ld_wait();
-                    if (!full) {
-#pragma unroll
-                        for (int c = 0; c < kDnBN; ++c)
-                            sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
-                    }
                     float mk[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -444,43 +455,26 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-                // pass 2: two halves of 64 scores (one wait each); P = exp2(s *
-                // scale - mu) as bf16 pairs over the first 64 columns of S, the
-                // A operand of O += P V (half h overwrites only columns the
-                // earlier loads already consumed)
-                // pass 2: two halves of 64 scores (one wait each); P = exp2(s *
-                // scale - mu) as bf16 pairs over the first 64 columns of S, the
-                // A operand of O += P V (half h overwrites only columns the
-                // earlier loads already consumed).  Row sums in four
+                // P = exp2(s * scale - mu) from the registers, as bf16 pairs over
+                // the first 64 columns of S (the A operand of O += P V; every
+                // score was loaded before the first store).  Row sums in four
                 // independent packed accumulators.
                 const uint64_t sc2 = f2(p.scale_log2, p.scale_log2);
                 const uint64_t nmu2 = f2(-mu, -mu);
                 uint64_t lacc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float sv[64];
-                    tmem_ld32(tS + hh * 64, *reinterpret_cast<float(*)[32]>(&sv[0]));
-                    tmem_ld32(tS + hh * 64 + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
-                    tmem_ld_wait();
+                for (int c = 0; c < kDnBN / 32; ++c) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int q = 0; q < 32; q += 2) {
-                            const int cc = hh * 64 + c * 32 + q;
-                            float x0, x1;
-                            f2_split(fma_f2(f2(sv[c * 32 + q], sv[c * 32 + q + 1]), sc2, nmu2), x0, x1);
-                            float e0 = ex2_approx(x0);
-                            float e1 = ex2_approx(x1);
-                            if (!full) {
-                                e0 = (cc >= c_lo && cc <= c_hi) ? e0 : 0.f;
-                                e1 = (cc + 1 >= c_lo && cc + 1 <= c_hi) ? e1 : 0.f;
-                            }
-                            lacc[(q >> 1) & 3] = add_f2(lacc[(q >> 1) & 3], f2(e0, e1));
-                            pk[q >> 1] = pack_bf16x2(e0, e1);
-                        }
-                        tmem_st16(tS + hh * 32 + c * 16, pk);
+                    for (int q = 0; q < 32; q += 2) {
+                        float x0, x1;
+                        f2_split(fma_f2(f2(sv[c * 32 + q], sv[c * 32 + q + 1]), sc2, nmu2), x0, x1);
+                        const float e0 = ex2_approx(x0);
+                        const float e1 = ex2_approx(x1);
+                        lacc[(q >> 1) & 3] = add_f2(lacc[(q >> 1) & 3], f2(e0, e1));
+                        pk[q >> 1] = pack_bf16x2(e0, e1);
                     }
+                    tmem_st16(tS + c * 16, pk);
                 }
                 float lsum;
                 {

@@ -179,10 +179,14 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
                  __nv_bfloat16 *__restrict__ out, int B, int L, int H, int dx, int m, int S)
 {
     extern __shared__ __align__(16) float sm_rg[];
-    float *red = sm_rg;                         // [S][dx] partial max, then partial sums
-    float *part = sm_rg + (size_t)S * dx;       // [2][S / groups per warp][ipc][8] partial sums
     const int tid = threadIdx.x;
     const int ipc = kMergeThreads / S;
+    const int gw = ipc < 32 ? 32 / ipc : 1;     // position groups per warp
+    const int np = S / gw;                      // partial sets after the warp fold
+    float *part = sm_rg;                        // [2][np][ipc][8] partial sums (S > 1)
+    float *ring_f = sm_rg + (S > 1 ? (size_t)2 * np * ipc * 8 : 0);
+    float *red = ring_f;                        // [S][dx] partial max, then sums (prologue only,
+                                                // before the ring is filled)
     const int s = tid / ipc;
     const int li = tid % ipc;
     const int c0 = (li * 8) % dx;               // fixed channel octet of this thread
@@ -255,9 +259,7 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
     const long long items = (long long)B * Nc * E8;
     const long long ntiles = (items + ipc - 1) / ipc;
     const size_t row_elems = (size_t)H * dx;
-    const int gw = ipc < 32 ? 32 / ipc : 1;     // position groups per warp
-    const int np = S / gw;                      // partial sets after the warp fold
-    const uint32_t ring = smem_u32(part + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0));
+    const uint32_t ring = smem_u32(ring_f);
     auto slot = [&](int stage, int k) -> uint32_t {
         return ring + (uint32_t)(((stage * NPOS + k) * kMergeThreads + tid) * 16);
     };
@@ -276,6 +278,7 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
         }
         cp_async_commit();   // one group per tile, empty past the end
     };
+    __syncthreads();   // every thread is done with `red`, which the ring overwrites
 #pragma unroll
     for (int d = 0; d < kMergeStages - 1; ++d)
         issue((long long)blockIdx.x + (long long)d * gridDim.x, d);
@@ -349,8 +352,11 @@ static cudaError_t launch_merge_regs(const void *x, int B, int L, int H, int dx,
                                      int num_sms)
 {
     const int ipc = kMergeThreads / S;
-    const size_t smem = sizeof(float) * ((size_t)S * dx + (S > 1 ? (size_t)2 * kMergeThreads * 8 : 0)) +
-                        (size_t)kMergeStages * NPOS * kMergeThreads * 16;
+    const int gw = ipc < 32 ? 32 / ipc : 1;
+    const int np = S / gw;
+    const size_t ring = (size_t)kMergeStages * NPOS * kMergeThreads * 16;
+    const size_t red = sizeof(float) * (size_t)S * dx;
+    const size_t smem = (S > 1 ? sizeof(float) * (size_t)2 * np * ipc * 8 : 0) + (ring > red ? ring : red);
     cudaError_t e = cudaFuncSetAttribute(block_merge_regs<NPOS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
