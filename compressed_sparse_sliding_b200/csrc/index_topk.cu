@@ -4,14 +4,14 @@
 // kept in fp32, over the entries visible to t; then an exact top-K with ties
 // resolved toward the lower entry index, written in ascending index order.
 //
-// Two kernels:
+// Kernels here (the tensor-core score kernels are in index_tc.cu):
 //   index_scores_simt  CUDA-core scores for a tile of query rows x keys into a
 //                      workspace row per query (only the visible prefix);
-//                      used for decode (one query row per sequence, the
-//                      kic stream from HBM is the bound) and small shapes.
-//   topk_regs          one CTA per query row, the row's keys in registers
-//                      (rows of up to 16384 entries); 4-bit digit search of
-//                      the K-th largest order key without shared atomics.
+//                      the fallback for shapes the tensor-core kernels do not
+//                      take (di != 64, more than 4 heads in prefill).
+//   topk_hist          one CTA per query row (rows of up to 16384 entries),
+//                      the row's keys in registers; histogram select of the
+//                      K-th largest order key by a narrowing key interval.
 //   topk_radix         rows longer than that: keys in shared memory, a
 //                      12 + 10 + 10-bit radix select.
 //   Both emit in index order: every key above the threshold and the
@@ -354,16 +354,7 @@ topk_radix(const float *__restrict__ scores, int B, int Lq, int Nc, int m, int W
     }
 }
 
-// ------------------------------------------------------------------------
-// Exact top-K with the row in registers.  Thread t owns entries
-// [t * 16, t * 16 + 16) of its row.  The K-th largest order key is found
-// digit by digit (4 bits per round, 8 rounds): every thread counts its
-// matching keys per digit in two packed 64-bit counters, warps add the counts
-// with __reduce_add_sync, and one scan over 16 digits picks the digit that
-// holds the K-th key.  No shared-memory atomics, so clustered scores cost the
-// same as spread ones.  Emission in index order as in topk_radix.
-// ------------------------------------------------------------------------
-constexpr int kRgPer = 16;
+// Block-wide exclusive prefix sum (thread order) for NT threads.
 
 template <int NT>
 __device__ __forceinline__ int blk_excl_scan(int v, int *warp_tot)
@@ -396,134 +387,6 @@ __device__ __forceinline__ int blk_excl_scan(int v, int *warp_tot)
     const int r = warp_tot[wid] + x - v;
     __syncthreads();
     return r;
-}
-
-template <int NT>
-__global__ void __launch_bounds__(NT)
-topk_regs(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
-          const int32_t *__restrict__ q_pos, int32_t *__restrict__ idx_out,
-          float *__restrict__ sel_scores)
-{
-    constexpr int NW = NT / 32;
-    __shared__ int s_cnt[NW][16];
-    __shared__ int s_tot[16];
-    __shared__ int s_scan[32];
-
-    const int row = blockIdx.x;
-    const int t = row % Lq;
-    const long long pos = q_pos ? q_pos[row] : t;
-    const int n = visible_entries(pos, m, W, Nc);
-    const int keff = n < K ? n : K;
-    const float *src = scores + (size_t)row * Nc;
-    int32_t *dst = idx_out + (size_t)row * K;
-    float *dsc = sel_scores ? sel_scores + (size_t)row * K : nullptr;
-
-    if (keff == n) {
-        for (int i = threadIdx.x; i < K; i += NT) {
-            dst[i] = i < n ? i : -1;
-            if (dsc)
-                dsc[i] = i < n ? src[i] : -INFINITY;
-        }
-        return;
-    }
-
-    const int i0 = threadIdx.x * kRgPer;
-    uint32_t key[kRgPer];
-    if ((Nc & 3) == 0 && i0 + kRgPer <= n) {
-#pragma unroll
-        for (int u = 0; u < kRgPer; u += 4) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i0 + u));
-            key[u] = order_key(v.x);
-            key[u + 1] = order_key(v.y);
-            key[u + 2] = order_key(v.z);
-            key[u + 3] = order_key(v.w);
-        }
-    } else {
-#pragma unroll
-        for (int u = 0; u < kRgPer; ++u)
-            key[u] = (i0 + u < n) ? order_key(__ldg(src + i0 + u)) : 0u;  // 0: below every score
-    }
-
-    // ---- digit-by-digit search of the K-th largest key ----
-    uint32_t prefix = 0, pmask = 0;
-    int need = keff;
-    for (int shift = 28; shift >= 0; shift -= 4) {
-        uint64_t c0 = 0, c1 = 0;
-#pragma unroll
-        for (int u = 0; u < kRgPer; ++u) {
-            const uint32_t k = key[u];
-            if ((k & pmask) == prefix) {
-                const uint32_t d = (k >> shift) & 15u;
-                const uint64_t one = 1ull << ((d & 7u) * 8u);
-                if (d < 8)
-                    c0 += one;
-                else
-                    c1 += one;
-            }
-        }
-        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-        for (int d = 0; d < 16; ++d) {
-            const int v = (int)(((d < 8 ? c0 : c1) >> ((d & 7) * 8)) & 0xffu);
-            const int sum = __reduce_add_sync(0xffffffffu, v);
-            if (lane == 0)
-                s_cnt[wid][d] = sum;
-        }
-        __syncthreads();
-        if (threadIdx.x < 16) {
-            int tot = 0;
-#pragma unroll
-            for (int w = 0; w < NW; ++w)
-                tot += s_cnt[w][threadIdx.x];
-            s_tot[threadIdx.x] = tot;
-        }
-        __syncthreads();
-        int cum = 0, dstar = 0;
-#pragma unroll
-        for (int d = 15; d >= 0; --d) {
-            const int c = s_tot[d];
-            if (cum + c >= need) {
-                dstar = d;
-                break;
-            }
-            cum += c;
-        }
-        need -= cum;
-        prefix |= (uint32_t)dstar << shift;
-        pmask |= 15u << shift;
-        __syncthreads();  // s_cnt / s_tot are rewritten next round
-    }
-    const uint32_t T = prefix;  // key of the K-th largest score; take `need` keys equal to it
-
-    int gt = 0, eq = 0;
-#pragma unroll
-    for (int u = 0; u < kRgPer; ++u) {
-        gt += key[u] > T;
-        eq += key[u] == T;
-    }
-    const int eq_before = blk_excl_scan<NT>(eq, s_scan);
-    const int take_eq = min(eq, max(0, need - eq_before));
-    int out = blk_excl_scan<NT>(gt + take_eq, s_scan);
-    int e_seen = 0;
-#pragma unroll
-    for (int u = 0; u < kRgPer; ++u) {
-        bool pick = key[u] > T;
-        if (key[u] == T) {
-            pick = e_seen < take_eq;
-            ++e_seen;
-        }
-        if (pick) {
-            dst[out] = i0 + u;
-            if (dsc)
-                dsc[out] = src[i0 + u];
-            ++out;
-        }
-    }
-    for (int i = keff + threadIdx.x; i < K; i += NT) {
-        dst[i] = -1;
-        if (dsc)
-            dsc[i] = -INFINITY;
-    }
 }
 
 // ------------------------------------------------------------------------
