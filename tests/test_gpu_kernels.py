@@ -137,7 +137,7 @@ def test_index_topk_many_rows(hb, Nc, pool):
 
 
 # ----------------------------------------------------------------- attention
-def _attn_case(hb, B, L, Hq, Hkv, d, m, W, K=0, seed=0, scale=None, lse=True):
+def _attn_case(hb, B, L, Hq, Hkv, d, m, W, K=0, seed=0, scale=None, lse=True, rows=None):
     g = torch.Generator().manual_seed(seed)
     q = _randn_bf16(g, (B, L, Hq, d))
     k = _randn_bf16(g, (B, L, Hkv, d))
@@ -164,10 +164,12 @@ def _attn_case(hb, B, L, Hq, Hkv, d, m, W, K=0, seed=0, scale=None, lse=True):
     torch.cuda.synchronize()
     assert hb.hyb_get_device_status() == hb.HYB_OK
     ref = oracle.hybrid_attention(bits(q), bits(kc), bits(vc), idx, bits(k), bits(v), m, W,
-                                  scale=scale)
-    check_output(o, ref["o"])
+                                  scale=scale, rows=rows)
+    og = o if rows is None else o.reshape(B * L, Hq, d)[torch.as_tensor(rows, device=o.device)]
+    check_output(og, ref["o"])
     if lse:
-        check_lse(lse_t.permute(0, 2, 1).reshape(B * L, Hq).cpu().numpy(), ref["lse"])
+        lg = lse_t.permute(0, 2, 1).reshape(B * L, Hq).cpu().numpy()
+        check_lse(lg if rows is None else lg[np.asarray(rows)], ref["lse"])
     return o, ref
 
 
@@ -187,6 +189,23 @@ def test_dense_attention_hca_blocks(hb):
 def test_sparse_attention_given_indices(hb, d):
     # CSA shape: MQA, K selected entries + 128-token window; several key tiles
     _attn_case(hb, 1, 700, 4, 1, d, 4, 128, K=160, seed=20 + d)
+
+
+@pytest.mark.parametrize("Hq,Hkv,K,W,L", [
+    (32, 1, 300, 128, 1700),     # 32-head group, ragged selection tile
+    (40, 2, 200, 64, 1300),      # GQA, 20 heads per group padded to 32
+    (32, 1, 768, 128, 3400),     # 6 + 1 tiles: a full 32-head token buffer
+    (16, 1, 1792, 128, 7400),    # 14 + 1 tiles: a full 16-head token buffer
+    (32, 1, 200, 0, 1000),       # no window
+    (32, 1, 1000, 128, 4300),    # 8 + 1 tiles: past the token buffer, lazy-softmax kernel
+])
+def test_sparse_attention_d128_groups(hb, Hq, Hkv, K, W, L):
+    # head dim 128 with every group width and tile count around the kernel limits;
+    # early, middle and late tokens plus a spread sample
+    rng = np.random.default_rng(L + K)
+    rows = sorted(set([0, 5, W + 3, L // 3, L // 2, L - 2, L - 1] +
+                      rng.choice(L, size=24, replace=False).tolist()))
+    _attn_case(hb, 1, L, Hq, Hkv, 128, 4, W, K=K, seed=60 + K, rows=rows)
 
 
 def test_sparse_attention_gqa_groups(hb):
@@ -231,9 +250,45 @@ def test_decode_form(hb):
         check_output(o, ref["o"])
 
 
-def test_out_of_range_index_is_reported_not_read(hb):
+@pytest.mark.parametrize("B,Hq,Hkv,K", [(5, 32, 1, 700), (4, 64, 2, 1024), (64, 64, 1, 1024)])
+def test_decode_group_widths(hb, B, Hq, Hkv, K):
+    # decode: one query per sequence, 32- and 64-head groups, GQA, selections
+    # of up to 1024 entries; early positions leave selection slots empty
+    g = torch.Generator().manual_seed(70 + K)
+    d, m, W, Nc = 128, 4, 128, 2048
+    rng = np.random.default_rng(70 + K)
+    pos = rng.integers(W + 1, Nc * m + W, size=B).astype(np.int32)
+    pos[0] = Nc * m + W - 1
+    pos[-1] = W + 40 * m          # only 40 visible entries
+    q = _randn_bf16(g, (B, 1, Hq, d))
+    kr = _randn_bf16(g, (B, W, Hkv, d))
+    vr = _randn_bf16(g, (B, W, Hkv, d))
+    kc = _randn_bf16(g, (B, Nc, Hkv, d))
+    vc = _randn_bf16(g, (B, Nc, Hkv, d))
+    idx = np.full((B, 1, K), -1, np.int32)
+    for b in range(B):
+        nv = oracle.visible_count(int(pos[b]), m, W, Nc)
+        n = min(K, nv)
+        idx[b, 0, :n] = np.sort(rng.choice(nv, size=n, replace=False))
+    qp = torch.from_numpy(pos.reshape(B, 1))
+    kv0 = torch.from_numpy(pos - W + 1)
+    p = hb.problem(B=B, Lq=1, Lkv=W, Hq=Hq, Hkv=Hkv, d=d, m=m, W=W, topk=K, Nc=Nc,
+                   q_pos=qp.cuda(), kv_pos0=kv0.cuda())
+    lse_t = torch.empty((B, Hq, 1), dtype=torch.float32, device="cuda")
+    o = hb.hyb_attn_fwd(p, q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(idx).cuda(), kr.cuda(),
+                        vr.cuda(), lse=lse_t)
+    torch.cuda.synchronize()
+    assert hb.hyb_get_device_status() == hb.HYB_OK
+    ref = oracle.hybrid_attention(bits(q), bits(kc), bits(vc), idx, bits(kr), bits(vr), m, W,
+                                  q_pos=pos.reshape(B, 1), kv_pos0=(pos - W + 1).astype(np.int32))
+    check_output(o, ref["o"])
+    check_lse(lse_t.reshape(B, Hq).cpu().numpy(), ref["lse"])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_out_of_range_index_is_reported_not_read(hb, d):
     g = torch.Generator().manual_seed(60)
-    B, L, Hq, d, m, W, K = 1, 64, 4, 64, 4, 8, 4
+    B, L, Hq, m, W, K = 1, 64, 4, 4, 8, 4
     Nc = L // m
     q = _randn_bf16(g, (B, L, Hq, d)).cuda()
     k = _randn_bf16(g, (B, L, 1, d)).cuda()
