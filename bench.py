@@ -5,7 +5,9 @@
 
 One step = one pass of the whole forward path over one batch of the workload:
 block_merge of K, V (and indexer keys for CSA) -> indexer scores + exact top-K
-(CSA) -> hybrid attention.  Default workload: the HCA+SWA batch (B=2, L=8192,
+(CSA) -> hybrid attention.  A decode step starts instead with the cache
+maintenance of the new token (window ring append; the block it closes becomes
+a compressed entry) and reads the window from the ring.  Default workload: the HCA+SWA batch (B=2, L=8192,
 16 query / 16 KV heads, d=128, m=128, W=128).  Inputs are synthetic, seeded and
 resident in HBM before the timed region; L2 is flushed between timed steps
 (a 256 MiB write, then a read of a separate 256 MiB buffer so that the step
@@ -101,11 +103,13 @@ def algorithmic_counts(w):
 
 
 # ----------------------------------------------------------------- GPU arm
-def problem_for(hb, w, inp):
+def problem_for(hb, w, inp, kv_pos0=None):
+    """Decode reads the window from the 2W-row ring that hyb_decode_append
+    maintains (kv_pos0: the [B] tensor that call writes)."""
     if w.is_decode:
-        return hb.problem(B=w.B, Lq=1, Lkv=w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
+        return hb.problem(B=w.B, Lq=1, Lkv=2 * w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
                           topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc, q_pos=inp["q_pos"],
-                          kv_pos0=inp["kv_pos0"])
+                          kv_pos0=kv_pos0)
     return hb.problem(B=w.B, Lq=w.L, Lkv=w.L, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
                       topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc)
 
@@ -116,8 +120,9 @@ class Step:
 
     def __init__(self, hb, w, inp):
         self.hb, self.w, self.inp = hb, w, inp
-        self.p = problem_for(hb, w, inp)
         dev = inp["q"].device
+        self.kv0 = torch.empty((w.B,), dtype=torch.int32, device=dev)
+        self.p = problem_for(hb, w, inp, self.kv0)
         if w.is_decode:
             self.kc, self.vc, self.kic = inp["kc"], inp["vc"], inp["kic"]
         else:
@@ -137,7 +142,14 @@ class Step:
         hb, w, inp, ev = self.hb, self.w, self.inp, self.ev
         launches = 0
         ev[0].record(stream)
-        if not w.is_decode:
+        if w.is_decode:
+            # cache maintenance of the new token: window ring + the closed block
+            hb.hyb_decode_append(self.p, inp["t_new"], inp["k_new"], inp["v_new"], inp["k_ring"],
+                                 inp["v_ring"], self.kc, self.vc, inp["wk"], inp["wv"],
+                                 ki_new=inp["ki_new"], wib=inp["wib"], ki_ring=inp["ki_ring"],
+                                 kic=self.kic, kv_pos0=self.kv0, stream=stream)
+            launches += 1
+        else:
             hb.hyb_hca_compress(inp["k"], inp["wk"], w.m, out=self.kc, stream=stream)
             hb.hyb_hca_compress(inp["v"], inp["wv"], w.m, out=self.vc, stream=stream)
             launches += 2
@@ -151,8 +163,8 @@ class Step:
             launches += 2
         ev[2].record(stream)
         hb.hyb_attn_fwd(self.p, inp["q"], self.kc, self.vc, self.idx,
-                        inp["k_raw"] if w.is_decode else inp["k"],
-                        inp["v_raw"] if w.is_decode else inp["v"], o=self.o, stream=stream)
+                        inp["k_ring"] if w.is_decode else inp["k"],
+                        inp["v_ring"] if w.is_decode else inp["v"], o=self.o, stream=stream)
         launches += 1
         ev[3].record(stream)
         self.launches = launches
@@ -342,27 +354,44 @@ def run_gpu(args, rank, world):
     tokens = w.B * w.Lq * world
     value = tokens / (ms_per_step / 1e3)
 
-    # ---- end to end through the fused C-ABI call with host buffers ----
-    host = {k: v.cpu().pin_memory() for k, v in inp.items()
-            if k in ("q", "k", "v", "wk", "wv", "qi", "wi", "ki", "wib", "kc", "vc", "kic",
-                     "k_raw", "v_raw", "q_pos", "kv_pos0")}
-    if not w.is_decode:
-        host.pop("k_raw", None)
-        host.pop("v_raw", None)
+    # ---- end to end through the public C-ABI calls with host buffers ----
+    # Prefill: every input of the step crosses from pinned host memory.  Decode:
+    # the step's own inputs do (the query, the indexer query and head weights,
+    # the new token's K / V / indexer-key rows and positions); the caches,
+    # rings and block weights are device-resident state the step maintains.
+    if w.is_decode:
+        per_step = ("q", "qi", "wi", "k_new", "v_new", "ki_new", "t_new", "q_pos")
+    else:
+        per_step = ("q", "k", "v", "wk", "wv", "qi", "wi", "ki", "wib")
+    host = {k: inp[k].cpu().pin_memory() for k in per_step if k in inp}
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    if w.is_decode:
+        for k in ("k_ring", "v_ring", "ki_ring", "kc", "vc", "kic", "wk", "wv", "wib"):
+            dev_in[k] = inp[k]
     o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o_host.numel() * o_host.element_size()
 
+    kv0_e2e = torch.empty((w.B,), dtype=torch.int32, device=dev)
+
     def e2e_step():
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
-        if not w.is_decode:
-            dev_in["k_raw"], dev_in["v_raw"] = dev_in["k"], dev_in["v"]
-        p = problem_for(hb, w, dev_in)
-        res = hb.hyb_fused_fwd(p, dev_in["q"], dev_in["k_raw"], dev_in["v_raw"], wk=dev_in.get("wk"),
-                               wv=dev_in.get("wv"), qi=dev_in.get("qi"), wi=dev_in.get("wi"),
-                               ki_raw=dev_in.get("ki"), wib=dev_in.get("wib"), kc=dev_in.get("kc"),
+        p = problem_for(hb, w, dev_in, kv0_e2e)
+        if w.is_decode:
+            hb.hyb_decode_append(p, dev_in["t_new"], dev_in["k_new"], dev_in["v_new"],
+                                 dev_in["k_ring"], dev_in["v_ring"], dev_in["kc"], dev_in["vc"],
+                                 dev_in["wk"], dev_in["wv"], ki_new=dev_in["ki_new"],
+                                 wib=dev_in["wib"], ki_ring=dev_in["ki_ring"], kic=dev_in["kic"],
+                                 kv_pos0=kv0_e2e, stream=stream)
+            raw_k, raw_v = dev_in["k_ring"], dev_in["v_ring"]
+        else:
+            raw_k, raw_v = dev_in["k"], dev_in["v"]
+        res = hb.hyb_fused_fwd(p, dev_in["q"], raw_k, raw_v,
+                               wk=None if w.is_decode else dev_in.get("wk"),
+                               wv=None if w.is_decode else dev_in.get("wv"), qi=dev_in.get("qi"),
+                               wi=dev_in.get("wi"), ki_raw=dev_in.get("ki"),
+                               wib=None if w.is_decode else dev_in.get("wib"), kc=dev_in.get("kc"),
                                vc=dev_in.get("vc"), kic=dev_in.get("kic"), o=step.o, ws=step.ws,
                                stream=stream)
         o_host.copy_(res["o"], non_blocking=True)
@@ -400,7 +429,7 @@ def run_gpu(args, rank, world):
     roof["kernel"] = kname
     roof["peak_source"] = peaks["source"]
     roof["traffic"] = kernel_traffic(kname, w.no)
-    stages = {"compress_ms": round(statistics.mean(comp), 4),
+    stages = {("append_ms" if w.is_decode else "compress_ms"): round(statistics.mean(comp), 4),
               "index_topk_ms": round(statistics.mean(idx), 4),
               "attention_ms": round(att_ms, 4)}
     if counts["compress_bytes"] and statistics.mean(comp) > 0:
@@ -438,9 +467,16 @@ def run_oracle(w, budget_s=12.0, rows_hint=None):
     cores = os.cpu_count()
     bits = {k: oracle.bf16_bits(v) for k, v in inp.items() if v.dtype == torch.bfloat16}
     t0 = time.perf_counter()
+    kv0_ring = None
     if w.is_decode:
-        kc, vc, kic = bits["kc"], bits["vc"], bits["kic"]
-        t_comp = 0.0
+        # the decode step's cache maintenance of the new token, then the ring
+        # holds the window
+        state = {n: bits[n] for n in ("k_ring", "v_ring", "ki_ring", "kc", "vc", "kic")}
+        kv0_ring = oracle.decode_append(state, inp["t_new"].numpy(), bits["k_new"], bits["v_new"],
+                                        inp["wk"].numpy(), inp["wv"].numpy(), w.m, w.W,
+                                        ki_new_bits=bits["ki_new"], wib=inp["wib"].numpy())
+        kc, vc, kic = state["kc"], state["vc"], state["kic"]
+        t_comp = time.perf_counter() - t0
     else:
         _, kc = oracle.block_merge(bits["k"], inp["wk"].numpy(), w.m)
         _, vc = oracle.block_merge(bits["v"], inp["wv"].numpy(), w.m)
@@ -463,8 +499,8 @@ def run_oracle(w, budget_s=12.0, rows_hint=None):
             idx[rows] = sel
             idx = idx.reshape(w.B, w.Lq, w.topk)
         if w.is_decode:
-            oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k_raw"], bits["v_raw"], w.m, w.W,
-                                    q_pos=qp, kv_pos0=inp["kv_pos0"].numpy(), rows=rows)
+            oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k_ring"], bits["v_ring"], w.m, w.W,
+                                    q_pos=qp, kv_pos0=kv0_ring, rows=rows)
         else:
             oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k"], bits["v"], w.m, w.W,
                                     rows=rows)
@@ -481,8 +517,9 @@ def run_oracle(w, budget_s=12.0, rows_hint=None):
     per_row = t_comp / total_rows + dt / len(rows)
     return {"value": round(1.0 / per_row, 3), "unit": "query-tokens/s", "cores": cores,
             "kind": "oracle",
-            "sample": (f"{len(rows)} of {total_rows} query rows (indexer, top-K, attention) + "
-                       f"compression of the whole batch ({t_comp:.2f} s) charged per token")}
+            "sample": (f"{len(rows)} of {total_rows} query rows (indexer, top-K, attention) + " +
+                       (f"cache maintenance of the new tokens ({t_comp:.2f} s)" if w.is_decode else
+                        f"compression of the whole batch ({t_comp:.2f} s)") + " charged per token")}
 
 
 def run_reference_arm(args):

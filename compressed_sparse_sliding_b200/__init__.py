@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
   hyb_attn_fwd         one softmax over compressed (selected / all visible)
                        keys and the raw sliding window
   hyb_fused_fwd        the three stages on one stream
+  hyb_decode_append    decode cache maintenance: window ring + compressed entries
   hyb_workspace_size, hyb_get_device_status, hyb_error_string
 """
 from __future__ import annotations
@@ -65,6 +66,8 @@ _lib.hyb_attn_fwd.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P]
 _lib.hyb_attn_fwd.restype = _I
 _lib.hyb_fused_fwd.argtypes = [_PP] + [_P] * 16 + [ctypes.c_size_t, _P]
 _lib.hyb_fused_fwd.restype = _I
+_lib.hyb_decode_append.argtypes = [_PP] + [_P] * 15
+_lib.hyb_decode_append.restype = _I
 _lib.hyb_get_device_status.argtypes = [_P]
 _lib.hyb_get_device_status.restype = _I
 _lib.hyb_error_string.argtypes = [_I]
@@ -174,6 +177,22 @@ def hyb_fused_fwd(p: HybProblem, q, k_raw, v_raw, wk=None, wv=None, qi=None, wi=
                             _stream(stream))
     _check(st, "hyb_fused_fwd")
     return dict(o=o, kc=kc, vc=vc, kic=kic, idx=idx)
+
+
+def hyb_decode_append(p: HybProblem, t_new, k_new, v_new, k_ring, v_ring, kc, vc, wk, wv,
+                      ki_new=None, wib=None, ki_ring=None, kic=None, kv_pos0=None, stream=None):
+    """Appends one token per sequence: t_new [B] int32, k_new/v_new [B, Hkv, d],
+    ki_new [B, di] (CSA); rings k_ring/v_ring [B, 2W, Hkv, d], ki_ring [B, W, di];
+    caches kc/vc [B, Nc, Hkv, d], kic [B, Nc, di] updated in place.  Returns the
+    kv_pos0 [B] int32 tensor to pass to the attention call (Lkv = 2W)."""
+    if kv_pos0 is None:
+        kv_pos0 = torch.empty((p.B,), dtype=torch.int32, device=k_new.device)
+    st = _lib.hyb_decode_append(ctypes.byref(p), _ptr(t_new), _ptr(k_new), _ptr(v_new), _ptr(ki_new),
+                                _ptr(wk), _ptr(wv), _ptr(wib), _ptr(k_ring), _ptr(v_ring),
+                                _ptr(ki_ring), _ptr(kc), _ptr(vc), _ptr(kic), _ptr(kv_pos0),
+                                _stream(stream))
+    _check(st, "hyb_decode_append")
+    return kv_pos0
 
 
 def hyb_get_device_status(stream=None) -> int:

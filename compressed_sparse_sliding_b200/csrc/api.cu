@@ -34,6 +34,9 @@ cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, i
                                const void *kr, const void *vr, void *o, float *lse,
                                cudaStream_t stream);
 
+struct AppendParams;
+cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream);
+
 static int num_sms_current()
 {
     int dev = 0, n = 148;
@@ -225,6 +228,53 @@ hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
             return st;
     }
     return hyb_attn_fwd(p, q, kc, vc, csa ? idx : nullptr, k_raw, v_raw, o, lse, stream);
+}
+
+hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                             const void *v_new, const void *ki_new, const float *wk, const float *wv,
+                             const float *wib, void *k_ring, void *v_ring, void *ki_ring, void *kc,
+                             void *vc, void *kic, int32_t *kv_pos0, cudaStream_t stream)
+{
+    if (!p || p->B <= 0 || p->Hkv <= 0 || p->d <= 0 || p->m <= 0 || p->W <= 0 || p->Nc <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (p->d % 8 != 0 || p->Lkv != 2 * p->W)
+        return HYB_ERR_INVALID_ARG;
+    if (p->m > p->W)
+        return HYB_ERR_UNSUPPORTED;   // a block must still be in the window when it completes
+    const bool csa = p->topk > 0;
+    if (!t_new || !k_new || !v_new || !wk || !wv || !k_ring || !v_ring || !kc || !vc || !kv_pos0)
+        return HYB_ERR_INVALID_ARG;
+    if (csa && (!ki_new || !wib || !ki_ring || !kic || p->di <= 0 || p->di % 8 != 0))
+        return HYB_ERR_INVALID_ARG;
+    const void *ptrs[] = {k_new, v_new, wk, wv, k_ring, v_ring, kc, vc};
+    for (const void *q : ptrs)
+        if (!aligned16(q))
+            return HYB_ERR_INVALID_ARG;
+    if (csa && (!aligned16(ki_new) || !aligned16(wib) || !aligned16(ki_ring) || !aligned16(kic)))
+        return HYB_ERR_INVALID_ARG;
+    AppendParams a;
+    a.B = p->B;
+    a.Hkv = p->Hkv;
+    a.d = p->d;
+    a.di = csa ? p->di : 0;
+    a.m = p->m;
+    a.W = p->W;
+    a.Nc = p->Nc;
+    a.t_new = t_new;
+    a.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    a.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    a.ki_new = csa ? static_cast<const __nv_bfloat16 *>(ki_new) : nullptr;
+    a.wk = wk;
+    a.wv = wv;
+    a.wib = csa ? wib : nullptr;
+    a.k_ring = static_cast<__nv_bfloat16 *>(k_ring);
+    a.v_ring = static_cast<__nv_bfloat16 *>(v_ring);
+    a.ki_ring = csa ? static_cast<__nv_bfloat16 *>(ki_ring) : nullptr;
+    a.kc = static_cast<__nv_bfloat16 *>(kc);
+    a.vc = static_cast<__nv_bfloat16 *>(vc);
+    a.kic = csa ? static_cast<__nv_bfloat16 *>(kic) : nullptr;
+    a.kv_pos0 = kv_pos0;
+    return cuda_status(launch_decode_append(a, stream));
 }
 
 hyb_status hyb_get_device_status(cudaStream_t stream)

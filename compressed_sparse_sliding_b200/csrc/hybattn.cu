@@ -6,5 +6,6 @@
 #include "attn.cu"
 #include "attn_dense.cu"
 #include "attn_sparse.cu"
+#include "decode_append.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -154,6 +154,34 @@ hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
                          void *vc, void *kic, int32_t *idx, void *o, float *lse, void *ws,
                          size_t ws_bytes, cudaStream_t stream);
 
+/* Decode cache maintenance (deepseek-v4 blog, section 1: the window's raw KV
+ * and the compressed KV are separate caches with different lifetimes).  For
+ * every sequence b the new token at absolute position t = t_new[b] is
+ * appended:
+ *   - its K and V rows go to the raw-window ring twice, rows t mod W and
+ *     t mod W + W, so that the window max(0, t-W+1) .. t is one contiguous
+ *     run of ring rows; kv_pos0[b] (output) is the absolute position of ring
+ *     row 0 for that run, i.e. lo - lo mod W with lo = max(0, t-W+1).  Call
+ *     hyb_attn_fwd / hyb_fused_fwd next with k_raw = k_ring, v_raw = v_ring,
+ *     Lkv = 2W, q_pos = t and this kv_pos0;
+ *   - its indexer key (CSA, p->topk > 0) goes to row t mod W of ki_ring;
+ *   - when (t + 1) is a multiple of m, block j = (t+1)/m - 1 (positions
+ *     j*m .. t) becomes compressed entry j of kc, vc (and kic): the block_merge
+ *     of hyb_hca_compress applied to that one block.
+ * p: B, Hkv, d, m, W, Nc (cache capacity), topk / di (CSA); requires
+ * Lkv == 2*W and m <= W (else HYB_ERR_INVALID_ARG / HYB_ERR_UNSUPPORTED).
+ * t_new: [B] int32; k_new, v_new: [B, Hkv, d] bf16; ki_new: [B, di] bf16;
+ * wk, wv: [m, d] fp32; wib: [m, di] fp32; k_ring, v_ring: [B, 2W, Hkv, d];
+ * ki_ring: [B, W, di]; kc, vc: [B, Nc, Hkv, d]; kic: [B, Nc, di]; kv_pos0:
+ * [B] int32 out.  A negative t, or an entry j >= Nc, is skipped and flagged
+ * as HYB_ERR_DEVICE_BOUNDS.  The rings start zeroed or filled by earlier
+ * calls; rows of positions outside the window are never read. */
+hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                             const void *v_new, const void *ki_new, const float *wk,
+                             const float *wv, const float *wib, void *k_ring, void *v_ring,
+                             void *ki_ring, void *kc, void *vc, void *kic, int32_t *kv_pos0,
+                             cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device (HYB_OK, HYB_ERR_DEVICE_TIMEOUT or HYB_ERR_DEVICE_BOUNDS). */
 hyb_status hyb_get_device_status(cudaStream_t stream);

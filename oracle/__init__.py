@@ -129,6 +129,48 @@ def block_merge(x_bits: np.ndarray, w: np.ndarray, m: int):
     return out, out_b
 
 
+def decode_append(state: dict, t_new, k_new_bits, v_new_bits, wk, wv, m: int, W: int,
+                  ki_new_bits=None, wib=None):
+    """Decode cache maintenance, one new token per sequence ("deepseek-v4"
+    blog, section 1: the window's raw KV and the compressed KV are separate
+    caches with different lifetimes).
+
+    state holds bf16 bits: k_ring / v_ring [B, 2W, Hkv, d], ki_ring [B, W, di]
+    (CSA), kc / vc [B, Nc, Hkv, d], kic [B, Nc, di]; updated in place.
+    The new row of position t goes to ring rows t mod W and t mod W + W (K, V)
+    and t mod W (indexer key).  When (t + 1) is a multiple of m the block of
+    positions j*m .. t, j = (t + 1) / m - 1, is compressed into entry j by
+    block_merge.  Returns kv_pos0 [B] int32: lo - lo mod W, lo = max(0,
+    t - W + 1), the position of ring row 0 for the contiguous window run.
+    """
+    t_new = np.asarray(t_new, dtype=np.int64).reshape(-1)
+    B = len(t_new)
+    kv_pos0 = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        t = int(t_new[b])
+        s = t % W
+        for name, new, two in (("k_ring", k_new_bits, True), ("v_ring", v_new_bits, True),
+                               ("ki_ring", ki_new_bits, False)):
+            if new is None:
+                continue
+            state[name][b, s] = new[b]
+            if two:
+                state[name][b, s + W] = new[b]
+        lo = max(0, t - W + 1)
+        kv_pos0[b] = lo - lo % W
+        if (t + 1) % m == 0:
+            j = (t + 1) // m - 1
+            block = [(j * m + i) % W for i in range(m)]
+            for ring, cache, w in (("k_ring", "kc", wk), ("v_ring", "vc", wv), ("ki_ring", "kic", wib)):
+                if cache not in state or w is None or state.get(ring) is None:
+                    continue
+                rows = state[ring][b, block]               # [m, ...] bits
+                x = rows.reshape(1, m, -1, rows.shape[-1]) if rows.ndim == 3 else rows.reshape(1, m, 1, -1)
+                _, out_b = block_merge(x, w, m)
+                state[cache][b, j] = out_b.reshape(state[cache][b, j].shape)
+    return kv_pos0
+
+
 def _rows(rows: Optional[Sequence[int]], total: int) -> np.ndarray:
     if rows is None:
         return np.arange(total, dtype=np.int64)

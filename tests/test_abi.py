@@ -26,7 +26,8 @@ def declared_symbols():
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
     assert {"hyb_hca_compress", "hyb_csa_index_topk", "hyb_attn_fwd", "hyb_fused_fwd",
-            "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string"} <= set(names)
+            "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string",
+            "hyb_decode_append"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -59,3 +60,19 @@ def test_host_side_argument_checks(lib):
     buf = ctypes.c_void_p(256)
     st = hb._lib.hyb_csa_index_topk(ctypes.byref(p), buf, buf, buf, buf, None, None, 0, None)
     assert st == hb.HYB_ERR_WORKSPACE
+
+
+def test_decode_append_argument_checks(lib):
+    import compressed_sparse_sliding_b200 as hb
+    buf = ctypes.c_void_p(256)
+    args = [buf] * 14 + [None]
+    # the ring must hold 2W rows
+    p = hb.problem(B=1, Lq=1, Lkv=8, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=16)
+    assert hb._lib.hyb_decode_append(ctypes.byref(p), *args) == hb.HYB_ERR_INVALID_ARG
+    # a block longer than the window cannot be merged from the ring
+    p = hb.problem(B=1, Lq=1, Lkv=16, Hq=4, Hkv=1, d=64, m=16, W=8, Nc=16)
+    assert hb._lib.hyb_decode_append(ctypes.byref(p), *args) == hb.HYB_ERR_UNSUPPORTED
+    # CSA needs the indexer-key ring and cache
+    p = hb.problem(B=1, Lq=1, Lkv=16, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=16, topk=4, Hi=2, di=32)
+    a = [buf] * 3 + [None] + [buf] * 11 + [None]
+    assert hb._lib.hyb_decode_append(ctypes.byref(p), *a) == hb.HYB_ERR_INVALID_ARG

@@ -30,12 +30,22 @@ def hb():
 
 
 def run_fused(hb, w, inp):
-    """The benchmark's call: hyb_fused_fwd on resident inputs."""
+    """The benchmark's calls on resident inputs: hyb_fused_fwd (prefill), or
+    for decode the cache maintenance of the new token followed by
+    hyb_fused_fwd reading the window from the ring."""
     if w.is_decode:
-        p = hb.problem(B=w.B, Lq=1, Lkv=w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W, topk=w.topk,
-                       Hi=w.Hi, di=w.di, Nc=w.Nc, q_pos=inp["q_pos"], kv_pos0=inp["kv_pos0"])
-        return hb.hyb_fused_fwd(p, inp["q"], inp["k_raw"], inp["v_raw"], qi=inp["qi"],
-                                wi=inp["wi"], kc=inp["kc"], vc=inp["vc"], kic=inp["kic"])
+        pa = hb.problem(B=w.B, Lq=1, Lkv=2 * w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
+                        topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc)
+        kv0 = hb.hyb_decode_append(pa, inp["t_new"], inp["k_new"], inp["v_new"], inp["k_ring"],
+                                   inp["v_ring"], inp["kc"], inp["vc"], inp["wk"], inp["wv"],
+                                   ki_new=inp["ki_new"], wib=inp["wib"], ki_ring=inp["ki_ring"],
+                                   kic=inp["kic"])
+        p = hb.problem(B=w.B, Lq=1, Lkv=2 * w.W, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W,
+                       topk=w.topk, Hi=w.Hi, di=w.di, Nc=w.Nc, q_pos=inp["q_pos"], kv_pos0=kv0)
+        out = hb.hyb_fused_fwd(p, inp["q"], inp["k_ring"], inp["v_ring"], qi=inp["qi"],
+                               wi=inp["wi"], kc=inp["kc"], vc=inp["vc"], kic=inp["kic"])
+        out["kv_pos0"] = kv0
+        return out
     p = hb.problem(B=w.B, Lq=w.L, Lkv=w.L, Hq=w.Hq, Hkv=w.Hkv, d=w.d, m=w.m, W=w.W, topk=w.topk,
                    Hi=w.Hi, di=w.di, Nc=w.Nc)
     return hb.hyb_fused_fwd(p, inp["q"], inp["k"], inp["v"], wk=inp["wk"], wv=inp["wv"],
@@ -71,6 +81,9 @@ def test_workload_end_to_end(hb, no):
     w = WORKLOADS[no]
     torch.cuda.empty_cache()
     inp = make_inputs(w, device="cuda")
+    pre = None
+    if w.is_decode:   # the state the decode step maintains, before it runs
+        pre = {n: bits(inp[n]).copy() for n in ("k_ring", "v_ring", "ki_ring", "kc", "vc", "kic")}
     out = run_fused(hb, w, inp)
     torch.cuda.synchronize()
     assert hb.hyb_get_device_status() == hb.HYB_OK
@@ -79,11 +92,27 @@ def test_workload_end_to_end(hb, no):
 
     if w.is_decode:
         B = w.B
-        rows_b = [np.arange(B)]
         q_pos = inp["q_pos"].cpu().numpy()
-        kv0 = inp["kv_pos0"].cpu().numpy()
-        kc_b, vc_b, kic_b = bits(inp["kc"]), bits(inp["vc"]), bits(inp["kic"])
-        kr_b, vr_b = bits(inp["k_raw"]), bits(inp["v_raw"])
+        # cache maintenance: rings exact, kv_pos0 exact, the closed block's entry
+        wk, wv, wib = (inp[n].cpu().numpy() for n in ("wk", "wv", "wib"))
+        t_new = inp["t_new"].cpu().numpy()
+        kv0 = oracle.decode_append(pre, t_new, bits(inp["k_new"]), bits(inp["v_new"]), wk, wv, w.m,
+                                   w.W, ki_new_bits=bits(inp["ki_new"]), wib=wib)
+        np.testing.assert_array_equal(out["kv_pos0"].cpu().numpy(), kv0)
+        for ring in ("k_ring", "v_ring", "ki_ring"):
+            np.testing.assert_array_equal(bits(inp[ring]), pre[ring])
+        j = (int(t_new[0]) + 1) // w.m - 1
+        blk = [(j * w.m + i) % w.W for i in range(w.m)]
+        for cache, ring, wt in (("kc", "k_ring", wk), ("vc", "v_ring", wv)):
+            xr = pre[ring][:, blk]
+            _, ref_c = oracle.block_merge(xr, wt, w.m)
+            check_bf16_cache(inp[cache][:, j:j + 1], ref_c, cache, abs_merge(xr, wt, w.m), w.m)
+        xr = pre["ki_ring"][:, blk][:, :, None, :]
+        _, ref_c = oracle.block_merge(xr, wib, w.m)
+        check_bf16_cache(inp["kic"][:, j:j + 1, None, :], ref_c, "kic", abs_merge(xr, wib, w.m), w.m)
+        # the step's index, top-K and attention on the maintained state
+        kc_b, vc_b, kic_b = pre["kc"], pre["vc"], pre["kic"]
+        kr_b, vr_b = pre["k_ring"], pre["v_ring"]
         q_b = bits(inp["q"])
         sc, nv = oracle.index_scores(bits(inp["qi"]), inp["wi"].cpu().numpy(), kic_b, w.m, w.W,
                                      q_pos=q_pos)

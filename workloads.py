@@ -134,6 +134,29 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None) -> Dict[s
         t["kic"] = _normal_bf16(gen, (B, Nc, w.di), sc, device)
         t["q_pos"] = torch.full((B, 1), w.L - 1, dtype=torch.int32, device=device)
         t["kv_pos0"] = torch.full((B,), w.L - w.W, dtype=torch.int32, device=device)
+        # decode step with cache maintenance: the new token is position L - 1
+        # (its K / V rows are the window's last rows); the window's rows sit in
+        # a 2W-row ring at rows p mod W and p mod W + W; block weights and the
+        # window's indexer keys are drawn after everything above, so the
+        # tensors above do not change
+        W = w.W
+        pos = torch.arange(w.L - W, w.L, device=device)
+        slot = pos % W
+        for name, raw in (("k_ring", t["k_raw"]), ("v_ring", t["v_raw"])):
+            ring = torch.zeros((B, 2 * W, Hkv, d), dtype=torch.bfloat16, device=device)
+            ring[:, slot] = raw
+            ring[:, slot + W] = raw
+            t[name] = ring
+        t["k_new"] = t["k_raw"][:, W - 1].contiguous()
+        t["v_new"] = t["v_raw"][:, W - 1].contiguous()
+        t["t_new"] = torch.full((B,), w.L - 1, dtype=torch.int32, device=device)
+        t["wk"] = torch.randn((w.m, d), generator=gen, dtype=torch.float32, device=device)
+        t["wv"] = torch.randn((w.m, d), generator=gen, dtype=torch.float32, device=device)
+        t["wib"] = torch.randn((w.m, w.di), generator=gen, dtype=torch.float32, device=device)
+        ki_win = _normal_bf16(gen, (B, W, w.di), sc, device)
+        t["ki_ring"] = torch.zeros((B, W, w.di), dtype=torch.bfloat16, device=device)
+        t["ki_ring"][:, slot] = ki_win
+        t["ki_new"] = ki_win[:, W - 1].contiguous()
         return t
     L = w.L
     t["k"] = _normal_bf16(gen, (B, L, Hkv, d), sc, device)
