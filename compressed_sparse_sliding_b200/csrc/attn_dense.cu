@@ -76,28 +76,33 @@ struct DenseItem {
     bool vA, vB;             // tile has at least one valid row
     int xA1, xB1;            // last valid token of each tile
     int nct, nrt, rlo;       // compressed tiles, raw tiles, first raw row
+    int nvA, nvB;            // compressed entries visible to the last row of each tile
 };
 
-__device__ __forceinline__ int dn_visible(long long t, int m, int W, int Nc)
+__device__ __forceinline__ int dn_visible(int t, int m, int W, int Nc)
 {
-    long long a = t - W + 1;
+    // positions fit in 32 bits (the launcher checks), so the division is 32-bit
+    const int a = t - W + 1;
     if (a <= 0)
         return 0;
-    long long n = a / m;
-    return n < Nc ? (int)n : Nc;
+    const int n = (int)((unsigned)a / (unsigned)m);
+    return n < Nc ? n : Nc;
 }
 
 __device__ __forceinline__ DenseItem dense_item(const DenseParams &p, long long w)
 {
+    // item counts fit in 32 bits (the launcher checks): 32-bit divisions only
     DenseItem it;
+    const unsigned wu = (unsigned)w;
     if (p.pair_heads) {
-        const long long per_t = (long long)p.B * p.Hkv * p.n_pairs;
-        const int trev = (int)(w / per_t);
-        long long r = w % per_t;
-        it.b = (int)(r / ((long long)p.Hkv * p.n_pairs));
-        r %= (long long)p.Hkv * p.n_pairs;
-        const int kvh = (int)(r / p.n_pairs);
-        const int hp = (int)(r % p.n_pairs);
+        const unsigned per_b = (unsigned)p.Hkv * (unsigned)p.n_pairs;
+        const unsigned per_t = (unsigned)p.B * per_b;
+        const int trev = (int)(wu / per_t);
+        unsigned r = wu % per_t;
+        it.b = (int)(r / per_b);
+        r %= per_b;
+        const int kvh = (int)(r / (unsigned)p.n_pairs);
+        const int hp = (int)(r % (unsigned)p.n_pairs);
         it.hA = kvh * p.g + 2 * hp;
         it.hB = it.hA + 1;
         it.tA = (p.n_ttiles - 1 - trev) * kDnBM;
@@ -105,11 +110,11 @@ __device__ __forceinline__ DenseItem dense_item(const DenseParams &p, long long 
         it.vA = true;
         it.vB = (2 * hp + 1) < p.g;
     } else {
-        const long long per_t = (long long)p.B * p.Hq;
-        const int trev = (int)(w / per_t);
-        long long r = w % per_t;
-        it.b = (int)(r / p.Hq);
-        it.hA = (int)(r % p.Hq);
+        const unsigned per_t = (unsigned)p.B * (unsigned)p.Hq;
+        const int trev = (int)(wu / per_t);
+        const unsigned r = wu % per_t;
+        it.b = (int)(r / (unsigned)p.Hq);
+        it.hA = (int)(r % (unsigned)p.Hq);
         it.hB = it.hA;
         it.tA = (p.n_pairs - 1 - trev) * 2 * kDnBM;
         it.tB = it.tA + kDnBM;
@@ -122,6 +127,8 @@ __device__ __forceinline__ DenseItem dense_item(const DenseParams &p, long long 
     const int tmax = it.vB ? max(it.xA1, it.xB1) : it.xA1;
     const int nv = dn_visible(tmax, p.m, p.W, p.Nc);
     it.nct = (nv + kDnBN - 1) / kDnBN;
+    it.nvA = dn_visible(it.xA1, p.m, p.W, p.Nc);
+    it.nvB = dn_visible(it.xB1, p.m, p.W, p.Nc);
     int lo = tmin - p.W + 1;
     if (lo < 0)
         lo = 0;
@@ -140,7 +147,7 @@ __device__ __forceinline__ bool dn_active(const DenseParams &p, const DenseItem 
     const int x0 = B_ ? it.tB : it.tA;
     const int x1 = B_ ? it.xB1 : it.xA1;
     if (i < it.nct)
-        return i * kDnBN < dn_visible(x1, p.m, p.W, p.Nc);
+        return i * kDnBN < (B_ ? it.nvB : it.nvA);
     const int r0 = it.rlo + (i - it.nct) * kDnBN;
     int need_lo = x0 - p.W + 1;
     if (need_lo < 0)
@@ -603,6 +610,8 @@ cudaError_t launch_hca_attn(int B, int L, int Lkv, int Hq, int Hkv, int d, int N
         p.n_pairs = (L + 2 * kDnBM - 1) / (2 * kDnBM);
         p.n_items = (long long)p.n_pairs * B * Hq;
     }
+    if (p.n_items >= (1LL << 31) || (long long)L + W >= (1LL << 30))
+        return cudaErrorInvalidValue;   // item indices and positions use 32-bit arithmetic
     p.scale_log2 = scale * 1.4426950408889634f;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
