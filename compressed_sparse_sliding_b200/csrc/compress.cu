@@ -185,8 +185,9 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
     const int np = S / gw;                      // partial sets after the warp fold
     float *part = sm_rg;                        // [2][np][ipc][8] partial sums (S > 1)
     float *ring_f = sm_rg + (S > 1 ? (size_t)2 * np * ipc * 8 : 0);
-    float *red = ring_f;                        // [S][dx] partial max, then sums (prologue only,
-                                                // before the ring is filled)
+    float *red = ring_f;                        // [S][dx] partial max, then sums, and [dx]
+    float *fin = ring_f + (size_t)S * dx;       // combined values (prologue only, before the
+                                                // ring is filled)
     const int s = tid / ipc;
     const int li = tid % ipc;
     const int c0 = (li * 8) % dx;               // fixed channel octet of this thread
@@ -210,19 +211,28 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
             v = fmaxf(v, P[k][q]);
         mx[q] = v;
     }
-    if (owner)
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            red[s * dx + c0 + q] = mx[q];
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        float v = red[c0 + q];
-        for (int g = 1; g < S; ++g)
-            v = fmaxf(v, red[g * dx + c0 + q]);
-        mx[q] = v;
+    // Per-channel max and sum over the S position groups: the groups' values go
+    // to red [S][dx]; thread c < dx combines channel c (consecutive threads,
+    // consecutive addresses) into fin [dx]; every thread reads its 8 channels
+    // back as two 16-byte loads.
+    if (owner) {
+        reinterpret_cast<float4 *>(red + s * dx + c0)[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+        reinterpret_cast<float4 *>(red + s * dx + c0)[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
     }
     __syncthreads();
+    if (tid < dx) {
+        float v = red[tid];
+        for (int g = 1; g < S; ++g)
+            v = fmaxf(v, red[g * dx + tid]);
+        fin[tid] = v;
+    }
+    __syncthreads();
+    {
+        const float4 a = reinterpret_cast<const float4 *>(fin + c0)[0];
+        const float4 b = reinterpret_cast<const float4 *>(fin + c0)[1];
+        mx[0] = a.x; mx[1] = a.y; mx[2] = a.z; mx[3] = a.w;
+        mx[4] = b.x; mx[5] = b.y; mx[6] = b.z; mx[7] = b.w;
+    }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         float acc = 0.f;
@@ -233,17 +243,27 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
         }
         den[q] = acc;
     }
-    if (owner)
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            red[s * dx + c0 + q] = den[q];
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    if (owner) {
+        reinterpret_cast<float4 *>(red + s * dx + c0)[0] = make_float4(den[0], den[1], den[2], den[3]);
+        reinterpret_cast<float4 *>(red + s * dx + c0)[1] = make_float4(den[4], den[5], den[6], den[7]);
+    }
+    __syncthreads();   // (every thread has read fin's maxima)
+    if (tid < dx) {
         float v = 0.f;
         for (int g = 0; g < S; ++g)
-            v += red[g * dx + c0 + q];
-        const float inv = 1.f / v;
+            v += red[g * dx + tid];
+        fin[tid] = v;
+    }
+    __syncthreads();
+    {
+        const float4 a = reinterpret_cast<const float4 *>(fin + c0)[0];
+        const float4 b = reinterpret_cast<const float4 *>(fin + c0)[1];
+        den[0] = a.x; den[1] = a.y; den[2] = a.z; den[3] = a.w;
+        den[4] = b.x; den[5] = b.y; den[6] = b.z; den[7] = b.w;
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float inv = 1.f / den[q];
 #pragma unroll
         for (int k = 0; k < NPOS; ++k)
             P[k][q] *= inv;
@@ -355,7 +375,7 @@ static cudaError_t launch_merge_regs(const void *x, int B, int L, int H, int dx,
     const int gw = ipc < 32 ? 32 / ipc : 1;
     const int np = S / gw;
     const size_t ring = (size_t)kMergeStages * NPOS * kMergeThreads * 16;
-    const size_t red = sizeof(float) * (size_t)S * dx;
+    const size_t red = sizeof(float) * (size_t)(S + 1) * dx;
     const size_t smem = (S > 1 ? sizeof(float) * (size_t)2 * np * ipc * 8 : 0) + (ring > red ? ring : red);
     cudaError_t e = cudaFuncSetAttribute(block_merge_regs<NPOS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
