@@ -193,6 +193,41 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
     const int c0 = (li * 8) % dx;               // fixed channel octet of this thread
     const bool owner = li < dx / 8;             // one thread per (s, channel octet) writes
 
+    // ---- the block stream ----
+    // Every thread copies its own NPOS 16-byte pieces of a tile into private
+    // slots of a kMergeStages-deep shared ring with cp.async, kMergeStages - 1
+    // tiles ahead of the one it reduces; a thread only ever reads the slots it
+    // filled, so the ring needs no barrier (cp.async.wait_group orders it).
+    // Tile k uses stage (k + 1) mod kMergeStages: the first tiles go to stages
+    // 1, 2, ... before the weight prologue, whose scratch lives in stage 0.
+    const int Nc = L / m;
+    const int E8 = H * dx / 8;
+    const long long items = (long long)B * Nc * E8;
+    const long long ntiles = (items + ipc - 1) / ipc;
+    const size_t row_elems = (size_t)H * dx;
+    const uint32_t ring = smem_u32(ring_f);
+    auto slot = [&](int stage, int k) -> uint32_t {
+        return ring + (uint32_t)(((stage * NPOS + k) * kMergeThreads + tid) * 16);
+    };
+    auto issue = [&](long long tile, int stage) {
+        const long long item = tile * ipc + li;
+        if (tile < ntiles && item < items) {
+            const long long unit = item / E8;
+            const int e8 = (int)(item % E8);
+            const int b = (int)(unit / Nc);
+            const int j = (int)(unit % Nc);
+            const __nv_bfloat16 *src =
+                x + ((size_t)b * L + (size_t)j * m + s) * row_elems + (size_t)e8 * 8;
+#pragma unroll
+            for (int k = 0; k < NPOS; ++k)
+                cp_async_16(slot(stage, k), src + (size_t)k * S * row_elems, 16u);
+        }
+        cp_async_commit();   // one group per tile, empty past the end
+    };
+#pragma unroll
+    for (int d = 0; d < kMergeStages - 1; ++d)
+        issue((long long)blockIdx.x + (long long)d * gridDim.x, d + 1);
+
     // ---- this thread's weights: positions s, s + S, ... (NPOS of them) ----
     float P[NPOS][8];
 #pragma unroll
@@ -269,40 +304,8 @@ block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ 
             P[k][q] *= inv;
     }
 
-    // ---- stream the blocks ----
-    // Every thread copies its own NPOS 16-byte pieces of a tile into private
-    // slots of a kMergeStages-deep shared ring with cp.async, kMergeStages - 1
-    // tiles ahead of the one it reduces; a thread only ever reads the slots it
-    // filled, so the ring needs no barrier (cp.async.wait_group orders it).
-    const int Nc = L / m;
-    const int E8 = H * dx / 8;
-    const long long items = (long long)B * Nc * E8;
-    const long long ntiles = (items + ipc - 1) / ipc;
-    const size_t row_elems = (size_t)H * dx;
-    const uint32_t ring = smem_u32(ring_f);
-    auto slot = [&](int stage, int k) -> uint32_t {
-        return ring + (uint32_t)(((stage * NPOS + k) * kMergeThreads + tid) * 16);
-    };
-    auto issue = [&](long long tile, int stage) {
-        const long long item = tile * ipc + li;
-        if (tile < ntiles && item < items) {
-            const long long unit = item / E8;
-            const int e8 = (int)(item % E8);
-            const int b = (int)(unit / Nc);
-            const int j = (int)(unit % Nc);
-            const __nv_bfloat16 *src =
-                x + ((size_t)b * L + (size_t)j * m + s) * row_elems + (size_t)e8 * 8;
-#pragma unroll
-            for (int k = 0; k < NPOS; ++k)
-                cp_async_16(slot(stage, k), src + (size_t)k * S * row_elems, 16u);
-        }
-        cp_async_commit();   // one group per tile, empty past the end
-    };
-    __syncthreads();   // every thread is done with `red`, which the ring overwrites
-#pragma unroll
-    for (int d = 0; d < kMergeStages - 1; ++d)
-        issue((long long)blockIdx.x + (long long)d * gridDim.x, d);
-    int parity = 0, stage = 0;
+    __syncthreads();   // every thread is done with `red` / `fin` (ring stage 0)
+    int parity = 0, stage = 1;
     for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         issue(tile + (long long)(kMergeStages - 1) * gridDim.x, (stage + kMergeStages - 1) % kMergeStages);
         cp_async_wait_group<kMergeStages - 1>();   // this tile's copies have landed
