@@ -7,8 +7,15 @@
 // the Hi accumulators of its row, forms the weighted ReLU sum and stores the
 // visible part of the tile into the token's score row.  Queries (one TMA box
 // per head) stay in shared memory; key tiles stream through a 4-stage ring.
+// When a score row is a multiple of 16 bytes the epilogue stages each 128 x 32
+// block of scores in shared memory (128-byte swizzle) and one thread writes it
+// with a TMA tensor store, so the rows leave as whole 128-byte lines instead of
+// 32 scattered 16-byte pieces per warp instruction (columns past a row's
+// visible prefix are written too; readers only use the prefix).
 // Roles (256 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 4-7
 // epilogue (TMEM lane quadrants 0-3); warps 2-3 idle.
+#include <cstring>
+
 #include "common.cuh"
 
 namespace hyb {
@@ -23,6 +30,7 @@ constexpr int kIxChunkTiles = 32; // key tiles per CTA (2048 entries)
 struct IndexParams {
     int B, Lq, Hi, Nc, m, W;
     int n_ttiles, n_chunks;       // token tiles, key chunks per token tile
+    int tma_store;                // 1: scores leave through the staged TMA store
     const int32_t *q_pos;
     const float *wi;              // [B, Lq, Hi]
     float *scores;                // [B * Lq, Nc]
@@ -36,13 +44,25 @@ struct IxSmem {
     static constexpr int OFF_K = HI * Q_BYTES;
     static constexpr int OFF_BAR = OFF_K + kIxStages * K_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
-    static constexpr int BYTES = OFF_MISC + 16 * 4;
+    static constexpr int OFF_ST = (OFF_MISC + 16 * 4 + 1023) & ~1023;  // 2 x [128][32] fp32 staging
+    static constexpr int ST_BYTES = kIxBM * 32 * 4;
+    static constexpr int BYTES = OFF_ST + 2 * ST_BYTES;
 };
+
+// TMA tensor store of one staged box (3-D map), as one bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
 
 template <int HI>
 __global__ void __launch_bounds__(kIxThreads, 1)
 index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const IndexParams p)
+                const __grid_constant__ CUtensorMap tm_s, const IndexParams p)
 {
     using SM = IxSmem<HI>;
     extern __shared__ __align__(1024) uint8_t ix_smem_raw[];
@@ -169,31 +189,64 @@ index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         float *srow = p.scores + ((size_t)b * p.Lq + (valid ? t : 0)) * p.Nc;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t stage0 = smem_u32(smem + SM::OFF_ST);
+        uint32_t u = 0;                                  // staged blocks written
+        // Every epilogue thread runs every iteration (the staged store meets a
+        // named barrier); after a failed wait it only skips the TMEM work.
+        bool ok = true;
         for (int i = 0; i < nt; ++i) {
             const int db = i & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (i >> 1) & 1, abort_flag)))
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (i >> 1) & 1, abort_flag));
+            if (!ok && !p.tma_store)
                 break;
             tc_fence_after();
             const int s0 = (j0 + i) * kIxBN;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                // the Hi accumulators of this row's 32 keys, one wait
-                float d[HI][32];
-#pragma unroll
-                for (int h = 0; h < HI; ++h)
-                    tmem_ld32(tl + (db * HI + h) * kIxBN + half * 32, d[h]);
-                tmem_ld_wait();
                 float acc[32];
+                if (ok) {
+                    // the Hi accumulators of this row's 32 keys, one wait
+                    float d[HI][32];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    float a = wv[0] * fmaxf(d[0][q], 0.f);
+                    for (int h = 0; h < HI; ++h)
+                        tmem_ld32(tl + (db * HI + h) * kIxBN + half * 32, d[h]);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int h = 1; h < HI; ++h)
-                        a = fmaf(wv[h], fmaxf(d[h][q], 0.f), a);
-                    acc[q] = a;
+                    for (int q = 0; q < 32; ++q) {
+                        float a = wv[0] * fmaxf(d[0][q], 0.f);
+#pragma unroll
+                        for (int h = 1; h < HI; ++h)
+                            a = fmaf(wv[h], fmaxf(d[h][q], 0.f), a);
+                        acc[q] = a;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        acc[q] = 0.f;
                 }
                 const int sb = s0 + half * 32;
-                if (valid && sb < nv) {
+                if (p.tma_store) {
+                    // this row's 32 scores into the staging block (128-byte swizzle:
+                    // 16-byte chunk c of row r at chunk c ^ (r & 7))
+                    const uint32_t buf = stage0 + (u & 1) * SM::ST_BYTES + row * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                         buf + ((c ^ (row & 7)) << 4)),
+                                     "f"(acc[4 * c]), "f"(acc[4 * c + 1]), "f"(acc[4 * c + 2]),
+                                     "f"(acc[4 * c + 3])
+                                     : "memory");
+                    fence_proxy_async_smem();
+                    // the other buffer's copy has read its rows before anyone
+                    // rewrites them (one copy in flight at most)
+                    if (row == 0)
+                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (row == 0)
+                        tma_store_3d(&tm_s, stage0 + (u & 1) * SM::ST_BYTES, sb, t0, b);
+                    ++u;
+                } else if (valid && sb < nv) {
                     if (sb + 32 <= nv && (p.Nc & 3) == 0) {
 #pragma unroll
                         for (int q = 0; q < 32; q += 4)
@@ -205,9 +258,13 @@ index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&bar[11 + db]);
+            if (ok) {
+                tc_fence_before();
+                mbar_arrive(&bar[11 + db]);
+            }
         }
+        if (row == 0)
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
@@ -229,6 +286,21 @@ static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const
     ok &= make_map(&mk, kic, kIxDi, 1, p.Nc, p.B, 1, kIxBN);
     if (!ok)
         return cudaErrorInvalidValue;
+    // scores [B, Lq, Nc] fp32 as (Nc, Lq, B) with a (32, 128, 1) box, 128-byte
+    // swizzle; rows past Lq and columns past Nc are clipped by the copy
+    CUtensorMap ms;
+    std::memset(&ms, 0, sizeof(ms));
+    if (p.tma_store) {
+        EncodeTiledFn fn = encode_fn();
+        cuuint64_t dims[3] = {(cuuint64_t)p.Nc, (cuuint64_t)p.Lq, (cuuint64_t)p.B};
+        cuuint64_t strides[2] = {(cuuint64_t)p.Nc * 4, (cuuint64_t)p.Nc * 4 * p.Lq};
+        cuuint32_t box[3] = {32, (cuuint32_t)kIxBM, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        if (!fn || fn(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.scores, dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     size_t smem = 1024 + SM::BYTES;
     if (smem < 120 * 1024)
         smem = 120 * 1024;  // one CTA per SM: each holds all 512 TMEM columns
@@ -237,7 +309,7 @@ static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const
     if (e != cudaSuccess)
         return e;
     dim3 grid(p.n_ttiles * p.n_chunks, p.B);
-    kern<<<grid, kIxThreads, smem, stream>>>(mq, mk, p);
+    kern<<<grid, kIxThreads, smem, stream>>>(mq, mk, ms, p);
     return cudaGetLastError();
 }
 
@@ -465,6 +537,8 @@ cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *
     p.q_pos = q_pos;
     p.wi = wi;
     p.scores = scores;
+    // the tensor store needs 16-byte row strides and a 16-byte aligned base
+    p.tma_store = (Nc % 4 == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) ? 1 : 0;
     switch (Hi) {
     case 1: return launch_index_tc_t<1>(p, qi, kic, stream);
     case 2: return launch_index_tc_t<2>(p, qi, kic, stream);
