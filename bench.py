@@ -62,8 +62,24 @@ def n_visible(t, m, W, Nc):
     return 0 if a <= 0 else min(a // m, Nc)
 
 
-def algorithmic_counts(w):
-    """Per step: attention keys and FLOP, indexer FLOP, unique bytes per stage."""
+def algorithmic_counts(w, gated=False):
+    """Per step: attention keys and FLOP, indexer FLOP, unique bytes per stage.
+    gated: the three-branch variant (all blocks ending at or before t, the
+    selected ones among them, the window; the selection sees the same blocks)."""
+    if gated:
+        t = np.arange(w.L, dtype=np.int64)
+        nv0 = np.minimum((t + 1) // w.m, w.Nc)
+        win = np.minimum(w.W, t + 1)
+        attn_keys = int(w.B * (nv0 + np.minimum(nv0, w.topk) + win).sum())
+        bf = 2
+        q_o = 2 * w.B * w.Lq * w.Hq * w.d * bf
+        return dict(attn_keys=attn_keys, attn_flop=4 * w.d * w.Hq * attn_keys,
+                    idx_flop=2 * w.Hi * w.di * int(w.B * nv0.sum()),
+                    attn_bytes=q_o + 2 * w.B * w.L * w.Hkv * w.d * bf + 2 * w.B * w.Nc * w.Hkv * w.d * bf
+                    + w.B * w.Lq * w.topk * 4 + w.B * w.Lq * w.Hq * 3 * 4,
+                    compress_bytes=2 * w.B * w.L * w.Hkv * w.d * bf + 2 * w.B * w.Nc * w.Hkv * w.d * bf
+                    + w.B * w.L * w.di * bf + w.B * w.Nc * w.di * bf,
+                    idx_bytes=0)
     if w.is_decode:
         t = w.L - 1
         nv = n_visible(t, w.m, w.W, w.Nc)
@@ -118,8 +134,8 @@ class Step:
     """One forward pass as the three C-ABI stages on one stream, with CUDA
     events between the stages (the same kernels hyb_fused_fwd launches)."""
 
-    def __init__(self, hb, w, inp):
-        self.hb, self.w, self.inp = hb, w, inp
+    def __init__(self, hb, w, inp, gated=False):
+        self.hb, self.w, self.inp, self.gated = hb, w, inp, gated
         dev = inp["q"].device
         self.kv0 = torch.empty((w.B,), dtype=torch.int32, device=dev)
         self.p = problem_for(hb, w, inp, self.kv0)
@@ -135,6 +151,12 @@ class Step:
         self.o = torch.empty((w.B, w.Lq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
         need = hb.hyb_workspace_size(self.p)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        if gated:
+            # the selection sees the same blocks as the compressed branch (W = 0)
+            self.p_sel = problem_for(hb, w, inp)
+            self.p_sel.W = 0
+            gneed = hb.hyb_gated_workspace_size(self.p)
+            self.gws = torch.empty(max(gneed, 256), dtype=torch.uint8, device=dev)
         self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         self.launches = 0
 
@@ -158,14 +180,19 @@ class Step:
                 launches += 1
         ev[1].record(stream)
         if w.topk:
-            hb.hyb_csa_index_topk(self.p, inp["qi"], inp["wi"], self.kic, idx=self.idx, ws=self.ws,
-                                  stream=stream)
+            hb.hyb_csa_index_topk(self.p_sel if self.gated else self.p, inp["qi"], inp["wi"], self.kic,
+                                  idx=self.idx, ws=self.ws, stream=stream)
             launches += 2
         ev[2].record(stream)
-        hb.hyb_attn_fwd(self.p, inp["q"], self.kc, self.vc, self.idx,
-                        inp["k_ring"] if w.is_decode else inp["k"],
-                        inp["v_ring"] if w.is_decode else inp["v"], o=self.o, stream=stream)
-        launches += 1
+        if self.gated:
+            hb.hyb_gated_fwd(self.p, inp["q"], self.kc, self.vc, self.idx, inp["k"], inp["v"],
+                             inp["gate"], o=self.o, ws=self.gws, stream=stream)
+            launches += 4
+        else:
+            hb.hyb_attn_fwd(self.p, inp["q"], self.kc, self.vc, self.idx,
+                            inp["k_ring"] if w.is_decode else inp["k"],
+                            inp["v_ring"] if w.is_decode else inp["v"], o=self.o, stream=stream)
+            launches += 1
         ev[3].record(stream)
         self.launches = launches
 
@@ -294,6 +321,13 @@ def kernel_traffic(kernel: str, config_no: int):
         return None
 
 
+def gate_logits(w, device, rank=0):
+    """Seeded gate logits [B, L, Hq, 3] for the gated variant (N(0, 2^2))."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(20360 + w.no + 1000 * rank)
+    return (torch.randn((w.B, w.Lq, w.Hq, 3), generator=g) * 2).to(device)
+
+
 def run_gpu(args, rank, world):
     import compressed_sparse_sliding_b200 as hb
     w = WORKLOADS[args.config]
@@ -301,8 +335,11 @@ def run_gpu(args, rank, world):
     inp = make_inputs(w, device=dev, seed=20260 + w.no + 1000 * rank)
     if not w.is_decode:
         inp["k_raw"], inp["v_raw"] = inp["k"], inp["v"]
+    gated = args.variant == "gated"
+    if gated:
+        inp["gate"] = gate_logits(w, dev, rank)
     stream = torch.cuda.current_stream()
-    step = Step(hb, w, inp)
+    step = Step(hb, w, inp, gated)
     # L2 flush: write 256 MiB, then read another 256 MiB so that no dirty line
     # of the flush buffer is left for the timed step to write back
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -312,7 +349,7 @@ def run_gpu(args, rank, world):
         flush.fill_(1)
         flush_rd.sum()
 
-    counts = algorithmic_counts(w)
+    counts = algorithmic_counts(w, gated)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -362,7 +399,7 @@ def run_gpu(args, rank, world):
     if w.is_decode:
         per_step = ("q", "qi", "wi", "k_new", "v_new", "ki_new", "t_new", "q_pos")
     else:
-        per_step = ("q", "k", "v", "wk", "wv", "qi", "wi", "ki", "wib")
+        per_step = ("q", "k", "v", "wk", "wv", "qi", "wi", "ki", "wib", "gate")
     host = {k: inp[k].cpu().pin_memory() for k in per_step if k in inp}
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     if w.is_decode:
@@ -378,6 +415,18 @@ def run_gpu(args, rank, world):
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
         p = problem_for(hb, w, dev_in, kv0_e2e)
+        if gated:
+            # the public calls of the gated variant: compression, the selection
+            # (W = 0 visibility) and the three-branch attention
+            hb.hyb_hca_compress(dev_in["k"], dev_in["wk"], w.m, out=step.kc, stream=stream)
+            hb.hyb_hca_compress(dev_in["v"], dev_in["wv"], w.m, out=step.vc, stream=stream)
+            hb.hyb_hca_compress(dev_in["ki"], dev_in["wib"], w.m, out=step.kic, stream=stream)
+            hb.hyb_csa_index_topk(step.p_sel, dev_in["qi"], dev_in["wi"], step.kic, idx=step.idx,
+                                  ws=step.ws, stream=stream)
+            hb.hyb_gated_fwd(p, dev_in["q"], step.kc, step.vc, step.idx, dev_in["k"], dev_in["v"],
+                             dev_in["gate"], o=step.o, ws=step.gws, stream=stream)
+            o_host.copy_(step.o, non_blocking=True)
+            return
         if w.is_decode:
             hb.hyb_decode_append(p, dev_in["t_new"], dev_in["k_new"], dev_in["v_new"],
                                  dev_in["k_ring"], dev_in["v_ring"], dev_in["kc"], dev_in["vc"],
@@ -426,6 +475,8 @@ def run_gpu(args, rank, world):
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4)}
     kname, ksrc = attention_kernel(w)
+    if gated:
+        kname = "hyb_gated_fwd (three attention kernels + combine)"
     roof["kernel"] = kname
     roof["peak_source"] = peaks["source"]
     roof["traffic"] = kernel_traffic(kname, w.no)
@@ -446,6 +497,7 @@ def run_gpu(args, rank, world):
         "data": "synthetic (seeded N(0,1) bf16 inputs, N(0,1) block weights, U(0,1) head weights)",
         "config": {"workload": w.name, "desc": w.describe(), "global_batch": w.B * world,
                    "seq_len": w.L, "parallelism": f"replicas{world}",
+                   "variant": args.variant,
                    "l2": "flushed between steps (256 MiB written, then a separate 256 MiB read)"},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "query-tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
@@ -458,7 +510,7 @@ def run_gpu(args, rank, world):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def run_oracle(w, budget_s=12.0, rows_hint=None):
+def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False):
     """Times the oracle on a bounded sample of the workload.  Compression of
     the whole batch is timed once and charged per query token; indexer, top-K
     and attention are timed on a sample of query rows."""
@@ -486,19 +538,24 @@ def run_oracle(w, budget_s=12.0, rows_hint=None):
             kic = kic[:, :, 0, :]
         t_comp = time.perf_counter() - t0
     total_rows = w.B * w.Lq
+    gate_np = gate_logits(w, "cpu").numpy() if gated else None
 
     def rows_work(rows):
         t1 = time.perf_counter()
         qp = inp["q_pos"].numpy() if w.is_decode else None
         idx = None
         if w.topk:
-            sc, nv = oracle.index_scores(bits["qi"], inp["wi"].numpy(), kic, w.m, w.W, q_pos=qp,
+            sc, nv = oracle.index_scores(bits["qi"], inp["wi"].numpy(), kic, w.m, 0 if gated else w.W,
+                                         q_pos=qp,
                                          rows=rows)
             sel = oracle.topk(sc, nv, w.topk)
             idx = np.full((total_rows, w.topk), -1, np.int32)
             idx[rows] = sel
             idx = idx.reshape(w.B, w.Lq, w.topk)
-        if w.is_decode:
+        if gated:
+            oracle.gated_attention(bits["q"], kc, vc, idx, bits["k"], bits["v"], w.m, w.W,
+                                   gate_np, rows=rows)
+        elif w.is_decode:
             oracle.hybrid_attention(bits["q"], kc, vc, idx, bits["k_ring"], bits["v_ring"], w.m, w.W,
                                     q_pos=qp, kv_pos0=kv0_ring, rows=rows)
         else:
@@ -526,10 +583,11 @@ def run_reference_arm(args):
     w = WORKLOADS[args.config]
     per_step = []
     base = None
+    gated = args.variant == "gated"
     for _ in range(args.warmup):
-        run_oracle(w, budget_s=2.0, rows_hint=4)
+        run_oracle(w, budget_s=2.0, rows_hint=4, gated=gated)
     for _ in range(args.steps):
-        base = run_oracle(w, budget_s=6.0, rows_hint=8)
+        base = run_oracle(w, budget_s=6.0, rows_hint=8, gated=gated)
         per_step.append(1.0 / base["value"])
     value = 1.0 / statistics.mean(per_step)
     cpu = dict(base)
@@ -541,7 +599,7 @@ def run_reference_arm(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded inputs as the GPU arm)",
         "config": {"workload": w.name, "desc": w.describe(), "global_batch": w.B, "seq_len": w.L,
-                   "parallelism": "host cores (OpenMP)"},
+                   "parallelism": "host cores (OpenMP)", "variant": args.variant},
         "cpu_baseline": cpu,
         "e2e": {"value": round(value, 3), "unit": "query-tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -556,8 +614,12 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated"],
+                    help="gated: the three-branch variant (CSA workloads with prefill)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.variant == "gated" and (not WORKLOADS[args.config].topk or WORKLOADS[args.config].is_decode):
+        ap.error("--variant gated needs a CSA prefill workload (configs 1 and 3)")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -577,7 +639,7 @@ def main():
     try:
         res = run_gpu(args, rank, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config])
+            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config], gated=args.variant == "gated")
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

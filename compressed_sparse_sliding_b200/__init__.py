@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
                        keys and the raw sliding window
   hyb_fused_fwd        the three stages on one stream
   hyb_decode_append    decode cache maintenance: window ring + compressed entries
+  hyb_gated_fwd        the gated three-branch variant (compressed, selected, window)
   hyb_workspace_size, hyb_get_device_status, hyb_error_string
 """
 from __future__ import annotations
@@ -68,6 +69,10 @@ _lib.hyb_fused_fwd.argtypes = [_PP] + [_P] * 16 + [ctypes.c_size_t, _P]
 _lib.hyb_fused_fwd.restype = _I
 _lib.hyb_decode_append.argtypes = [_PP] + [_P] * 15
 _lib.hyb_decode_append.restype = _I
+_lib.hyb_gated_workspace_size.argtypes = [_PP]
+_lib.hyb_gated_workspace_size.restype = ctypes.c_size_t
+_lib.hyb_gated_fwd.argtypes = [_PP] + [_P] * 9 + [ctypes.c_size_t, _P]
+_lib.hyb_gated_fwd.restype = _I
 _lib.hyb_get_device_status.argtypes = [_P]
 _lib.hyb_get_device_status.restype = _I
 _lib.hyb_error_string.argtypes = [_I]
@@ -193,6 +198,23 @@ def hyb_decode_append(p: HybProblem, t_new, k_new, v_new, k_ring, v_ring, kc, vc
                                 _stream(stream))
     _check(st, "hyb_decode_append")
     return kv_pos0
+
+
+def hyb_gated_workspace_size(p: HybProblem) -> int:
+    return int(_lib.hyb_gated_workspace_size(ctypes.byref(p)))
+
+
+def hyb_gated_fwd(p: HybProblem, q, kc, vc, idx, k_raw, v_raw, gate, o=None, ws=None, stream=None):
+    """Gated three-branch attention; gate [B, Lq, Hq, 3] fp32 logits."""
+    if o is None:
+        o = torch.empty((p.B, p.Lq, p.Hq, p.d), dtype=torch.bfloat16, device=q.device)
+    need = int(_lib.hyb_gated_workspace_size(ctypes.byref(p)))
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = _lib.hyb_gated_fwd(ctypes.byref(p), _ptr(q), _ptr(kc), _ptr(vc), _ptr(idx), _ptr(k_raw),
+                            _ptr(v_raw), _ptr(gate), _ptr(o), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "hyb_gated_fwd")
+    return o
 
 
 def hyb_get_device_status(stream=None) -> int:

@@ -36,6 +36,8 @@ cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, i
 
 struct AppendParams;
 cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream);
+cudaError_t launch_gated_combine(const void *o1, const void *o2, const void *o3, const float *gate,
+                                 void *o, long long rows, int d, cudaStream_t stream, int num_sms);
 
 static int num_sms_current()
 {
@@ -275,6 +277,53 @@ hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const v
     a.kic = csa ? static_cast<__nv_bfloat16 *>(kic) : nullptr;
     a.kv_pos0 = kv_pos0;
     return cuda_status(launch_decode_append(a, stream));
+}
+
+size_t hyb_gated_workspace_size(const hyb_problem *p)
+{
+    if (!p || p->B <= 0 || p->Lq <= 0 || p->Hq <= 0 || p->d <= 0)
+        return 0;
+    const size_t one = ((size_t)p->B * p->Lq * p->Hq * p->d * 2 + 255) & ~(size_t)255;
+    return 3 * one;
+}
+
+hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                         const int32_t *idx, const void *k_raw, const void *v_raw, const float *gate,
+                         void *o, void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, false);
+    if (st != HYB_OK)
+        return st;
+    if (!idx || p->topk <= 0 || !gate || !o || !q || p->Nc <= 0 || p->W <= 0 || p->d % 8 != 0)
+        return HYB_ERR_INVALID_ARG;
+    const size_t need = hyb_gated_workspace_size(p);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return HYB_ERR_WORKSPACE;
+    const size_t one = need / 3;
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    // branch 1: every compressed block that ends at or before t (no window)
+    hyb_problem p1 = *p;
+    p1.W = 0;
+    p1.topk = 0;
+    st = hyb_attn_fwd(&p1, q, kc, vc, nullptr, k_raw, v_raw, w8, nullptr, stream);
+    if (st != HYB_OK)
+        return st;
+    // branch 2: the selected blocks among those (no window)
+    hyb_problem p2 = *p;
+    p2.W = 0;
+    st = hyb_attn_fwd(&p2, q, kc, vc, idx, k_raw, v_raw, w8 + one, nullptr, stream);
+    if (st != HYB_OK)
+        return st;
+    // branch 3: the raw window only
+    hyb_problem p3 = *p;
+    p3.Nc = 0;
+    p3.topk = 0;
+    st = hyb_attn_fwd(&p3, q, nullptr, nullptr, nullptr, k_raw, v_raw, w8 + 2 * one, nullptr, stream);
+    if (st != HYB_OK)
+        return st;
+    return cuda_status(launch_gated_combine(w8, w8 + one, w8 + 2 * one, gate, o,
+                                            (long long)p->B * p->Lq * p->Hq, p->d, stream,
+                                            num_sms_current()));
 }
 
 hyb_status hyb_get_device_status(cudaStream_t stream)

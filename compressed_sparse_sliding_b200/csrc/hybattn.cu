@@ -7,5 +7,6 @@
 #include "attn_dense.cu"
 #include "attn_sparse.cu"
 #include "decode_append.cu"
+#include "gated.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -176,6 +176,24 @@ hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
  * [B] int32 out.  A negative t, or an entry j >= Nc, is skipped and flagged
  * as HYB_ERR_DEVICE_BOUNDS.  The rings start zeroed or filled by earlier
  * calls; rows of positions outside the window are never read. */
+/* The gated three-branch variant (Tiny-R2 README, "Attention Computation",
+ * "branch_gate"): three attentions with separate softmaxes, then
+ *   o[b,t,h] = sum_k softmax(gate[b,t,h,:])_k * o_k[b,t,h]
+ * with
+ *   o_1: every compressed block ending at or before t (all visible with W=0),
+ *   o_2: the blocks of idx among those (the selection made with W = 0),
+ *   o_3: the raw keys max(0, t-W+1) .. t;
+ * a branch with no key gives 0.  Inputs as hyb_attn_fwd (idx required);
+ * gate: [B, Lq, Hq, 3] fp32 logits (the output of the page's gate Linear,
+ * which is out of scope here); o: [B, Lq, Hq, d] bf16.  ws: device
+ * workspace of >= hyb_gated_workspace_size(p) bytes, 256-byte aligned (the
+ * three branch outputs, bf16). */
+size_t hyb_gated_workspace_size(const hyb_problem *p);
+hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                         const int32_t *idx, const void *k_raw, const void *v_raw,
+                         const float *gate, void *o, void *ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
 hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const void *k_new,
                              const void *v_new, const void *ki_new, const float *wk,
                              const float *wv, const float *wib, void *k_ring, void *v_ring,

@@ -255,6 +255,38 @@ def hybrid_attention(q_bits, kc_bits, vc_bits, idx, k_raw_bits, v_raw_bits, m: i
     return res
 
 
+def gated_attention(q_bits, kc_bits, vc_bits, idx, k_raw_bits, v_raw_bits, m: int, W: int,
+                    gate_logits, scale: Optional[float] = None, q_pos=None, kv_pos0=None, rows=None):
+    """The gated three-branch variant (Tiny-R2 README, "Attention Computation"
+    and "branch_gate"): three attentions with separate softmaxes, then a
+    softmax over the branches of per-(token, head) gate logits weights them.
+
+      branch 1, compressed: every compressed block that ends at or before t
+                (hybrid_attention with no selection and W = 0);
+      branch 2, selected:   the listed blocks among those (idx, W = 0);
+      branch 3, window:     the raw keys max(0, t-W+1) .. t (no compressed).
+    A branch with no key contributes 0.  gate_logits [B, Lq, Hq, 3] (fp32).
+    Returns dict(o [nrows, Hq, d], branches [3, nrows, Hq, d]).
+    """
+    kc_bits = _c(kc_bits, np.uint16)
+    B, Nc, Hkv, d = kc_bits.shape
+    none = np.zeros((B, 0, Hkv, d), dtype=np.uint16)
+    o1 = hybrid_attention(q_bits, kc_bits, vc_bits, None, k_raw_bits, v_raw_bits, m, 0, scale=scale,
+                          q_pos=q_pos, kv_pos0=kv_pos0, rows=rows)["o"]
+    o2 = hybrid_attention(q_bits, kc_bits, vc_bits, idx, k_raw_bits, v_raw_bits, m, 0, scale=scale,
+                          q_pos=q_pos, kv_pos0=kv_pos0, rows=rows)["o"]
+    o3 = hybrid_attention(q_bits, none, none, None, k_raw_bits, v_raw_bits, m, W, scale=scale,
+                          q_pos=q_pos, kv_pos0=kv_pos0, rows=rows)["o"]
+    g = np.asarray(gate_logits, dtype=np.float64)
+    Lq, Hq = g.shape[1], g.shape[2]
+    g = g.reshape(-1, Hq, 3)[_rows(rows, B * Lq)]
+    g = np.exp(g - g.max(axis=-1, keepdims=True))
+    g /= g.sum(axis=-1, keepdims=True)
+    br = np.stack([o1, o2, o3])
+    o = np.einsum("nhk,knhd->nhd", g, br)
+    return dict(o=o, branches=br)
+
+
 def forward(inp: dict, m: int, W: int, topk_k: int, rows=None, scale=None):
     """The whole forward pass for prefill inputs (see workloads.make_inputs).
 

@@ -27,7 +27,7 @@ def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
     assert {"hyb_hca_compress", "hyb_csa_index_topk", "hyb_attn_fwd", "hyb_fused_fwd",
             "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string",
-            "hyb_decode_append"} <= set(names)
+            "hyb_decode_append", "hyb_gated_fwd", "hyb_gated_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -76,3 +76,16 @@ def test_decode_append_argument_checks(lib):
     p = hb.problem(B=1, Lq=1, Lkv=16, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=16, topk=4, Hi=2, di=32)
     a = [buf] * 3 + [None] + [buf] * 11 + [None]
     assert hb._lib.hyb_decode_append(ctypes.byref(p), *a) == hb.HYB_ERR_INVALID_ARG
+
+
+def test_gated_argument_checks(lib):
+    import compressed_sparse_sliding_b200 as hb
+    buf = ctypes.c_void_p(256)
+    p = hb.problem(B=1, Lq=16, Lkv=16, Hq=4, Hkv=1, d=64, m=4, W=8, topk=4, Nc=4)
+    # the selection branch needs idx
+    assert hb._lib.hyb_gated_fwd(ctypes.byref(p), buf, buf, buf, None, buf, buf, buf, buf, buf,
+                                 1 << 20, None) == hb.HYB_ERR_INVALID_ARG
+    # workspace: three bf16 branch outputs, each 256-byte rounded
+    assert hb._lib.hyb_gated_workspace_size(ctypes.byref(p)) == 3 * ((16 * 4 * 64 * 2 + 255) // 256 * 256)
+    assert hb._lib.hyb_gated_fwd(ctypes.byref(p), buf, buf, buf, buf, buf, buf, buf, buf, None, 0,
+                                 None) == hb.HYB_ERR_WORKSPACE
