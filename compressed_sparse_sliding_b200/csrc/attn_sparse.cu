@@ -11,12 +11,15 @@
 // where NH is the group's head count padded to 16, 32 or 64.  No MMA row is
 // padding for the 32- and 64-head groups of the CSA workloads.
 //
-// Softmax: thread = key (TMEM lane), holding that key's NH scores.  A per-head
-// reference max lives in shared memory; it is moved (with a block-wide max
-// reduction, and a rescale of O^T and of the partial sums) only when some key
-// exceeds it by more than 2^8, i.e. on the first tile of a token and rarely
-// after.  Partial row sums stay per thread and are reduced once per token.
-// P^T is written to shared memory in the 32/64/128-byte swizzle matching NH.
+// Softmax: thread = key (TMEM lane).  For 32- and 64-head groups two
+// warpgroups share the keys and split the heads (TMEM columns), each thread
+// holding NH / 2 scores of its key; 16-head groups use one warpgroup.  A
+// per-head reference max lives in shared memory; it is moved (with a
+// block-wide max reduction, and a rescale of O^T and of the partial sums) only
+// when some key exceeds it by more than 2^8, i.e. on the first tile of a token
+// and rarely after.  Partial row sums stay per thread and are reduced once per
+// token.  P^T is written to shared memory in the 32/64/128-byte swizzle
+// matching NH.
 //
 // Gathers: four producer warps copy the selected compressed rows and the
 // window rows with 16-byte cp.async (16 lanes per 256-byte row, so every warp
@@ -24,19 +27,25 @@
 // layout; each thread then arms the stage's mbarrier with an asynchronous
 // arrive that fires when its copies land, so the producers never block on a
 // copy.  (Random 256-byte rows move through this path about nine times faster
-// than through TMA tile::gather4 on B200.)  The token's selection is decoded
-// once into a shared table of source rows (-1: unselected, invisible or out
-// of range; those slots are zero-filled and masked).
-// Roles: warps 0-3 softmax + epilogue, then four producer warps (two for
-// 64-head groups, whose softmax needs more registers), then one MMA warp;
-// work items (b, t, KV head) go round-robin to persistent CTAs.
+// than through TMA tile::gather4 on B200, and about three times faster than
+// through 256-byte bulk copies.)  K copies run one tile ahead of V copies.
+// The token's selection is decoded once into one of two shared tables of
+// source rows (-1: unselected, invisible or out of range; those slots are
+// zero-filled and masked); the softmax reads key validity from the same
+// table, published through its own mbarrier.
+// Roles: softmax warpgroup(s), then four producer warps (two for 64-head
+// groups, whose softmax needs more registers), then one MMA warp; work items
+// (b, t, KV head) go round-robin to persistent CTAs.  Every role agrees once
+// per item whether to go on, so a failed (bounded) wait never leaves a
+// thread waiting at a named barrier.
 #include "common.cuh"
 
 namespace hyb {
 
-constexpr int kSpBN = 128;     // keys per tile (the M of S^T)
-constexpr int kSpVS = 2;       // V ring depth
-constexpr int kSpD = 128;      // head dim handled by this kernel
+constexpr int kSpBN = 128;       // keys per tile (the M of S^T)
+constexpr int kSpSelBatch = 8;   // selection entries a producer thread loads at once
+constexpr int kSpLead = 1;       // tiles by which the K copies run ahead of the V copies
+constexpr int kSpD = 128;        // head dim handled by this kernel
 
 struct SparseParams {
     int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
@@ -54,24 +63,25 @@ struct SparseSmem {
     static constexpr int KV_BYTES = kSpBN * kSpD * 2;
     static constexpr int P_BYTES = kSpBN * NH * 2;
     static constexpr int P_STRIDE = (P_BYTES + 1023) & ~1023;
-    static constexpr int KS = NH == 64 ? 2 : 3;                    // K ring depth
+    static constexpr int KS = 2;                                   // K ring depth
+    static constexpr int VS = NH == 64 ? 2 : 3;                    // V ring depth
     static constexpr int OFF_Q = 0;                                // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + kSpVS * KV_BYTES;         // 2 buffers
+    static constexpr int OFF_P = OFF_V + VS * KV_BYTES;            // 2 buffers
     static constexpr int OFF_RED = OFF_P + 2 * P_STRIDE;           // [NH][4] floats
     static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;          // [2][NH] floats
     static constexpr int OFF_INV = OFF_MREF + 2 * NH * 4;          // [NH] floats
     static constexpr int OFF_BAR = OFF_INV + NH * 4;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
-    static constexpr int OFF_VAL = OFF_MISC + 16 * 4;               // [kSpVS][128] slot validity
-    static constexpr int OFF_IDX = OFF_VAL + kSpVS * kSpBN;         // producer's selection list
-    static constexpr int BASE_BYTES = OFF_IDX;                      // + topk * 4
+    static constexpr int OFF_IDX = OFF_MISC + 16 * 4;               // [2][topk] decoded selections
+    static constexpr int BASE_BYTES = OFF_IDX;                      // + 2 topk * 4
 };
 
+// mbarriers (two of each per-item or per-buffer kind, three per ring stage)
 enum {
-    SB_QF = 0, SB_QE = 2, SB_KF = 4, SB_KE = 7, SB_VF = 10, SB_VE = 12, SB_SF = 14, SB_PF = 16,
-    SB_OD = 18, SB_OE = 20, SB_DONE = 22
+    SB_QF = 0, SB_QE = 2, SB_KF = 4, SB_KE = 7, SB_VF = 10, SB_VE = 13, SB_SF = 16, SB_PF = 18,
+    SB_OD = 20, SB_OE = 22, SB_IF = 24, SB_DONE = 26, SB_COUNT = 27
 };
 
 struct SparseTok {
@@ -119,6 +129,22 @@ __device__ __forceinline__ void prod_sync()
     asm volatile("bar.sync 2, %0;" ::"n"(N) : "memory");
 }
 
+// AND of a predicate over the producer threads (named barrier 2).
+template <int N>
+__device__ __forceinline__ bool prod_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 2, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(N)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
 {
     asm volatile(
@@ -128,24 +154,42 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// OR-reduction of a predicate over the 128 softmax threads (named barrier 1).
+// OR-reduction of a predicate over the N softmax threads (named barrier 1).
+template <int N>
 __device__ __forceinline__ bool sm_any(bool v)
 {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "bar.red.or.pred p, 1, %2, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v)
+        : "r"((uint32_t)v), "n"(N)
         : "memory");
     return r != 0;
 }
 
+// AND of a predicate over the N softmax threads (named barrier 1).
+template <int N>
+__device__ __forceinline__ bool sm_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(N)
+        : "memory");
+    return r != 0;
+}
+
+template <int N>
 __device__ __forceinline__ void sm_sync()
 {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
 
 // Per-head totals over the 32 lanes of a warp by recursive halving: at each
@@ -252,8 +296,12 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float (&v)[N]
 // threads need up to 255 registers (8 warps in all).
 template <int NH>
 struct SpRoles {
-    static constexpr int PW = NH == 64 ? 2 : 4;
-    static constexpr int MMA_WARP = 4 + PW;
+    static constexpr int HS = NH >= 32 ? 2 : 1;       // softmax warpgroups (head halves)
+    static constexpr int NHW = NH / HS;               // heads per softmax thread
+    static constexpr int SMT = 128 * HS;              // softmax threads
+    static constexpr int PW = NH == 64 ? 2 : 4;       // producer warps
+    static constexpr int PROD_WARP0 = 4 * HS;
+    static constexpr int MMA_WARP = PROD_WARP0 + PW;
     static constexpr int THREADS = 32 * (MMA_WARP + 1);
 };
 
@@ -265,6 +313,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 {
     using SM = SparseSmem<NH>;
     constexpr int KS = SM::KS;
+    constexpr int VS = SM::VS;
     constexpr int RB = NH * 2;                                  // bytes of one P^T row
     constexpr uint32_t PLAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
     constexpr int PCH = RB / 16;                                // 16-byte chunks per row
@@ -281,27 +330,29 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     int *sIdx = reinterpret_cast<int *>(smem + SM::OFF_IDX);
-    uint8_t *sVal = smem + SM::OFF_VAL;
     volatile int *abort_flag = misc + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    constexpr int PW = SpRoles<NH>::PW;
+    constexpr int NPT = 32 * PW;                // producer threads
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[SB_QF + s], 1);
             mbar_init(&bar[SB_QE + s], 1);
             mbar_init(&bar[SB_SF + s], 1);
-            mbar_init(&bar[SB_OE + s], 128);
-            mbar_init(&bar[SB_PF + s], 128);
+            mbar_init(&bar[SB_OE + s], SpRoles<NH>::SMT);
+            mbar_init(&bar[SB_PF + s], SpRoles<NH>::SMT);
             mbar_init(&bar[SB_OD + s], 1);
+            mbar_init(&bar[SB_IF + s], NPT);
         }
         for (int s = 0; s < KS; ++s) {
-            mbar_init(&bar[SB_KF + s], 32 * SpRoles<NH>::PW);
+            mbar_init(&bar[SB_KF + s], NPT);
             mbar_init(&bar[SB_KE + s], 1);
         }
-        for (int s = 0; s < kSpVS; ++s) {
-            mbar_init(&bar[SB_VF + s], 32 * SpRoles<NH>::PW);
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(&bar[SB_VF + s], NPT);
             mbar_init(&bar[SB_VE + s], 1);
         }
         mbar_init(&bar[SB_DONE], 1);
@@ -319,26 +370,44 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // TMEM columns: S^T buffers at 0 and NH, O^T buffers at 2NH and 3NH
     const uint32_t TM_S0 = 0, TM_O0 = 2 * NH;
 
-    constexpr int PW = SpRoles<NH>::PW;
-    constexpr int NPT = 32 * PW;                // producer threads
     constexpr int RPI = NPT / 16;               // rows per copy round
     constexpr int CPT = kSpBN / RPI;            // copies per thread per tile and operand
     constexpr int MMA_WARP = SpRoles<NH>::MMA_WARP;
-    if (warp >= 4 && warp < MMA_WARP) {
+    if (warp >= SpRoles<NH>::PROD_WARP0 && warp < MMA_WARP) {
         // ================================ producer ================================
-        // 16 lanes per 256-byte row, two rows per warp instruction
-        const int pt = threadIdx.x - 128;
+        // 16 lanes per 256-byte row, two rows per warp instruction.  Within an
+        // item no thread leaves early: a failed wait clears `ok`, the copies
+        // go on (every source row stays in range), and the producers agree
+        // on `ok` once per item before its named barrier.
+        const int pt = threadIdx.x - 32 * SpRoles<NH>::PROD_WARP0;
         const int c8 = pt & 15;                 // 16-byte chunk of the row
         const int rsub = pt >> 4;               // rows rsub, rsub + RPI, ...
         const uint32_t dchunk = (uint32_t)(c8 >> 3) * kSpBN * 128;
         uint32_t kc = 0, vc = 0, nq = 0;
         bool ok = true;
-        for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+        // entries q0 + e NPT + pt of item w's selection (-1 past topk); item
+        // w = (b Lq + t) Hkv + KV head, and items number below 2^31
+        auto load_sel = [&](long long w, int q0, int (&jv)[kSpSelBatch]) {
+            const int32_t *irow = p.idx + (size_t)((uint32_t)w / (uint32_t)p.Hkv) * p.topk;
+#pragma unroll
+            for (int e = 0; e < kSpSelBatch; ++e) {
+                const int q = q0 + e * NPT + pt;
+                jv[e] = q < p.topk ? __ldg(irow + q) : -1;
+            }
+        };
+        int jnext[kSpSelBatch];
+        if (blockIdx.x < p.n_items)
+            load_sel(blockIdx.x, 0, jnext);
+        for (long long w = blockIdx.x; w < p.n_items; w += gridDim.x, ++nq) {
+            if (!prod_all<NPT>(ok && !*abort_flag))
+                break;
             const SparseTok k = sparse_tok(p, w);
             const int qb = nq & 1;
-            if (nq >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_QE + qb], ((nq >> 1) - 1) & 1, abort_flag))) {
-                ok = false;
-                break;
+            if (nq >= 2) {
+                // Q buffer qb: the last scores of item nq - 2 are done;
+                // selection buffer qb: so is that item's softmax
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_QE + qb], ((nq >> 1) - 1) & 1, abort_flag));
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OE + qb], ((nq >> 1) - 1) & 1, abort_flag));
             }
             if (pt == 0) {
                 mbar_arrive_expect_tx(&bar[SB_QF + qb], SM::Q_BYTES);
@@ -347,82 +416,109 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tma_load_2d(sQ + qb * SM::Q_BYTES + cb * NH * 128, &tm_q, &bar[SB_QF + qb], cb * 64,
                                 qrow);
             }
-            // decode the token's selection once: source row of every slot, or -1
-            prod_sync<NPT>();
+            // decode the item's selection once into buffer qb: source row of
+            // every slot, or -1 (unselected, invisible or out of range).  A
+            // batch's loads are all in flight together; the first batch was
+            // loaded during the previous item's copies.
+            int *sSel = sIdx + qb * p.topk;
             {
-                const int32_t *irow = p.idx + ((size_t)k.b * p.Lq + k.t) * p.topk;
                 const long long wstart = k.pos - p.W + 1;
-                for (int q = pt; q < p.topk; q += NPT) {
-                    const int j = __ldg(irow + q);
-                    if (j >= p.Nc)
-                        set_error(HYB_ERR_DEVICE_BOUNDS);
-                    const bool v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < wstart);
-                    sIdx[q] = v ? (k.b * p.Nc + j) * p.Hkv + k.kvh : -1;
-                }
-            }
-            prod_sync<NPT>();
-            const int nt = k.nct + k.nrt;
-            for (int i = 0; i < nt && ok; ++i) {
-                const bool comp = i < k.nct;
-                const __nv_bfloat16 *bk = comp ? p.kc : p.kr;
-                const __nv_bfloat16 *bv = comp ? p.vc : p.vr;
-                int src[CPT];
+#pragma unroll 1
+                for (int q0 = 0; q0 < p.topk; q0 += kSpSelBatch * NPT) {
+                    int jv[kSpSelBatch];
+                    if (q0 == 0) {
 #pragma unroll
-                for (int u = 0; u < CPT; ++u) {
-                    const int r = u * RPI + rsub;
-                    if (comp) {
-                        const int sidx = i * kSpBN + r;
-                        src[u] = sidx < p.topk ? sIdx[sidx] : -1;
+                        for (int e = 0; e < kSpSelBatch; ++e)
+                            jv[e] = jnext[e];
                     } else {
-                        const int rr = k.rlo + (i - k.nct) * kSpBN + r;
-                        src[u] = rr <= k.rhi ? (k.b * p.Lkv + rr) * p.Hkv + k.kvh : -1;
+                        load_sel(w, q0, jv);
+                    }
+#pragma unroll
+                    for (int e = 0; e < kSpSelBatch; ++e) {
+                        const int q = q0 + e * NPT + pt;
+                        if (q < p.topk) {
+                            const int j = jv[e];
+                            if (j >= p.Nc)
+                                set_error(HYB_ERR_DEVICE_BOUNDS);
+                            const bool v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < wstart);
+                            sSel[q] = v ? (k.b * p.Nc + j) * p.Hkv + k.kvh : -1;
+                        }
                     }
                 }
-                const uint32_t ks = kc % KS;
-                if (kc >= KS &&
-                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_KE + ks], ((kc / KS) - 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
+            }
+            mbar_arrive(&bar[SB_IF + qb]);      // the softmax reads key validity from it
+            prod_sync<NPT>();
+            // the next item's first batch, in flight during this item's copies
+            // (issued after the barrier, which would otherwise wait for it)
+            if (w + gridDim.x < p.n_items)
+                load_sel(w + gridDim.x, 0, jnext);
+            const int nt = k.nct + k.nrt;
+            // source row of copy u of tile i, or -1 (zero-filled)
+            auto src_of = [&](int i, int u) -> int {
+                const int r = u * RPI + rsub;
+                if (i < k.nct) {
+                    const int sidx = i * kSpBN + r;
+                    return sidx < p.topk ? sSel[sidx] : -1;
                 }
-                {
+                const int rr = k.rlo + (i - k.nct) * kSpBN + r;
+                return rr <= k.rhi ? (k.b * p.Lkv + rr) * p.Hkv + k.kvh : -1;
+            };
+            // K of tile i goes out kSpLead tiles ahead of V of the same tile, so
+            // that the next scores need not queue behind a V stage that a PV
+            // still holds.  A tile's source rows are read into registers
+            // before its copies (each copy is a compiler barrier).
+            int srcv[CPT];
+            for (int i = 0; i < nt + kSpLead; ++i) {
+                int srck[CPT];
+                if (i < nt) {
+#pragma unroll
+                    for (int u = 0; u < CPT; ++u)
+                        srck[u] = src_of(i, u);
+                    const __nv_bfloat16 *bk = i < k.nct ? p.kc : p.kr;
+                    const uint32_t ks = kc % KS;
+                    if (kc >= KS)
+                        ok &= __all_sync(0xffffffffu,
+                                         mbar_wait(&bar[SB_KE + ks], ((kc / KS) - 1) & 1, abort_flag));
                     const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
 #pragma unroll
                     for (int u = 0; u < CPT; ++u) {
                         const int r = u * RPI + rsub;
-                        const bool v = src[u] >= 0;
+                        const int sr = srck[u];
                         cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                    bk + (size_t)(v ? src[u] : 0) * kSpD + c8 * 8, v ? 16u : 0u);
+                                    bk + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
                     }
                     cp_async_mbar_arrive(&bar[SB_KF + ks]);
                     mbar_arrive(&bar[SB_KF + ks]);
+                    ++kc;
                 }
-                ++kc;
-                const uint32_t vs = vc % kSpVS;
-                if (vc >= kSpVS &&
-                    !__all_sync(0xffffffffu, mbar_wait(&bar[SB_VE + vs], ((vc / kSpVS) - 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                if (c8 == 0) {
-                    // which slots are real keys, published with the V stage (the
-                    // softmax reads them after waiting on it)
+                if (kSpLead == 0) {
 #pragma unroll
                     for (int u = 0; u < CPT; ++u)
-                        sVal[vs * kSpBN + u * RPI + rsub] = src[u] >= 0 ? 1 : 0;
+                        srcv[u] = srck[u];
                 }
-                {
+                if (i >= kSpLead) {
+                    const __nv_bfloat16 *bv = i - kSpLead < k.nct ? p.vc : p.vr;
+                    const uint32_t vs = vc % VS;
+                    if (vc >= VS)
+                        ok &= __all_sync(0xffffffffu,
+                                         mbar_wait(&bar[SB_VE + vs], ((vc / VS) - 1) & 1, abort_flag));
                     const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
 #pragma unroll
                     for (int u = 0; u < CPT; ++u) {
                         const int r = u * RPI + rsub;
-                        const bool v = src[u] >= 0;
+                        const int sr = srcv[u];
                         cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                    bv + (size_t)(v ? src[u] : 0) * kSpD + c8 * 8, v ? 16u : 0u);
+                                    bv + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
                     }
                     cp_async_mbar_arrive(&bar[SB_VF + vs]);
                     mbar_arrive(&bar[SB_VF + vs]);
+                    ++vc;
                 }
-                ++vc;
+                if (kSpLead == 1) {
+#pragma unroll
+                    for (int u = 0; u < CPT; ++u)
+                        srcv[u] = srck[u];
+                }
             }
         }
         // unwinding: every copy issued by this thread has landed
@@ -448,10 +544,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     break;
                 }
                 auto issue_pv = [&](bool first) -> bool {
-                    const uint32_t vs = vc % kSpVS;
+                    const uint32_t vs = vc % VS;
                     const uint32_t pb = pcnt & 1;
                     if (!mbar_wait(&bar[SB_PF + pb], (pcnt >> 1) & 1, abort_flag) ||
-                        !mbar_wait(&bar[SB_VF + vs], (vc / kSpVS) & 1, abort_flag))
+                        !mbar_wait(&bar[SB_VF + vs], (vc / VS) & 1, abort_flag))
                         return false;
                     if (first && nq >= 2 &&
                         !mbar_wait(&bar[SB_OE + ob], ((nq >> 1) - 1) & 1, abort_flag))
@@ -511,11 +607,18 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ========================== softmax + epilogue ==========================
+        // HS warpgroups share the tile's keys (TMEM lanes) and split its heads
+        // (TMEM columns): warpgroup x owns heads x NHW .. x NHW + NHW - 1.
         // The reference maxima live in shared memory in two buffers, sMref[mb]
         // current; a move writes the other buffer and flips mb after a barrier,
-        // so readers of the old values never race the writers.
-        using HD = SpHeads<NH>;
-        const int quad = warp;                       // warps 0-3
+        // so readers of the old values never race the writers.  The softmax
+        // threads agree once per item whether to go on; within an item every
+        // thread takes the same named barriers (a failed wait clears `ok`).
+        constexpr int NHW = SpRoles<NH>::NHW;
+        constexpr int SMT = SpRoles<NH>::SMT;
+        using HD = SpHeads<NHW>;
+        const int hb = (warp >> 2) * NHW;            // first head of this warpgroup
+        const int quad = warp & 3;
         const int r = quad * 32 + lane;              // key lane (S^T) / d lane (O^T)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const bool head_owner = (lane % HD::LPH) == 0;
@@ -523,106 +626,109 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         const uint32_t prow = smem_u32(sP) + r * RB;
         const float4 *red4 = reinterpret_cast<const float4 *>(sRed);
-        for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+        for (long long w = blockIdx.x; w < p.n_items; w += gridDim.x, ++nq) {
+            if (!sm_all<SMT>(ok && !*abort_flag))
+                break;
             const SparseTok k = sparse_tok(p, w);
             const int nt = k.nct + k.nrt;
             const int ob = nq & 1;
-            float lpart[NH];
+            // the item's decoded selection (key validity of its compressed tiles)
+            const int *sSel = sIdx + ob * p.topk;
+            ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_IF + ob], (nq >> 1) & 1, abort_flag));
+            float lpart[NHW];
 #pragma unroll
-            for (int h = 0; h < NH; ++h)
+            for (int h = 0; h < NHW; ++h)
                 lpart[h] = 0.f;
             // No global memory access inside this loop: a CTA barrier (the
             // votes below) waits for every outstanding access of its threads.
             for (int i = 0; i < nt; ++i, ++gt) {
-                const int vs = gt % kSpVS;
                 const uint32_t sb = gt & 1;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag) &&
-                                                 mbar_wait(&bar[SB_VF + vs], (gt / kSpVS) & 1, abort_flag))) {
-                    ok = false;
-                    break;
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag));
+                bool valid;
+                if (i < k.nct) {
+                    const int slot = i * kSpBN + r;
+                    valid = slot < p.topk && sSel[slot] >= 0;
+                } else {
+                    valid = k.rlo + (i - k.nct) * kSpBN + r <= k.rhi;
                 }
-                const bool valid = sVal[vs * kSpBN + r] != 0;
                 tc_fence_after();
-                float s[NH];
-                tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, s);
+                float s[NHW];
+                tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
                 tmem_ld_wait();
 #pragma unroll
-                for (int h = 0; h < NH; ++h)
+                for (int h = 0; h < NHW; ++h)
                     s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
-                bool need = i == 0;   // the first tile of a token always sets the reference
+                bool need = i == 0;   // the first tile of an item always sets the reference
                 if (!need) {
-                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH);
+                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH + hb);
                     bool exceed = false;
 #pragma unroll
-                    for (int h = 0; h < NH; h += 4) {
+                    for (int h = 0; h < NHW; h += 4) {
                         const float4 mr = m4[h >> 2];
                         exceed |= (s[h] > mr.x + 8.f) | (s[h + 1] > mr.y + 8.f) | (s[h + 2] > mr.z + 8.f) |
                                   (s[h + 3] > mr.w + 8.f);
                     }
-                    need = sm_any(exceed);
+                    need = sm_any<SMT>(exceed);
                 }
                 if (need) {
                     // per-head max over the tile: warp halving, then the four
-                    // warps' values through sRed [head][warp]
-                    warp_reduce_heads<NH, true>(s, lane);
+                    // quadrants' values through sRed [head][quadrant]
+                    warp_reduce_heads<NHW, true>(s, lane);
                     if (head_owner) {
 #pragma unroll
                         for (int e = 0; e < HD::VPL; ++e)
-                            sRed[HD::head(lane, e) * 4 + quad] = s[e];
+                            sRed[(hb + HD::head(lane, e)) * 4 + quad] = s[e];
                     }
-                    sm_sync();
+                    sm_sync<SMT>();
                     const float *mold = sMref + mb * NH;
                     bool moved = false;
                     if (i > 0) {
 #pragma unroll
-                        for (int h = 0; h < NH; ++h) {
-                            const float old = mold[h];
-                            const float a = sp_factor(old, sp_new_ref(red4[h], old));
+                        for (int h = 0; h < NHW; ++h) {
+                            const float old = mold[hb + h];
+                            const float a = sp_factor(old, sp_new_ref(red4[hb + h], old));
                             moved |= a != 1.f;
                             lpart[h] *= a;
                         }
                     }
                     if (moved) {
-                        // O^T holds every earlier PV of this token: wait for the
-                        // last one, then scale column h by its factor
-                        if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)],
-                                                               ((gt - 1) >> 1) & 1, abort_flag))) {
-                            ok = false;
-                            break;
-                        }
+                        // O^T holds every earlier PV of this item: wait for the
+                        // last one, then scale this warpgroup's columns
+                        ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)],
+                                                                ((gt - 1) >> 1) & 1, abort_flag));
                         tc_fence_after();
 #pragma unroll 1
-                        for (int c = 0; c < NH; c += 16) {
+                        for (int c = 0; c < NHW; c += 16) {
                             float ov[16];
-                            tmem_ld_cols<16>(tl + TM_O0 + ob * NH + c, ov);
+                            tmem_ld_cols<16>(tl + TM_O0 + ob * NH + hb + c, ov);
                             tmem_ld_wait();
 #pragma unroll
                             for (int q = 0; q < 16; ++q) {
-                                const float old = mold[c + q];
-                                ov[q] *= sp_factor(old, sp_new_ref(red4[c + q], old));
+                                const float old = mold[hb + c + q];
+                                ov[q] *= sp_factor(old, sp_new_ref(red4[hb + c + q], old));
                             }
-                            tmem_st_cols<16>(tl + TM_O0 + ob * NH + c, ov);
+                            tmem_st_cols<16>(tl + TM_O0 + ob * NH + hb + c, ov);
                         }
                         tmem_st_wait();
                     }
                     if (threadIdx.x < NH)
                         sMref[(mb ^ 1) * NH + threadIdx.x] =
                             sp_new_ref(red4[threadIdx.x], mold[threadIdx.x]);
-                    sm_sync();
+                    sm_sync<SMT>();
                     mb ^= 1;
                     // the halving consumed the scores: load them again
-                    tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, s);
+                    tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int h = 0; h < NH; ++h)
+                    for (int h = 0; h < NHW; ++h)
                         s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
                 }
                 // P^T row of this key: exp2(s - mref), 0 for masked keys
-                uint32_t pk[NH / 2];
+                uint32_t pk[NHW / 2];
                 {
-                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH);
+                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH + hb);
 #pragma unroll
-                    for (int h = 0; h < NH; h += 4) {
+                    for (int h = 0; h < NHW; h += 4) {
                         const float4 mr = m4[h >> 2];
                         const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
                         float e[4];
@@ -636,14 +742,12 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 // P^T buffer sb is free once the PV of tile gt - 2 completed
-                if (gt >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1,
-                                                                  abort_flag))) {
-                    ok = false;
-                    break;
-                }
+                if (gt >= 2)
+                    ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1, abort_flag));
                 const uint32_t prow_b = prow + sb * SM::P_STRIDE;
 #pragma unroll
-                for (int c = 0; c < PCH; ++c) {
+                for (int cl = 0; cl < NHW / 8; ++cl) {
+                    const int c = hb / 8 + cl;               // 16-byte chunk of the row
                     uint32_t phys;
                     if (RB == 128)
                         phys = c ^ (r & 7);
@@ -652,65 +756,64 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     else
                         phys = c ^ ((r >> 2) & 1);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_b + phys * 16),
-                                 "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                                 "r"(pk[4 * cl]), "r"(pk[4 * cl + 1]), "r"(pk[4 * cl + 2]), "r"(pk[4 * cl + 3])
                                  : "memory");
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
             }
-            if (!ok)
-                break;
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
-            warp_reduce_heads<NH, false>(lpart, lane);
+            warp_reduce_heads<NHW, false>(lpart, lane);
             if (head_owner) {
 #pragma unroll
                 for (int e = 0; e < HD::VPL; ++e)
-                    sRed[HD::head(lane, e) * 4 + quad] = lpart[e];
+                    sRed[(hb + HD::head(lane, e)) * 4 + quad] = lpart[e];
             }
             const bool have_o = nt > 0;
             if (have_o) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1,
-                                                       abort_flag))) {
-                    ok = false;
-                    break;
-                }
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1,
+                                                        abort_flag));
                 tc_fence_after();
             }
-            sm_sync();
+            sm_sync<SMT>();
+            // thread h < NH (all in the first warpgroup) finishes head h
+            const int th = threadIdx.x;
             float lse_v = -INFINITY;
-            if (r < NH) {
-                const float4 q4 = red4[r];
+            if (th < NH) {
+                const float4 q4 = red4[th];
                 const float l = (q4.x + q4.y) + (q4.z + q4.w);
-                sInv[r] = l > 0.f ? 1.f / l : 0.f;
-                lse_v = l > 0.f ? (sMref[mb * NH + r] + log2f(l)) * 0.6931471805599453f : -INFINITY;
-                sMref[(mb ^ 1) * NH + r] = -INFINITY;   // the next token's reference
+                sInv[th] = l > 0.f ? 1.f / l : 0.f;
+                lse_v = l > 0.f ? (sMref[mb * NH + th] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                sMref[(mb ^ 1) * NH + th] = -INFINITY;   // the next item's reference
             }
-            sm_sync();  // sRed / sMref read, sInv written, next reference cleared
+            sm_sync<SMT>();  // sRed / sMref read, sInv written, next reference cleared
             mb ^= 1;
-            float ov[NH];
+            float ov[NHW];
             if (have_o) {
-                tmem_ld_cols<NH>(tl + TM_O0 + ob * NH, ov);
+                tmem_ld_cols<NHW>(tl + TM_O0 + ob * NH + hb, ov);
                 tmem_ld_wait();
             } else {
 #pragma unroll
-                for (int h = 0; h < NH; ++h)
+                for (int h = 0; h < NHW; ++h)
                     ov[h] = 0.f;
             }
-            // global stores only after the last barrier of the token
-            const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
-            const float4 *inv4 = reinterpret_cast<const float4 *>(sInv);
+            // global stores only after the last barrier of the item
+            if (ok) {
+                const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+                const float4 *inv4 = reinterpret_cast<const float4 *>(sInv + hb);
 #pragma unroll
-            for (int h = 0; h < NH; h += 4) {
-                const float4 iv = inv4[h >> 2];
-                const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
+                for (int h = 0; h < NHW; h += 4) {
+                    const float4 iv = inv4[h >> 2];
+                    const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (h + q < p.g)
-                        p.o[obase + (size_t)(h + q) * kSpD + r] = __float2bfloat16_rn(ov[h + q] * ivs[q]);
+                    for (int q = 0; q < 4; ++q)
+                        if (hb + h + q < p.g)
+                            p.o[obase + (size_t)(hb + h + q) * kSpD + r] = __float2bfloat16_rn(ov[h + q] * ivs[q]);
+                }
+                if (p.lse && th < p.g)
+                    p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + th) * p.Lq + k.t] = lse_v;
             }
-            if (p.lse && r < p.g)
-                p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + r) * p.Lq + k.t] = lse_v;
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
         }
@@ -753,7 +856,7 @@ static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void
     ok &= make_map_2d(&mvr, vr, (long long)p.B * p.Lkv * p.Hkv, 1);
     if (!ok)
         return cudaErrorInvalidValue;
-    size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.topk * 4;
+    size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.topk * 8;
     auto kern = csa_attn_kernel<NH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
@@ -792,6 +895,8 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
     p.topk = topk;
     p.NH = p.g <= 16 ? 16 : (p.g <= 32 ? 32 : 64);
     p.n_items = (long long)B * Lq * Hkv;
+    if (p.n_items >= (1ll << 31))
+        return cudaErrorInvalidValue;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.q_pos = q_pos;
     p.kv_pos0 = kv_pos0;
