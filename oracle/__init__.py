@@ -20,6 +20,12 @@ Parity status per function (what pins it, in tests/test_oracle_*.py):
   hybrid_attention  brute-force masked attention (brute.py), torch SDPA for
                     m=1/W=0, K >= n_vis equals dense, softmax rows sum to 1,
                     label-counting pins for the key sets, window-count pin
+  decode_append     ring rows and emitted entries against block_merge of the
+                    same positions, kv_pos0 closed form
+  gated_attention   one-hot gates give one branch (brute-force masks per
+                    branch), the output is the gate-weighted combination
+  fp4_quantize /    exact levels, ties to even, constant rows, nibble order,
+  fp4_dequantize    the half-step error bound, nearest level by brute force
 """
 from __future__ import annotations
 
@@ -169,6 +175,55 @@ def decode_append(state: dict, t_new, k_new_bits, v_new_bits, wk, wv, m: int, W:
                 _, out_b = block_merge(x, w, m)
                 state[cache][b, j] = out_b.reshape(state[cache][b, j].shape)
     return kv_pos0
+
+
+def fp4_quantize(x_bits):
+    """4-bit min/max affine quantization of every row (the last axis) of a bf16
+    tensor, as the "FP4" cache storage of the DeepSeek-V4 CSDN article
+    ("compress_to_fp4"): scale = (max - min) / 15, code = round((x - min) /
+    scale) clamped to 0..15.
+
+    Readings: min and max are taken per row (one compressed entry of one
+    head), so that a cache can grow one entry at a time; round is to nearest,
+    ties to even (torch.round); a row with max == min gets scale 0 and codes 0.
+    The arithmetic that decides a code is fp32, one IEEE operation at a time.
+    Codes are packed two per byte, element 2i in the low nibble of byte i.
+
+    Returns (codes uint8 [..., dx / 2], qp float32 [..., 2] = (min, scale)).
+    """
+    bits = np.asarray(x_bits, dtype=np.uint16)
+    if bits.shape[-1] % 2:
+        raise ValueError("rows must have an even number of elements")
+    x = (bits.astype(np.uint32) << 16).view(np.float32)
+    mn = x.min(axis=-1)
+    mx = x.max(axis=-1)
+    scale = np.float32(mx - mn) / np.float32(15.0)
+    scale = np.asarray(scale, dtype=np.float32)
+    q = np.zeros(x.shape, dtype=np.float32)
+    pos = scale > 0
+    if np.any(pos):
+        diff = (x - mn[..., None]).astype(np.float32)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = (diff / np.where(pos, scale, np.float32(1.0))[..., None]).astype(np.float32)
+        q = np.where(pos[..., None], np.rint(ratio), np.float32(0.0))
+    q = np.clip(q, 0, 15).astype(np.uint8)
+    codes = (q[..., 0::2] | (q[..., 1::2] << 4)).astype(np.uint8)
+    qp = np.stack([mn, scale], axis=-1).astype(np.float32)
+    return codes, qp
+
+
+def fp4_dequantize(codes, qp):
+    """Inverse of fp4_quantize ("decompress_from_fp4"): code * scale + min,
+    the product and the sum each rounded to fp32, the result rounded to bf16
+    (nearest, ties to even).  Returns bf16 bits [..., 2 * codes.shape[-1]]."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    qp = np.asarray(qp, dtype=np.float32)
+    q = np.empty(codes.shape[:-1] + (2 * codes.shape[-1],), dtype=np.float32)
+    q[..., 0::2] = codes & 15
+    q[..., 1::2] = codes >> 4
+    prod = (q * qp[..., 1:2]).astype(np.float32)
+    v = (prod + qp[..., 0:1]).astype(np.float32)
+    return round_bf16(v.astype(np.float64))
 
 
 def _rows(rows: Optional[Sequence[int]], total: int) -> np.ndarray:
