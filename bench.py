@@ -62,10 +62,12 @@ def n_visible(t, m, W, Nc):
     return 0 if a <= 0 else min(a // m, Nc)
 
 
-def algorithmic_counts(w, gated=False):
+def algorithmic_counts(w, gated=False, fp4=False):
     """Per step: attention keys and FLOP, indexer FLOP, unique bytes per stage.
     gated: the three-branch variant (all blocks ending at or before t, the
-    selected ones among them, the window; the selection sees the same blocks)."""
+    selected ones among them, the window; the selection sees the same blocks).
+    fp4: decode over 4-bit compressed caches (a row of dx channels is dx/2
+    bytes of codes and 8 bytes of (min, scale))."""
     if gated:
         t = np.arange(w.L, dtype=np.int64)
         nv0 = np.minimum((t + 1) // w.m, w.Nc)
@@ -102,9 +104,12 @@ def algorithmic_counts(w, gated=False):
     q_o = 2 * B * Lq * Hq * d * bf
     if w.is_decode:
         # unique bytes: q/o, the selected compressed rows, the raw window rows, the indexer keys
-        attn_bytes = q_o + (w.B * keys_per_tok) * Hkv * d * bf * 2 + w.B * w.topk * 4
+        row_c = (d // 2 + 8) if fp4 else d * bf             # one compressed K or V row
+        row_i = (w.di // 2 + 8) if fp4 else w.di * bf       # one compressed indexer key
+        win = min(w.W, t + 1)
+        attn_bytes = q_o + w.B * (sel * row_c + win * d * bf) * Hkv * 2 + w.B * w.topk * 4
         compress_bytes = 0
-        idx_bytes = B * nv * w.di * bf + B * w.Hi * w.di * bf + B * w.topk * 4
+        idx_bytes = B * nv * row_i + B * w.Hi * w.di * bf + B * w.topk * 4
     else:
         attn_bytes = q_o + 2 * B * w.L * Hkv * d * bf + 2 * B * Nc * Hkv * d * bf
         if w.topk:
@@ -134,13 +139,20 @@ class Step:
     """One forward pass as the three C-ABI stages on one stream, with CUDA
     events between the stages (the same kernels hyb_fused_fwd launches)."""
 
-    def __init__(self, hb, w, inp, gated=False):
-        self.hb, self.w, self.inp, self.gated = hb, w, inp, gated
+    def __init__(self, hb, w, inp, gated=False, fp4=False):
+        self.hb, self.w, self.inp, self.gated, self.fp4 = hb, w, inp, gated, fp4
         dev = inp["q"].device
         self.kv0 = torch.empty((w.B,), dtype=torch.int32, device=dev)
         self.p = problem_for(hb, w, inp, self.kv0)
         if w.is_decode:
             self.kc, self.vc, self.kic = inp["kc"], inp["vc"], inp["kic"]
+            if fp4:
+                # the caches as stored in 4 bits (quantized once, before timing)
+                self.kq = hb.hyb_fp4_quantize(self.kc)
+                self.vq = hb.hyb_fp4_quantize(self.vc)
+                self.kiq = hb.hyb_fp4_quantize(self.kic)
+                self.fws = torch.empty(max(hb.hyb_fp4_workspace_size(self.p), 256), dtype=torch.uint8,
+                                       device=dev)
         else:
             self.kc = torch.empty((w.B, w.Nc, w.Hkv, w.d), dtype=torch.bfloat16, device=dev)
             self.vc = torch.empty_like(self.kc)
@@ -164,7 +176,13 @@ class Step:
         hb, w, inp, ev = self.hb, self.w, self.inp, self.ev
         launches = 0
         ev[0].record(stream)
-        if w.is_decode:
+        if w.is_decode and self.fp4:
+            hb.hyb_decode_append_fp4(self.p, inp["t_new"], inp["k_new"], inp["v_new"], inp["k_ring"],
+                                     inp["v_ring"], self.kq, self.vq, inp["wk"], inp["wv"],
+                                     ki_new=inp["ki_new"], wib=inp["wib"], ki_ring=inp["ki_ring"],
+                                     kic=self.kiq, kv_pos0=self.kv0, stream=stream)
+            launches += 1
+        elif w.is_decode:
             # cache maintenance of the new token: window ring + the closed block
             hb.hyb_decode_append(self.p, inp["t_new"], inp["k_new"], inp["v_new"], inp["k_ring"],
                                  inp["v_ring"], self.kc, self.vc, inp["wk"], inp["wv"],
@@ -179,12 +197,20 @@ class Step:
                 hb.hyb_hca_compress(inp["ki"], inp["wib"], w.m, out=self.kic, stream=stream)
                 launches += 1
         ev[1].record(stream)
-        if w.topk:
+        if self.fp4:
+            hb.hyb_csa_index_topk_fp4(self.p, inp["qi"], inp["wi"], self.kiq, idx=self.idx, ws=self.fws,
+                                      stream=stream)
+            launches += 2
+        elif w.topk:
             hb.hyb_csa_index_topk(self.p_sel if self.gated else self.p, inp["qi"], inp["wi"], self.kic,
                                   idx=self.idx, ws=self.ws, stream=stream)
             launches += 2
         ev[2].record(stream)
-        if self.gated:
+        if self.fp4:
+            hb.hyb_attn_fwd_fp4(self.p, inp["q"], self.kq, self.vq, self.idx, inp["k_ring"], inp["v_ring"],
+                                o=self.o, ws=self.fws, stream=stream)
+            launches += 2
+        elif self.gated:
             hb.hyb_gated_fwd(self.p, inp["q"], self.kc, self.vc, self.idx, inp["k"], inp["v"],
                              inp["gate"], o=self.o, ws=self.gws, stream=stream)
             launches += 4
@@ -336,10 +362,11 @@ def run_gpu(args, rank, world):
     if not w.is_decode:
         inp["k_raw"], inp["v_raw"] = inp["k"], inp["v"]
     gated = args.variant == "gated"
+    fp4 = args.variant == "fp4"
     if gated:
         inp["gate"] = gate_logits(w, dev, rank)
     stream = torch.cuda.current_stream()
-    step = Step(hb, w, inp, gated)
+    step = Step(hb, w, inp, gated, fp4)
     # L2 flush: write 256 MiB, then read another 256 MiB so that no dirty line
     # of the flush buffer is left for the timed step to write back
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -349,7 +376,7 @@ def run_gpu(args, rank, world):
         flush.fill_(1)
         flush_rd.sum()
 
-    counts = algorithmic_counts(w, gated)
+    counts = algorithmic_counts(w, gated, fp4)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -427,6 +454,19 @@ def run_gpu(args, rank, world):
                              dev_in["gate"], o=step.o, ws=step.gws, stream=stream)
             o_host.copy_(step.o, non_blocking=True)
             return
+        if fp4:
+            # the public calls over the 4-bit caches
+            hb.hyb_decode_append_fp4(p, dev_in["t_new"], dev_in["k_new"], dev_in["v_new"],
+                                     dev_in["k_ring"], dev_in["v_ring"], step.kq, step.vq, dev_in["wk"],
+                                     dev_in["wv"], ki_new=dev_in["ki_new"], wib=dev_in["wib"],
+                                     ki_ring=dev_in["ki_ring"], kic=step.kiq, kv_pos0=kv0_e2e,
+                                     stream=stream)
+            hb.hyb_csa_index_topk_fp4(p, dev_in["qi"], dev_in["wi"], step.kiq, idx=step.idx, ws=step.fws,
+                                      stream=stream)
+            hb.hyb_attn_fwd_fp4(p, dev_in["q"], step.kq, step.vq, step.idx, dev_in["k_ring"],
+                                dev_in["v_ring"], o=step.o, ws=step.fws, stream=stream)
+            o_host.copy_(step.o, non_blocking=True)
+            return
         if w.is_decode:
             hb.hyb_decode_append(p, dev_in["t_new"], dev_in["k_new"], dev_in["v_new"],
                                  dev_in["k_ring"], dev_in["v_ring"], dev_in["kc"], dev_in["vc"],
@@ -477,6 +517,8 @@ def run_gpu(args, rank, world):
     kname, ksrc = attention_kernel(w)
     if gated:
         kname = "hyb_gated_fwd (three attention kernels + combine)"
+    if fp4:
+        kname = "hyb_attn_fwd_fp4 (fp4_gather_kernel + csa_attn_kernel)"
     roof["kernel"] = kname
     roof["peak_source"] = peaks["source"]
     roof["traffic"] = kernel_traffic(kname, w.no)
@@ -510,14 +552,19 @@ def run_gpu(args, rank, world):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False):
+def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False, fp4=False):
     """Times the oracle on a bounded sample of the workload.  Compression of
     the whole batch is timed once and charged per query token; indexer, top-K
-    and attention are timed on a sample of query rows."""
+    and attention are timed on a sample of query rows.  fp4: the decode caches
+    are the 4-bit round trip of the inputs (the stored form, made before
+    timing)."""
     import oracle
     inp = make_inputs(w, device="cpu")
     cores = os.cpu_count()
     bits = {k: oracle.bf16_bits(v) for k, v in inp.items() if v.dtype == torch.bfloat16}
+    if fp4:
+        for n in ("kc", "vc", "kic"):
+            bits[n] = oracle.fp4_dequantize(*oracle.fp4_quantize(bits[n]))
     t0 = time.perf_counter()
     kv0_ring = None
     if w.is_decode:
@@ -584,10 +631,11 @@ def run_reference_arm(args):
     per_step = []
     base = None
     gated = args.variant == "gated"
+    fp4 = args.variant == "fp4"
     for _ in range(args.warmup):
-        run_oracle(w, budget_s=2.0, rows_hint=4, gated=gated)
+        run_oracle(w, budget_s=2.0, rows_hint=4, gated=gated, fp4=fp4)
     for _ in range(args.steps):
-        base = run_oracle(w, budget_s=6.0, rows_hint=8, gated=gated)
+        base = run_oracle(w, budget_s=6.0, rows_hint=8, gated=gated, fp4=fp4)
         per_step.append(1.0 / base["value"])
     value = 1.0 / statistics.mean(per_step)
     cpu = dict(base)
@@ -614,12 +662,15 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated"],
-                    help="gated: the three-branch variant (CSA workloads with prefill)")
+    ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated", "fp4"],
+                    help="gated: the three-branch variant (CSA workloads with prefill); "
+                         "fp4: decode over 4-bit compressed caches (config 5)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.variant == "gated" and (not WORKLOADS[args.config].topk or WORKLOADS[args.config].is_decode):
         ap.error("--variant gated needs a CSA prefill workload (configs 1 and 3)")
+    if args.variant == "fp4" and not WORKLOADS[args.config].is_decode:
+        ap.error("--variant fp4 needs the decode workload (config 5)")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -639,7 +690,8 @@ def main():
     try:
         res = run_gpu(args, rank, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config], gated=args.variant == "gated")
+            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config], gated=args.variant == "gated",
+                                             fp4=args.variant == "fp4")
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -14,6 +14,8 @@ Entry points (same names as the C ABI):
   hyb_fused_fwd        the three stages on one stream
   hyb_decode_append    decode cache maintenance: window ring + compressed entries
   hyb_gated_fwd        the gated three-branch variant (compressed, selected, window)
+  hyb_fp4_*            4-bit compressed caches: quantize / dequantize, and the
+                       indexer, attention and decode append over them
   hyb_workspace_size, hyb_get_device_status, hyb_error_string
 """
 from __future__ import annotations
@@ -27,10 +29,10 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhybattn.so")
 
+_BUILD_HINT = ("build it with `python compressed_sparse_sliding_b200/build.py` (nvcc, sm_100a). "
+               "There is no fallback implementation.")
 if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_sliding_b200.build` "
-        "(nvcc, sm_100a). There is no fallback implementation.")
+    raise ImportError(f"{LIB_PATH} is missing: {_BUILD_HINT}")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -57,26 +59,41 @@ class HybProblem(ctypes.Structure):
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _PP = ctypes.POINTER(HybProblem)
-_lib.hyb_workspace_size.argtypes = [_PP]
-_lib.hyb_workspace_size.restype = ctypes.c_size_t
-_lib.hyb_hca_compress.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
-_lib.hyb_hca_compress.restype = _I
-_lib.hyb_csa_index_topk.argtypes = [_PP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
-_lib.hyb_csa_index_topk.restype = _I
-_lib.hyb_attn_fwd.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P]
-_lib.hyb_attn_fwd.restype = _I
-_lib.hyb_fused_fwd.argtypes = [_PP] + [_P] * 16 + [ctypes.c_size_t, _P]
-_lib.hyb_fused_fwd.restype = _I
-_lib.hyb_decode_append.argtypes = [_PP] + [_P] * 15
-_lib.hyb_decode_append.restype = _I
-_lib.hyb_gated_workspace_size.argtypes = [_PP]
-_lib.hyb_gated_workspace_size.restype = ctypes.c_size_t
-_lib.hyb_gated_fwd.argtypes = [_PP] + [_P] * 9 + [ctypes.c_size_t, _P]
-_lib.hyb_gated_fwd.restype = _I
-_lib.hyb_get_device_status.argtypes = [_P]
-_lib.hyb_get_device_status.restype = _I
-_lib.hyb_error_string.argtypes = [_I]
-_lib.hyb_error_string.restype = ctypes.c_char_p
+try:
+    _lib.hyb_workspace_size.argtypes = [_PP]
+    _lib.hyb_workspace_size.restype = ctypes.c_size_t
+    _lib.hyb_hca_compress.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
+    _lib.hyb_hca_compress.restype = _I
+    _lib.hyb_csa_index_topk.argtypes = [_PP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    _lib.hyb_csa_index_topk.restype = _I
+    _lib.hyb_attn_fwd.argtypes = [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+    _lib.hyb_attn_fwd.restype = _I
+    _lib.hyb_fused_fwd.argtypes = [_PP] + [_P] * 16 + [ctypes.c_size_t, _P]
+    _lib.hyb_fused_fwd.restype = _I
+    _lib.hyb_decode_append.argtypes = [_PP] + [_P] * 15
+    _lib.hyb_decode_append.restype = _I
+    _lib.hyb_gated_workspace_size.argtypes = [_PP]
+    _lib.hyb_gated_workspace_size.restype = ctypes.c_size_t
+    _lib.hyb_gated_fwd.argtypes = [_PP] + [_P] * 9 + [ctypes.c_size_t, _P]
+    _lib.hyb_gated_fwd.restype = _I
+    _lib.hyb_fp4_quantize.argtypes = [_P, ctypes.c_longlong, _I, _P, _P, _P]
+    _lib.hyb_fp4_quantize.restype = _I
+    _lib.hyb_fp4_dequantize.argtypes = [_P, _P, ctypes.c_longlong, _I, _P, _P]
+    _lib.hyb_fp4_dequantize.restype = _I
+    _lib.hyb_fp4_workspace_size.argtypes = [_PP]
+    _lib.hyb_fp4_workspace_size.restype = ctypes.c_size_t
+    _lib.hyb_csa_index_topk_fp4.argtypes = [_PP] + [_P] * 7 + [ctypes.c_size_t, _P]
+    _lib.hyb_csa_index_topk_fp4.restype = _I
+    _lib.hyb_attn_fwd_fp4.argtypes = [_PP] + [_P] * 11 + [ctypes.c_size_t, _P]
+    _lib.hyb_attn_fwd_fp4.restype = _I
+    _lib.hyb_decode_append_fp4.argtypes = [_PP] + [_P] * 18
+    _lib.hyb_decode_append_fp4.restype = _I
+    _lib.hyb_get_device_status.argtypes = [_P]
+    _lib.hyb_get_device_status.restype = _I
+    _lib.hyb_error_string.argtypes = [_I]
+    _lib.hyb_error_string.restype = ctypes.c_char_p
+except AttributeError as exc:   # a library built from older sources
+    raise ImportError(f"{LIB_PATH} lacks an entry point ({exc}); rebuild: {_BUILD_HINT}") from exc
 
 
 class HybError(RuntimeError):
@@ -197,6 +214,94 @@ def hyb_decode_append(p: HybProblem, t_new, k_new, v_new, k_ring, v_ring, kc, vc
                                 _ptr(ki_ring), _ptr(kc), _ptr(vc), _ptr(kic), _ptr(kv_pos0),
                                 _stream(stream))
     _check(st, "hyb_decode_append")
+    return kv_pos0
+
+
+class Fp4Cache:
+    """A 4-bit cache: codes [..., dx/2] uint8 and qp [..., 2] fp32 (min, scale) per row."""
+
+    def __init__(self, codes: torch.Tensor, qp: torch.Tensor):
+        self.codes = codes
+        self.qp = qp
+
+    @staticmethod
+    def empty(shape, device):
+        """Storage for a cache of bf16 shape [..., dx]."""
+        *lead, dx = shape
+        return Fp4Cache(torch.zeros((*lead, dx // 2), dtype=torch.uint8, device=device),
+                        torch.zeros((*lead, 2), dtype=torch.float32, device=device))
+
+
+def hyb_fp4_quantize(x: torch.Tensor, out: Optional[Fp4Cache] = None, stream=None) -> Fp4Cache:
+    """Per-row 4-bit min/max quantization of a bf16 tensor [..., dx]."""
+    if out is None:
+        out = Fp4Cache.empty(tuple(x.shape), x.device)
+    rows = x.numel() // x.shape[-1]
+    st = _lib.hyb_fp4_quantize(_ptr(x), rows, x.shape[-1], _ptr(out.codes), _ptr(out.qp), _stream(stream))
+    _check(st, "hyb_fp4_quantize")
+    return out
+
+
+def hyb_fp4_dequantize(c: Fp4Cache, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 values [..., dx] of a 4-bit cache."""
+    dx = 2 * c.codes.shape[-1]
+    if out is None:
+        out = torch.empty((*c.codes.shape[:-1], dx), dtype=torch.bfloat16, device=c.codes.device)
+    rows = c.codes.numel() // c.codes.shape[-1]
+    st = _lib.hyb_fp4_dequantize(_ptr(c.codes), _ptr(c.qp), rows, dx, _ptr(out), _stream(stream))
+    _check(st, "hyb_fp4_dequantize")
+    return out
+
+
+def hyb_fp4_workspace_size(p: HybProblem) -> int:
+    return int(_lib.hyb_fp4_workspace_size(ctypes.byref(p)))
+
+
+def _fp4_ws(p, ws, device):
+    need = max(hyb_fp4_workspace_size(p), 256)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def hyb_csa_index_topk_fp4(p: HybProblem, qi, wi, kic: Fp4Cache, idx=None, sel_scores=None, ws=None,
+                           stream=None):
+    """hyb_csa_index_topk over a 4-bit indexer-key cache [B, Nc, di]."""
+    if idx is None:
+        idx = torch.empty((p.B, p.Lq, p.topk), dtype=torch.int32, device=qi.device)
+    ws = _fp4_ws(p, ws, qi.device)
+    st = _lib.hyb_csa_index_topk_fp4(ctypes.byref(p), _ptr(qi), _ptr(wi), _ptr(kic.codes), _ptr(kic.qp),
+                                     _ptr(idx), _ptr(sel_scores), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "hyb_csa_index_topk_fp4")
+    return idx
+
+
+def hyb_attn_fwd_fp4(p: HybProblem, q, kc: Fp4Cache, vc: Fp4Cache, idx, k_raw, v_raw, o=None, lse=None,
+                     ws=None, stream=None):
+    """hyb_attn_fwd over 4-bit K / V caches [B, Nc, Hkv, d]."""
+    if o is None:
+        o = torch.empty((p.B, p.Lq, p.Hq, p.d), dtype=torch.bfloat16, device=q.device)
+    ws = _fp4_ws(p, ws, q.device)
+    st = _lib.hyb_attn_fwd_fp4(ctypes.byref(p), _ptr(q), _ptr(kc.codes), _ptr(kc.qp), _ptr(vc.codes),
+                               _ptr(vc.qp), _ptr(idx), _ptr(k_raw), _ptr(v_raw), _ptr(o), _ptr(lse),
+                               _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "hyb_attn_fwd_fp4")
+    return o
+
+
+def hyb_decode_append_fp4(p: HybProblem, t_new, k_new, v_new, k_ring, v_ring, kc: Fp4Cache, vc: Fp4Cache,
+                          wk, wv, ki_new=None, wib=None, ki_ring=None, kic: Optional[Fp4Cache] = None,
+                          kv_pos0=None, stream=None):
+    """hyb_decode_append with 4-bit caches (entries quantized as they close)."""
+    if kv_pos0 is None:
+        kv_pos0 = torch.empty((p.B,), dtype=torch.int32, device=k_new.device)
+    st = _lib.hyb_decode_append_fp4(ctypes.byref(p), _ptr(t_new), _ptr(k_new), _ptr(v_new), _ptr(ki_new),
+                                    _ptr(wk), _ptr(wv), _ptr(wib), _ptr(k_ring), _ptr(v_ring), _ptr(ki_ring),
+                                    _ptr(kc.codes), _ptr(kc.qp), _ptr(vc.codes), _ptr(vc.qp),
+                                    _ptr(kic.codes if kic is not None else None),
+                                    _ptr(kic.qp if kic is not None else None), _ptr(kv_pos0),
+                                    _stream(stream))
+    _check(st, "hyb_decode_append_fp4")
     return kv_pos0
 
 

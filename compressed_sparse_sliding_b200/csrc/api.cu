@@ -27,14 +27,24 @@ cudaError_t launch_hca_attn(int B, int L, int Lkv, int Hq, int Hkv, int d, int N
 cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int m, int W, int topk,
                             float scale, const int32_t *q_pos, const int32_t *kv_pos0, const void *q,
                             const void *kc, const void *vc, const int32_t *idx, const void *kr,
-                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms);
+                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms,
+                            int pregathered);
+cudaError_t launch_fp4_quantize(const void *x, long long rows, int dx, uint8_t *codes, float *qp,
+                                cudaStream_t stream, int num_sms);
+cudaError_t launch_fp4_dequantize(const uint8_t *codes, const float *qp, long long rows, int dx,
+                                  void *out, cudaStream_t stream, int num_sms);
+cudaError_t launch_fp4_gather(const uint8_t *kcodes, const float *kqp, const uint8_t *vcodes,
+                              const float *vqp, const int32_t *idx, void *kout, void *vout, int B, int Lq,
+                              int topk, int Hkv, int Nc, int d, cudaStream_t stream, int num_sms);
+cudaError_t launch_index_dec_fp4(const void *qi, const float *wi, const uint8_t *kic_codes,
+                                 const float *kic_qp, float *scores, int B, int Lq, int Hi, int di, int Nc,
+                                 int m, int W, const int32_t *q_pos, cudaStream_t stream);
 cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, int Nc, int m, int W,
                                int topk, float scale, const int32_t *q_pos, const int32_t *kv_pos0,
                                const void *q, const void *kc, const void *vc, const int32_t *idx,
                                const void *kr, const void *vr, void *o, float *lse,
                                cudaStream_t stream);
 
-struct AppendParams;
 cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream);
 cudaError_t launch_gated_combine(const void *o1, const void *o2, const void *o3, const float *gate,
                                  void *o, long long rows, int d, cudaStream_t stream, int num_sms);
@@ -116,6 +126,78 @@ static float softmax_scale(const hyb_problem *p)
     return p->scale != 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
 }
 
+// 4-bit caches.  Attention: when a query batch selects fewer rows than the
+// cache holds (decode), only those are dequantized, in slot order (the CSA
+// kernel then reads them as its "pre-gathered" rows); otherwise the whole K
+// and V caches are dequantized once.  The workspace holds the bf16 K rows,
+// then the V rows.
+static bool fp4_attn_pregather(const hyb_problem *p)
+{
+    return p->topk > 0 && p->d == 128 && (long long)p->Lq * p->topk < (long long)p->Nc;
+}
+
+static size_t fp4_attn_bytes(const hyb_problem *p)
+{
+    const long long rows = fp4_attn_pregather(p) ? (long long)p->B * p->Lq * p->topk * p->Hkv
+                                                 : (long long)p->B * p->Nc * p->Hkv;
+    const size_t one = ((size_t)rows * p->d * 2 + 255) & ~(size_t)255;
+    return 2 * one;
+}
+
+// Indexer: the decode form (few query rows, di = 64) dequantizes key tiles
+// on chip; other shapes dequantize the indexer-key cache into the workspace
+// after the score buffer.
+static bool fp4_index_in_kernel(const hyb_problem *p)
+{
+    return p->di == 64 && p->Lq < 64 && p->Hi <= 16;
+}
+
+// Checks shared by the two decode-append entry points (the caches are
+// checked by each); fills everything but the cache pointers.
+static hyb_status append_common(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                                const void *v_new, const void *ki_new, const float *wk, const float *wv,
+                                const float *wib, void *k_ring, void *v_ring, void *ki_ring,
+                                int32_t *kv_pos0, AppendParams &a)
+{
+    if (!p || p->B <= 0 || p->Hkv <= 0 || p->d <= 0 || p->m <= 0 || p->W <= 0 || p->Nc <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (p->d % 8 != 0 || p->Lkv != 2 * p->W)
+        return HYB_ERR_INVALID_ARG;
+    if (p->m > p->W)
+        return HYB_ERR_UNSUPPORTED;   // a block must still be in the window when it completes
+    const bool csa = p->topk > 0;
+    if (!t_new || !k_new || !v_new || !wk || !wv || !k_ring || !v_ring || !kv_pos0)
+        return HYB_ERR_INVALID_ARG;
+    if (csa && (!ki_new || !wib || !ki_ring || p->di <= 0 || p->di % 8 != 0))
+        return HYB_ERR_INVALID_ARG;
+    const void *ptrs[] = {k_new, v_new, wk, wv, k_ring, v_ring};
+    for (const void *q : ptrs)
+        if (!aligned16(q))
+            return HYB_ERR_INVALID_ARG;
+    if (csa && (!aligned16(ki_new) || !aligned16(wib) || !aligned16(ki_ring)))
+        return HYB_ERR_INVALID_ARG;
+    a = AppendParams{};
+    a.B = p->B;
+    a.Hkv = p->Hkv;
+    a.d = p->d;
+    a.di = csa ? p->di : 0;
+    a.m = p->m;
+    a.W = p->W;
+    a.Nc = p->Nc;
+    a.t_new = t_new;
+    a.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    a.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    a.ki_new = csa ? static_cast<const __nv_bfloat16 *>(ki_new) : nullptr;
+    a.wk = wk;
+    a.wv = wv;
+    a.wib = csa ? wib : nullptr;
+    a.k_ring = static_cast<__nv_bfloat16 *>(k_ring);
+    a.v_ring = static_cast<__nv_bfloat16 *>(v_ring);
+    a.ki_ring = csa ? static_cast<__nv_bfloat16 *>(ki_ring) : nullptr;
+    a.kv_pos0 = kv_pos0;
+    return HYB_OK;
+}
+
 }  // namespace hyb
 
 using namespace hyb;
@@ -187,7 +269,7 @@ hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, con
         // CSA: per-token selections, transposed tcgen05 kernel
         return cuda_status(launch_csa_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->Nc, p->m, p->W,
                                            p->topk, softmax_scale(p), p->q_pos, p->kv_pos0, q, kc, vc,
-                                           idx, k_raw, v_raw, o, lse, stream, num_sms_current()));
+                                           idx, k_raw, v_raw, o, lse, stream, num_sms_current(), 0));
     }
     cudaError_t e = launch_hybrid_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->d, p->Nc, p->m, p->W,
                                        p->topk, softmax_scale(p), p->q_pos, p->kv_pos0, q, kc, vc, idx,
@@ -237,46 +319,157 @@ hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const v
                              const float *wib, void *k_ring, void *v_ring, void *ki_ring, void *kc,
                              void *vc, void *kic, int32_t *kv_pos0, cudaStream_t stream)
 {
-    if (!p || p->B <= 0 || p->Hkv <= 0 || p->d <= 0 || p->m <= 0 || p->W <= 0 || p->Nc <= 0)
-        return HYB_ERR_INVALID_ARG;
-    if (p->d % 8 != 0 || p->Lkv != 2 * p->W)
-        return HYB_ERR_INVALID_ARG;
-    if (p->m > p->W)
-        return HYB_ERR_UNSUPPORTED;   // a block must still be in the window when it completes
-    const bool csa = p->topk > 0;
-    if (!t_new || !k_new || !v_new || !wk || !wv || !k_ring || !v_ring || !kc || !vc || !kv_pos0)
-        return HYB_ERR_INVALID_ARG;
-    if (csa && (!ki_new || !wib || !ki_ring || !kic || p->di <= 0 || p->di % 8 != 0))
-        return HYB_ERR_INVALID_ARG;
-    const void *ptrs[] = {k_new, v_new, wk, wv, k_ring, v_ring, kc, vc};
-    for (const void *q : ptrs)
-        if (!aligned16(q))
-            return HYB_ERR_INVALID_ARG;
-    if (csa && (!aligned16(ki_new) || !aligned16(wib) || !aligned16(ki_ring) || !aligned16(kic)))
-        return HYB_ERR_INVALID_ARG;
     AppendParams a;
-    a.B = p->B;
-    a.Hkv = p->Hkv;
-    a.d = p->d;
-    a.di = csa ? p->di : 0;
-    a.m = p->m;
-    a.W = p->W;
-    a.Nc = p->Nc;
-    a.t_new = t_new;
-    a.k_new = static_cast<const __nv_bfloat16 *>(k_new);
-    a.v_new = static_cast<const __nv_bfloat16 *>(v_new);
-    a.ki_new = csa ? static_cast<const __nv_bfloat16 *>(ki_new) : nullptr;
-    a.wk = wk;
-    a.wv = wv;
-    a.wib = csa ? wib : nullptr;
-    a.k_ring = static_cast<__nv_bfloat16 *>(k_ring);
-    a.v_ring = static_cast<__nv_bfloat16 *>(v_ring);
-    a.ki_ring = csa ? static_cast<__nv_bfloat16 *>(ki_ring) : nullptr;
+    hyb_status st = append_common(p, t_new, k_new, v_new, ki_new, wk, wv, wib, k_ring, v_ring, ki_ring,
+                                  kv_pos0, a);
+    if (st != HYB_OK)
+        return st;
+    const bool csa = p->topk > 0;
+    if (!kc || !vc || !aligned16(kc) || !aligned16(vc) || (csa && (!kic || !aligned16(kic))))
+        return HYB_ERR_INVALID_ARG;
     a.kc = static_cast<__nv_bfloat16 *>(kc);
     a.vc = static_cast<__nv_bfloat16 *>(vc);
     a.kic = csa ? static_cast<__nv_bfloat16 *>(kic) : nullptr;
-    a.kv_pos0 = kv_pos0;
     return cuda_status(launch_decode_append(a, stream));
+}
+
+hyb_status hyb_decode_append_fp4(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                                 const void *v_new, const void *ki_new, const float *wk, const float *wv,
+                                 const float *wib, void *k_ring, void *v_ring, void *ki_ring,
+                                 uint8_t *kc_codes, float *kc_qp, uint8_t *vc_codes, float *vc_qp,
+                                 uint8_t *kic_codes, float *kic_qp, int32_t *kv_pos0, cudaStream_t stream)
+{
+    AppendParams a;
+    hyb_status st = append_common(p, t_new, k_new, v_new, ki_new, wk, wv, wib, k_ring, v_ring, ki_ring,
+                                  kv_pos0, a);
+    if (st != HYB_OK)
+        return st;
+    const bool csa = p->topk > 0;
+    if (p->d > 256 || (csa && p->di > 256))
+        return HYB_ERR_UNSUPPORTED;
+    if (!kc_codes || !kc_qp || !vc_codes || !vc_qp || (csa && (!kic_codes || !kic_qp)))
+        return HYB_ERR_INVALID_ARG;
+    if (!aligned16(kc_codes) || !aligned16(kc_qp) || !aligned16(vc_codes) || !aligned16(vc_qp) ||
+        (csa && (!aligned16(kic_codes) || !aligned16(kic_qp))))
+        return HYB_ERR_INVALID_ARG;
+    a.kcq = kc_codes;
+    a.vcq = vc_codes;
+    a.kicq = csa ? kic_codes : nullptr;
+    a.kqp = reinterpret_cast<float2 *>(kc_qp);
+    a.vqp = reinterpret_cast<float2 *>(vc_qp);
+    a.kiqp = csa ? reinterpret_cast<float2 *>(kic_qp) : nullptr;
+    return cuda_status(launch_decode_append(a, stream));
+}
+
+hyb_status hyb_fp4_quantize(const void *x, long long rows, int dx, uint8_t *codes, float *qp,
+                            cudaStream_t stream)
+{
+    if (!x || !codes || !qp || rows < 0)
+        return HYB_ERR_INVALID_ARG;
+    if (dx != 64 && dx != 128 && dx != 256)
+        return HYB_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(qp))
+        return HYB_ERR_INVALID_ARG;
+    return cuda_status(launch_fp4_quantize(x, rows, dx, codes, qp, stream, num_sms_current()));
+}
+
+hyb_status hyb_fp4_dequantize(const uint8_t *codes, const float *qp, long long rows, int dx, void *out,
+                              cudaStream_t stream)
+{
+    if (!codes || !qp || !out || rows < 0 || dx <= 0 || dx % 8 != 0)
+        return HYB_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(codes) || !aligned16(qp))
+        return HYB_ERR_INVALID_ARG;
+    return cuda_status(launch_fp4_dequantize(codes, qp, rows, dx, out, stream, num_sms_current()));
+}
+
+size_t hyb_fp4_workspace_size(const hyb_problem *p)
+{
+    if (!p || p->B <= 0 || p->Lq <= 0 || p->Hkv <= 0 || p->d <= 0 || p->Nc < 0)
+        return 0;
+    const size_t attn = fp4_attn_bytes(p);
+    size_t index = 0;
+    if (p->topk > 0 && p->Hi > 0 && p->di > 0) {
+        index = hyb_workspace_size(p);
+        if (!fp4_index_in_kernel(p))
+            index += ((size_t)p->B * p->Nc * p->di * 2 + 255) & ~(size_t)255;
+    }
+    return attn > index ? attn : index;
+}
+
+hyb_status hyb_csa_index_topk_fp4(const hyb_problem *p, const void *qi, const float *wi,
+                                  const uint8_t *kic_codes, const float *kic_qp, int32_t *idx,
+                                  float *sel_scores, void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, true);
+    if (st != HYB_OK)
+        return st;
+    if (!qi || !wi || !kic_codes || !kic_qp || !idx || !aligned16(qi) || !aligned16(kic_codes) ||
+        !aligned16(kic_qp))
+        return HYB_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < hyb_fp4_workspace_size(p) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return HYB_ERR_WORKSPACE;
+    float *scores = static_cast<float *>(ws);
+    if (fp4_index_in_kernel(p)) {
+        // decode: the indexer dequantizes key tiles on chip
+        cudaError_t e = launch_index_dec_fp4(qi, wi, kic_codes, kic_qp, scores, p->B, p->Lq, p->Hi,
+                                             p->di, p->Nc, p->m, p->W, p->q_pos, stream);
+        if (e != cudaSuccess)
+            return cuda_status(e);
+        return cuda_status(launch_topk_radix(scores, p->B, p->Lq, p->Nc, p->m, p->W, p->topk, p->q_pos,
+                                             idx, sel_scores, stream));
+    }
+    // otherwise the whole indexer-key cache is dequantized once
+    uint8_t *kic = static_cast<uint8_t *>(ws) + hyb_workspace_size(p);
+    cudaError_t e = launch_fp4_dequantize(kic_codes, kic_qp, (long long)p->B * p->Nc, p->di, kic, stream,
+                                          num_sms_current());
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, scores, stream));
+}
+
+hyb_status hyb_attn_fwd_fp4(const hyb_problem *p, const void *q, const uint8_t *kc_codes,
+                            const float *kc_qp, const uint8_t *vc_codes, const float *vc_qp,
+                            const int32_t *idx, const void *k_raw, const void *v_raw, void *o, float *lse,
+                            void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, false);
+    if (st != HYB_OK)
+        return st;
+    if (p->Nc <= 0 || !kc_codes || !kc_qp || !vc_codes || !vc_qp)
+        return HYB_ERR_INVALID_ARG;
+    if (!aligned16(kc_codes) || !aligned16(kc_qp) || !aligned16(vc_codes) || !aligned16(vc_qp))
+        return HYB_ERR_INVALID_ARG;
+    if (idx && p->topk <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < fp4_attn_bytes(p) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return HYB_ERR_WORKSPACE;
+    uint8_t *wk = static_cast<uint8_t *>(ws);
+    const int n = num_sms_current();
+    if (idx && fp4_attn_pregather(p)) {
+        // decode: only the selected rows, dequantized in slot order
+        if (!q || !o || !k_raw || !v_raw || !aligned16(q) || !aligned16(o) || !aligned16(k_raw) ||
+            !aligned16(v_raw) || (p->Lkv <= 0 && p->W > 0))
+            return HYB_ERR_INVALID_ARG;
+        const size_t half = fp4_attn_bytes(p) / 2;
+        cudaError_t e = launch_fp4_gather(kc_codes, kc_qp, vc_codes, vc_qp, idx, wk, wk + half, p->B, p->Lq,
+                                          p->topk, p->Hkv, p->Nc, p->d, stream, n);
+        if (e != cudaSuccess)
+            return cuda_status(e);
+        const int Lkv = p->Lkv > 0 ? p->Lkv : 1;
+        return cuda_status(launch_csa_attn(p->B, p->Lq, Lkv, p->Hq, p->Hkv, p->Nc, p->m, p->W, p->topk,
+                                           softmax_scale(p), p->q_pos, p->kv_pos0, q, wk, wk + half, idx,
+                                           k_raw, v_raw, o, lse, stream, n, 1));
+    }
+    // otherwise the whole K / V caches are dequantized once
+    const long long rows = (long long)p->B * p->Nc * p->Hkv;
+    const size_t half = fp4_attn_bytes(p) / 2;
+    cudaError_t e = launch_fp4_dequantize(kc_codes, kc_qp, rows, p->d, wk, stream, n);
+    if (e == cudaSuccess)
+        e = launch_fp4_dequantize(vc_codes, vc_qp, rows, p->d, wk + half, stream, n);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    return hyb_attn_fwd(p, q, wk, wk + half, idx, k_raw, v_raw, o, lse, stream);
 }
 
 size_t hyb_gated_workspace_size(const hyb_problem *p)

@@ -49,6 +49,7 @@ constexpr int kSpD = 128;        // head dim handled by this kernel
 
 struct SparseParams {
     int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
+    int pregathered;   // kc / vc hold each token's selected rows in slot order: [B Lq, topk, Hkv, 128]
     long long n_items;
     float scale_log2;
     const int32_t *q_pos, *kv_pos0, *idx;
@@ -316,7 +317,6 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr int VS = SM::VS;
     constexpr int RB = NH * 2;                                  // bytes of one P^T row
     constexpr uint32_t PLAYOUT = RB == 128 ? 2u : (RB == 64 ? 4u : 6u);
-    constexpr int PCH = RB / 16;                                // 16-byte chunks per row
     extern __shared__ __align__(1024) uint8_t sp_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sp_smem_raw) + 1023) &
                                                 ~(uintptr_t)1023);
@@ -441,7 +441,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             if (j >= p.Nc)
                                 set_error(HYB_ERR_DEVICE_BOUNDS);
                             const bool v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < wstart);
-                            sSel[q] = v ? (k.b * p.Nc + j) * p.Hkv + k.kvh : -1;
+                            const int srow = p.pregathered
+                                                 ? ((int)((uint32_t)w / (uint32_t)p.Hkv) * p.topk + q) * p.Hkv + k.kvh
+                                                 : (k.b * p.Nc + j) * p.Hkv + k.kvh;
+                            sSel[q] = v ? srow : -1;
                         }
                     }
                 }
@@ -850,8 +853,9 @@ static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void
     using SM = SparseSmem<NH>;
     CUtensorMap mq, mkc, mvc, mkr, mvr;
     bool ok = make_map_2d(&mq, q, (long long)p.B * p.Lq * p.Hq, NH);
-    ok &= make_map_2d(&mkc, kc, (long long)p.B * p.Nc * p.Hkv, 1);
-    ok &= make_map_2d(&mvc, vc, (long long)p.B * p.Nc * p.Hkv, 1);
+    const long long crow = p.pregathered ? (long long)p.B * p.Lq * p.topk * p.Hkv : (long long)p.B * p.Nc * p.Hkv;
+    ok &= make_map_2d(&mkc, kc, crow, 1);
+    ok &= make_map_2d(&mvc, vc, crow, 1);
     ok &= make_map_2d(&mkr, kr, (long long)p.B * p.Lkv * p.Hkv, 1);
     ok &= make_map_2d(&mvr, vr, (long long)p.B * p.Lkv * p.Hkv, 1);
     if (!ok)
@@ -880,7 +884,8 @@ static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void
 cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int m, int W, int topk,
                             float scale, const int32_t *q_pos, const int32_t *kv_pos0, const void *q,
                             const void *kc, const void *vc, const int32_t *idx, const void *kr,
-                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms)
+                            const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms,
+                            int pregathered)
 {
     SparseParams p;
     p.B = B;
@@ -896,6 +901,9 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
     p.NH = p.g <= 16 ? 16 : (p.g <= 32 ? 32 : 64);
     p.n_items = (long long)B * Lq * Hkv;
     if (p.n_items >= (1ll << 31))
+        return cudaErrorInvalidValue;
+    p.pregathered = pregathered;
+    if (pregathered && (long long)B * Lq * topk * Hkv >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.q_pos = q_pos;

@@ -1,6 +1,7 @@
 // hybattn.cu -- single translation unit of libhybattn.so (keeps the device
 // status word and every kernel in one module without relocatable device code).
 #include "compress.cu"
+#include "fp4.cu"
 #include "index_topk.cu"
 #include "index_tc.cu"
 #include "attn.cu"

@@ -321,8 +321,15 @@ static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const
 // indexer-key cache once (HBM bound).  One CTA per (query row, run of tiles).
 // Roles (192 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 2-5
 // epilogue (warp w reads TMEM lane quadrant w % 4).
+// With a 4-bit key cache (codes and per-row (min, scale), see fp4.cu) four
+// converter warps replace the TMA producer (288 threads): thread r copies
+// key r's codes of tiles kDcAhead ahead into a staging ring with cp.async,
+// and, when they have landed, writes the row's bf16 values into the K stage
+// in the 128-byte swizzle; the MMA warp is then warp 4, the epilogue warps
+// 5-8.
 // ------------------------------------------------------------------------
 constexpr int kDcThreads = 192;
+constexpr int kDcAhead = 8;      // 4-bit form: tiles of codes in flight per converter thread
 constexpr int kDcBM = 128;       // keys per tile
 constexpr int kDcN = 16;         // padded indexer heads
 constexpr int kDcStages = 4;
@@ -333,14 +340,30 @@ struct DecIndexParams {
     const int32_t *q_pos;
     const float *wi;
     float *scores;
+    const uint8_t *kcodes;   // 4-bit form: [B Nc, 32] codes, [B Nc] (min, scale)
+    const float2 *kqp;
 };
 
-__global__ void __launch_bounds__(kDcThreads, 1)
+template <bool Q4>
+struct DecRoles {
+    static constexpr int PW = Q4 ? 4 : 1;            // producer (converter) warps
+    static constexpr int MMA_WARP = PW;
+    static constexpr int THREADS = 32 * (PW + 5);
+    static constexpr int Q_BYTES = kDcN * kIxDi * 2;       // 2 KB
+    static constexpr int K_BYTES = kDcBM * kIxDi * 2;      // 16 KB
+    static constexpr int ST_CODES = kDcBM * kIxDi / 2;     // 4 KB of codes per staged tile
+    static constexpr int ST_BYTES = Q4 ? kDcAhead * (ST_CODES + kDcBM * 8) : 0;
+    static constexpr int SMEM = 1024 + kDcStages * K_BYTES + Q_BYTES + 16 * 8 + 16 * 4 + ST_BYTES;
+};
+
+template <bool Q4>
+__global__ void __launch_bounds__(DecRoles<Q4>::THREADS, 1)
 index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const DecIndexParams p)
 {
-    constexpr int Q_BYTES = kDcN * kIxDi * 2;      // 2 KB
-    constexpr int K_BYTES = kDcBM * kIxDi * 2;     // 16 KB
+    using RL = DecRoles<Q4>;
+    constexpr int Q_BYTES = RL::Q_BYTES;
+    constexpr int K_BYTES = RL::K_BYTES;
     extern __shared__ __align__(1024) uint8_t dc_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dc_smem_raw) + 1023) &
                                                 ~(uintptr_t)1023);
@@ -349,6 +372,7 @@ index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t *bar = reinterpret_cast<uint64_t *>(sQ + Q_BYTES);
     int *misc = reinterpret_cast<int *>(bar + 16);
     volatile int *abort_flag = misc + 1;
+    uint8_t *sSt = reinterpret_cast<uint8_t *>(misc + 16);   // 4-bit staging: codes, then (min, scale)
     // bars: 0 Q, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -370,18 +394,77 @@ index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 16; ++i)
-            mbar_init(&bar[i], (i == 11 || i == 12) ? 128 : 1);
+            mbar_init(&bar[i], (i == 11 || i == 12 || (Q4 && i >= 1 && i <= 4)) ? 128 : 1);
         mbar_fence_init();
         misc[1] = 0;
     }
-    if (warp == 1)
+    if (warp == RL::MMA_WARP)
         tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 32);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
 
-    if (warp == 0) {
+    if (Q4 && warp < RL::PW) {
+        // converters: thread r owns key row r of every tile
+        const int r = threadIdx.x;
+        if (r == 0) {
+            mbar_arrive_expect_tx(&bar[0], Q_BYTES);
+            tma_load_2d_box(sQ, &tm_q, &bar[0], 0, row * p.Hi);
+        }
+        const uint32_t st_codes = smem_u32(sSt), st_qp = st_codes + kDcAhead * RL::ST_CODES;
+        // copies of tile i's row r into staging slot i % kDcAhead (zero past the cache)
+        auto stage = [&](int i) {
+            const int s = i % kDcAhead;
+            const long long kr = (long long)(j0 + i) * kDcBM + r;
+            const bool in = kr < p.Nc;
+            const long long src = (long long)b * p.Nc + (in ? kr : 0);
+            const uint32_t n = in ? 16u : 0u;
+            const uint8_t *cs = p.kcodes + src * (kIxDi / 2);
+            cp_async_16(st_codes + s * RL::ST_CODES + r * 32, cs, n);
+            cp_async_16(st_codes + s * RL::ST_CODES + r * 32 + 16, cs + 16, n);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(st_qp + s * kDcBM * 8 + r * 8),
+                         "l"(p.kqp + src), "r"(in ? 8u : 0u)
+                         : "memory");
+        };
+#pragma unroll 1
+        for (int i = 0; i < kDcAhead - 1; ++i) {
+            if (i < nt)
+                stage(i);
+            cp_async_commit();
+        }
+        bool ok = true;
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kDcStages;
+            if (i + kDcAhead - 1 < nt)
+                stage(i + kDcAhead - 1);
+            cp_async_commit();
+            cp_async_wait_group<kDcAhead - 1>();     // tile i's copies of this thread have landed
+            if (i >= kDcStages)
+                ok &= mbar_wait(&bar[5 + s], ((i / kDcStages) - 1) & 1, abort_flag);
+            const int ss = i % kDcAhead;
+            const uint8_t *cr = sSt + ss * RL::ST_CODES + r * 32;
+            const float2 qv = *reinterpret_cast<const float2 *>(sSt + kDcAhead * RL::ST_CODES +
+                                                                ss * kDcBM * 8 + r * 8);
+            const uint4 c0 = *reinterpret_cast<const uint4 *>(cr);
+            const uint4 c1 = *reinterpret_cast<const uint4 *>(cr + 16);
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const uint32_t dst = smem_u32(sK + s * K_BYTES);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = fp4_dequant8(cw[c], qv.x, qv.y);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128_offset(r, c)),
+                             "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar[1 + s]);
+        }
+        (void)ok;
+        cp_async_wait_group<0>();
+        if (r == 0)
+            drain_wait(&bar[0], 0);
+    } else if (!Q4 && warp == 0) {
         if (lane == 0) {
             mbar_arrive_expect_tx(&bar[0], Q_BYTES);
             // rows row*Hi .. row*Hi+15 of the [B*Lq*Hi, 64] view; rows past this
@@ -400,7 +483,7 @@ index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int i = max(0, issued - kDcStages); i < issued; ++i)
                 drain_wait(&bar[1 + i % kDcStages], (i / kDcStages) & 1);
         }
-    } else if (warp == 1) {
+    } else if (warp == RL::MMA_WARP) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(kDcBM, kDcN, false, false);
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
@@ -459,15 +542,16 @@ index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == RL::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc((uint32_t)misc[0], 32);
     }
 }
 
-static cudaError_t launch_index_dec(const void *qi, const float *wi, const void *kic, float *scores,
-                                    int B, int Lq, int Hi, int Nc, int m, int W, const int32_t *q_pos,
-                                    cudaStream_t stream)
+// kic: bf16 cache (TMA tiles), or nullptr with kcodes / kqp set (4-bit form).
+static cudaError_t launch_index_dec(const void *qi, const float *wi, const void *kic,
+                                    const uint8_t *kcodes, const float *kqp, float *scores, int B, int Lq,
+                                    int Hi, int Nc, int m, int W, const int32_t *q_pos, cudaStream_t stream)
 {
     CUtensorMap mq, mk;
     EncodeTiledFn fn = encode_fn();
@@ -483,7 +567,10 @@ static cudaError_t launch_index_dec(const void *qi, const float *wi, const void 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    if (!make_map(&mk, kic, kIxDi, 1, Nc, B, 1, kDcBM))
+    const bool q4 = kic == nullptr;
+    if (q4)
+        mk = mq;   // unused by the 4-bit form
+    else if (!make_map(&mk, kic, kIxDi, 1, Nc, B, 1, kDcBM))
         return cudaErrorInvalidValue;
     DecIndexParams p;
     p.B = B;
@@ -498,13 +585,36 @@ static cudaError_t launch_index_dec(const void *qi, const float *wi, const void 
     p.q_pos = q_pos;
     p.wi = wi;
     p.scores = scores;
-    const size_t smem = 1024 + kDcStages * kDcBM * kIxDi * 2 + kDcN * kIxDi * 2 + 16 * 8 + 16 * 4;
-    cudaError_t e = cudaFuncSetAttribute(index_scores_dec, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess)
-        return e;
-    index_scores_dec<<<(unsigned)(B * Lq * p.n_chunks), kDcThreads, smem, stream>>>(mq, mk, p);
+    p.kcodes = kcodes;
+    p.kqp = reinterpret_cast<const float2 *>(kqp);
+    const unsigned grid = (unsigned)(B * Lq * p.n_chunks);
+    if (q4) {
+        const size_t smem = DecRoles<true>::SMEM;
+        cudaError_t e = cudaFuncSetAttribute(index_scores_dec<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        index_scores_dec<true><<<grid, DecRoles<true>::THREADS, smem, stream>>>(mq, mk, p);
+    } else {
+        const size_t smem = DecRoles<false>::SMEM;
+        cudaError_t e = cudaFuncSetAttribute(index_scores_dec<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        index_scores_dec<false><<<grid, DecRoles<false>::THREADS, smem, stream>>>(mq, mk, p);
+    }
     return cudaGetLastError();
+}
+
+// Decode indexer scores over a 4-bit indexer-key cache (di = 64, Hi <= 16).
+cudaError_t launch_index_dec_fp4(const void *qi, const float *wi, const uint8_t *kic_codes,
+                                 const float *kic_qp, float *scores, int B, int Lq, int Hi, int di, int Nc,
+                                 int m, int W, const int32_t *q_pos, cudaStream_t stream)
+{
+    if (di != kIxDi || Hi < 1 || Hi > kDcN)
+        return cudaErrorNotSupported;
+    return launch_index_dec(qi, wi, nullptr, kic_codes, kic_qp, scores, B, Lq, Hi, Nc, m, W, q_pos,
+                            stream);
 }
 
 // Prefill indexer scores on tensor cores (di = 64, Hi <= 4).  Returns
@@ -519,7 +629,7 @@ cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *
         // decode: one tile of keys per MMA, the query's heads in N
         if (Hi > kDcN)
             return cudaErrorNotSupported;
-        return launch_index_dec(qi, wi, kic, scores, B, Lq, Hi, Nc, m, W, q_pos, stream);
+        return launch_index_dec(qi, wi, kic, nullptr, nullptr, scores, B, Lq, Hi, Nc, m, W, q_pos, stream);
     }
     if (Hi > 4)
         return cudaErrorNotSupported;

@@ -176,6 +176,12 @@ hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
  * [B] int32 out.  A negative t, or an entry j >= Nc, is skipped and flagged
  * as HYB_ERR_DEVICE_BOUNDS.  The rings start zeroed or filled by earlier
  * calls; rows of positions outside the window are never read. */
+hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                             const void *v_new, const void *ki_new, const float *wk,
+                             const float *wv, const float *wib, void *k_ring, void *v_ring,
+                             void *ki_ring, void *kc, void *vc, void *kic, int32_t *kv_pos0,
+                             cudaStream_t stream);
+
 /* The gated three-branch variant (Tiny-R2 README, "Attention Computation",
  * "branch_gate"): three attentions with separate softmaxes, then
  *   o[b,t,h] = sum_k softmax(gate[b,t,h,:])_k * o_k[b,t,h]
@@ -194,11 +200,51 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
                          const float *gate, void *o, void *ws, size_t ws_bytes,
                          cudaStream_t stream);
 
-hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const void *k_new,
-                             const void *v_new, const void *ki_new, const float *wk,
-                             const float *wv, const float *wib, void *k_ring, void *v_ring,
-                             void *ki_ring, void *kc, void *vc, void *kic, int32_t *kv_pos0,
-                             cudaStream_t stream);
+/* 4-bit compressed caches (CSDN code page, section 1, compress_to_fp4 /
+ * decompress_from_fp4).  Every row of dx channels -- one compressed entry
+ * of one head (K, V) or one indexer key -- is stored as dx/2 bytes of codes
+ * (element 2i in the low nibble of byte i) and one fp32 pair (min, scale):
+ *   scale = (max - min) / 15,  code = clamp(rint((x - min) / scale), 0, 15),
+ *   value = code * scale + min, rounded to bf16,
+ * each step one IEEE fp32 operation (ties to even; a row with max == min
+ * has scale 0 and codes 0).  The page takes min and max over the whole
+ * tensor; here they are per row, so a cache grows one entry at a time.
+ * codes: [rows, dx/2] uint8, qp: [rows, 2] fp32; all pointers device,
+ * 16-byte aligned, caller-owned. */
+hyb_status hyb_fp4_quantize(const void *x /*[rows, dx] bf16*/, long long rows, int dx,
+                            uint8_t *codes, float *qp, cudaStream_t stream);   /* dx 64/128/256 */
+hyb_status hyb_fp4_dequantize(const uint8_t *codes, const float *qp, long long rows, int dx,
+                              void *out /*[rows, dx] bf16*/, cudaStream_t stream);
+/* Workspace (bytes, 256-aligned use) for hyb_csa_index_topk_fp4 and
+ * hyb_attn_fwd_fp4 with this problem. */
+size_t hyb_fp4_workspace_size(const hyb_problem *p);
+/* hyb_csa_index_topk over a 4-bit indexer-key cache (kic_codes [B, Nc,
+ * di/2], kic_qp [B, Nc, 2]); results as hyb_csa_index_topk on the
+ * dequantized cache.  Decode shapes (Lq < 64, di = 64, Hi <= 16) dequantize
+ * key tiles on chip; others dequantize the cache into ws first. */
+hyb_status hyb_csa_index_topk_fp4(const hyb_problem *p, const void *qi, const float *wi,
+                                  const uint8_t *kic_codes, const float *kic_qp, int32_t *idx,
+                                  float *sel_scores, void *ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+/* hyb_attn_fwd over 4-bit K / V caches (codes [B, Nc, Hkv, d/2], qp [B, Nc,
+ * Hkv, 2]); results as hyb_attn_fwd on the dequantized caches.  When the
+ * query batch selects fewer rows than the cache holds (CSA, d = 128, Lq *
+ * topk < Nc) only the selected rows are dequantized into ws; otherwise the
+ * whole K and V caches are. */
+hyb_status hyb_attn_fwd_fp4(const hyb_problem *p, const void *q, const uint8_t *kc_codes,
+                            const float *kc_qp, const uint8_t *vc_codes, const float *vc_qp,
+                            const int32_t *idx, const void *k_raw, const void *v_raw, void *o,
+                            float *lse, void *ws, size_t ws_bytes, cudaStream_t stream);
+/* hyb_decode_append with 4-bit caches: a closing block is merged into its
+ * bf16 entry as in hyb_decode_append, and each (entry, head) row of it is
+ * then quantized as hyb_fp4_quantize does.  Requires d, di <= 256. */
+hyb_status hyb_decode_append_fp4(const hyb_problem *p, const int32_t *t_new, const void *k_new,
+                                 const void *v_new, const void *ki_new, const float *wk,
+                                 const float *wv, const float *wib, void *k_ring, void *v_ring,
+                                 void *ki_ring, uint8_t *kc_codes, float *kc_qp,
+                                 uint8_t *vc_codes, float *vc_qp, uint8_t *kic_codes,
+                                 float *kic_qp, int32_t *kv_pos0, cudaStream_t stream);
+
 
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device (HYB_OK, HYB_ERR_DEVICE_TIMEOUT or HYB_ERR_DEVICE_BOUNDS). */

@@ -27,7 +27,9 @@ def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
     assert {"hyb_hca_compress", "hyb_csa_index_topk", "hyb_attn_fwd", "hyb_fused_fwd",
             "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string",
-            "hyb_decode_append", "hyb_gated_fwd", "hyb_gated_workspace_size"} <= set(names)
+            "hyb_decode_append", "hyb_gated_fwd", "hyb_gated_workspace_size",
+            "hyb_fp4_quantize", "hyb_fp4_dequantize", "hyb_fp4_workspace_size",
+            "hyb_csa_index_topk_fp4", "hyb_attn_fwd_fp4", "hyb_decode_append_fp4"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -89,3 +91,28 @@ def test_gated_argument_checks(lib):
     assert hb._lib.hyb_gated_workspace_size(ctypes.byref(p)) == 3 * ((16 * 4 * 64 * 2 + 255) // 256 * 256)
     assert hb._lib.hyb_gated_fwd(ctypes.byref(p), buf, buf, buf, buf, buf, buf, buf, buf, None, 0,
                                  None) == hb.HYB_ERR_WORKSPACE
+
+
+def test_fp4_argument_checks(lib):
+    import compressed_sparse_sliding_b200 as hb
+    buf = ctypes.c_void_p(256)
+    # row widths the quantizer handles: 64, 128, 256 channels
+    assert hb._lib.hyb_fp4_quantize(buf, 4, 96, buf, buf, None) == hb.HYB_ERR_UNSUPPORTED
+    assert hb._lib.hyb_fp4_quantize(None, 4, 64, buf, buf, None) == hb.HYB_ERR_INVALID_ARG
+    assert hb._lib.hyb_fp4_dequantize(buf, buf, 4, 12, buf, None) == hb.HYB_ERR_INVALID_ARG
+    # decode (Lq * topk < Nc): workspace = the selected K rows, then V rows, bf16
+    p = hb.problem(B=2, Lq=1, Lkv=256, Hq=64, Hkv=1, d=128, m=4, W=128, topk=64, Hi=4, di=64, Nc=512)
+    attn = 2 * ((2 * 64 * 128 * 2 + 255) // 256 * 256)
+    index = (2 * 1 * 512 * 4 + 255) // 256 * 256          # scores; keys dequantized on chip
+    assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
+    # prefill: the whole caches are dequantized
+    p = hb.problem(B=1, Lq=64, Lkv=64, Hq=4, Hkv=1, d=64, m=4, W=8, topk=4, Hi=2, di=32, Nc=16)
+    attn = 2 * ((16 * 64 * 2 + 255) // 256 * 256)
+    index = (64 * 16 * 4 + 255) // 256 * 256 + (16 * 32 * 2 + 255) // 256 * 256
+    assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
+    assert hb._lib.hyb_attn_fwd_fp4(ctypes.byref(p), *([buf] * 10), None, 0, None) == hb.HYB_ERR_WORKSPACE
+    assert hb._lib.hyb_csa_index_topk_fp4(ctypes.byref(p), *([buf] * 5), None, None, 0,
+                                          None) == hb.HYB_ERR_WORKSPACE
+    # the append shares the checks of hyb_decode_append
+    p = hb.problem(B=1, Lq=1, Lkv=8, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=16)
+    assert hb._lib.hyb_decode_append_fp4(ctypes.byref(p), *([buf] * 17), None) == hb.HYB_ERR_INVALID_ARG
