@@ -347,6 +347,21 @@ def kernel_traffic(kernel: str, config_no: int):
         return None
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (each rank's time is its own
+    device time; the job takes as long as its slowest replica)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(w, rank: int) -> int:
+    """Seed of a replica's synthetic inputs: every rank its own batch."""
+    return 20260 + w.no + 1000 * rank
+
+
 def gate_logits(w, device, rank=0):
     """Seeded gate logits [B, L, Hq, 3] for the gated variant (N(0, 2^2))."""
     g = torch.Generator(device="cpu")
@@ -358,7 +373,7 @@ def run_gpu(args, rank, world):
     import compressed_sparse_sliding_b200 as hb
     w = WORKLOADS[args.config]
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp = make_inputs(w, device=dev, seed=20260 + w.no + 1000 * rank)
+    inp = make_inputs(w, device=dev, seed=replica_seed(w, rank))
     if not w.is_decode:
         inp["k_raw"], inp["v_raw"] = inp["k"], inp["v"]
     gated = args.variant == "gated"
@@ -409,11 +424,7 @@ def run_gpu(args, rank, world):
     if st != 0:
         raise RuntimeError(f"device status after timing: {hb.hyb_error_string(st)}")
 
-    total_ms = float(sum(tot))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(tot)), world, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.B * w.Lq * world
     value = tokens / (ms_per_step / 1e3)
@@ -495,11 +506,7 @@ def run_gpu(args, rank, world):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
 
     peaks = load_peaks()
     att_ms = statistics.mean(att)
