@@ -26,6 +26,8 @@ Parity status per function (what pins it, in tests/test_oracle_*.py):
                     branch), the output is the gate-weighted combination
   fp4_quantize /    exact levels, ties to even, constant rows, nibble order,
   fp4_dequantize    the half-step error bound, nearest level by brute force
+  backward.*        (oracle/backward.py) attention and block_merge gradients:
+                    central finite differences of the scalar losses in fp64
 """
 from __future__ import annotations
 
