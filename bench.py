@@ -139,8 +139,8 @@ class Step:
     """One forward pass as the three C-ABI stages on one stream, with CUDA
     events between the stages (the same kernels hyb_fused_fwd launches)."""
 
-    def __init__(self, hb, w, inp, gated=False, fp4=False):
-        self.hb, self.w, self.inp, self.gated, self.fp4 = hb, w, inp, gated, fp4
+    def __init__(self, hb, w, inp, gated=False, fp4=False, train=False):
+        self.hb, self.w, self.inp, self.gated, self.fp4, self.train = hb, w, inp, gated, fp4, train
         dev = inp["q"].device
         self.kv0 = torch.empty((w.B,), dtype=torch.int32, device=dev)
         self.p = problem_for(hb, w, inp, self.kv0)
@@ -169,7 +169,17 @@ class Step:
             self.p_sel.W = 0
             gneed = hb.hyb_gated_workspace_size(self.p)
             self.gws = torch.empty(max(gneed, 256), dtype=torch.uint8, device=dev)
-        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        if train:
+            # the backward of the step: a seeded output gradient, lse from the forward
+            self.lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+            gen = torch.Generator(device="cpu")
+            gen.manual_seed(30260 + w.no)
+            self.dout = torch.randn(self.o.shape, generator=gen).to(torch.bfloat16).to(dev)
+            self.bws = torch.empty(max(hb._lib.hyb_hca_compress_bwd_workspace_size(w.d, w.m), 256),
+                                   dtype=torch.uint8, device=dev)
+            self.dwk = torch.empty((w.m, w.d), dtype=torch.float32, device=dev)
+            self.dwv = torch.empty_like(self.dwk)
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         self.launches = 0
 
     def run(self, stream):
@@ -206,6 +216,23 @@ class Step:
                                   idx=self.idx, ws=self.ws, stream=stream)
             launches += 2
         ev[2].record(stream)
+        if self.train:
+            hb.hyb_attn_fwd(self.p, inp["q"], self.kc, self.vc, self.idx, inp["k"], inp["v"], o=self.o,
+                            lse=self.lse, stream=stream)
+            launches += 1
+            ev[3].record(stream)
+            # backward: attention (window and compressed paths), then block_merge of K and V,
+            # whose x gradients add into the raw K / V gradients
+            self.grads = hb.hyb_attn_bwd(self.p, inp["q"], self.kc, self.vc, self.idx, inp["k"], inp["v"],
+                                         self.o, self.lse, self.dout, stream=stream)
+            hb.hyb_hca_compress_bwd(inp["k"], inp["wk"], w.m, self.grads["dkc"], dx=self.grads["dk_raw"],
+                                    dw=self.dwk, ws=self.bws, stream=stream)
+            hb.hyb_hca_compress_bwd(inp["v"], inp["wv"], w.m, self.grads["dvc"], dx=self.grads["dv_raw"],
+                                    dw=self.dwv, ws=self.bws, stream=stream)
+            launches += 5
+            ev[4].record(stream)
+            self.launches = launches
+            return
         if self.fp4:
             hb.hyb_attn_fwd_fp4(self.p, inp["q"], self.kq, self.vq, self.idx, inp["k_ring"], inp["v_ring"],
                                 o=self.o, ws=self.fws, stream=stream)
@@ -224,8 +251,9 @@ class Step:
 
     def times_ms(self):
         e = self.ev
-        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
-                e[2].elapsed_time(e[3]))
+        last = e[4] if self.train else e[3]
+        return (e[0].elapsed_time(last), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                e[2].elapsed_time(e[3]), e[3].elapsed_time(e[4]) if self.train else 0.0)
 
 
 class ClockSampler:
@@ -378,10 +406,11 @@ def run_gpu(args, rank, world):
         inp["k_raw"], inp["v_raw"] = inp["k"], inp["v"]
     gated = args.variant == "gated"
     fp4 = args.variant == "fp4"
+    train = args.variant == "train"
     if gated:
         inp["gate"] = gate_logits(w, dev, rank)
     stream = torch.cuda.current_stream()
-    step = Step(hb, w, inp, gated, fp4)
+    step = Step(hb, w, inp, gated, fp4, train)
     # L2 flush: write 256 MiB, then read another 256 MiB so that no dirty line
     # of the flush buffer is left for the timed step to write back
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -407,14 +436,14 @@ def run_gpu(args, rank, world):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    tot, comp, idx, att = [], [], [], []
+    tot, comp, idx, att, back = [], [], [], [], []
     launches = 0
     for _ in range(args.steps):
         flush_l2()  # outside the step's events
         step.run(stream)
         torch.cuda.synchronize()
-        a, b, c, d = step.times_ms()
-        tot.append(a); comp.append(b); idx.append(c); att.append(d)
+        a, b, c, d, e = step.times_ms()
+        tot.append(a); comp.append(b); idx.append(c); att.append(d); back.append(e)
         launches += step.launches
     torch.cuda.synchronize()
     if world > 1:
@@ -452,6 +481,14 @@ def run_gpu(args, rank, world):
     def e2e_step():
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
+        if train:
+            # the training step through the public calls, on the copied inputs
+            saved = step.inp
+            step.inp = dict(saved, **dev_in)
+            step.run(stream)
+            step.inp = saved
+            o_host.copy_(step.grads["dq"].to(torch.bfloat16), non_blocking=True)
+            return
         p = problem_for(hb, w, dev_in, kv0_e2e)
         if gated:
             # the public calls of the gated variant: compression, the selection
@@ -511,7 +548,17 @@ def run_gpu(args, rank, world):
     peaks = load_peaks()
     att_ms = statistics.mean(att)
     hbm_bound = w.is_decode or w.no == 2
-    if hbm_bound:
+    if train:
+        # the attention backward on CUDA cores: 10 d FLOP per (query head, key)
+        # (the scores again, dP, dq, dk, dv); peak = 148 SMs x 128 fp32 lanes x
+        # 2 FLOP x the clock measured during the run
+        bwd_ms = statistics.mean(back)
+        mhz = (clocks or {}).get("sm_mhz") or 1965.0
+        peak = round(148 * 128 * 2 * mhz * 1e6 / 1e12, 1)
+        achieved = 2.5 * counts["attn_flop"] / (bwd_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4)}
+    elif hbm_bound:
         achieved = counts["attn_bytes"] / (att_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -526,8 +573,10 @@ def run_gpu(args, rank, world):
         kname = "hyb_gated_fwd (three attention kernels + combine)"
     if fp4:
         kname = "hyb_attn_fwd_fp4 (fp4_gather_kernel + csa_attn_kernel)"
+    if train:
+        kname = "attn_bwd_kernel"
     roof["kernel"] = kname
-    roof["peak_source"] = peaks["source"]
+    roof["peak_source"] = "derived (unit counts x measured clock)" if train else peaks["source"]
     roof["traffic"] = kernel_traffic(kname, w.no)
     stages = {("append_ms" if w.is_decode else "compress_ms"): round(statistics.mean(comp), 4),
               "index_topk_ms": round(statistics.mean(idx), 4),
@@ -537,6 +586,8 @@ def run_gpu(args, rank, world):
     if w.topk and statistics.mean(idx) > 0:
         stages["index_topk_TFLOPs"] = round(counts["idx_flop"] / (statistics.mean(idx) / 1e3) / 1e12, 2)
     stages["attention_TFLOPs"] = round(counts["attn_flop"] / (att_ms / 1e3) / 1e12, 1)
+    if train:
+        stages["backward_ms"] = round(statistics.mean(back), 4)
     stages["attention_GBps"] = round(counts["attn_bytes"] / (att_ms / 1e3) / 1e9, 1)
 
     res = {
@@ -559,7 +610,7 @@ def run_gpu(args, rank, world):
 
 
 # ----------------------------------------------------------------- CPU oracle
-def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False, fp4=False):
+def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False, fp4=False, train=False):
     """Times the oracle on a bounded sample of the workload.  Compression of
     the whole batch is timed once and charged per query token; indexer, top-K
     and attention are timed on a sample of query rows.  fp4: the decode caches
@@ -626,11 +677,32 @@ def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False, fp4=False):
             break
         n = min(total_rows, int(n * max(2.0, (budget_s / 2) / max(dt, 1e-3))))
     per_row = t_comp / total_rows + dt / len(rows)
+    note = ""
+    if train:
+        # the backward oracle works on one whole sequence (dense masked form)
+        if w.L * (w.Nc + w.L) * 8 <= (1 << 28):
+            from oracle import backward as bwd
+            f64 = lambda t: t.double().numpy()
+            t1 = time.perf_counter()
+            bwd.attention_bwd(f64(inp["q"][0]), kc_f64(kc, 0), kc_f64(vc, 0), f64(inp["k"][0]), f64(inp["v"][0]),
+                              w.m, w.W, np.ones((w.L, w.Hq, w.d)), idx=None)
+            for x, wt in ((inp["k"], inp["wk"]), (inp["v"], inp["wv"])):
+                bwd.block_merge_bwd(f64(x[:1]), wt.double().numpy(), w.m, np.ones((1, w.Nc, w.Hkv, w.d)))
+            per_row += (time.perf_counter() - t1) / w.Lq
+            note = "; backward of one sequence (dense masked oracle) charged per token"
+        else:
+            note = "; backward not sampled (the dense backward oracle is too large for this sequence length)"
     return {"value": round(1.0 / per_row, 3), "unit": "query-tokens/s", "cores": cores,
             "kind": "oracle",
             "sample": (f"{len(rows)} of {total_rows} query rows (indexer, top-K, attention) + " +
                        (f"cache maintenance of the new tokens ({t_comp:.2f} s)" if w.is_decode else
-                        f"compression of the whole batch ({t_comp:.2f} s)") + " charged per token")}
+                        f"compression of the whole batch ({t_comp:.2f} s)") + " charged per token" + note)}
+
+
+def kc_f64(bits, b):
+    """One sequence of a bf16-bits cache as fp64."""
+    import oracle
+    return oracle.bf16_to_f64(bits[b])
 
 
 def run_reference_arm(args):
@@ -639,10 +711,11 @@ def run_reference_arm(args):
     base = None
     gated = args.variant == "gated"
     fp4 = args.variant == "fp4"
+    train = args.variant == "train"
     for _ in range(args.warmup):
-        run_oracle(w, budget_s=2.0, rows_hint=4, gated=gated, fp4=fp4)
+        run_oracle(w, budget_s=2.0, rows_hint=4, gated=gated, fp4=fp4, train=train)
     for _ in range(args.steps):
-        base = run_oracle(w, budget_s=6.0, rows_hint=8, gated=gated, fp4=fp4)
+        base = run_oracle(w, budget_s=6.0, rows_hint=8, gated=gated, fp4=fp4, train=train)
         per_step.append(1.0 / base["value"])
     value = 1.0 / statistics.mean(per_step)
     cpu = dict(base)
@@ -669,15 +742,18 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated", "fp4"],
+    ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated", "fp4", "train"],
                     help="gated: the three-branch variant (CSA workloads with prefill); "
-                         "fp4: decode over 4-bit compressed caches (config 5)")
+                         "fp4: decode over 4-bit compressed caches (config 5); "
+                         "train: forward + backward (prefill workloads)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.variant == "gated" and (not WORKLOADS[args.config].topk or WORKLOADS[args.config].is_decode):
         ap.error("--variant gated needs a CSA prefill workload (configs 1 and 3)")
     if args.variant == "fp4" and not WORKLOADS[args.config].is_decode:
         ap.error("--variant fp4 needs the decode workload (config 5)")
+    if args.variant == "train" and WORKLOADS[args.config].is_decode:
+        ap.error("--variant train needs a prefill workload (configs 1-4)")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -698,7 +774,7 @@ def main():
         res = run_gpu(args, rank, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = run_oracle(WORKLOADS[args.config], gated=args.variant == "gated",
-                                             fp4=args.variant == "fp4")
+                                             fp4=args.variant == "fp4", train=args.variant == "train")
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -16,6 +16,8 @@ Entry points (same names as the C ABI):
   hyb_gated_fwd        the gated three-branch variant (compressed, selected, window)
   hyb_fp4_*            4-bit compressed caches: quantize / dequantize, and the
                        indexer, attention and decode append over them
+  hyb_attn_bwd,        gradients for training: through the attention (fixed
+  hyb_hca_compress_bwd selection) and through block_merge
   hyb_workspace_size, hyb_get_device_status, hyb_error_string
 """
 from __future__ import annotations
@@ -88,6 +90,12 @@ try:
     _lib.hyb_attn_fwd_fp4.restype = _I
     _lib.hyb_decode_append_fp4.argtypes = [_PP] + [_P] * 18
     _lib.hyb_decode_append_fp4.restype = _I
+    _lib.hyb_attn_bwd.argtypes = [_PP] + [_P] * 15
+    _lib.hyb_attn_bwd.restype = _I
+    _lib.hyb_hca_compress_bwd_workspace_size.argtypes = [_I, _I]
+    _lib.hyb_hca_compress_bwd_workspace_size.restype = ctypes.c_size_t
+    _lib.hyb_hca_compress_bwd.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    _lib.hyb_hca_compress_bwd.restype = _I
     _lib.hyb_get_device_status.argtypes = [_P]
     _lib.hyb_get_device_status.restype = _I
     _lib.hyb_error_string.argtypes = [_I]
@@ -303,6 +311,41 @@ def hyb_decode_append_fp4(p: HybProblem, t_new, k_new, v_new, k_ring, v_ring, kc
                                     _stream(stream))
     _check(st, "hyb_decode_append_fp4")
     return kv_pos0
+
+
+def hyb_attn_bwd(p: HybProblem, q, kc, vc, idx, k_raw, v_raw, o, lse, dout, stream=None):
+    """Gradients of sum(dout * o) through hyb_attn_fwd (o, lse: its outputs;
+    the selection idx is taken as fixed).  Returns dict(dq, dkc, dvc, dk_raw,
+    dv_raw), fp32 tensors shaped like q, kc, vc, k_raw, v_raw."""
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = dict(dq=torch.empty(q.shape, **f32), dk_raw=torch.empty(k_raw.shape, **f32),
+             dv_raw=torch.empty(v_raw.shape, **f32),
+             dkc=torch.empty(kc.shape, **f32) if kc is not None else None,
+             dvc=torch.empty(vc.shape, **f32) if vc is not None else None)
+    st = _lib.hyb_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(kc), _ptr(vc), _ptr(idx), _ptr(k_raw), _ptr(v_raw),
+                           _ptr(o), _ptr(lse), _ptr(dout), _ptr(g["dq"]), _ptr(g["dkc"]), _ptr(g["dvc"]),
+                           _ptr(g["dk_raw"]), _ptr(g["dv_raw"]), _stream(stream))
+    _check(st, "hyb_attn_bwd")
+    return g
+
+
+def hyb_hca_compress_bwd(x: torch.Tensor, w: torch.Tensor, m: int, dc: torch.Tensor,
+                         dx: Optional[torch.Tensor] = None, dw: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of sum(dc * hyb_hca_compress(x, w, m)): adds the x gradient
+    into dx (fp32, zero-initialised when not given) and returns (dx, dw)."""
+    B, L, H, D = x.shape if x.dim() == 4 else (x.shape[0], x.shape[1], 1, x.shape[2])
+    if dx is None:
+        dx = torch.zeros(x.shape, dtype=torch.float32, device=x.device)
+    if dw is None:
+        dw = torch.empty((m, D), dtype=torch.float32, device=x.device)
+    need = max(int(_lib.hyb_hca_compress_bwd_workspace_size(D, m)), 256)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=x.device)
+    st = _lib.hyb_hca_compress_bwd(_ptr(x), B, L, H, D, m, _ptr(w), _ptr(dc), _ptr(dx), _ptr(dw), _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    _check(st, "hyb_hca_compress_bwd")
+    return dx, dw
 
 
 def hyb_gated_workspace_size(p: HybProblem) -> int:

@@ -46,6 +46,9 @@ cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, i
                                cudaStream_t stream);
 
 cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream);
+cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream);
+cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, int m, const float *w,
+                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream);
 cudaError_t launch_gated_combine(const void *o1, const void *o2, const void *o3, const float *gate,
                                  void *o, long long rows, int d, cudaStream_t stream, int num_sms);
 
@@ -470,6 +473,95 @@ hyb_status hyb_attn_fwd_fp4(const hyb_problem *p, const void *q, const uint8_t *
     if (e != cudaSuccess)
         return cuda_status(e);
     return hyb_attn_fwd(p, q, wk, wk + half, idx, k_raw, v_raw, o, lse, stream);
+}
+
+hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                        const int32_t *idx, const void *k_raw, const void *v_raw, const void *o,
+                        const float *lse, const void *dout, float *dq, float *dkc, float *dvc,
+                        float *dk_raw, float *dv_raw, cudaStream_t stream)
+{
+    hyb_status st = check_problem(p, false);
+    if (st != HYB_OK)
+        return st;
+    if (!q || !o || !lse || !dout || !dq || !dk_raw || !dv_raw || !k_raw || !v_raw)
+        return HYB_ERR_INVALID_ARG;
+    if (p->Nc > 0 && (!kc || !vc || !dkc || !dvc))
+        return HYB_ERR_INVALID_ARG;
+    if (idx && p->topk <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (p->Lkv <= 0)
+        return HYB_ERR_INVALID_ARG;
+    const size_t ck = (size_t)p->B * p->Nc * p->Hkv * p->d * sizeof(float);
+    const size_t rk = (size_t)p->B * p->Lkv * p->Hkv * p->d * sizeof(float);
+    cudaError_t e = cudaSuccess;
+    if (ck) {
+        e = cudaMemsetAsync(dkc, 0, ck, stream);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(dvc, 0, ck, stream);
+    }
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(dk_raw, 0, rk, stream);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(dv_raw, 0, rk, stream);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    BwdParams b;
+    b.B = p->B;
+    b.Lq = p->Lq;
+    b.Lkv = p->Lkv;
+    b.Hq = p->Hq;
+    b.Hkv = p->Hkv;
+    b.g = p->Hq / p->Hkv;
+    b.d = p->d;
+    b.Nc = p->Nc;
+    b.m = p->m;
+    b.W = p->W;
+    b.topk = idx ? p->topk : 0;
+    b.scale = softmax_scale(p);
+    b.q_pos = p->q_pos;
+    b.kv_pos0 = p->kv_pos0;
+    b.idx = idx;
+    b.q = static_cast<const __nv_bfloat16 *>(q);
+    b.kc = static_cast<const __nv_bfloat16 *>(kc);
+    b.vc = static_cast<const __nv_bfloat16 *>(vc);
+    b.kr = static_cast<const __nv_bfloat16 *>(k_raw);
+    b.vr = static_cast<const __nv_bfloat16 *>(v_raw);
+    b.o = static_cast<const __nv_bfloat16 *>(o);
+    b.dout = static_cast<const __nv_bfloat16 *>(dout);
+    b.lse = lse;
+    b.dq = dq;
+    b.dkc = dkc;
+    b.dvc = dvc;
+    b.dkr = dk_raw;
+    b.dvr = dv_raw;
+    return cuda_status(launch_attn_bwd(b, stream));
+}
+
+size_t hyb_hca_compress_bwd_workspace_size(int dx, int m)
+{
+    if (dx <= 0 || m <= 0)
+        return 0;
+    return ((size_t)m * dx * sizeof(float) + 255) & ~(size_t)255;
+}
+
+hyb_status hyb_hca_compress_bwd(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                                const float *dc, float *dx_acc, float *dw, void *ws, size_t ws_bytes,
+                                cudaStream_t stream)
+{
+    if (!x || !w || !dc || !dx_acc || !dw || B <= 0 || L < 0 || H <= 0 || dx <= 0 || m <= 0)
+        return HYB_ERR_INVALID_ARG;
+    if (dx % 32 != 0)
+        return HYB_ERR_UNSUPPORTED;
+    if (m > 256)
+        return HYB_ERR_UNSUPPORTED;
+    const size_t need = hyb_hca_compress_bwd_workspace_size(dx, m);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return HYB_ERR_WORKSPACE;
+    float *G = static_cast<float *>(ws);
+    cudaError_t e = cudaMemsetAsync(G, 0, (size_t)m * dx * sizeof(float), stream);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(launch_block_merge_bwd(x, B, L, H, dx, m, w, dc, dx_acc, dw, G, stream));
 }
 
 size_t hyb_gated_workspace_size(const hyb_problem *p)

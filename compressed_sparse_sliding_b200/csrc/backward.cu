@@ -1,0 +1,311 @@
+// backward.cu -- gradients for training (Tiny-R2 README, "Training"): the
+// hybrid attention step and block_merge.  The top-K selection is taken as
+// fixed (the pages define no gradient for it).
+//
+// Attention, per query row with key set S (the forward's: selected or all
+// visible compressed entries, and the raw window), with the forward's lse:
+//     P_j = exp(scale q.k_j - lse),  dP_j = dO.v_j,  D = dO.o = sum_j P_j dP_j
+//     dS_j = P_j (dP_j - D)
+//     dq = scale sum_j dS_j k_j,  dk_j += scale dS_j q,  dv_j += P_j dO
+// One CTA per (token, KV head): warp w holds heads w, w + 8, ... of the group
+// (q, dO and the dq accumulators in registers; lane = d/32 channels).  Keys go
+// four at a time: each warp adds its heads' dk / dv parts into shared
+// memory, then the CTA adds the keys' sums to the fp32 gradients with one
+// atomic per element.  CUDA cores throughout: a correct first form.
+//
+// block_merge, c_j = sum_i P[i] x_{jm+i} with P = softmax over i of w (per
+// channel):  dx_{jm+i} += P[i] dc_j  (each raw row belongs to one block, so
+// plain read-modify-write), dw[i] = P[i] (G[i] - sum_k P[k] G[k]) with
+// G[i] = sum over blocks, batches, heads of dc_j x_{jm+i}; a CTA owns 32
+// channels and a run of rows, reduces its share of G in shared memory and
+// adds it to a global G with one atomic per (i, channel); a last small
+// kernel forms dw from G.
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kBwWarps = 8;
+constexpr int kBwKeys = 4;      // keys per shared-memory round (2 x 16 KB of partials)
+
+struct BwdParams {
+    int B, Lq, Lkv, Hq, Hkv, g, d, Nc, m, W, topk;
+    float scale;
+    const int32_t *q_pos, *kv_pos0, *idx;
+    const __nv_bfloat16 *q, *kc, *vc, *kr, *vr, *o, *dout;
+    const float *lse;
+    float *dq, *dkc, *dvc, *dkr, *dvr;
+};
+
+__device__ __forceinline__ float bw_warp_sum(float v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+template <int CPL, int HPW>
+__global__ void __launch_bounds__(32 * kBwWarps)
+attn_bwd_kernel(const BwdParams p)
+{
+    // item = (b, t, KV head)
+    const long long item = blockIdx.x;
+    const int kvh = (int)(item % p.Hkv);
+    const long long bt = item / p.Hkv;
+    const int b = (int)(bt / p.Lq), t = (int)(bt % p.Lq);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d = 32 * CPL;
+    const long long pos = p.q_pos ? p.q_pos[bt] : t;
+    const long long kv0 = p.kv_pos0 ? p.kv_pos0[b] : 0;
+    long long lo = pos - p.W + 1;
+    if (lo < 0)
+        lo = 0;
+    lo -= kv0;
+    if (lo < 0)
+        lo = 0;
+    long long hi = pos - kv0;
+    if (hi > p.Lkv - 1)
+        hi = p.Lkv - 1;
+    const int nwin = (p.W > 0 && hi >= lo) ? (int)(hi - lo + 1) : 0;
+    const long long wstart = pos - p.W + 1;
+    int nvis = 0;
+    if (wstart > 0)
+        nvis = (int)min((long long)p.Nc, wstart / p.m);
+    const int ncomp = p.idx ? p.topk : nvis;
+
+    // this warp's heads: h = warp + kBwWarps * e
+    float qv[HPW][CPL], dov[HPW][CPL], dqv[HPW][CPL], lse[HPW], Dh[HPW];
+#pragma unroll
+    for (int e = 0; e < HPW; ++e) {
+        const int h = warp + kBwWarps * e;
+        const bool on = h < p.g;
+        const size_t row = ((size_t)bt * p.Hq + (size_t)kvh * p.g + (on ? h : 0)) * d + lane * CPL;
+        float od = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            qv[e][c] = on ? __bfloat162float(p.q[row + c]) : 0.f;
+            dov[e][c] = on ? __bfloat162float(p.dout[row + c]) : 0.f;
+            od += on ? dov[e][c] * __bfloat162float(p.o[row + c]) : 0.f;
+            dqv[e][c] = 0.f;
+        }
+        Dh[e] = bw_warp_sum(od);
+        lse[e] = on ? p.lse[((size_t)b * p.Hq + (size_t)kvh * p.g + h) * p.Lq + t] : -INFINITY;
+    }
+
+    __shared__ float sdk[kBwKeys][kBwWarps][128];
+    __shared__ float sdv[kBwKeys][kBwWarps][128];
+    __shared__ long long srow[kBwKeys];     // source row of each key (-1: none)
+    __shared__ int scomp[kBwKeys];          // compressed (1) or raw (0)
+    const int total = ncomp + nwin;
+    for (int k0 = 0; k0 < total; k0 += kBwKeys) {
+        if (threadIdx.x < kBwKeys) {
+            const int kk = k0 + threadIdx.x;
+            long long r = -1;
+            int comp = 0;
+            if (kk < ncomp) {
+                comp = 1;
+                int j = p.idx ? p.idx[(size_t)bt * p.topk + kk] : kk;
+                if (p.idx && j >= p.Nc)
+                    set_error(HYB_ERR_DEVICE_BOUNDS);
+                const bool v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < wstart);
+                r = v ? ((long long)b * p.Nc + j) * p.Hkv + kvh : -1;
+            } else if (kk < total) {
+                r = ((long long)b * p.Lkv + lo + (kk - ncomp)) * p.Hkv + kvh;
+            }
+            srow[threadIdx.x] = r;
+            scomp[threadIdx.x] = comp;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int u = 0; u < kBwKeys; ++u) {
+            const long long r = srow[u];
+            float dkp[CPL], dvp[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                dkp[c] = 0.f;
+                dvp[c] = 0.f;
+            }
+            if (r >= 0) {
+                const __nv_bfloat16 *kp = (scomp[u] ? p.kc : p.kr) + r * d + lane * CPL;
+                const __nv_bfloat16 *vp = (scomp[u] ? p.vc : p.vr) + r * d + lane * CPL;
+                float kv[CPL], vv[CPL];
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    kv[c] = __bfloat162float(kp[c]);
+                    vv[c] = __bfloat162float(vp[c]);
+                }
+#pragma unroll
+                for (int e = 0; e < HPW; ++e) {
+                    if (warp + kBwWarps * e >= p.g)
+                        continue;
+                    float s = 0.f, dp = 0.f;
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+                        s = fmaf(qv[e][c], kv[c], s);
+                        dp = fmaf(dov[e][c], vv[c], dp);
+                    }
+                    s = bw_warp_sum(s);
+                    dp = bw_warp_sum(dp);
+                    const float pr = expf(s * p.scale - lse[e]);
+                    const float ds = pr * (dp - Dh[e]);
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+                        dqv[e][c] = fmaf(ds, kv[c], dqv[e][c]);
+                        dkp[c] = fmaf(ds, qv[e][c], dkp[c]);
+                        dvp[c] = fmaf(pr, dov[e][c], dvp[c]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                sdk[u][warp][lane * CPL + c] = dkp[c];
+                sdv[u][warp][lane * CPL + c] = dvp[c];
+            }
+        }
+        __syncthreads();
+        // thread -> (key, channel) sums over the warps, one atomic each
+        for (int e = threadIdx.x; e < kBwKeys * d; e += 32 * kBwWarps) {
+            const int u = e / d, c = e % d;
+            const long long r = srow[u];
+            if (r < 0)
+                continue;
+            float sk = 0.f, sv = 0.f;
+#pragma unroll
+            for (int w = 0; w < kBwWarps; ++w) {
+                sk += sdk[u][w][c];
+                sv += sdv[u][w][c];
+            }
+            atomicAdd((scomp[u] ? p.dkc : p.dkr) + r * d + c, sk * p.scale);
+            atomicAdd((scomp[u] ? p.dvc : p.dvr) + r * d + c, sv);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int e = 0; e < HPW; ++e) {
+        const int h = warp + kBwWarps * e;
+        if (h >= p.g)
+            continue;
+        const size_t row = ((size_t)bt * p.Hq + (size_t)kvh * p.g + h) * d + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+            p.dq[row + c] = dqv[e][c] * p.scale;
+    }
+}
+
+template <int CPL>
+static cudaError_t launch_attn_bwd_c(const BwdParams &p, long long items, cudaStream_t stream)
+{
+    const int hpw = (p.g + kBwWarps - 1) / kBwWarps;
+    if (hpw <= 1)
+        attn_bwd_kernel<CPL, 1><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
+    else if (hpw <= 2)
+        attn_bwd_kernel<CPL, 2><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
+    else if (hpw <= 4)
+        attn_bwd_kernel<CPL, 4><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
+    else
+        attn_bwd_kernel<CPL, 8><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
+{
+    const long long items = (long long)p.B * p.Lq * p.Hkv;
+    if (items <= 0)
+        return cudaSuccess;
+    if (items >= (1ll << 31) || p.g > 64)
+        return cudaErrorInvalidValue;
+    return p.d == 128 ? launch_attn_bwd_c<4>(p, items, stream) : launch_attn_bwd_c<2>(p, items, stream);
+}
+
+// ---------------------------------------------------------------- block_merge
+constexpr int kBmbRows = 64;    // (block, batch, head) rows per CTA
+
+// grid (dx / 32, row groups); warp w of the CTA takes rows w, w + 8, ... of
+// its group; lane = channel.  G partials in shared memory [m][32].
+__global__ void __launch_bounds__(256)
+block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
+                       const float *__restrict__ dc, float *__restrict__ dx, float *__restrict__ G,
+                       int B, int L, int H, int D, int m)
+{
+    extern __shared__ float bm_smem[];
+    float *sP = bm_smem;                  // [m][32] softmax weights of the CTA's channels
+    float *sG = bm_smem + m * 32;         // [m][32] G partials
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + lane;
+    const int Nc = L / m;
+    const long long rows = (long long)B * Nc * H;
+    if (warp == 0) {
+        float mx = -INFINITY;
+        for (int i = 0; i < m; ++i)
+            mx = fmaxf(mx, w[(size_t)i * D + c]);
+        float den = 0.f;
+        for (int i = 0; i < m; ++i)
+            den += expf(w[(size_t)i * D + c] - mx);
+        for (int i = 0; i < m; ++i)
+            sP[i * 32 + lane] = expf(w[(size_t)i * D + c] - mx) / den;
+    }
+    for (int e = threadIdx.x; e < m * 32; e += 256)
+        sG[e] = 0.f;
+    __syncthreads();
+    const long long r0 = (long long)blockIdx.y * kBmbRows;
+    for (long long r = r0 + warp; r < r0 + kBmbRows && r < rows; r += 8) {
+        const int h = (int)(r % H);
+        const long long bj = r / H;
+        const int b = (int)(bj / Nc), j = (int)(bj % Nc);
+        const float g = dc[((size_t)bj * H + h) * D + c];
+        const size_t xrow0 = (((size_t)b * L + (size_t)j * m) * H + h) * D + c;
+        for (int i = 0; i < m; ++i) {
+            const size_t at = xrow0 + (size_t)i * H * D;
+            dx[at] += sP[i * 32 + lane] * g;
+            atomicAdd(&sG[i * 32 + lane], g * __bfloat162float(x[at]));
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < m * 32; e += 256)
+        atomicAdd(&G[(size_t)(e / 32) * D + blockIdx.x * 32 + (e % 32)], sG[e]);
+}
+
+// dw[i, c] = P[i, c] (G[i, c] - sum_k P[k, c] G[k, c]); thread per channel.
+__global__ void block_merge_dw_kernel(const float *__restrict__ w, const float *__restrict__ G,
+                                      float *__restrict__ dw, int D, int m)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= D)
+        return;
+    float mx = -INFINITY;
+    for (int i = 0; i < m; ++i)
+        mx = fmaxf(mx, w[(size_t)i * D + c]);
+    float den = 0.f;
+    for (int i = 0; i < m; ++i)
+        den += expf(w[(size_t)i * D + c] - mx);
+    float pg = 0.f;
+    for (int i = 0; i < m; ++i)
+        pg += expf(w[(size_t)i * D + c] - mx) / den * G[(size_t)i * D + c];
+    for (int i = 0; i < m; ++i) {
+        const float pi = expf(w[(size_t)i * D + c] - mx) / den;
+        dw[(size_t)i * D + c] = pi * (G[(size_t)i * D + c] - pg);
+    }
+}
+
+// G: m * D floats of workspace, zeroed by the caller.
+cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, int m, const float *w,
+                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream)
+{
+    const long long rows = (long long)B * (L / m) * H;
+    if (rows > 0) {
+        const long long groups = (rows + kBmbRows - 1) / kBmbRows;
+        if (groups > 65535)
+            return cudaErrorInvalidValue;
+        const size_t smem = (size_t)2 * m * 32 * sizeof(float);
+        dim3 grid(D / 32, (unsigned)groups);
+        block_merge_bwd_kernel<<<grid, 256, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x), w, dc, dx,
+                                                            G, B, L, H, D, m);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    block_merge_dw_kernel<<<(D + 127) / 128, 128, 0, stream>>>(w, G, dw, D, m);
+    return cudaGetLastError();
+}
+
+}  // namespace hyb

@@ -9,5 +9,6 @@
 #include "attn_sparse.cu"
 #include "decode_append.cu"
 #include "gated.cu"
+#include "backward.cu"
 #include "api.cu"
 #include "noalloc.cu"

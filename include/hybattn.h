@@ -200,6 +200,33 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
                          const float *gate, void *o, void *ws, size_t ws_bytes,
                          cudaStream_t stream);
 
+/* Backward pass for training (Tiny-R2 README, "Training"), with the top-K
+ * selection taken as fixed (the pages define no gradient for it).
+ * hyb_attn_bwd: gradients of sum(dout * o) through hyb_attn_fwd for the same
+ * problem and inputs; o [B, Lq, Hq, d] bf16 and lse [B, Hq, Lq] fp32 are
+ * that call's outputs, dout [B, Lq, Hq, d] bf16.  Per query row with key set
+ * S: P_j = exp(scale q.k_j - lse), dS_j = P_j (dout.v_j - dout.o),
+ * dq = scale sum_j dS_j k_j, dk_j += scale dS_j q, dv_j += P_j dout.
+ * Outputs fp32, caller-owned, overwritten: dq [B, Lq, Hq, d]; dkc, dvc
+ * [B, Nc, Hkv, d]; dk_raw, dv_raw [B, Lkv, Hkv, d] (the window path only:
+ * the path through the compression is hyb_hca_compress_bwd's). */
+hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
+                        const int32_t *idx, const void *k_raw, const void *v_raw, const void *o,
+                        const float *lse, const void *dout, float *dq, float *dkc, float *dvc,
+                        float *dk_raw, float *dv_raw, cudaStream_t stream);
+/* hyb_hca_compress_bwd: gradients of sum(dc * c), c = hyb_hca_compress(x, w,
+ * m): dx_acc [B, L, H, dx] fp32 += P[i] dc_j at row j m + i (rows of a
+ * trailing partial block get nothing), dw [m, dx] fp32 overwritten with
+ * P (G - sum_k P_k G_k), G[i] = sum of dc_j x_{jm+i} over blocks, batches and
+ * heads (P = softmax over positions of w, per channel).  dc [B, L/m, H, dx]
+ * fp32; x bf16 as the forward; dx a multiple of 32, m <= 256.  ws: device
+ * workspace of hyb_hca_compress_bwd_workspace_size(dx, m) bytes, 256-byte
+ * aligned. */
+size_t hyb_hca_compress_bwd_workspace_size(int dx, int m);
+hyb_status hyb_hca_compress_bwd(const void *x, int B, int L, int H, int dx, int m, const float *w,
+                                const float *dc, float *dx_acc, float *dw, void *ws, size_t ws_bytes,
+                                cudaStream_t stream);
+
 /* 4-bit compressed caches (CSDN code page, section 1, compress_to_fp4 /
  * decompress_from_fp4).  Every row of dx channels -- one compressed entry
  * of one head (K, V) or one indexer key -- is stored as dx/2 bytes of codes

@@ -29,7 +29,8 @@ def test_every_declared_symbol_is_exported(lib):
             "hyb_workspace_size", "hyb_get_device_status", "hyb_error_string",
             "hyb_decode_append", "hyb_gated_fwd", "hyb_gated_workspace_size",
             "hyb_fp4_quantize", "hyb_fp4_dequantize", "hyb_fp4_workspace_size",
-            "hyb_csa_index_topk_fp4", "hyb_attn_fwd_fp4", "hyb_decode_append_fp4"} <= set(names)
+            "hyb_csa_index_topk_fp4", "hyb_attn_fwd_fp4", "hyb_decode_append_fp4",
+            "hyb_attn_bwd", "hyb_hca_compress_bwd", "hyb_hca_compress_bwd_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -116,3 +117,18 @@ def test_fp4_argument_checks(lib):
     # the append shares the checks of hyb_decode_append
     p = hb.problem(B=1, Lq=1, Lkv=8, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=16)
     assert hb._lib.hyb_decode_append_fp4(ctypes.byref(p), *([buf] * 17), None) == hb.HYB_ERR_INVALID_ARG
+
+
+def test_backward_argument_checks(lib):
+    import compressed_sparse_sliding_b200 as hb
+    buf = ctypes.c_void_p(256)
+    p = hb.problem(B=1, Lq=16, Lkv=16, Hq=4, Hkv=1, d=64, m=4, W=8, Nc=4)
+    # lse is required (P is recomputed from it)
+    args = [buf] * 7 + [None] + [buf] * 6 + [None]
+    assert hb._lib.hyb_attn_bwd(ctypes.byref(p), *args) == hb.HYB_ERR_INVALID_ARG
+    # block_merge backward: channels in multiples of 32, a G buffer of m * dx floats
+    assert hb._lib.hyb_hca_compress_bwd_workspace_size(64, 4) == 1024
+    assert hb._lib.hyb_hca_compress_bwd(buf, 1, 8, 1, 48, 4, buf, buf, buf, buf, buf, 1024,
+                                        None) == hb.HYB_ERR_UNSUPPORTED
+    assert hb._lib.hyb_hca_compress_bwd(buf, 1, 8, 1, 64, 4, buf, buf, buf, buf, buf, 512,
+                                        None) == hb.HYB_ERR_WORKSPACE
