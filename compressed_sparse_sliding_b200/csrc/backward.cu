@@ -8,7 +8,8 @@
 //     dS_j = P_j (dP_j - D)
 //     dq = scale sum_j dS_j k_j,  dk_j += scale dS_j q,  dv_j += P_j dO
 // One CTA per (token, KV head): warp w holds heads w, w + 8, ... of the group
-// (q, dO and the dq accumulators in registers; lane = d/32 channels).  Keys go
+// (q, dO and the dq accumulators in registers; lane = d/32 channels); warps
+// without a head (groups of fewer than eight) only take part in the sums.  Keys go
 // four at a time: each warp adds its heads' dk / dv parts into shared
 // memory, then the CTA adds the keys' sums to the fp32 gradients with one
 // atomic per element.  CUDA cores throughout: a correct first form.
@@ -17,7 +18,8 @@
 // channel):  dx_{jm+i} += P[i] dc_j  (each raw row belongs to one block, so
 // plain read-modify-write), dw[i] = P[i] (G[i] - sum_k P[k] G[k]) with
 // G[i] = sum over blocks, batches, heads of dc_j x_{jm+i}; a CTA owns 32
-// channels and a run of rows, reduces its share of G in shared memory and
+// channels and eight rows (more when the grid would be too tall), reduces its
+// share of G in shared memory and
 // adds it to a global G with one atomic per (i, channel); a last small
 // kernel forms dw from G.
 #include "common.cuh"
@@ -97,6 +99,7 @@ attn_bwd_kernel(const BwdParams p)
     __shared__ long long srow[kBwKeys];     // source row of each key (-1: none)
     __shared__ int scomp[kBwKeys];          // compressed (1) or raw (0)
     const int total = ncomp + nwin;
+    const int nw = p.g < kBwWarps ? p.g : kBwWarps;   // warps holding a head
     for (int k0 = 0; k0 < total; k0 += kBwKeys) {
         if (threadIdx.x < kBwKeys) {
             const int kk = k0 + threadIdx.x;
@@ -117,7 +120,7 @@ attn_bwd_kernel(const BwdParams p)
         }
         __syncthreads();
 #pragma unroll 1
-        for (int u = 0; u < kBwKeys; ++u) {
+        for (int u = 0; u < kBwKeys && warp < nw; ++u) {
             const long long r = srow[u];
             float dkp[CPL], dvp[CPL];
 #pragma unroll
@@ -170,8 +173,7 @@ attn_bwd_kernel(const BwdParams p)
             if (r < 0)
                 continue;
             float sk = 0.f, sv = 0.f;
-#pragma unroll
-            for (int w = 0; w < kBwWarps; ++w) {
+            for (int w = 0; w < nw; ++w) {
                 sk += sdk[u][w][c];
                 sv += sdv[u][w][c];
             }
@@ -218,14 +220,12 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
 }
 
 // ---------------------------------------------------------------- block_merge
-constexpr int kBmbRows = 64;    // (block, batch, head) rows per CTA
-
-// grid (dx / 32, row groups); warp w of the CTA takes rows w, w + 8, ... of
-// its group; lane = channel.  G partials in shared memory [m][32].
+// grid (dx / 32, row groups of rpc rows); warp w of the CTA takes rows w,
+// w + 8, ... of its group; lane = channel.  G partials in shared memory [m][32].
 __global__ void __launch_bounds__(256)
 block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
                        const float *__restrict__ dc, float *__restrict__ dx, float *__restrict__ G,
-                       int B, int L, int H, int D, int m)
+                       int B, int L, int H, int D, int m, int rpc)
 {
     extern __shared__ float bm_smem[];
     float *sP = bm_smem;                  // [m][32] softmax weights of the CTA's channels
@@ -247,8 +247,8 @@ block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restr
     for (int e = threadIdx.x; e < m * 32; e += 256)
         sG[e] = 0.f;
     __syncthreads();
-    const long long r0 = (long long)blockIdx.y * kBmbRows;
-    for (long long r = r0 + warp; r < r0 + kBmbRows && r < rows; r += 8) {
+    const long long r0 = (long long)blockIdx.y * rpc;
+    for (long long r = r0 + warp; r < r0 + rpc && r < rows; r += 8) {
         const int h = (int)(r % H);
         const long long bj = r / H;
         const int b = (int)(bj / Nc), j = (int)(bj % Nc);
@@ -293,13 +293,15 @@ cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, in
 {
     const long long rows = (long long)B * (L / m) * H;
     if (rows > 0) {
-        const long long groups = (rows + kBmbRows - 1) / kBmbRows;
-        if (groups > 65535)
-            return cudaErrorInvalidValue;
+        // one row per warp where the grid allows, more rows per CTA beyond
+        long long rpc = 8;
+        while ((rows + rpc - 1) / rpc > 65535)
+            rpc += 8;
+        const long long groups = (rows + rpc - 1) / rpc;
         const size_t smem = (size_t)2 * m * 32 * sizeof(float);
         dim3 grid(D / 32, (unsigned)groups);
         block_merge_bwd_kernel<<<grid, 256, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x), w, dc, dx,
-                                                            G, B, L, H, D, m);
+                                                            G, B, L, H, D, m, (int)rpc);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
