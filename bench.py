@@ -693,10 +693,23 @@ def run_oracle(w, budget_s=12.0, rows_hint=None, gated=False, fp4=False, train=F
         else:
             note = "; backward not sampled (the dense backward oracle is too large for this sequence length)"
     return {"value": round(1.0 / per_row, 3), "unit": "query-tokens/s", "cores": cores,
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": (f"{len(rows)} of {total_rows} query rows (indexer, top-K, attention) + " +
                        (f"cache maintenance of the new tokens ({t_comp:.2f} s)" if w.is_decode else
                         f"compression of the whole batch ({t_comp:.2f} s)") + " charged per token" + note)}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (for the oracle baseline's record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def kc_f64(bits, b):
