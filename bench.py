@@ -7,8 +7,9 @@ One step = one pass of the whole forward path over one batch of the workload:
 block_merge of K, V (and indexer keys for CSA) -> indexer scores + exact top-K
 (CSA) -> hybrid attention.  A decode step starts instead with the cache
 maintenance of the new token (window ring append; the block it closes becomes
-a compressed entry) and reads the window from the ring.  Default workload: the HCA+SWA batch (B=2, L=8192,
-16 query / 16 KV heads, d=128, m=128, W=128).  Inputs are synthetic, seeded and
+a compressed entry) and reads the window from the ring.  Default workload: the
+CSA+SWA prefill (B=1, L=32768, 32 query heads sharing one KV head, d=128, m=4,
+top-K=512, W=128, indexer 4 heads x 64).  Inputs are synthetic, seeded and
 resident in HBM before the timed region; L2 is flushed between timed steps
 (a 256 MiB write, then a read of a separate 256 MiB buffer so that the step
 does not pay for writing back the flush's dirty lines), outside the per-step
@@ -40,7 +41,7 @@ import torch  # noqa: E402
 from workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "query-tokens/s"
-DEFAULT_CONFIG = 2
+DEFAULT_CONFIG = 3
 
 
 def load_peaks():

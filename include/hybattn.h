@@ -117,6 +117,10 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
  *   - Every GPU that loads the library holds the array until the process
  *     exits.  The first call on a device looks up the array's address with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process: do not use this entry
+ *     point after cudaDeviceReset() on that device, or from a CUDA context
+ *     other than the device's primary context (the library's copy of the
+ *     array lives at another address there).
  *   - All calls share the array: calls whose kernels overlap on the GPU (for
  *     example on different streams) race and must be serialised by the
  *     caller.  Nothing in it needs clearing between calls. */
@@ -139,7 +143,11 @@ hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, con
                         const int32_t *idx, const void *k_raw, const void *v_raw, void *o,
                         float *lse, cudaStream_t stream);
 
-/* The whole forward pass on one stream:
+/* The whole forward pass on one stream (deepseek-v4 blog, section 1: CSA
+ * compresses every m raw KV rows into one entry and its lightning indexer
+ * picks the top-K entries for each query; HCA attends densely to every
+ * compressed entry; SWA adds the raw KV of the latest W tokens, and the
+ * compressed and raw keys enter one attention):
  *   prefill (wk != NULL): kc = block_merge(k_raw, wk), vc = block_merge(v_raw, wv)
  *     and, for CSA, kic = block_merge(ki_raw, wib); Nc must equal Lkv / m.
  *   decode (wk == NULL): kc, vc, kic are read as ready caches of Nc entries.

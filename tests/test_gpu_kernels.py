@@ -103,6 +103,15 @@ def test_index_topk_decode_positions(hb):
     _index_case(hb, B, 1, 4, 64, Nc, 4, 128, 256, q_pos=pos, seed=4)
 
 
+def test_index_topk_decode_workload_shape(hb):
+    # the decode workload's selection: K = 1024 of 16352 visible entries of a
+    # 16384-entry cache, one query per sequence at the last context position
+    B, Nc = 8, 16384
+    pos = [[65535 - 5 * b] for b in range(B)]
+    exact = _index_case(hb, B, 1, 4, 64, Nc, 4, 128, 1024, q_pos=pos, seed=6)
+    assert exact.sum() >= 1
+
+
 def test_index_topk_large_rows_sampled(hb):
     # entries per row as in the long CSA prefill (up to 8160 visible), sampled rows
     rows = list(range(0, 32768, 997)) + [32767, 520, 521]

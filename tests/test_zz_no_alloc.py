@@ -73,7 +73,8 @@ def test_noalloc_matches_the_workspace_entry_point(hb, name):
 
 def test_noalloc_rejects_problems_beyond_its_scratch(hb):
     f = _entry(hb)
-    # 64 rows x 65536 entries x 4 B = 16 MiB > the 8 MiB scratch: refused, nothing launched
+    # 64 rows x 40000 entries x 4 B ~ 10 MB > the 8 MiB scratch: refused, nothing launched (Nc
+    # stays under the top-K's shared-memory limit, so only the scratch size refuses it)
     p = hb.problem(B=64, Lq=1, Lkv=128, Hq=4, Hkv=1, d=64, m=4, W=128, topk=64, Hi=4, di=64,
                    Nc=40000)
     buf = torch.empty(256, dtype=torch.uint8, device="cuda")
