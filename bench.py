@@ -748,6 +748,60 @@ def run_reference_arm(args):
     }
 
 
+def run_micro(args):
+    """The measured roofline denominators on this GPU: an HBM copy, the
+    L2-resident random-row gather (the CSA attention's data path, through the
+    library's probe kernel) and a cuBLAS bf16 GEMM.  CUDA events, best of N."""
+    import compressed_sparse_sliding_b200 as hb
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def best_ms(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(reps):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return best
+
+    clk = sample_clocks_start()
+    a = torch.ones(1 << 30, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    ms = best_ms(lambda: b.copy_(a), 10)
+    hbm = 2 * a.numel() * 2 / (ms / 1e3) / 1e9
+    del a, b
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    table = torch.randint(0, 1 << 30, ((4 << 20) // 4,), dtype=torch.int32, device=dev)
+    sink = torch.zeros(256, dtype=torch.int32, device=dev)
+    rows = 128 * 2048
+    gather = {}
+    for stages in range(2, 7):
+        ms = best_ms(lambda: hb.hyb_probe_l2_gather(table, rows, stages, sink, stream), 10)
+        gather[str(stages)] = round(sms * rows * 256 / (ms / 1e3) / 1e9, 1)
+    n = 8192
+    x = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    y = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    ms = best_ms(lambda: torch.matmul(x, y), 10)
+    gemm = 2 * n ** 3 / (ms / 1e3) / 1e12
+    clocks = sample_clocks_stop(clk)
+    return {"metric": "roofline denominators", "hbm_copy_GBps": round(hbm, 1),
+            "l2_gather_GBps_by_stages": gather, "l2_gather_GBps": max(gather.values()),
+            "l2_gather_B_per_clk_per_sm": round(max(gather.values()) * 1e9 / sms /
+                                               (((clocks or {}).get("sm_mhz") or 1965.0) * 1e6), 1),
+            "bf16_gemm_TFLOPs": round(gemm, 1), "sms": sms,
+            "how": "HBM: 1 GiB bf16 copy (read + write bytes); L2 gather: random 256-byte rows of a 4 MB "
+                   "table into 32 KB shared-memory stages with 16-byte cp.async, one CTA per SM, "
+                   f"{rows} rows per SM (hyb_probe_l2_gather); GEMM: torch.matmul bf16 {n}^3; "
+                   "best of 10 with CUDA events",
+            "clocks": clocks}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -756,6 +810,8 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--micro", action="store_true",
+                    help="print the measured roofline denominators (HBM copy, L2 gather, bf16 GEMM) and exit")
     ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated", "fp4", "train"],
                     help="gated: the three-branch variant (CSA workloads with prefill); "
                          "fp4: decode over 4-bit compressed caches (config 5); "
@@ -768,6 +824,10 @@ def main():
         ap.error("--variant fp4 needs the decode workload (config 5)")
     if args.variant == "train" and WORKLOADS[args.config].is_decode:
         ap.error("--variant train needs a prefill workload (configs 1-4)")
+
+    if args.micro:
+        print(json.dumps(run_micro(args)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

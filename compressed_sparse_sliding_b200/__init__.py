@@ -100,6 +100,10 @@ try:
     _lib.hyb_get_device_status.restype = _I
     _lib.hyb_error_string.argtypes = [_I]
     _lib.hyb_error_string.restype = ctypes.c_char_p
+    _lib.hyb_trace_attach.argtypes = [_P, ctypes.c_size_t]
+    _lib.hyb_trace_attach.restype = _I
+    _lib.hyb_probe_l2_gather.argtypes = [_P, ctypes.c_longlong, ctypes.c_longlong, _I, _P, _P]
+    _lib.hyb_probe_l2_gather.restype = _I
 except AttributeError as exc:   # a library built from older sources
     raise ImportError(f"{LIB_PATH} lacks an entry point ({exc}); rebuild: {_BUILD_HINT}") from exc
 
@@ -367,3 +371,45 @@ def hyb_gated_fwd(p: HybProblem, q, kc, vc, idx, k_raw, v_raw, gate, o=None, ws=
 
 def hyb_get_device_status(stream=None) -> int:
     return int(_lib.hyb_get_device_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------- timeline
+TRACE_ROLES = {1: "gather", 2: "mma", 3: "softmax"}
+
+
+def hyb_trace_attach(buf: Optional[torch.Tensor]) -> None:
+    """Attach (or, with None, detach) a device buffer for the per-role timeline
+    of CTA 0 of the kernels that record one (see hyb_trace_attach in the C
+    header).  The record count in the buffer's first word is cleared here."""
+    if buf is None:
+        st = _lib.hyb_trace_attach(None, 0)
+    else:
+        if buf.device.type != "cuda" or not buf.is_contiguous():
+            raise ValueError("trace buffer: a contiguous CUDA tensor")
+        buf.view(torch.uint8)[:16].zero_()
+        st = _lib.hyb_trace_attach(_ptr(buf), buf.numel() * buf.element_size())
+    if st != HYB_OK:
+        raise HybError(st, "hyb_trace_attach")
+
+
+def trace_records(buf: torch.Tensor):
+    """The records of an attached buffer as a list of dicts (clock, role,
+    event, item, tile), in the order they were appended."""
+    words = buf.view(torch.int64).cpu().numpy().view("uint64")
+    n = int(words[0] & 0xFFFFFFFF)
+    cap = (words.size - 2) // 2
+    out = []
+    for r in range(min(n, cap)):
+        clk, tag = int(words[2 + 2 * r]), int(words[3 + 2 * r])
+        out.append(dict(clock=clk, role=tag >> 56, event=(tag >> 48) & 0xFF,
+                        item=(tag >> 16) & 0xFFFFFFFF, tile=tag & 0xFFFF))
+    return out
+
+
+def hyb_probe_l2_gather(table: torch.Tensor, rows_per_sm: int, stages: int, sink: torch.Tensor,
+                        stream=None) -> None:
+    """One launch of the L2-resident random-row gather probe (see the C header)."""
+    st = _lib.hyb_probe_l2_gather(_ptr(table), table.numel() * table.element_size(), int(rows_per_sm),
+                                  int(stages), _ptr(sink), _stream(stream))
+    if st != HYB_OK:
+        raise HybError(st, "hyb_probe_l2_gather")

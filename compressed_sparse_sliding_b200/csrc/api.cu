@@ -4,9 +4,20 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace hyb {
+
+// An NVTX range around each entry point (host side), so that a profiler's
+// timeline names the stage that launched each kernel.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 
 
@@ -21,6 +32,10 @@ cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *
 cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m, int W, int K,
                               const int32_t *q_pos, int32_t *idx, float *sel_scores,
                               cudaStream_t stream);
+bool index_fused_supported(int Lq, int Hi, int di, int Nc, int K);
+cudaError_t launch_index_topk_fused(const void *qi, const float *wi, const void *kic, int32_t *idx,
+                                    float *sel, int B, int Lq, int Hi, int di, int Nc, int m, int W, int K,
+                                    const int32_t *q_pos, cudaStream_t stream);
 cudaError_t launch_hca_attn(int B, int L, int Lkv, int Hq, int Hkv, int d, int Nc, int m, int W,
                             float scale, const void *q, const void *kc, const void *vc, const void *kr,
                             const void *vr, void *o, float *lse, cudaStream_t stream, int num_sms);
@@ -124,6 +139,13 @@ static cudaError_t index_topk_into(const hyb_problem *p, const void *qi, const f
                              sel_scores, stream);
 }
 
+// Stage 2 in one kernel (scores recomputed on chip, no score rows stored) for
+// the shapes it takes; the two-kernel path above for the others.
+static bool index_topk_fused_path(const hyb_problem *p)
+{
+    return index_fused_supported(p->Lq, p->Hi, p->di, p->Nc, p->topk);
+}
+
 static float softmax_scale(const hyb_problem *p)
 {
     return p->scale != 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
@@ -209,7 +231,7 @@ extern "C" {
 
 size_t hyb_workspace_size(const hyb_problem *p)
 {
-    if (!p || p->topk <= 0)
+    if (!p || p->topk <= 0 || index_topk_fused_path(p))
         return 0;
     size_t scores = (size_t)p->B * p->Lq * p->Nc * sizeof(float);
     return (scores + 255) & ~(size_t)255;
@@ -218,6 +240,7 @@ size_t hyb_workspace_size(const hyb_problem *p)
 hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m, const float *w,
                             void *out, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_hca_compress");
     if (!x || !w || !out || B <= 0 || L < 0 || H <= 0 || dx <= 0 || m <= 0)
         return HYB_ERR_INVALID_ARG;
     if (dx % 8 != 0 || !aligned16(x) || !aligned16(out) || !aligned16(w))
@@ -231,11 +254,15 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
                               int32_t *idx, float *sel_scores, void *ws, size_t ws_bytes,
                               cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_csa_index_topk");
     hyb_status st = check_problem(p, true);
     if (st != HYB_OK)
         return st;
     if (!qi || !wi || !kic || !idx || !aligned16(qi) || !aligned16(kic))
         return HYB_ERR_INVALID_ARG;
+    if (index_topk_fused_path(p))
+        return cuda_status(launch_index_topk_fused(qi, wi, kic, idx, sel_scores, p->B, p->Lq, p->Hi, p->di,
+                                                   p->Nc, p->m, p->W, p->topk, p->q_pos, stream));
     const size_t need = hyb_workspace_size(p);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return HYB_ERR_WORKSPACE;
@@ -247,6 +274,7 @@ hyb_status hyb_attn_fwd(const hyb_problem *p, const void *q, const void *kc, con
                         const int32_t *idx, const void *k_raw, const void *v_raw, void *o, float *lse,
                         cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_attn_fwd");
     hyb_status st = check_problem(p, false);
     if (st != HYB_OK)
         return st;
@@ -286,6 +314,7 @@ hyb_status hyb_fused_fwd(const hyb_problem *p, const void *q, const void *k_raw,
                          int32_t *idx, void *o, float *lse, void *ws, size_t ws_bytes,
                          cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_fused_fwd");
     const bool csa = p && p->topk > 0;
     hyb_status st = check_problem(p, csa);
     if (st != HYB_OK)
@@ -322,6 +351,7 @@ hyb_status hyb_decode_append(const hyb_problem *p, const int32_t *t_new, const v
                              const float *wib, void *k_ring, void *v_ring, void *ki_ring, void *kc,
                              void *vc, void *kic, int32_t *kv_pos0, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_decode_append");
     AppendParams a;
     hyb_status st = append_common(p, t_new, k_new, v_new, ki_new, wk, wv, wib, k_ring, v_ring, ki_ring,
                                   kv_pos0, a);
@@ -342,6 +372,7 @@ hyb_status hyb_decode_append_fp4(const hyb_problem *p, const int32_t *t_new, con
                                  uint8_t *kc_codes, float *kc_qp, uint8_t *vc_codes, float *vc_qp,
                                  uint8_t *kic_codes, float *kic_qp, int32_t *kv_pos0, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_decode_append_fp4");
     AppendParams a;
     hyb_status st = append_common(p, t_new, k_new, v_new, ki_new, wk, wv, wib, k_ring, v_ring, ki_ring,
                                   kv_pos0, a);
@@ -367,6 +398,7 @@ hyb_status hyb_decode_append_fp4(const hyb_problem *p, const int32_t *t_new, con
 hyb_status hyb_fp4_quantize(const void *x, long long rows, int dx, uint8_t *codes, float *qp,
                             cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_fp4_quantize");
     if (!x || !codes || !qp || rows < 0)
         return HYB_ERR_INVALID_ARG;
     if (dx != 64 && dx != 128 && dx != 256)
@@ -379,6 +411,7 @@ hyb_status hyb_fp4_quantize(const void *x, long long rows, int dx, uint8_t *code
 hyb_status hyb_fp4_dequantize(const uint8_t *codes, const float *qp, long long rows, int dx, void *out,
                               cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_fp4_dequantize");
     if (!codes || !qp || !out || rows < 0 || dx <= 0 || dx % 8 != 0)
         return HYB_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(codes) || !aligned16(qp))
@@ -404,6 +437,7 @@ hyb_status hyb_csa_index_topk_fp4(const hyb_problem *p, const void *qi, const fl
                                   const uint8_t *kic_codes, const float *kic_qp, int32_t *idx,
                                   float *sel_scores, void *ws, size_t ws_bytes, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_csa_index_topk_fp4");
     hyb_status st = check_problem(p, true);
     if (st != HYB_OK)
         return st;
@@ -428,6 +462,9 @@ hyb_status hyb_csa_index_topk_fp4(const hyb_problem *p, const void *qi, const fl
                                           num_sms_current());
     if (e != cudaSuccess)
         return cuda_status(e);
+    if (index_topk_fused_path(p))
+        return cuda_status(launch_index_topk_fused(qi, wi, kic, idx, sel_scores, p->B, p->Lq, p->Hi, p->di,
+                                                   p->Nc, p->m, p->W, p->topk, p->q_pos, stream));
     return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, scores, stream));
 }
 
@@ -436,6 +473,7 @@ hyb_status hyb_attn_fwd_fp4(const hyb_problem *p, const void *q, const uint8_t *
                             const int32_t *idx, const void *k_raw, const void *v_raw, void *o, float *lse,
                             void *ws, size_t ws_bytes, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_attn_fwd_fp4");
     hyb_status st = check_problem(p, false);
     if (st != HYB_OK)
         return st;
@@ -480,6 +518,7 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
                         const float *lse, const void *dout, float *dq, float *dkc, float *dvc,
                         float *dk_raw, float *dv_raw, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_attn_bwd");
     hyb_status st = check_problem(p, false);
     if (st != HYB_OK)
         return st;
@@ -548,6 +587,7 @@ hyb_status hyb_hca_compress_bwd(const void *x, int B, int L, int H, int dx, int 
                                 const float *dc, float *dx_acc, float *dw, void *ws, size_t ws_bytes,
                                 cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_hca_compress_bwd");
     if (!x || !w || !dc || !dx_acc || !dw || B <= 0 || L < 0 || H <= 0 || dx <= 0 || m <= 0)
         return HYB_ERR_INVALID_ARG;
     if (dx % 32 != 0)
@@ -576,6 +616,7 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
                          const int32_t *idx, const void *k_raw, const void *v_raw, const float *gate,
                          void *o, void *ws, size_t ws_bytes, cudaStream_t stream)
 {
+    NvtxRange nvtx_range("hyb_gated_fwd");
     hyb_status st = check_problem(p, false);
     if (st != HYB_OK)
         return st;
@@ -621,6 +662,22 @@ hyb_status hyb_get_device_status(cudaStream_t stream)
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess)
         return HYB_ERR_CUDA;
     return (hyb_status)v;
+}
+
+hyb_status hyb_trace_attach(void *buf, size_t bytes)
+{
+    unsigned long long *b = static_cast<unsigned long long *>(buf);
+    unsigned int cap = 0;
+    if (b) {
+        if ((reinterpret_cast<uintptr_t>(buf) & 15u) || bytes < 32)
+            return HYB_ERR_INVALID_ARG;
+        const size_t recs = (bytes - 16) / 16;
+        cap = recs > 0xFFFFFFFFull ? 0xFFFFFFFFu : (unsigned int)recs;
+    }
+    if (cudaMemcpyToSymbol(g_trace_cap, &cap, sizeof(cap)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_trace_buf, &b, sizeof(b)) != cudaSuccess)
+        return HYB_ERR_CUDA;
+    return HYB_OK;
 }
 
 const char *hyb_error_string(hyb_status s)

@@ -334,6 +334,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    unsigned long long *const tb = trace_buffer();   // timeline of CTA 0, when attached
     constexpr int PW = SpRoles<NH>::PW;
     constexpr int NPT = 32 * PW;                // producer threads
 
@@ -492,6 +493,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     cp_async_mbar_arrive(&bar[SB_KF + ks]);
                     mbar_arrive(&bar[SB_KF + ks]);
+                    if (pt == 0)
+                        trace_ev(tb, 1, 1, w, i);
                     ++kc;
                 }
                 if (kSpLead == 0) {
@@ -515,6 +518,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     cp_async_mbar_arrive(&bar[SB_VF + vs]);
                     mbar_arrive(&bar[SB_VF + vs]);
+                    if (pt == 0)
+                        trace_ev(tb, 1, 2, w, i - kSpLead);
                     ++vc;
                 }
                 if (kSpLead == 1) {
@@ -567,6 +572,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_OD + pb]);
                     mma_commit(&bar[SB_VE + vs]);
+                    trace_ev(tb, 2, 2, w, (int)pcnt);
                     ++vc;
                     ++pcnt;
                     return true;
@@ -588,6 +594,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_SF + (gt & 1)]);
                     mma_commit(&bar[SB_KE + ks]);
+                    trace_ev(tb, 2, 1, w, i);
                     ++kc;
                     if (i == nt - 1)
                         mma_commit(&bar[SB_QE + qb]);
@@ -658,6 +665,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float s[NHW];
                 tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
                 tmem_ld_wait();
+                if (threadIdx.x == 0)
+                    trace_ev(tb, 3, 1, w, i);
 #pragma unroll
                 for (int h = 0; h < NHW; ++h)
                     s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
@@ -765,8 +774,12 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
+                if (threadIdx.x == 0)
+                    trace_ev(tb, 3, 2, w, i);
             }
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
+            if (threadIdx.x == 0)
+                trace_ev(tb, 3, 3, w, nt);
             warp_reduce_heads<NHW, false>(lpart, lane);
             if (head_owner) {
 #pragma unroll
@@ -819,6 +832,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
+            if (threadIdx.x == 0)
+                trace_ev(tb, 3, 4, w, nt);
         }
     }
 

@@ -41,6 +41,35 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
+// ---------------------------------------------------------------------------
+// Optional per-role timeline (a debug aid; see hyb_trace_attach).  When a
+// buffer is attached, CTA 0 of a kernel that supports it appends one record
+// per event: word 0 of the buffer counts records, record r occupies words
+// 2 + 2r (the SM clock) and 3 + 2r (role << 56 | event << 48 | item << 16 |
+// tile).  Other CTAs, and every CTA without a buffer, skip the records.
+// ---------------------------------------------------------------------------
+__device__ unsigned long long *g_trace_buf = nullptr;
+__device__ unsigned int g_trace_cap = 0;     // records the buffer holds
+
+__device__ __forceinline__ unsigned long long *trace_buffer()
+{
+    return blockIdx.x == 0 && blockIdx.y == 0 ? g_trace_buf : nullptr;
+}
+
+__device__ __forceinline__ void trace_ev(unsigned long long *tb, int role, int ev, long long item, int tile)
+{
+    if (!tb)
+        return;
+    const unsigned long long clk = clock64();
+    const unsigned int r = atomicAdd(reinterpret_cast<unsigned int *>(tb), 1u);
+    if (r < g_trace_cap) {
+        tb[2 + 2 * (size_t)r] = clk;
+        tb[3 + 2 * (size_t)r] = ((unsigned long long)role << 56) | ((unsigned long long)ev << 48) |
+                                (((unsigned long long)item & 0xFFFFFFFFull) << 16) |
+                                ((unsigned long long)tile & 0xFFFFull);
+    }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -1,0 +1,690 @@
+// index_fused.cu -- stage 2 of CSA for prefill-shaped problems in one kernel:
+// the lightning-indexer scores and the exact per-query top-K ("deepseek-v4"
+// blog, section 1, CSA: a lightning indexer scores the compressed entries and
+// the top-K of them are kept for the current query; score = ReLU-weighted
+// head sum, fp32), without ever storing a row of scores.
+//
+//     I[t, s] = sum_h wi[t, h] * max(0, qi[t, h, :] . kic[s, :])
+//
+// A CTA owns 128 query rows of one sequence (one TMEM lane each).  Key tiles
+// of 64 entries stream through a TMA ring; per tile one tcgen05 MMA per
+// indexer head writes D_h [128 rows x 64 keys] into TMEM (double-buffered), and
+// the epilogue thread of a row forms the row's 64 scores.  The scores are
+// recomputed pass after pass (the GEMM is cheap next to moving the score rows
+// through HBM) and only per-row summaries stay on chip:
+//   S  (sample)    two tiles spread over the visible range; each row keeps the
+//                  order keys of its <= 128 sampled scores and derives a key
+//                  window that very likely holds its K-th largest score;
+//   H  (histogram) every visible key; each row counts its scores above the
+//                  window and histograms those inside it (128 bins, u16
+//                  counters in shared memory), then finds the bin holding the
+//                  K-th largest.  A row whose window missed (or whose bin is too
+//                  full to keep) moves or narrows its window and the CTA runs
+//                  H again, so the result never depends on the sample;
+//   E  (emit)      every visible key again; scores above the bin are written
+//                  straight to the row's index list (ascending, since keys are
+//                  visited in order), scores inside the bin are kept in a
+//                  per-row buffer of <= 64 entries.  Afterwards the row takes
+//                  the largest of them (lower index first on equal scores) and
+//                  merges them into its list; when the bin is a single score
+//                  value (an exact tie) the first entries in index order are
+//                  taken during E itself.
+// Order keys are the fp32 scores mapped to uint32 so that larger scores give
+// larger keys (-0.0 folded onto +0.0), as in the two-kernel path.
+// Roles (256 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 4-7 the
+// row epilogue (TMEM lane quadrants 0-3); warps 2-3 idle.  The epilogue
+// decides after each H pass whether another H or the E pass follows; the
+// producer and MMA warps learn it through two shared words and stop after E.
+#include "common.cuh"
+
+namespace hyb {
+
+constexpr int kFxThreads = 256;
+constexpr int kFxBM = 128;          // query rows per CTA
+constexpr int kFxBN = 64;           // keys per tile
+constexpr int kFxStages = 4;
+constexpr int kFxSampleTiles = 2;
+constexpr int kFxBins = 128;        // histogram bins per row
+constexpr int kFxCap = 64;          // boundary-bin entries kept per row
+constexpr int kFxMaxPasses = 16;    // S + H rounds + E, far above what the window moves need
+constexpr int kFxMaxNc = 65535;     // index and list position share one 32-bit word
+
+struct FusedIndexParams {
+    int B, Lq, Hi, Nc, m, W, K;
+    int n_ttiles;
+    const int32_t *q_pos;
+    const float *wi;          // [B, Lq, Hi]
+    int32_t *idx;             // [B, Lq, K]
+    float *sel;               // [B, Lq, K] or nullptr
+};
+
+template <int HI, int DI>
+struct FxSmem {
+    static constexpr int Q_BYTES = kFxBM * DI * 2;                   // one head
+    static constexpr int K_BYTES = kFxBN * DI * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = HI * Q_BYTES;
+    static constexpr int OFF_U = OFF_K + kFxStages * K_BYTES;        // union below
+    // pass S: sample keys [slot][row]; later passes: histogram [bin / 2][row]
+    // (two u16 counters per word) followed by the boundary buffer: keys
+    // [slot][row], then (index | list position << 16) [slot][row]
+    static constexpr int SAMPLE_BYTES = kFxSampleTiles * kFxBN * kFxBM * 4;
+    static constexpr int HIST_BYTES = (kFxBins / 2) * kFxBM * 4;
+    static constexpr int BND_BYTES = 2 * kFxCap * kFxBM * 4;
+    static constexpr int U_BYTES = SAMPLE_BYTES > HIST_BYTES + BND_BYTES ? SAMPLE_BYTES
+                                                                         : HIST_BYTES + BND_BYTES;
+    static constexpr int OFF_BAR = OFF_U + U_BYTES;
+    static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+    static constexpr int BYTES = OFF_MISC + 16 * 4;
+};
+
+// 128-byte swizzle for 64-element bf16 rows, 64-byte swizzle for 32-element rows.
+template <int DI>
+struct FxLayout {
+    static constexpr uint32_t SWZ = DI == 64 ? 2u : 4u;             // descriptor layout field
+    static constexpr uint32_t SBO = DI * 2 * 8;                      // bytes per 8-row group
+};
+
+__device__ __forceinline__ uint64_t fx_desc(uint32_t saddr, uint32_t sbo, uint32_t layout)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                      // leading byte offset (unused when swizzled)
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+
+// Larger float -> larger key; -0.0 folded onto +0.0.
+__device__ __forceinline__ uint32_t fx_key(float f)
+{
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float fx_score(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Last key of a window of `n` bins of 2^sh keys starting at lo (saturating).
+__device__ __forceinline__ uint32_t fx_last(uint32_t lo, int sh, uint32_t n)
+{
+    const unsigned long long e = (unsigned long long)lo + ((unsigned long long)n << sh) - 1ull;
+    return e > 0xFFFFFFFFull ? 0xFFFFFFFFu : (uint32_t)e;
+}
+
+// AND of a predicate over the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ bool fx_all(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+// Bounded wait until the shared decision word reaches `p` (or the CTA aborts).
+__device__ __forceinline__ bool fx_wait_decided(volatile int *decided, int p, volatile int *abort_flag)
+{
+    const uint64_t t0 = global_ns();
+    while (*decided < p) {
+        if (*abort_flag)
+            return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            set_error(HYB_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+        __nanosleep(64);
+    }
+    __threadfence_block();
+    return true;
+}
+
+// Row modes of the epilogue
+enum { FX_ALL = 0, FX_BIN = 1, FX_TIE = 2, FX_OPEN = 3, FX_NONE = 4 };
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(kFxThreads, 1)
+index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const FusedIndexParams p)
+{
+    using SM = FxSmem<HI, DI>;
+    using LY = FxLayout<DI>;
+    extern __shared__ __align__(1024) uint8_t fx_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(fx_smem_raw) + 1023) &
+                                                ~(uintptr_t)1023);
+    uint8_t *sQ = smem + SM::OFF_Q;
+    uint8_t *sK = smem + SM::OFF_K;
+    uint32_t *sU = reinterpret_cast<uint32_t *>(smem + SM::OFF_U);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
+    int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
+    volatile int *abort_flag = misc + 1;
+    volatile int *decided = misc + 2;      // passes 0 .. *decided are known to exist (or not)
+    volatile int *last_pass = misc + 3;    // index of the E pass once known
+    // bars: 0 Q full, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // heavy token tiles first, all sequences of one weight class together
+    const int ttile = p.n_ttiles - 1 - (int)(blockIdx.x / p.B);
+    const int b = (int)(blockIdx.x % p.B);
+    const int t0 = ttile * kFxBM;
+    const int t_last = min(t0 + kFxBM - 1, p.Lq - 1);
+    auto nvis_of = [&](int t) -> int {
+        const long long pos = p.q_pos ? p.q_pos[(size_t)b * p.Lq + t] : t;
+        const long long a = pos - p.W + 1;
+        return a > 0 ? (int)min((long long)p.Nc, a / p.m) : 0;
+    };
+    int nv_max = 0;
+    if (p.q_pos) {
+        for (int t = t0; t <= t_last; ++t)
+            nv_max = max(nv_max, nvis_of(t));
+    } else {
+        nv_max = nvis_of(t_last);
+    }
+    const bool has_sel = nv_max > p.K;
+    const int t_vis = (nv_max + kFxBN - 1) / kFxBN;     // key tiles of a full pass
+    // sample tiles: disjoint, each starting inside the visible range (a tile
+    // that would start past it repeats the first and is ignored: slot_lo)
+    int soff[kFxSampleTiles];
+    for (int s = 0; s < kFxSampleTiles; ++s) {
+        if (nv_max <= kFxSampleTiles * kFxBN) {
+            soff[s] = s * kFxBN < nv_max ? s * kFxBN : 0;
+        } else {
+            const int c = (int)(((2ll * s + 1) * nv_max) / (2 * kFxSampleTiles)) - kFxBN / 2;
+            soff[s] = max(0, min(c, nv_max - kFxBN));
+        }
+    }
+    // sampled keys of tile s count only from slot_lo(s) on (no key counted twice)
+    auto slot_lo = [&](int s) -> int { return s == 0 ? 0 : soff[s - 1] + kFxBN; };
+    // tiles of pass q: the sample pass has its own tiles, every other pass all visible ones
+    auto pass_tiles = [&](int q) -> int { return (has_sel && q == 0) ? kFxSampleTiles : t_vis; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        for (int s = 0; s < kFxStages; ++s) {
+            mbar_init(&bar[1 + s], 1);
+            mbar_init(&bar[5 + s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[9 + s], 1);
+            mbar_init(&bar[11 + s], 128);
+        }
+        mbar_init(&bar[13], 1);
+        mbar_fence_init();
+        misc[1] = 0;
+        // with a selection to make: S, H and one more pass (H or E) always run
+        misc[2] = has_sel ? 2 : 0x7fffffff;
+        misc[3] = has_sel ? 0x7fffffff : (t_vis > 0 ? 0 : -1);
+    }
+    if (warp == 1)
+        tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[0], HI * SM::Q_BYTES);
+            for (int h = 0; h < HI; ++h)
+                tma_load_4d(sQ + h * SM::Q_BYTES, &tm_q, &bar[0], 0, h, t0, b);
+            int issued = 0;
+            bool ok = true;
+            for (int q = 0; ok && q < kFxMaxPasses; ++q) {
+                if (q >= 3 && !fx_wait_decided(decided, q, abort_flag))
+                    break;
+                if (q > *last_pass)
+                    break;
+                const int nt = pass_tiles(q);
+                for (int i = 0; i < nt; ++i) {
+                    const int s = issued % kFxStages;
+                    if (issued >= kFxStages &&
+                        !mbar_wait(&bar[5 + s], ((issued / kFxStages) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int start = (has_sel && q == 0) ? soff[i] : i * kFxBN;
+                    mbar_arrive_expect_tx(&bar[1 + s], SM::K_BYTES);
+                    tma_load_4d(sK + s * SM::K_BYTES, &tm_k, &bar[1 + s], 0, 0, start, b);
+                    ++issued;
+                }
+            }
+            drain_wait(&bar[0], 0);
+            for (int i = max(0, issued - kFxStages); i < issued; ++i)
+                drain_wait(&bar[1 + i % kFxStages], (i / kFxStages) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kFxBM, kFxBN, false, false);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+            bool ok = *last_pass < 0 ? true : mbar_wait(&bar[0], 0, abort_flag);
+            int g = 0;
+            for (int q = 0; ok && q < kFxMaxPasses; ++q) {
+                if (q >= 3 && !fx_wait_decided(decided, q, abort_flag))
+                    break;
+                if (q > *last_pass)
+                    break;
+                const int nt = pass_tiles(q);
+                for (int i = 0; i < nt; ++i, ++g) {
+                    const int s = g % kFxStages, db = g & 1;
+                    if (!mbar_wait(&bar[1 + s], (g / kFxStages) & 1, abort_flag) ||
+                        (g >= 2 && !mbar_wait(&bar[11 + db], ((g >> 1) - 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int h = 0; h < HI; ++h) {
+#pragma unroll
+                        for (int kk = 0; kk < DI / 16; ++kk) {
+                            const uint64_t da = fx_desc(aQ + h * SM::Q_BYTES + kk * 32, LY::SBO, LY::SWZ);
+                            const uint64_t dbk = fx_desc(aK + s * SM::K_BYTES + kk * 32, LY::SBO, LY::SWZ);
+                            mma_bf16_ss(tmem + (db * HI + h) * kFxBN, da, dbk, idesc, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&bar[9 + db]);
+                    mma_commit(&bar[5 + s]);
+                }
+            }
+            mma_commit(&bar[13]);
+            drain_wait(&bar[13], 0);
+        }
+    } else if (warp >= 4) {
+        // ================================ row epilogue ================================
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int t = t0 + row;
+        const bool valid = t < p.Lq;
+        const int nv = valid ? nvis_of(t) : 0;
+        const int K = p.K;
+        float wv[HI];
+#pragma unroll
+        for (int h = 0; h < HI; ++h)
+            wv[h] = valid ? p.wi[((size_t)b * p.Lq + t) * HI + h] : 0.f;
+        int32_t *orow = p.idx + ((size_t)b * p.Lq + (valid ? t : 0)) * K;
+        float *srow = p.sel ? p.sel + ((size_t)b * p.Lq + (valid ? t : 0)) * K : nullptr;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        uint32_t *col = sU + row;                         // this row's column of the union area
+        uint32_t *hist = col;                             // [bin / 2] stride kFxBM
+        uint32_t *bkey = col + (kFxBins / 2) * kFxBM;     // [slot] stride kFxBM
+        uint32_t *bpk = bkey + kFxCap * kFxBM;
+
+        int mode = !valid ? FX_NONE : (nv > K ? FX_OPEN : FX_ALL);
+        uint32_t lo = 0, top_m1 = 0xFFFFFFFFu, blo = 0, bhi_m1 = 0;
+        int sh = 25, need = 0, a_cnt = 0;
+        int ab = 0, ns = 0, pos = 0, taken = 0, nb = 0;
+        bool ok = true, emitted = false;
+        int g = 0;
+        // index of the E pass as this thread knows it (every epilogue thread
+        // takes the same decisions from the same barrier votes)
+        int lastp = has_sel ? 0x7fffffff : (t_vis > 0 ? 0 : -1);
+        for (int q = 0; q < kFxMaxPasses; ++q) {
+            if (q > lastp)
+                break;
+            const int ptype = (has_sel && q == 0) ? 0 : (q == lastp ? 2 : 1);   // S / H / E
+            const int nt = pass_tiles(q);
+            for (int i = 0; i < nt; ++i, ++g) {
+                const int db = g & 1;
+                if (ok)
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (g >> 1) & 1, abort_flag));
+                if (!ok)
+                    continue;
+                tc_fence_after();
+                const int kbase = ptype == 0 ? soff[i] : i * kFxBN;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float d[HI][32];
+#pragma unroll
+                    for (int h = 0; h < HI; ++h)
+                        tmem_ld32(tl + (db * HI + h) * kFxBN + half * 32, d[h]);
+                    tmem_ld_wait();
+                    if (half == 1) {
+                        // both halves are in registers: the MMA may refill this buffer
+                        tc_fence_before();
+                        mbar_arrive(&bar[11 + db]);
+                    }
+                    const int j0 = kbase + half * 32;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        float s = wv[0] * fmaxf(d[0][c], 0.f);
+#pragma unroll
+                        for (int h = 1; h < HI; ++h)
+                            s = fmaf(wv[h], fmaxf(d[h][c], 0.f), s);
+                        const int j = j0 + c;
+                        const bool vis = j < nv;
+                        if (ptype == 0) {
+                            const bool in = vis && j >= slot_lo(i);
+                            col[(i * kFxBN + half * 32 + c) * kFxBM] = in ? fx_key(s) : 0u;
+                            ns += in;
+                        } else if (ptype == 1) {
+                            if (mode == FX_OPEN && vis) {
+                                const uint32_t k = fx_key(s);
+                                if (k >= lo) {
+                                    if (k > top_m1) {
+                                        ++ab;
+                                    } else {
+                                        const uint32_t bin = (k - lo) >> sh;
+                                        atomicAdd(hist + (bin >> 1) * kFxBM, 1u << ((bin & 1u) * 16u));
+                                    }
+                                }
+                            }
+                        } else if (vis && mode != FX_NONE) {
+                            bool pick = mode == FX_ALL;
+                            if (!pick) {
+                                const uint32_t k = fx_key(s);
+                                if (k > bhi_m1) {
+                                    pick = true;
+                                } else if (k >= blo) {
+                                    if (mode == FX_TIE) {
+                                        pick = taken < need;
+                                        taken += pick;
+                                    } else if (nb < kFxCap) {
+                                        bkey[nb * kFxBM] = k;
+                                        bpk[nb * kFxBM] = (uint32_t)j | ((uint32_t)pos << 16);
+                                        ++nb;
+                                    }
+                                }
+                            }
+                            if (pick && pos < K) {
+                                orow[pos] = j;
+                                if (srow)
+                                    srow[pos] = s;
+                                ++pos;
+                            }
+                        }
+                    }
+                }
+            }
+            // ------------------------------ end of pass q ------------------------------
+            if (!fx_all(ok)) {
+                if (threadIdx.x == 128) {
+                    *abort_flag = 1;
+                    *last_pass = -1;
+                    __threadfence_block();
+                    *decided = 0x7fffffff;
+                }
+                break;
+            }
+            if (ptype == 2) {
+                emitted = true;
+                break;
+            }
+            if (ptype == 0) {
+                // window from the sample: its lower edge is (a lower bound of) the
+                // sample key of rank klo, a rank that the row's K-th largest key
+                // reaches with a wide margin; its 96 lower bins span up to the
+                // sample maximum, the 32 upper bins leave room above it
+                if (mode == FX_OPEN) {
+                    uint32_t kmax = 0;
+                    for (int u = 0; u < kFxSampleTiles * kFxBN; ++u)
+                        kmax = max(kmax, col[u * kFxBM]);
+                    if (ns > 0) {
+                        const float e = (float)K * (float)ns / (float)nv;
+                        int klo = (int)ceilf(e + 3.f * sqrtf(e) + 2.f);
+                        klo = max(1, min(klo, ns));
+                        // largest 16-bit prefix P with #(key >> 16 >= P) >= klo
+                        uint32_t pfx = 0;
+                        for (int bit = 15; bit >= 0; --bit) {
+                            const uint32_t cand = pfx | (1u << bit);
+                            int cnt = 0;
+                            for (int u = 0; u < kFxSampleTiles * kFxBN; ++u)
+                                cnt += (col[u * kFxBM] >> 16) >= cand;
+                            if (cnt >= klo)
+                                pfx = cand;
+                        }
+                        lo = pfx << 16;
+                        const uint32_t span = kmax > lo ? kmax - lo : 0u;
+                        sh = 0;
+                        while (sh < 25 && (span >> sh) >= 96u)
+                            ++sh;
+                    } else {
+                        lo = 0;
+                        sh = 25;
+                    }
+                    top_m1 = fx_last(lo, sh, kFxBins);
+                }
+                // the sample area becomes the histogram: clear this row's column
+#pragma unroll 4
+                for (int w = 0; w < kFxBins / 2; ++w)
+                    hist[w * kFxBM] = 0u;
+            } else {
+                // after H: find the bin holding the K-th largest key
+                if (mode == FX_OPEN) {
+                    int cum = ab, bstar = -1, cnt = 0;
+                    for (int w = kFxBins / 2 - 1; w >= 0; --w) {
+                        const uint32_t v = hist[w * kFxBM];
+                        hist[w * kFxBM] = 0u;
+                        if (bstar >= 0)
+                            continue;
+                        const int c_hi = (int)(v >> 16), c_lo = (int)(v & 0xFFFFu);
+                        if (cum + c_hi >= K) {
+                            bstar = 2 * w + 1;
+                            cnt = c_hi;
+                        } else if (cum + c_hi + c_lo >= K) {
+                            cum += c_hi;
+                            bstar = 2 * w;
+                            cnt = c_lo;
+                        } else {
+                            cum += c_hi + c_lo;
+                        }
+                    }
+                    if (ab >= K) {
+                        // the K-th key lies above the window: move up, wider
+                        lo = top_m1 + 1u;
+                        sh = min(sh + 7, 25);
+                    } else if (bstar < 0) {
+                        // below the window: take the whole key range
+                        lo = 0;
+                        sh = 25;
+                    } else {
+                        const uint32_t bl = lo + ((uint32_t)bstar << sh);
+                        if (sh == 0 || cnt <= kFxCap) {
+                            mode = sh == 0 ? FX_TIE : FX_BIN;
+                            blo = bl;
+                            bhi_m1 = fx_last(bl, sh, 1);
+                            a_cnt = cum;
+                            need = K - cum;
+                        } else {
+                            // too many keys share the bin: narrow to it
+                            lo = bl;
+                            sh = max(sh - 7, 0);
+                        }
+                    }
+                    top_m1 = fx_last(lo, sh, kFxBins);
+                    ab = 0;
+                }
+                const bool all_set = fx_all(mode != FX_OPEN);
+                if (all_set)
+                    lastp = q + 1;
+                if (threadIdx.x == 128) {
+                    if (all_set) {
+                        *last_pass = q + 1;       // the next pass emits
+                        __threadfence_block();
+                        *decided = 0x7fffffff;
+                    } else {
+                        __threadfence_block();
+                        *decided = q + 2;         // another H pass, then at least one more
+                    }
+                }
+            }
+        }
+        // ---- boundary bin: take the `need` largest (lower index first), merge ----
+        if (emitted && mode == FX_BIN) {
+            // largest key T in [blo, bhi_m1] with #(key >= T) >= need
+            uint32_t lo_b = blo, hi_b = bhi_m1;
+            while (lo_b < hi_b) {
+                const uint32_t mid = lo_b + ((hi_b - lo_b) >> 1) + 1u;
+                int cnt = 0;
+                for (int e = 0; e < nb; ++e)
+                    cnt += bkey[e * kFxBM] >= mid;
+                if (cnt >= need)
+                    lo_b = mid;
+                else
+                    hi_b = mid - 1u;
+            }
+            const uint32_t T = lo_b;
+            int gt = 0, eq = 0;
+            for (int e = 0; e < nb; ++e) {
+                const uint32_t k = bkey[e * kFxBM];
+                gt += k > T;
+                eq += k == T;
+            }
+            const int take_eq = need - gt;
+            // chosen entries in reverse list order: the m-th chosen one goes to
+            // its above-count + m - 1; the above entries after it move right by m
+            int m = need, hi_end = a_cnt, eq_back = 0;
+            for (int e = nb - 1; e >= 0 && m > 0; --e) {
+                const uint32_t k = bkey[e * kFxBM];
+                bool ch = k > T;
+                if (k == T) {
+                    ch = (eq - 1 - eq_back) < take_eq;
+                    ++eq_back;
+                }
+                if (!ch)
+                    continue;
+                const uint32_t pk = bpk[e * kFxBM];
+                const int j = (int)(pk & 0xFFFFu), abf = (int)(pk >> 16);
+                if (abf > hi_end || abf + m > K) {   // cannot happen: E recomputes H's scores exactly
+                    set_error(HYB_ERR_DEVICE_BOUNDS);
+                    break;
+                }
+                int qq = hi_end - 1;
+                for (; qq - 7 >= abf; qq -= 8) {
+                    int32_t v[8];
+                    float sv[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        v[u] = orow[qq - u];
+                        if (srow)
+                            sv[u] = srow[qq - u];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        orow[qq - u + m] = v[u];
+                        if (srow)
+                            srow[qq - u + m] = sv[u];
+                    }
+                }
+                for (; qq >= abf; --qq) {
+                    orow[qq + m] = orow[qq];
+                    if (srow)
+                        srow[qq + m] = srow[qq];
+                }
+                orow[abf + m - 1] = j;
+                if (srow)
+                    srow[abf + m - 1] = fx_score(k);
+                hi_end = abf;
+                --m;
+            }
+            pos = K;
+        }
+        if ((emitted || lastp < 0) && mode != FX_NONE) {
+            for (int u = pos; u < K; ++u) {
+                orow[u] = -1;
+                if (srow)
+                    srow[u] = -INFINITY;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc((uint32_t)misc[0], 512);
+    }
+}
+
+// 4-D map over a [B][rows][heads][DI] bf16 tensor, box (DI, 1, box_rows, 1),
+// 128-byte swizzle for DI = 64, 64-byte swizzle for DI = 32.
+template <int DI>
+static bool fx_map(CUtensorMap *map, const void *base, int n1, int n2, int n3, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[4] = {(cuuint64_t)DI, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+    cuuint64_t strides[3] = {(cuuint64_t)DI * 2, (cuuint64_t)DI * 2 * n1, (cuuint64_t)DI * 2 * n1 * n2};
+    cuuint32_t box[4] = {(cuuint32_t)DI, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    DI == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int HI, int DI>
+static cudaError_t launch_fx_t(const FusedIndexParams &p, const void *qi, const void *kic, cudaStream_t stream)
+{
+    using SM = FxSmem<HI, DI>;
+    CUtensorMap mq, mk;
+    // qi [B, Lq, Hi, DI] as (DI, Hi, Lq, B): one head's 128 rows per box
+    bool ok = fx_map<DI>(&mq, qi, HI, p.Lq, p.B, kFxBM);
+    // kic [B, Nc, DI] as (DI, 1, Nc, B): 64 entries per box (zeros past Nc)
+    ok &= fx_map<DI>(&mk, kic, 1, p.Nc, p.B, kFxBN);
+    if (!ok)
+        return cudaErrorInvalidValue;
+    size_t smem = 1024 + SM::BYTES;
+    if (smem < 120 * 1024)
+        smem = 120 * 1024;   // one CTA per SM: each holds all 512 TMEM columns
+    auto kern = index_topk_fused<HI, DI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    const unsigned grid = (unsigned)p.n_ttiles * (unsigned)p.B;
+    kern<<<grid, kFxThreads, smem, stream>>>(mq, mk, p);
+    return cudaGetLastError();
+}
+
+// Shapes the fused kernel takes: query tiles of many rows (not the decode
+// form), di in {32, 64}, at most 4 indexer heads, entries and K small enough
+// for the packed (index, list position) words.
+bool index_fused_supported(int Lq, int Hi, int di, int Nc, int K)
+{
+    return Lq >= 64 && Hi >= 1 && Hi <= 4 && (di == 32 || di == 64) && Nc <= kFxMaxNc && K >= 1 &&
+           K <= 2048;
+}
+
+cudaError_t launch_index_topk_fused(const void *qi, const float *wi, const void *kic, int32_t *idx,
+                                    float *sel, int B, int Lq, int Hi, int di, int Nc, int m, int W, int K,
+                                    const int32_t *q_pos, cudaStream_t stream)
+{
+    if (!index_fused_supported(Lq, Hi, di, Nc, K))
+        return cudaErrorNotSupported;
+    FusedIndexParams p;
+    p.B = B;
+    p.Lq = Lq;
+    p.Hi = Hi;
+    p.Nc = Nc;
+    p.m = m;
+    p.W = W;
+    p.K = K;
+    p.n_ttiles = (Lq + kFxBM - 1) / kFxBM;
+    p.q_pos = q_pos;
+    p.wi = wi;
+    p.idx = idx;
+    p.sel = sel;
+    if (di == 64) {
+        switch (Hi) {
+        case 1: return launch_fx_t<1, 64>(p, qi, kic, stream);
+        case 2: return launch_fx_t<2, 64>(p, qi, kic, stream);
+        case 3: return launch_fx_t<3, 64>(p, qi, kic, stream);
+        default: return launch_fx_t<4, 64>(p, qi, kic, stream);
+        }
+    }
+    switch (Hi) {
+    case 1: return launch_fx_t<1, 32>(p, qi, kic, stream);
+    case 2: return launch_fx_t<2, 32>(p, qi, kic, stream);
+    case 3: return launch_fx_t<3, 32>(p, qi, kic, stream);
+    default: return launch_fx_t<4, 32>(p, qi, kic, stream);
+    }
+}
+
+}  // namespace hyb

@@ -75,8 +75,11 @@ typedef struct hyb_problem {
     const int32_t *kv_pos0;  /* [B] position of raw row 0, or NULL (0)        */
 } hyb_problem;
 
-/* Bytes of device workspace hyb_csa_index_topk / hyb_fused_fwd need for `p`
- * (0 for HCA).  The workspace must be 256-byte aligned. */
+/* Bytes of device workspace hyb_csa_index_topk / hyb_fused_fwd need for `p`:
+ * 0 for HCA, and 0 for CSA problems whose selection runs in one kernel
+ * (Lq >= 64 query rows per sequence, Hi <= 4, Nc <= 65535: the scores are
+ * recomputed on chip and never stored); otherwise B * Lq * Nc fp32 score rows.
+ * A nonzero workspace must be 256-byte aligned; with 0, ws may be NULL. */
 size_t hyb_workspace_size(const hyb_problem *p);
 
 /* Stage 1, block_merge (CSDN code page, section 1):
@@ -96,7 +99,11 @@ hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m,
  * padded when fewer than K are visible.  sel_scores (nullable) receives the
  * fp32 score of each idx slot (-inf for padding).
  * qi: [B, Lq, Hi, di] bf16; wi: [B, Lq, Hi] fp32; kic: [B, Nc, di] bf16;
- * idx: [B, Lq, topk] int32; ws: workspace of >= hyb_workspace_size(p) bytes. */
+ * idx: [B, Lq, topk] int32; ws: workspace of >= hyb_workspace_size(p) bytes.
+ * Problems of 64 or more query rows per sequence (Hi <= 4, Nc <= 65535) are
+ * scored and selected in one kernel that keeps only per-row histograms on
+ * chip; decode-shaped problems (few query rows) score into the workspace and
+ * select from it. */
 hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float *wi,
                               const void *kic, int32_t *idx, float *sel_scores,
                               void *ws, size_t ws_bytes, cudaStream_t stream);
@@ -287,6 +294,32 @@ hyb_status hyb_get_device_status(cudaStream_t stream);
 
 /* Static description of a status code. */
 const char *hyb_error_string(hyb_status status);
+
+/* Debug aid (the pages have no counterpart): a per-role timeline of one CTA.
+ * Attaches a caller-owned device buffer of `bytes` bytes (16-byte aligned,
+ * >= 32) for the kernels launched afterwards on the current device; NULL
+ * detaches.  CTA 0 of a kernel that supports it (the CSA attention kernel)
+ * then appends a record per event: the first 8-byte word counts records (set
+ * it to 0 before the launch), record r is two words at 8 * (2 + 2r) bytes --
+ * the SM clock, then role << 56 | event << 48 | item << 16 | tile.  Records
+ * past the buffer are dropped (the count still grows).  Roles and events of
+ * the CSA attention kernel: 1 gather (1 K tile issued, 2 V tile issued),
+ * 2 MMA (1 QK^T issued, 2 PV issued), 3 softmax warpgroup 0 (1 scores read,
+ * 2 P written, 3 item epilogue begun, 4 item done).  Tracing serialises a
+ * little work of CTA 0 only; detach it before timing anything. */
+hyb_status hyb_trace_attach(void *buf, size_t bytes);
+
+/* Measurement kernel (the pages have no counterpart): the rate at which the
+ * SMs gather random rows held in L2 into shared memory -- the data path of the
+ * CSA attention, whose selected compressed rows differ per query token.  One
+ * CTA per SM copies rows_per_sm random 256-byte rows of `table` (device, 16-byte
+ * aligned, table_bytes bytes; keep it well under the L2 size) into a ring of
+ * `stages` (2..6) 32 KB shared-memory stages with 16-byte cp.async, rows
+ * chosen by a hash.  sink: device array of 256 uint32 receiving a checksum.
+ * Time the call with events on `stream`: bytes moved = SMs * rows_per_sm * 256
+ * (rows_per_sm is rounded down to a multiple of 128). */
+hyb_status hyb_probe_l2_gather(const void *table, long long table_bytes, long long rows_per_sm,
+                               int stages, unsigned int *sink, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -53,9 +53,17 @@ def test_host_side_argument_checks(lib):
     p = hb.problem(B=1, Lq=16, Lkv=16, Hq=4, Hkv=1, d=96, m=4, W=8)
     assert hb._lib.hyb_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, None,
                                 None) == hb.HYB_ERR_UNSUPPORTED
-    # workspace: scores of every (query row, entry) pair, fp32, 256-byte rounded
+    # workspace: none when the selection runs in one kernel (64 or more query
+    # rows per sequence, at most 4 indexer heads, Nc <= 65535) ...
     p = hb.problem(B=2, Lq=100, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=2, di=32, Nc=25)
-    assert hb.hyb_workspace_size(p) == (2 * 100 * 25 * 4 + 255) // 256 * 256
+    assert hb.hyb_workspace_size(p) == 0
+    p.Lq = 2048
+    p.Nc = 65535
+    assert hb.hyb_workspace_size(p) == 0
+    # ... otherwise the scores of every (query row, entry) pair, fp32, 256-byte rounded
+    for lq, hi, nc in ((63, 2, 25), (100, 5, 25), (100, 2, 65536)):
+        p = hb.problem(B=2, Lq=lq, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=hi, di=32, Nc=nc)
+        assert hb.hyb_workspace_size(p) == (2 * lq * nc * 4 + 255) // 256 * 256
     p.topk = 0
     assert hb.hyb_workspace_size(p) == 0
     # missing workspace is reported as such
@@ -109,8 +117,12 @@ def test_fp4_argument_checks(lib):
     # prefill: the whole caches are dequantized
     p = hb.problem(B=1, Lq=64, Lkv=64, Hq=4, Hkv=1, d=64, m=4, W=8, topk=4, Hi=2, di=32, Nc=16)
     attn = 2 * ((16 * 64 * 2 + 255) // 256 * 256)
+    index = (16 * 32 * 2 + 255) // 256 * 256    # keys dequantized once; no score rows (one-kernel selection)
+    assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
+    p.Hi = 5                                     # selection from stored score rows
     index = (64 * 16 * 4 + 255) // 256 * 256 + (16 * 32 * 2 + 255) // 256 * 256
     assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
+    p.Hi = 2
     assert hb._lib.hyb_attn_fwd_fp4(ctypes.byref(p), *([buf] * 10), None, 0, None) == hb.HYB_ERR_WORKSPACE
     assert hb._lib.hyb_csa_index_topk_fp4(ctypes.byref(p), *([buf] * 5), None, None, 0,
                                           None) == hb.HYB_ERR_WORKSPACE

@@ -49,11 +49,19 @@ def test_block_merge_matches_oracle(hb, B, L, H, dx, m):
 
 
 # ------------------------------------------------------------ indexer + top-K
-def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, pool=0):
+def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, pool=0, neg_w=False,
+                ramp=False):
     g = torch.Generator().manual_seed(seed)
     qi = _randn_bf16(g, (B, Lq, Hi, di))
     wi = torch.rand((B, Lq, Hi), generator=g)
+    if neg_w:
+        wi = wi * 2 - 1          # signed head weights: scores of either sign
     kic = _randn_bf16(g, (B, Nc, di))
+    if ramp:
+        # every key a scaled copy of one vector: each row's scores grow with
+        # the entry index, so its largest scores sit past any sampled entry
+        base = torch.randn((B, 1, di), generator=g)
+        kic = (base * (0.5 + torch.arange(Nc).reshape(1, Nc, 1) / Nc)).to(torch.bfloat16)
     if pool:
         # entries drawn from `pool` distinct rows: every score value repeats,
         # so the K-th score is an exact tie broken toward the lower index
@@ -143,6 +151,32 @@ def test_index_topk_many_rows(hb, Nc, pool):
                         rows=rows)
     if pool:
         assert exact.all()
+
+
+@pytest.mark.parametrize("case", ["ramp", "signed", "two_values", "random_pos", "all_visible", "k1",
+                                  "short_rows"])
+def test_index_topk_selection_paths(hb, case):
+    # prefill-shaped problems select in one kernel that recomputes the scores
+    # pass by pass and moves or narrows a per-row key window until the K-th
+    # score is pinned; each case drives one of its paths
+    rng = np.random.default_rng(len(case))
+    if case == "ramp":          # the K-th score lies above every sampled score
+        _index_case(hb, 1, 700, 4, 64, 3000, 4, 128, 300, seed=11, ramp=True)
+    elif case == "signed":      # negative scores (order keys below +0)
+        _index_case(hb, 2, 400, 3, 64, 2500, 4, 64, 200, seed=12, neg_w=True)
+    elif case == "two_values":  # two distinct keys: the threshold bin is one exact score
+        exact = _index_case(hb, 1, 520, 4, 32, 2000, 4, 128, 100, seed=13, pool=2)
+        assert exact.all()
+    elif case == "random_pos":  # rows of one tile with very different visible counts
+        L = 4000 * 4 + 128
+        pos = rng.integers(0, L, size=(2, 300)).astype(np.int32)
+        _index_case(hb, 2, 300, 4, 64, 4000, 4, 128, 256, q_pos=pos, seed=14)
+    elif case == "all_visible":  # K >= every row's visible count
+        _index_case(hb, 1, 777, 2, 64, 190, 4, 16, 200, seed=15)
+    elif case == "k1":
+        _index_case(hb, 1, 300, 4, 64, 500, 4, 32, 1, seed=16)
+    else:                       # rows shorter than one sampled tile
+        _index_case(hb, 1, 200, 2, 32, 60, 2, 64, 7, seed=17)
 
 
 # ----------------------------------------------------------------- attention

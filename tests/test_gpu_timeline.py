@@ -1,0 +1,60 @@
+"""The per-role timeline of the CSA attention kernel (a debug aid): CTA 0
+records, per work item, a gather, an MMA and a softmax event for every key tile,
+with clocks that never go backwards within a role; with no buffer attached
+nothing is recorded and the output is unchanged."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hb():
+    import compressed_sparse_sliding_b200 as hb
+    return hb
+
+
+def _case(hb):
+    g = torch.Generator().manual_seed(77)
+    B, L, Hq, d, m, W, K, Nc = 1, 600, 32, 128, 4, 128, 256, 150
+    q = torch.randn((B, L, Hq, d), generator=g).to(torch.bfloat16).cuda()
+    kv = [torch.randn((B, L, 1, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
+    kc = [torch.randn((B, Nc, 1, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
+    idx = torch.stack([torch.randperm(Nc, generator=g)[:K].sort().values for _ in range(L)])
+    idx = idx.to(torch.int32).reshape(B, L, K).cuda()
+    p = hb.problem(B=B, Lq=L, Lkv=L, Hq=Hq, Hkv=1, d=d, m=m, W=W, topk=K, Nc=Nc)
+    return p, q, kc, idx, kv
+
+
+def test_csa_attention_timeline(hb):
+    p, q, kc, idx, kv = _case(hb)
+    ref = hb.hyb_attn_fwd(p, q, kc[0], kc[1], idx, kv[0], kv[1])
+    buf = torch.zeros(1 << 20, dtype=torch.int64, device="cuda")
+    hb.hyb_trace_attach(buf)
+    try:
+        out = hb.hyb_attn_fwd(p, q, kc[0], kc[1], idx, kv[0], kv[1])
+        torch.cuda.synchronize()
+    finally:
+        hb.hyb_trace_attach(None)
+    assert hb.hyb_get_device_status() == hb.HYB_OK
+    assert torch.equal(out, ref)
+    rec = hb.trace_records(buf)
+    assert rec, "no records"
+    items = sorted({r["item"] for r in rec})
+    for role in (1, 2, 3):
+        clk = [r["clock"] for r in rec if r["role"] == role]
+        assert clk and np.all(np.diff(clk) >= 0), f"role {role}: clocks out of order"
+    # every item of CTA 0: K and V gathered, QK^T and PV issued, scores read and
+    # P written for each of its key tiles (2 selected tiles of 128 + the window)
+    for it in items:
+        ev = {(r["role"], r["event"]) for r in rec if r["item"] == it}
+        assert {(1, 1), (1, 2), (2, 1), (2, 2), (3, 1), (3, 2), (3, 3), (3, 4)} <= ev
+        n_qk = sum(1 for r in rec if r["item"] == it and r["role"] == 2 and r["event"] == 1)
+        n_p = sum(1 for r in rec if r["item"] == it and r["role"] == 3 and r["event"] == 2)
+        assert n_qk == n_p >= 2
+    # detached: nothing more is appended
+    n0 = int(buf[0].item())
+    hb.hyb_attn_fwd(p, q, kc[0], kc[1], idx, kv[0], kv[1])
+    torch.cuda.synchronize()
+    assert int(buf[0].item()) == n0
