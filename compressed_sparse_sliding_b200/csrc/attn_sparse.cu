@@ -50,6 +50,7 @@ constexpr int kSpD = 128;        // head dim handled by this kernel
 struct SparseParams {
     int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
     int pregathered;   // kc / vc hold each token's selected rows in slot order: [B Lq, topk, Hkv, 128]
+    int split;         // CTAs (one cluster) sharing each item's key tiles: 1 or 2
     long long n_items;
     float scale_log2;
     const int32_t *q_pos, *kv_pos0, *idx;
@@ -75,14 +76,19 @@ struct SparseSmem {
     static constexpr int OFF_INV = OFF_MREF + 2 * NH * 4;          // [NH] floats
     static constexpr int OFF_BAR = OFF_INV + NH * 4;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
-    static constexpr int OFF_IDX = OFF_MISC + 16 * 4;               // [2][topk] decoded selections
+    static constexpr int OFF_PML = OFF_MISC + 16 * 4;               // split: peer's [max, sum] per head
+    static constexpr int OFF_CMB = OFF_PML + 2 * NH * 4;            // split: [2][NH] combine factors
+    static constexpr int OFF_IDX = OFF_CMB + 2 * NH * 4;            // [2][topk] decoded selections
     static constexpr int BASE_BYTES = OFF_IDX;                      // + 2 topk * 4
 };
 
 // mbarriers (two of each per-item or per-buffer kind, three per ring stage)
 enum {
     SB_QF = 0, SB_QE = 2, SB_KF = 4, SB_KE = 7, SB_VF = 10, SB_VE = 13, SB_SF = 16, SB_PF = 18,
-    SB_OD = 20, SB_OE = 22, SB_IF = 24, SB_DONE = 26, SB_COUNT = 27
+    SB_OD = 20, SB_OE = 22, SB_IF = 24, SB_DONE = 26,
+    SB_GO = 27,      // split, rank 1: rank 0 can take this item's partial (arrived by rank 0)
+    SB_PFULL = 28,   // split, rank 0: rank 1's partial has landed (arrived by rank 1's softmax threads)
+    SB_COUNT = 29
 };
 
 struct SparseTok {
@@ -334,7 +340,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    unsigned long long *const tb = trace_buffer();   // timeline of CTA 0, when attached
+    unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
     constexpr int PW = SpRoles<NH>::PW;
     constexpr int NPT = 32 * PW;                // producer threads
 
@@ -357,6 +363,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bar[SB_VE + s], 1);
         }
         mbar_init(&bar[SB_DONE], 1);
+        mbar_init(&bar[SB_GO], 1);
+        mbar_init(&bar[SB_PFULL], SpRoles<NH>::SMT);
         mbar_fence_init();
         misc[1] = 0;
     }
@@ -368,6 +376,15 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
+    // Items go round-robin to CTAs, or to clusters of `split` CTAs that share
+    // each item's key tiles: CTA rank r takes tiles [nt r / split, nt (r+1) / split).
+    const int split = p.split;
+    const uint32_t crank = split > 1 ? cluster_ctarank() : 0u;
+    const long long w0 = blockIdx.x / split, wstep = gridDim.x / split;
+    auto tile_lo = [&](int nt) -> int { return (int)((nt * (int)crank) / split); };
+    auto tile_hi = [&](int nt) -> int { return (int)((nt * ((int)crank + 1)) / split); };
+    if (split > 1)
+        cluster_sync_all();   // the peer's barriers are initialised before any remote arrival
     // TMEM columns: S^T buffers at 0 and NH, O^T buffers at 2NH and 3NH
     const uint32_t TM_S0 = 0, TM_O0 = 2 * NH;
 
@@ -397,9 +414,9 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         };
         int jnext[kSpSelBatch];
-        if (blockIdx.x < p.n_items)
-            load_sel(blockIdx.x, 0, jnext);
-        for (long long w = blockIdx.x; w < p.n_items; w += gridDim.x, ++nq) {
+        if (w0 < p.n_items)
+            load_sel(w0, 0, jnext);
+        for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
             if (!prod_all<NPT>(ok && !*abort_flag))
                 break;
             const SparseTok k = sparse_tok(p, w);
@@ -454,9 +471,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             prod_sync<NPT>();
             // the next item's first batch, in flight during this item's copies
             // (issued after the barrier, which would otherwise wait for it)
-            if (w + gridDim.x < p.n_items)
-                load_sel(w + gridDim.x, 0, jnext);
+            if (w + wstep < p.n_items)
+                load_sel(w + wstep, 0, jnext);
             const int nt = k.nct + k.nrt;
+            const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             // source row of copy u of tile i, or -1 (zero-filled)
             auto src_of = [&](int i, int u) -> int {
                 const int r = u * RPI + rsub;
@@ -472,9 +490,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // still holds.  A tile's source rows are read into registers
             // before its copies (each copy is a compiler barrier).
             int srcv[CPT];
-            for (int i = 0; i < nt + kSpLead; ++i) {
+            for (int ii = 0; ii < ntl + kSpLead; ++ii) {
+                const int i = tb + ii;
                 int srck[CPT];
-                if (i < nt) {
+                if (ii < ntl) {
 #pragma unroll
                     for (int u = 0; u < CPT; ++u)
                         srck[u] = src_of(i, u);
@@ -494,7 +513,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     cp_async_mbar_arrive(&bar[SB_KF + ks]);
                     mbar_arrive(&bar[SB_KF + ks]);
                     if (pt == 0)
-                        trace_ev(tb, 1, 1, w, i);
+                        trace_ev(trb, 1, 1, w, i);
                     ++kc;
                 }
                 if (kSpLead == 0) {
@@ -502,7 +521,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int u = 0; u < CPT; ++u)
                         srcv[u] = srck[u];
                 }
-                if (i >= kSpLead) {
+                if (ii >= kSpLead) {
                     const __nv_bfloat16 *bv = i - kSpLead < k.nct ? p.vc : p.vr;
                     const uint32_t vs = vc % VS;
                     if (vc >= VS)
@@ -519,7 +538,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     cp_async_mbar_arrive(&bar[SB_VF + vs]);
                     mbar_arrive(&bar[SB_VF + vs]);
                     if (pt == 0)
-                        trace_ev(tb, 1, 2, w, i - kSpLead);
+                        trace_ev(trb, 1, 2, w, i - kSpLead);
                     ++vc;
                 }
                 if (kSpLead == 1) {
@@ -543,9 +562,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
             uint32_t kc = 0, vc = 0, nq = 0, gt = 0, pcnt = 0;
             bool ok = true;
-            for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x, ++nq) {
+            for (long long w = w0; ok && w < p.n_items; w += wstep, ++nq) {
                 const SparseTok k = sparse_tok(p, w);
                 const int nt = k.nct + k.nrt;
+                const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
                 const int qb = nq & 1, ob = nq & 1;
                 if (!mbar_wait(&bar[SB_QF + qb], (nq >> 1) & 1, abort_flag)) {
                     ok = false;
@@ -572,12 +592,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_OD + pb]);
                     mma_commit(&bar[SB_VE + vs]);
-                    trace_ev(tb, 2, 2, w, (int)pcnt);
+                    trace_ev(trb, 2, 2, w, (int)pcnt);
                     ++vc;
                     ++pcnt;
                     return true;
                 };
-                for (int i = 0; i < nt; ++i, ++gt) {
+                for (int ii = 0; ii < ntl; ++ii, ++gt) {
+                    const int i = tb + ii;
                     const uint32_t ks = kc % KS;
                     if (!mbar_wait(&bar[SB_KF + ks], (kc / KS) & 1, abort_flag)) {
                         ok = false;
@@ -594,20 +615,20 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_SF + (gt & 1)]);
                     mma_commit(&bar[SB_KE + ks]);
-                    trace_ev(tb, 2, 1, w, i);
+                    trace_ev(trb, 2, 1, w, i);
                     ++kc;
-                    if (i == nt - 1)
+                    if (ii == ntl - 1)
                         mma_commit(&bar[SB_QE + qb]);
-                    if (i > 0 && !issue_pv(i == 1)) {
+                    if (ii > 0 && !issue_pv(ii == 1)) {
                         ok = false;
                         break;
                     }
                 }
                 if (!ok)
                     break;
-                if (nt == 0) {
+                if (ntl == 0) {
                     mma_commit(&bar[SB_QE + qb]);
-                } else if (!issue_pv(nt == 1)) {
+                } else if (!issue_pv(ntl == 1)) {
                     ok = false;
                     break;
                 }
@@ -636,11 +657,14 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bool ok = true;
         const uint32_t prow = smem_u32(sP) + r * RB;
         const float4 *red4 = reinterpret_cast<const float4 *>(sRed);
-        for (long long w = blockIdx.x; w < p.n_items; w += gridDim.x, ++nq) {
+        float *sPml = reinterpret_cast<float *>(smem + SM::OFF_PML);   // split: peer's [max | sum]
+        float *sCmb = reinterpret_cast<float *>(smem + SM::OFF_CMB);   // split: [2][NH]
+        for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
             if (!sm_all<SMT>(ok && !*abort_flag))
                 break;
             const SparseTok k = sparse_tok(p, w);
             const int nt = k.nct + k.nrt;
+            const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             const int ob = nq & 1;
             // the item's decoded selection (key validity of its compressed tiles)
             const int *sSel = sIdx + ob * p.topk;
@@ -651,7 +675,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 lpart[h] = 0.f;
             // No global memory access inside this loop: a CTA barrier (the
             // votes below) waits for every outstanding access of its threads.
-            for (int i = 0; i < nt; ++i, ++gt) {
+            for (int ii = 0; ii < ntl; ++ii, ++gt) {
+                const int i = tb + ii;
                 const uint32_t sb = gt & 1;
                 ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag));
                 bool valid;
@@ -666,11 +691,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
                 tmem_ld_wait();
                 if (threadIdx.x == 0)
-                    trace_ev(tb, 3, 1, w, i);
+                    trace_ev(trb, 3, 1, w, i);
 #pragma unroll
                 for (int h = 0; h < NHW; ++h)
                     s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
-                bool need = i == 0;   // the first tile of an item always sets the reference
+                bool need = ii == 0;   // this CTA's first tile of an item always sets the reference
                 if (!need) {
                     const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH + hb);
                     bool exceed = false;
@@ -694,7 +719,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     sm_sync<SMT>();
                     const float *mold = sMref + mb * NH;
                     bool moved = false;
-                    if (i > 0) {
+                    if (ii > 0) {
 #pragma unroll
                         for (int h = 0; h < NHW; ++h) {
                             const float old = mold[hb + h];
@@ -775,35 +800,68 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
                 if (threadIdx.x == 0)
-                    trace_ev(tb, 3, 2, w, i);
+                    trace_ev(trb, 3, 2, w, i);
             }
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
             if (threadIdx.x == 0)
-                trace_ev(tb, 3, 3, w, nt);
+                trace_ev(trb, 3, 3, w, nt);
             warp_reduce_heads<NHW, false>(lpart, lane);
             if (head_owner) {
 #pragma unroll
                 for (int e = 0; e < HD::VPL; ++e)
                     sRed[(hb + HD::head(lane, e)) * 4 + quad] = lpart[e];
             }
-            const bool have_o = nt > 0;
+            const bool have_o = ntl > 0;
             if (have_o) {
                 ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1,
                                                         abort_flag));
                 tc_fence_after();
             }
             sm_sync<SMT>();
-            // thread h < NH (all in the first warpgroup) finishes head h
+            // thread h < NH (all in the first warpgroup) finishes head h.  With a
+            // split item, rank 1 hands its unnormalised O^T and its (max, sum)
+            // per head to rank 0 (into rank 0's P buffers, free once rank 0's
+            // last PV of the item has completed), and rank 0 combines:
+            //   M = max(m0, m1),  a_r = 2^(m_r - M),  L = a0 l0 + a1 l1,
+            //   o = (a0 O0 + a1 O1) / L,  lse = (M + log2 L) ln 2.
             const int th = threadIdx.x;
             float lse_v = -INFINITY;
-            if (th < NH) {
-                const float4 q4 = red4[th];
-                const float l = (q4.x + q4.y) + (q4.z + q4.w);
-                sInv[th] = l > 0.f ? 1.f / l : 0.f;
-                lse_v = l > 0.f ? (sMref[mb * NH + th] + log2f(l)) * 0.6931471805599453f : -INFINITY;
-                sMref[(mb ^ 1) * NH + th] = -INFINITY;   // the next item's reference
+            if (split == 1) {
+                if (th < NH) {
+                    const float4 q4 = red4[th];
+                    const float l = (q4.x + q4.y) + (q4.z + q4.w);
+                    sInv[th] = l > 0.f ? 1.f / l : 0.f;
+                    lse_v = l > 0.f ? (sMref[mb * NH + th] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                    sMref[(mb ^ 1) * NH + th] = -INFINITY;   // the next item's reference
+                }
+            } else if (crank == 0) {
+                if (th == 0)
+                    mbar_arrive_remote(cluster_addr(&bar[SB_GO], 1));
+                ok &= __all_sync(0xffffffffu, mbar_wait_cluster(&bar[SB_PFULL], nq & 1, abort_flag));
+                if (th < NH) {
+                    const float4 q4 = red4[th];
+                    const float l0 = (q4.x + q4.y) + (q4.z + q4.w);
+                    const float m0 = sMref[mb * NH + th];
+                    const float m1 = sPml[th], l1 = sPml[NH + th];
+                    const float M = fmaxf(m0, m1);
+                    const float a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M);
+                    const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+                    const float L = a0 * l0 + a1 * l1;
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    sCmb[th] = a0 * inv;
+                    sCmb[NH + th] = a1 * inv;
+                    lse_v = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+                    sMref[(mb ^ 1) * NH + th] = -INFINITY;
+                }
+            } else {
+                if (th < NH) {
+                    const float4 q4 = red4[th];
+                    sCmb[th] = sMref[mb * NH + th];
+                    sCmb[NH + th] = (q4.x + q4.y) + (q4.z + q4.w);
+                    sMref[(mb ^ 1) * NH + th] = -INFINITY;
+                }
             }
-            sm_sync<SMT>();  // sRed / sMref read, sInv written, next reference cleared
+            sm_sync<SMT>();  // sRed / sMref read, sInv / sCmb written, next reference cleared
             mb ^= 1;
             float ov[NHW];
             if (have_o) {
@@ -814,9 +872,35 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int h = 0; h < NHW; ++h)
                     ov[h] = 0.f;
             }
-            // global stores only after the last barrier of the item
-            if (ok) {
-                const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+            const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+            if (split > 1 && crank != 0) {
+                // rank 1: wait until rank 0 takes the partial, then write it there
+                ok &= __all_sync(0xffffffffu, mbar_wait_cluster(&bar[SB_GO], nq & 1, abort_flag));
+                if (ok) {
+                    const uint32_t part0 = cluster_addr(sP, 0);
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h)
+                        cluster_st_f32(part0 + (uint32_t)(((hb + h) * kSpD + r) * 4), ov[h]);
+                    if (th < NH) {
+                        cluster_st_f32(cluster_addr(sPml + th, 0), sCmb[th]);
+                        cluster_st_f32(cluster_addr(sPml + NH + th, 0), sCmb[NH + th]);
+                    }
+                }
+                mbar_arrive_remote(cluster_addr(&bar[SB_PFULL], 0));
+            } else if (ok && split > 1) {
+                // rank 0: combine with rank 1's partial ([head][d] fp32 in the P buffers)
+                const float *part = reinterpret_cast<const float *>(sP);
+#pragma unroll
+                for (int h = 0; h < NHW; ++h) {
+                    const int hh = hb + h;
+                    if (hh < p.g)
+                        p.o[obase + (size_t)hh * kSpD + r] =
+                            __float2bfloat16_rn(ov[h] * sCmb[hh] + part[hh * kSpD + r] * sCmb[NH + hh]);
+                }
+                if (p.lse && th < p.g)
+                    p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + th) * p.Lq + k.t] = lse_v;
+            } else if (ok) {
+                // global stores only after the last barrier of the item
                 const float4 *inv4 = reinterpret_cast<const float4 *>(sInv + hb);
 #pragma unroll
                 for (int h = 0; h < NHW; h += 4) {
@@ -833,11 +917,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
             if (threadIdx.x == 0)
-                trace_ev(tb, 3, 4, w, nt);
+                trace_ev(trb, 3, 4, w, nt);
         }
     }
 
     tc_fence_before();
+    if (split > 1)
+        cluster_sync_all();   // no CTA leaves while its peer may still touch its shared memory
     __syncthreads();
     if (warp == SpRoles<NH>::MMA_WARP) {
         tc_fence_after();
@@ -862,7 +948,7 @@ static bool make_map_2d(CUtensorMap *map, const void *base, long long rows, int 
 }
 
 template <int NH>
-static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void *kc, const void *vc,
+static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, const void *vc,
                                 const void *kr, const void *vr, cudaStream_t stream, int num_sms)
 {
     using SM = SparseSmem<NH>;
@@ -886,13 +972,38 @@ static cudaError_t launch_csa_t(const SparseParams &p, const void *q, const void
         return e;
     if (per_sm < 1)
         return cudaErrorLaunchOutOfResources;
-    long long grid = (long long)num_sms * per_sm;
-    if (grid > p.n_items)
-        grid = p.n_items;
-    if (grid < 1)
-        return cudaSuccess;
-    kern<<<(unsigned)grid, SpRoles<NH>::THREADS, smem, stream>>>(mq, mkc, mvc, mkr, mvr, p);
-    return cudaGetLastError();
+    const long long slots = (long long)num_sms * per_sm;
+    // Few items (decode): two CTAs, one cluster, share each item's key tiles,
+    // so that twice as many SMs gather; otherwise one CTA per item.
+    p.split = (p.n_items * 2 <= slots) ? 2 : 1;
+    if (p.split == 1) {
+        long long grid = slots < p.n_items ? slots : p.n_items;
+        if (grid < 1)
+            return cudaSuccess;
+        kern<<<(unsigned)grid, SpRoles<NH>::THREADS, smem, stream>>>(mq, mkc, mvc, mkr, mvr, p);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(SpRoles<NH>::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int max_clusters = 0;
+    cfg.gridDim = dim3(2 * (unsigned)p.n_items, 1, 1);
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    if (e != cudaSuccess)
+        return e;
+    if (max_clusters < 1)
+        return cudaErrorLaunchOutOfResources;
+    const long long clusters = max_clusters < p.n_items ? max_clusters : p.n_items;
+    cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+    return cudaLaunchKernelEx(&cfg, kern, mq, mkc, mvc, mkr, mvr, p);
 }
 
 // CSA attention with per-token selections, head dim 128, Hq / Hkv <= 64.
@@ -918,6 +1029,7 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
     if (p.n_items >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.pregathered = pregathered;
+    p.split = 1;
     if (pregathered && (long long)B * Lq * topk * Hkv >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.scale_log2 = scale * 1.4426950408889634f;

@@ -567,33 +567,6 @@ topk_hist(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
 constexpr int kTcThreads = 256;
 constexpr int kTcCS = 8;
 
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of the same shared variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ int cluster_ld(uint32_t addr)
-{
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 template <int KPT>
 __global__ void __launch_bounds__(kTcThreads)
 topk_cluster(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
