@@ -100,6 +100,8 @@ try:
     _lib.hyb_get_device_status.restype = _I
     _lib.hyb_error_string.argtypes = [_I]
     _lib.hyb_error_string.restype = ctypes.c_char_p
+    _lib.hyb_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    _lib.hyb_set_wait_limit_ns.restype = _I
     _lib.hyb_trace_attach.argtypes = [_P, ctypes.c_size_t]
     _lib.hyb_trace_attach.restype = _I
     _lib.hyb_probe_l2_gather.argtypes = [_P, ctypes.c_longlong, ctypes.c_longlong, _I, _P, _P]
@@ -413,3 +415,10 @@ def hyb_probe_l2_gather(table: torch.Tensor, rows_per_sm: int, stages: int, sink
                                   int(stages), _ptr(sink), _stream(stream))
     if st != HYB_OK:
         raise HybError(st, "hyb_probe_l2_gather")
+
+
+def hyb_set_wait_limit_ns(ns: int) -> None:
+    """Bound of the kernels' waits for later launches (0: the default 200 ms)."""
+    st = _lib.hyb_set_wait_limit_ns(int(ns))
+    if st != HYB_OK:
+        raise HybError(st, "hyb_set_wait_limit_ns")

@@ -664,6 +664,12 @@ hyb_status hyb_get_device_status(cudaStream_t stream)
     return (hyb_status)v;
 }
 
+hyb_status hyb_set_wait_limit_ns(unsigned long long ns)
+{
+    const uint64_t v = ns ? (uint64_t)ns : kWaitLimitNs;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? HYB_OK : HYB_ERR_CUDA;
+}
+
 hyb_status hyb_trace_attach(void *buf, size_t bytes)
 {
     unsigned long long *b = static_cast<unsigned long long *>(buf);

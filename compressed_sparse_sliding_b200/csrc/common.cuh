@@ -29,6 +29,12 @@ __device__ __forceinline__ void set_error(int code)
 // host reads the status word: waits of every other CTA then give up at once.
 constexpr uint64_t kWaitLimitNs = 200000000ull;
 
+// The bound that ordinary waits use, settable by hyb_set_wait_limit_ns (a
+// failure-detection test shortens it so that waits run out).  Waits that
+// drain a CTA's own asynchronous copies and MMAs while it unwinds keep
+// kWaitLimitNs, so that nothing is left in flight when the CTA exits.
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+
 __device__ __forceinline__ bool timed_out_somewhere()
 {
     return *reinterpret_cast<volatile int *>(&g_status) == HYB_ERR_DEVICE_TIMEOUT;
@@ -120,7 +126,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     uint32_t addr = smem_u32(bar);
     if (mbar_try_wait(addr, parity))
         return true;
-    uint64_t t0 = global_ns();
+    const uint64_t t0 = global_ns();
+    const uint64_t lim = *reinterpret_cast<volatile uint64_t *>(&g_wait_limit_ns);
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(addr, parity))
             return true;
@@ -130,7 +137,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             *abort_flag = 1;
             return false;
         }
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > lim) {
             set_error(HYB_ERR_DEVICE_TIMEOUT);
             *abort_flag = 1;
             return false;
@@ -201,6 +208,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
     if (try_once())
         return true;
     const uint64_t t0 = global_ns();
+    const uint64_t lim = *reinterpret_cast<volatile uint64_t *>(&g_wait_limit_ns);
     for (uint32_t it = 1;; ++it) {
         if (try_once())
             return true;
@@ -210,7 +218,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
             *abort_flag = 1;
             return false;
         }
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > lim) {
             set_error(HYB_ERR_DEVICE_TIMEOUT);
             *abort_flag = 1;
             return false;

@@ -134,10 +134,11 @@ __device__ __forceinline__ bool fx_all(bool v)
 __device__ __forceinline__ bool fx_wait_decided(volatile int *decided, int p, volatile int *abort_flag)
 {
     const uint64_t t0 = global_ns();
+    const uint64_t lim = *reinterpret_cast<volatile uint64_t *>(&g_wait_limit_ns);
     while (*decided < p) {
         if (*abort_flag)
             return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > lim) {
             set_error(HYB_ERR_DEVICE_TIMEOUT);
             *abort_flag = 1;
             return false;

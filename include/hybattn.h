@@ -295,6 +295,17 @@ hyb_status hyb_get_device_status(cudaStream_t stream);
 /* Static description of a status code. */
 const char *hyb_error_string(hyb_status status);
 
+/* Failure detection (the pages have no counterpart): every wait inside a
+ * kernel is bounded; when one runs out the kernel records
+ * HYB_ERR_DEVICE_TIMEOUT in the status word and every CTA unwinds (waits for
+ * its own copies and MMAs in flight, frees its tensor memory, returns).  The
+ * bound is 200 ms; this sets it for later launches on the current device
+ * (0 restores 200 ms).  A tiny bound makes the first wait that is not already
+ * satisfied run out -- the way a test exercises the error path without a
+ * fault.  Read the status (hyb_get_device_status) before launching with the
+ * normal bound again: a recorded timeout makes later waits give up too. */
+hyb_status hyb_set_wait_limit_ns(unsigned long long ns);
+
 /* Debug aid (the pages have no counterpart): a per-role timeline of one CTA.
  * Attaches a caller-owned device buffer of `bytes` bytes (16-byte aligned,
  * >= 32) for the kernels launched afterwards on the current device; NULL
