@@ -152,6 +152,15 @@ __device__ __forceinline__ bool prod_all(bool v)
     return r != 0;
 }
 
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
 {
     asm volatile(
@@ -494,24 +503,40 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int i = tb + ii;
                 int srck[CPT];
                 if (ii < ntl) {
-#pragma unroll
-                    for (int u = 0; u < CPT; ++u)
-                        srck[u] = src_of(i, u);
-                    const __nv_bfloat16 *bk = i < k.nct ? p.kc : p.kr;
                     const uint32_t ks = kc % KS;
                     if (kc >= KS)
                         ok &= __all_sync(0xffffffffu,
                                          mbar_wait(&bar[SB_KE + ks], ((kc / KS) - 1) & 1, abort_flag));
-                    const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
+                    if (i >= k.nct) {
+                        // window tile: 128 consecutive raw rows, two TMA boxes
+                        // (rows past the window are masked by the softmax)
+                        if (pt == 0) {
+                            const int r0 = k.b * p.Lkv + k.rlo + (i - k.nct) * kSpBN;
+                            mbar_arrive_expect_tx(&bar[SB_KF + ks], SM::KV_BYTES);
+                            tma_load_3d(sK + ks * SM::KV_BYTES, &tm_kr, &bar[SB_KF + ks], 0, k.kvh, r0);
+                            tma_load_3d(sK + ks * SM::KV_BYTES + kSpBN * 128, &tm_kr, &bar[SB_KF + ks], 64,
+                                        k.kvh, r0);
+                        } else {
+                            mbar_arrive(&bar[SB_KF + ks]);
+                        }
 #pragma unroll
-                    for (int u = 0; u < CPT; ++u) {
-                        const int r = u * RPI + rsub;
-                        const int sr = srck[u];
-                        cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                    bk + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
+                        for (int u = 0; u < CPT; ++u)
+                            srck[u] = -1;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < CPT; ++u)
+                            srck[u] = src_of(i, u);
+                        const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
+#pragma unroll
+                        for (int u = 0; u < CPT; ++u) {
+                            const int r = u * RPI + rsub;
+                            const int sr = srck[u];
+                            cp_async_16(dst + sw128_offset(r, c8 & 7),
+                                        p.kc + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
+                        }
+                        cp_async_mbar_arrive(&bar[SB_KF + ks]);
+                        mbar_arrive(&bar[SB_KF + ks]);
                     }
-                    cp_async_mbar_arrive(&bar[SB_KF + ks]);
-                    mbar_arrive(&bar[SB_KF + ks]);
                     if (pt == 0)
                         trace_ev(trb, 1, 1, w, i);
                     ++kc;
@@ -522,21 +547,33 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         srcv[u] = srck[u];
                 }
                 if (ii >= kSpLead) {
-                    const __nv_bfloat16 *bv = i - kSpLead < k.nct ? p.vc : p.vr;
+                    const int iv = i - kSpLead;
                     const uint32_t vs = vc % VS;
                     if (vc >= VS)
                         ok &= __all_sync(0xffffffffu,
                                          mbar_wait(&bar[SB_VE + vs], ((vc / VS) - 1) & 1, abort_flag));
-                    const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
+                    if (iv >= k.nct) {
+                        if (pt == 0) {
+                            const int r0 = k.b * p.Lkv + k.rlo + (iv - k.nct) * kSpBN;
+                            mbar_arrive_expect_tx(&bar[SB_VF + vs], SM::KV_BYTES);
+                            tma_load_3d(sV + vs * SM::KV_BYTES, &tm_vr, &bar[SB_VF + vs], 0, k.kvh, r0);
+                            tma_load_3d(sV + vs * SM::KV_BYTES + kSpBN * 128, &tm_vr, &bar[SB_VF + vs], 64,
+                                        k.kvh, r0);
+                        } else {
+                            mbar_arrive(&bar[SB_VF + vs]);
+                        }
+                    } else {
+                        const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
 #pragma unroll
-                    for (int u = 0; u < CPT; ++u) {
-                        const int r = u * RPI + rsub;
-                        const int sr = srcv[u];
-                        cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                    bv + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
+                        for (int u = 0; u < CPT; ++u) {
+                            const int r = u * RPI + rsub;
+                            const int sr = srcv[u];
+                            cp_async_16(dst + sw128_offset(r, c8 & 7),
+                                        p.vc + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
+                        }
+                        cp_async_mbar_arrive(&bar[SB_VF + vs]);
+                        mbar_arrive(&bar[SB_VF + vs]);
                     }
-                    cp_async_mbar_arrive(&bar[SB_VF + vs]);
-                    mbar_arrive(&bar[SB_VF + vs]);
                     if (pt == 0)
                         trace_ev(trb, 1, 2, w, i - kSpLead);
                     ++vc;
@@ -931,6 +968,22 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
+// 3-D map over a [rows, heads, 128] bf16 view with a (64, 1, 128) box, 128-byte swizzle.
+static bool make_map_3d_rows(CUtensorMap *map, const void *base, int heads, long long rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kSpD, (cuuint64_t)heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)kSpD * 2, (cuuint64_t)kSpD * 2 * heads};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kSpBN};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 2-D map over a [rows, 128] bf16 view with a (64, box_rows) box, 128-byte swizzle.
 static bool make_map_2d(CUtensorMap *map, const void *base, long long rows, int box_rows)
 {
@@ -957,8 +1010,10 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
     const long long crow = p.pregathered ? (long long)p.B * p.Lq * p.topk * p.Hkv : (long long)p.B * p.Nc * p.Hkv;
     ok &= make_map_2d(&mkc, kc, crow, 1);
     ok &= make_map_2d(&mvc, vc, crow, 1);
-    ok &= make_map_2d(&mkr, kr, (long long)p.B * p.Lkv * p.Hkv, 1);
-    ok &= make_map_2d(&mvr, vr, (long long)p.B * p.Lkv * p.Hkv, 1);
+    // raw rows [B Lkv, Hkv, 128] as (128, Hkv, B Lkv): one box = 64 channels of
+    // 128 consecutive rows of one KV head (a window tile half)
+    ok &= make_map_3d_rows(&mkr, kr, p.Hkv, (long long)p.B * p.Lkv);
+    ok &= make_map_3d_rows(&mvr, vr, p.Hkv, (long long)p.B * p.Lkv);
     if (!ok)
         return cudaErrorInvalidValue;
     size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.topk * 8;
@@ -1026,7 +1081,7 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
     p.topk = topk;
     p.NH = p.g <= 16 ? 16 : (p.g <= 32 ? 32 : 64);
     p.n_items = (long long)B * Lq * Hkv;
-    if (p.n_items >= (1ll << 31))
+    if (p.n_items >= (1ll << 31) || (long long)B * Lkv >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.pregathered = pregathered;
     p.split = 1;

@@ -172,6 +172,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     volatile int *last_pass = misc + 3;    // index of the E pass once known
     // bars: 0 Q full, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
 
     // heavy token tiles first, all sequences of one weight class together
     const int ttile = p.n_ttiles - 1 - (int)(blockIdx.x / p.B);
@@ -255,6 +256,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int start = (has_sel && q == 0) ? soff[i] : i * kFxBN;
                     mbar_arrive_expect_tx(&bar[1 + s], SM::K_BYTES);
                     tma_load_4d(sK + s * SM::K_BYTES, &tm_k, &bar[1 + s], 0, 0, start, b);
+                    trace_ev(trb, 1, 1, q, i);
                     ++issued;
                 }
             }
@@ -292,6 +294,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     mma_commit(&bar[9 + db]);
                     mma_commit(&bar[5 + s]);
+                    trace_ev(trb, 2, 1, q, i);
                 }
             }
             mma_commit(&bar[13]);
@@ -402,6 +405,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     }
                 }
+                if (threadIdx.x == 128)
+                    trace_ev(trb, 3, 1, q, i);
             }
             // ------------------------------ end of pass q ------------------------------
             if (!fx_all(ok)) {
@@ -504,6 +509,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const bool all_set = fx_all(mode != FX_OPEN);
                 if (all_set)
                     lastp = q + 1;
+                if (threadIdx.x == 128)
+                    trace_ev(trb, 3, 2, q, all_set ? 1 : 0);
                 if (threadIdx.x == 128) {
                     if (all_set) {
                         *last_pass = q + 1;       // the next pass emits
@@ -517,6 +524,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         // ---- boundary bin: take the `need` largest (lower index first), merge ----
+        if (threadIdx.x == 128)
+            trace_ev(trb, 3, 3, lastp, nb);
         if (emitted && mode == FX_BIN) {
             // largest key T in [blo, bhi_m1] with #(key >= T) >= need
             uint32_t lo_b = blo, hi_b = bhi_m1;
@@ -586,6 +595,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             pos = K;
         }
+        if (threadIdx.x == 128)
+            trace_ev(trb, 3, 4, lastp, mode);
         if ((emitted || lastp < 0) && mode != FX_NONE) {
             for (int u = pos; u < K; ++u) {
                 orow[u] = -1;

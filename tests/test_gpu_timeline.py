@@ -17,7 +17,7 @@ def hb():
 
 def _case(hb):
     g = torch.Generator().manual_seed(77)
-    B, L, Hq, d, m, W, K, Nc = 1, 600, 32, 128, 4, 128, 256, 150
+    B, L, Hq, d, m, W, K, Nc = 1, 600, 32, 128, 4, 128, 256, 400
     q = torch.randn((B, L, Hq, d), generator=g).to(torch.bfloat16).cuda()
     kv = [torch.randn((B, L, 1, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
     kc = [torch.randn((B, Nc, 1, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
