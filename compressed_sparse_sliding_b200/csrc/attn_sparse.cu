@@ -46,6 +46,11 @@ constexpr int kSpBN = 128;       // keys per tile (the M of S^T)
 constexpr int kSpSelBatch = 8;   // selection entries a producer thread loads at once
 constexpr int kSpLead = 1;       // tiles by which the K copies run ahead of the V copies
 constexpr int kSpD = 128;        // head dim handled by this kernel
+// Selected rows of K / V through TMA tile::gather4 (four rows of one 64-column
+// half per instruction, issued by 64 producer threads per tile) instead of
+// 16-byte cp.async.
+constexpr bool kSpGatherK4 = false;
+constexpr bool kSpGatherV4 = false;
 
 struct SparseParams {
     int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
@@ -158,6 +163,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Rows r0..r3 (64 columns from column c) of a 2-D map with a one-row box.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int c, int r0, int r1,
+                                            int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -522,6 +538,25 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int u = 0; u < CPT; ++u)
                             srck[u] = -1;
+                    } else if (kSpGatherK4) {
+                        if (pt < 64) {
+                            const int grp = pt >> 1, hf = pt & 1;
+                            int rr[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int sidx = i * kSpBN + 4 * grp + j;
+                                const int sr = sidx < p.topk ? sSel[sidx] : -1;
+                                rr[j] = sr >= 0 ? sr : 0;
+                            }
+                            mbar_arrive_expect_tx(&bar[SB_KF + ks], 4 * 128);
+                            tma_gather4(sK + ks * SM::KV_BYTES + hf * kSpBN * 128 + grp * 4 * 128, &tm_kc,
+                                        &bar[SB_KF + ks], hf * 64, rr[0], rr[1], rr[2], rr[3]);
+                        } else {
+                            mbar_arrive(&bar[SB_KF + ks]);
+                        }
+#pragma unroll
+                        for (int u = 0; u < CPT; ++u)
+                            srck[u] = src_of(i, u);
                     } else {
 #pragma unroll
                         for (int u = 0; u < CPT; ++u)
@@ -559,6 +594,22 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             tma_load_3d(sV + vs * SM::KV_BYTES, &tm_vr, &bar[SB_VF + vs], 0, k.kvh, r0);
                             tma_load_3d(sV + vs * SM::KV_BYTES + kSpBN * 128, &tm_vr, &bar[SB_VF + vs], 64,
                                         k.kvh, r0);
+                        } else {
+                            mbar_arrive(&bar[SB_VF + vs]);
+                        }
+                    } else if (kSpGatherV4) {
+                        if (pt < 64) {
+                            const int grp = pt >> 1, hf = pt & 1;
+                            int rr[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int sidx = iv * kSpBN + 4 * grp + j;
+                                const int sr = sidx < p.topk ? sSel[sidx] : -1;
+                                rr[j] = sr >= 0 ? sr : 0;
+                            }
+                            mbar_arrive_expect_tx(&bar[SB_VF + vs], 4 * 128);
+                            tma_gather4(sV + vs * SM::KV_BYTES + hf * kSpBN * 128 + grp * 4 * 128, &tm_vc,
+                                        &bar[SB_VF + vs], hf * 64, rr[0], rr[1], rr[2], rr[3]);
                         } else {
                             mbar_arrive(&bar[SB_VF + vs]);
                         }

@@ -573,8 +573,9 @@ topk_cluster(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int
              const int32_t *__restrict__ q_pos, int32_t *__restrict__ idx_out, float *__restrict__ sel_scores)
 {
     constexpr int NT = kTcThreads;
-    constexpr int PER = kHbBins / NT;
-    __shared__ int hist[2][kHbBins];
+    constexpr int PER = kHbBins / NT;   // bins per thread, contiguous
+    __shared__ int hist[kHbBins];       // this CTA's counts of the round
+    __shared__ int tot[3][kHbBins];     // rank 0: the cluster's counts, buffer (round mod 3)
     __shared__ int s_scan[32];
     __shared__ int s_sel[3];
     __shared__ int s_cnt[2];            // this CTA's (greater, equal) counts, read by peers
@@ -625,54 +626,69 @@ topk_cluster(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int
         for (int u = 0; u < KPT; ++u)
             key[u] = u < nv ? order_key(__ldg(src + i0 + u)) : 0u;
     }
-    for (int i = threadIdx.x; i < kHbBins; i += NT)
-        hist[0][i] = 0;
-    __syncthreads();
+    for (int i = threadIdx.x; i < kHbBins; i += NT) {
+        hist[i] = 0;
+        tot[0][i] = 0;
+        tot[1][i] = 0;
+        tot[2][i] = 0;
+    }
+    // rank 0's totals are zero before any peer adds into them
+    cluster_sync_all();
 
     uint32_t lo = 0u, hi = 0xFFFFFFFFu;
     int need = keff;
     bool whole = false;
     uint32_t T = lo;
+    const int b0 = (int)threadIdx.x * PER;    // this thread's bins (descending scan order below)
 #pragma unroll 1
     for (int rnd = 0; lo < hi; ++rnd) {
         const uint32_t span = hi - lo;
         const int bits = 32 - __clz(span);
         const int sh = bits > 11 ? bits - 11 : 0;
-        int *h = hist[rnd & 1];
-        int *hn = hist[(rnd + 1) & 1];
 #pragma unroll
         for (int u = 0; u < KPT; ++u)
             if (u < nv && key[u] >= lo && key[u] <= hi)
-                atomicAdd(&h[(key[u] - lo) >> sh], 1);
-        // every CTA's histogram of this round is complete; every peer has
-        // finished reading the other buffer (last round's)
-        cluster_sync_all();
-        for (int i = threadIdx.x; i < kHbBins; i += NT)
-            hn[i] = 0;
-        int mine = 0;
+                atomicAdd(&hist[(key[u] - lo) >> sh], 1);
+        __syncthreads();
+        // add this CTA's counts into rank 0's totals of the round, and clear
+        // them for the next round (each thread its own bins)
+        const uint32_t tr = cluster_addr(&tot[rnd % 3][0], 0);
 #pragma unroll
         for (int q = 0; q < PER; ++q) {
-            const int bin = kHbBins - 1 - ((int)threadIdx.x * PER + q);
-#pragma unroll
-            for (int c = 0; c < kTcCS; ++c)
-                mine += cluster_ld(cluster_addr(&h[bin], (uint32_t)c));
+            const int c = hist[b0 + q];
+            if (c) {
+                asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(tr + (uint32_t)(b0 + q) * 4u), "r"(c)
+                             : "memory");
+                hist[b0 + q] = 0;
+            }
         }
+        cluster_sync_all();   // every CTA's counts are in rank 0's totals
+        if (rank == 0) {
+            // the buffer of the previous round: its readers passed the barrier above
+            for (int i = threadIdx.x; i < kHbBins; i += NT)
+                tot[(rnd + 2) % 3][i] = 0;
+        }
+        // this thread's PER bins counted down from the top: bins NB-1-b0-q
+        int v[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q)
+            v[q] = cluster_ld(tr + (uint32_t)(kHbBins - 1 - (b0 + q)) * 4u);
+        int mine = 0;
+#pragma unroll
+        for (int q = 0; q < PER; ++q)
+            mine += v[q];
         const int ex = blk_excl_scan<NT>(mine, s_scan);
         if (ex < need && ex + mine >= need) {
             int acc = ex;
-#pragma unroll 1
+#pragma unroll
             for (int q = 0; q < PER; ++q) {
-                const int bin = kHbBins - 1 - ((int)threadIdx.x * PER + q);
-                int c = 0;
-                for (int cc = 0; cc < kTcCS; ++cc)
-                    c += cluster_ld(cluster_addr(&h[bin], (uint32_t)cc));
-                if (acc + c >= need) {
-                    s_sel[0] = bin;
+                if (acc + v[q] >= need) {
+                    s_sel[0] = kHbBins - 1 - (b0 + q);
                     s_sel[1] = acc;
-                    s_sel[2] = c;
+                    s_sel[2] = v[q];
                     break;
                 }
-                acc += c;
+                acc += v[q];
             }
         }
         __syncthreads();
