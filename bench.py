@@ -398,9 +398,19 @@ def gate_logits(w, device, rank=0):
     return (torch.randn((w.B, w.Lq, w.Hq, 3), generator=g) * 2).to(device)
 
 
+def workload_of(args):
+    """The workload of --config, with --seq-len (prefill only) shortening its
+    sequences for small profiler captures; the full sizes otherwise."""
+    import dataclasses
+    w = WORKLOADS[args.config]
+    if getattr(args, "seq_len", None) and not w.is_decode:
+        w = dataclasses.replace(w, L=int(args.seq_len), name=f"{w.name}_l{int(args.seq_len)}")
+    return w
+
+
 def run_gpu(args, rank, world):
     import compressed_sparse_sliding_b200 as hb
-    w = WORKLOADS[args.config]
+    w = workload_of(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_inputs(w, device=dev, seed=replica_seed(w, rank))
     if not w.is_decode:
@@ -720,7 +730,7 @@ def kc_f64(bits, b):
 
 
 def run_reference_arm(args):
-    w = WORKLOADS[args.config]
+    w = workload_of(args)
     per_step = []
     base = None
     gated = args.variant == "gated"
@@ -810,6 +820,9 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="shorter sequences of a prefill workload (small profiler captures); "
+                         "the full workload when absent")
     ap.add_argument("--micro", action="store_true",
                     help="print the measured roofline denominators (HBM copy, L2 gather, bf16 GEMM) and exit")
     ap.add_argument("--variant", default="hybrid", choices=["hybrid", "gated", "fp4", "train"],
@@ -847,7 +860,7 @@ def main():
     try:
         res = run_gpu(args, rank, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = run_oracle(WORKLOADS[args.config], gated=args.variant == "gated",
+            res["cpu_baseline"] = run_oracle(workload_of(args), gated=args.variant == "gated",
                                              fp4=args.variant == "fp4", train=args.variant == "train")
         if rank == 0:
             print(json.dumps(res), flush=True)

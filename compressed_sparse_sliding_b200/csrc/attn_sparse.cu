@@ -46,16 +46,12 @@ constexpr int kSpBN = 128;       // keys per tile (the M of S^T)
 constexpr int kSpSelBatch = 8;   // selection entries a producer thread loads at once
 constexpr int kSpLead = 1;       // tiles by which the K copies run ahead of the V copies
 constexpr int kSpD = 128;        // head dim handled by this kernel
-// Selected rows of K / V through TMA tile::gather4 (four rows of one 64-column
-// half per instruction, issued by 64 producer threads per tile) instead of
-// 16-byte cp.async.
-constexpr bool kSpGatherK4 = false;
-constexpr bool kSpGatherV4 = false;
 
 struct SparseParams {
     int B, Lq, Lkv, Hq, Hkv, g, Nc, m, W, topk, NH;
     int pregathered;   // kc / vc hold each token's selected rows in slot order: [B Lq, topk, Hkv, 128]
     int split;         // CTAs (one cluster) sharing each item's key tiles: 1 or 2
+    int tsel;          // entries of a decoded selection table: topk rounded up to whole tiles
     long long n_items;
     float scale_log2;
     const int32_t *q_pos, *kv_pos0, *idx;
@@ -83,8 +79,8 @@ struct SparseSmem {
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
     static constexpr int OFF_PML = OFF_MISC + 16 * 4;               // split: peer's [max, sum] per head
     static constexpr int OFF_CMB = OFF_PML + 2 * NH * 4;            // split: [2][NH] combine factors
-    static constexpr int OFF_IDX = OFF_CMB + 2 * NH * 4;            // [2][topk] decoded selections
-    static constexpr int BASE_BYTES = OFF_IDX;                      // + 2 topk * 4
+    static constexpr int OFF_IDX = OFF_CMB + 2 * NH * 4;            // [2][tsel] decoded selections
+    static constexpr int BASE_BYTES = OFF_IDX;                      // + 2 tsel * 4, tsel = topk rounded up to 128
 };
 
 // mbarriers (two of each per-item or per-buffer kind, three per ring stage)
@@ -163,17 +159,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Rows r0..r3 (64 columns from column c) of a 2-D map with a one-row box.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int c, int r0, int r1,
-                                            int r2, int r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -463,7 +448,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // every slot, or -1 (unselected, invisible or out of range).  A
             // batch's loads are all in flight together; the first batch was
             // loaded during the previous item's copies.
-            int *sSel = sIdx + qb * p.topk;
+            int *sSel = sIdx + qb * p.tsel;
             {
                 const long long wstart = k.pos - p.W + 1;
 #pragma unroll 1
@@ -491,6 +476,9 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                     }
                 }
+                // slots past topk in the last selected tile
+                for (int q = p.topk + pt; q < p.tsel; q += NPT)
+                    sSel[q] = -1;
             }
             mbar_arrive(&bar[SB_IF + qb]);      // the softmax reads key validity from it
             prod_sync<NPT>();
@@ -501,15 +489,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int nt = k.nct + k.nrt;
             const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             // source row of copy u of tile i, or -1 (zero-filled)
-            auto src_of = [&](int i, int u) -> int {
-                const int r = u * RPI + rsub;
-                if (i < k.nct) {
-                    const int sidx = i * kSpBN + r;
-                    return sidx < p.topk ? sSel[sidx] : -1;
-                }
-                const int rr = k.rlo + (i - k.nct) * kSpBN + r;
-                return rr <= k.rhi ? (k.b * p.Lkv + rr) * p.Hkv + k.kvh : -1;
-            };
+            // source row of copy u of selected tile i; an unselected slot reads
+            // row 0 (finite data the softmax masks) rather than a zero fill
+            auto src_of = [&](int i, int u) -> int { return max(sSel[i * kSpBN + u * RPI + rsub], 0); };
+            const __nv_bfloat16 *kc8 = p.kc + c8 * 8, *vc8 = p.vc + c8 * 8;   // this thread's chunk
             // K of tile i goes out kSpLead tiles ahead of V of the same tile, so
             // that the next scores need not queue behind a V stage that a PV
             // still holds.  A tile's source rows are read into registers
@@ -538,37 +521,14 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int u = 0; u < CPT; ++u)
                             srck[u] = -1;
-                    } else if (kSpGatherK4) {
-                        if (pt < 64) {
-                            const int grp = pt >> 1, hf = pt & 1;
-                            int rr[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int sidx = i * kSpBN + 4 * grp + j;
-                                const int sr = sidx < p.topk ? sSel[sidx] : -1;
-                                rr[j] = sr >= 0 ? sr : 0;
-                            }
-                            mbar_arrive_expect_tx(&bar[SB_KF + ks], 4 * 128);
-                            tma_gather4(sK + ks * SM::KV_BYTES + hf * kSpBN * 128 + grp * 4 * 128, &tm_kc,
-                                        &bar[SB_KF + ks], hf * 64, rr[0], rr[1], rr[2], rr[3]);
-                        } else {
-                            mbar_arrive(&bar[SB_KF + ks]);
-                        }
-#pragma unroll
-                        for (int u = 0; u < CPT; ++u)
-                            srck[u] = src_of(i, u);
                     } else {
 #pragma unroll
                         for (int u = 0; u < CPT; ++u)
                             srck[u] = src_of(i, u);
                         const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
 #pragma unroll
-                        for (int u = 0; u < CPT; ++u) {
-                            const int r = u * RPI + rsub;
-                            const int sr = srck[u];
-                            cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                        p.kc + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
-                        }
+                        for (int u = 0; u < CPT; ++u)
+                            cp_async_16_full(dst + sw128_offset(u * RPI + rsub, c8 & 7), kc8 + (size_t)srck[u] * kSpD);
                         cp_async_mbar_arrive(&bar[SB_KF + ks]);
                         mbar_arrive(&bar[SB_KF + ks]);
                     }
@@ -597,31 +557,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         } else {
                             mbar_arrive(&bar[SB_VF + vs]);
                         }
-                    } else if (kSpGatherV4) {
-                        if (pt < 64) {
-                            const int grp = pt >> 1, hf = pt & 1;
-                            int rr[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const int sidx = iv * kSpBN + 4 * grp + j;
-                                const int sr = sidx < p.topk ? sSel[sidx] : -1;
-                                rr[j] = sr >= 0 ? sr : 0;
-                            }
-                            mbar_arrive_expect_tx(&bar[SB_VF + vs], 4 * 128);
-                            tma_gather4(sV + vs * SM::KV_BYTES + hf * kSpBN * 128 + grp * 4 * 128, &tm_vc,
-                                        &bar[SB_VF + vs], hf * 64, rr[0], rr[1], rr[2], rr[3]);
-                        } else {
-                            mbar_arrive(&bar[SB_VF + vs]);
-                        }
                     } else {
                         const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
 #pragma unroll
-                        for (int u = 0; u < CPT; ++u) {
-                            const int r = u * RPI + rsub;
-                            const int sr = srcv[u];
-                            cp_async_16(dst + sw128_offset(r, c8 & 7),
-                                        p.vc + (size_t)(sr >= 0 ? sr : 0) * kSpD + c8 * 8, sr >= 0 ? 16u : 0u);
-                        }
+                        for (int u = 0; u < CPT; ++u)
+                            cp_async_16_full(dst + sw128_offset(u * RPI + rsub, c8 & 7), vc8 + (size_t)srcv[u] * kSpD);
                         cp_async_mbar_arrive(&bar[SB_VF + vs]);
                         mbar_arrive(&bar[SB_VF + vs]);
                     }
@@ -744,6 +684,15 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t nq = 0, gt = 0, mb = 0;
         bool ok = true;
         const uint32_t prow = smem_u32(sP) + r * RB;
+        // byte offsets of this thread's 16-byte chunks in its P^T row (swizzle matching NH)
+        uint32_t pphys[NHW / 8];
+#pragma unroll
+        for (int cl = 0; cl < NHW / 8; ++cl) {
+            const uint32_t c = (uint32_t)(hb / 8 + cl);
+            const uint32_t ph = RB == 128 ? (c ^ (r & 7)) : (RB == 64 ? (c ^ ((r >> 1) & 3)) : (c ^ ((r >> 2) & 1)));
+            pphys[cl] = ph * 16u;
+        }
+        const bool trace0 = trb != nullptr && threadIdx.x == 0;
         const float4 *red4 = reinterpret_cast<const float4 *>(sRed);
         float *sPml = reinterpret_cast<float *>(smem + SM::OFF_PML);   // split: peer's [max | sum]
         float *sCmb = reinterpret_cast<float *>(smem + SM::OFF_CMB);   // split: [2][NH]
@@ -755,12 +704,39 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             const int ob = nq & 1;
             // the item's decoded selection (key validity of its compressed tiles)
-            const int *sSel = sIdx + ob * p.topk;
+            const int *sSel = sIdx + ob * p.tsel;
             ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_IF + ob], (nq >> 1) & 1, abort_flag));
-            float lpart[NHW];
+            // partial row sums (packed pairs), the warpgroup's reference maxima
+            // as -m and as raw-score thresholds (m + 8) / scale, kept in
+            // registers and reloaded only when a tile moves them
+            uint64_t lp2[NHW / 2];
 #pragma unroll
-            for (int h = 0; h < NHW; ++h)
-                lpart[h] = 0.f;
+            for (int h = 0; h < NHW / 2; ++h)
+                lp2[h] = f2(0.f, 0.f);
+            constexpr bool NM_REGS = NHW <= 16;     // -m in registers (else read from shared memory)
+            float nm[NM_REGS ? NHW : 1];
+            const float sl = p.scale_log2;
+            // x[h] = s[h] scale - m[h]: the exponent of this key's P^T entry
+            auto exps_of = [&](const float (&sr)[NHW], float (&x)[NHW]) {
+#pragma unroll
+                for (int h = 0; h < NHW; h += 4) {
+                    float n0, n1, n2, n3;
+                    if constexpr (NM_REGS) {
+                        n0 = nm[h];
+                        n1 = nm[h + 1];
+                        n2 = nm[h + 2];
+                        n3 = nm[h + 3];
+                    } else {
+                        const float4 m4 = *reinterpret_cast<const float4 *>(sMref + mb * NH + hb + h);
+                        n0 = -m4.x;
+                        n1 = -m4.y;
+                        n2 = -m4.z;
+                        n3 = -m4.w;
+                    }
+                    f2_split(fma_f2(f2(sr[h], sr[h + 1]), f2(sl, sl), f2(n0, n1)), x[h], x[h + 1]);
+                    f2_split(fma_f2(f2(sr[h + 2], sr[h + 3]), f2(sl, sl), f2(n2, n3)), x[h + 2], x[h + 3]);
+                }
+            };
             // No global memory access inside this loop: a CTA barrier (the
             // votes below) waits for every outstanding access of its threads.
             for (int ii = 0; ii < ntl; ++ii, ++gt) {
@@ -769,51 +745,55 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag));
                 bool valid;
                 if (i < k.nct) {
-                    const int slot = i * kSpBN + r;
-                    valid = slot < p.topk && sSel[slot] >= 0;
+                    valid = sSel[i * kSpBN + r] >= 0;   // the table is padded with -1 to whole tiles
                 } else {
                     valid = k.rlo + (i - k.nct) * kSpBN + r <= k.rhi;
                 }
                 tc_fence_after();
-                float s[NHW];
-                tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
-                tmem_ld_wait();
-                if (threadIdx.x == 0)
-                    trace_ev(trb, 3, 1, w, i);
-#pragma unroll
-                for (int h = 0; h < NHW; ++h)
-                    s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
+                float x[NHW];
                 bool need = ii == 0;   // this CTA's first tile of an item always sets the reference
+                {
+                    float sr[NHW];                  // raw scores q . k of this key
+                    tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, sr);
+                    tmem_ld_wait();
+                    if (!need)
+                        exps_of(sr, x);
+                }
+                if (trace0)
+                    trace_ev(trb, 3, 1, w, i);
                 if (!need) {
-                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH + hb);
                     bool exceed = false;
 #pragma unroll
-                    for (int h = 0; h < NHW; h += 4) {
-                        const float4 mr = m4[h >> 2];
-                        exceed |= (s[h] > mr.x + 8.f) | (s[h + 1] > mr.y + 8.f) | (s[h + 2] > mr.z + 8.f) |
-                                  (s[h + 3] > mr.w + 8.f);
-                    }
-                    need = sm_any<SMT>(exceed);
+                    for (int h = 0; h < NHW; ++h)
+                        exceed |= x[h] > 8.f;
+                    need = sm_any<SMT>(valid && exceed);
                 }
                 if (need) {
-                    // per-head max over the tile: warp halving, then the four
-                    // quadrants' values through sRed [head][quadrant]
-                    warp_reduce_heads<NHW, true>(s, lane);
+                    // per-head max over the tile (scaled, masked keys -inf): warp
+                    // halving, then the four quadrants' values through sRed [head][quadrant]
+                    float sc[NHW];
+                    tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, sc);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < NHW; ++h)
+                        sc[h] = valid ? sc[h] * sl : -INFINITY;
+                    warp_reduce_heads<NHW, true>(sc, lane);
                     if (head_owner) {
 #pragma unroll
                         for (int e = 0; e < HD::VPL; ++e)
-                            sRed[(hb + HD::head(lane, e)) * 4 + quad] = s[e];
+                            sRed[(hb + HD::head(lane, e)) * 4 + quad] = sc[e];
                     }
                     sm_sync<SMT>();
                     const float *mold = sMref + mb * NH;
                     bool moved = false;
                     if (ii > 0) {
 #pragma unroll
-                        for (int h = 0; h < NHW; ++h) {
-                            const float old = mold[hb + h];
-                            const float a = sp_factor(old, sp_new_ref(red4[hb + h], old));
-                            moved |= a != 1.f;
-                            lpart[h] *= a;
+                        for (int h = 0; h < NHW; h += 2) {
+                            const float o0 = mold[hb + h], o1 = mold[hb + h + 1];
+                            const float a0 = sp_factor(o0, sp_new_ref(red4[hb + h], o0));
+                            const float a1 = sp_factor(o1, sp_new_ref(red4[hb + h + 1], o1));
+                            moved |= (a0 != 1.f) | (a1 != 1.f);
+                            lp2[h >> 1] = fma_f2(lp2[h >> 1], f2(a0, a1), f2(0.f, 0.f));
                         }
                     }
                     if (moved) {
@@ -841,57 +821,53 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             sp_new_ref(red4[threadIdx.x], mold[threadIdx.x]);
                     sm_sync<SMT>();
                     mb ^= 1;
-                    // the halving consumed the scores: load them again
-                    tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, s);
-                    tmem_ld_wait();
+                    if constexpr (NM_REGS) {
 #pragma unroll
-                    for (int h = 0; h < NHW; ++h)
-                        s[h] = valid ? s[h] * p.scale_log2 : -INFINITY;
-                }
-                // P^T row of this key: exp2(s - mref), 0 for masked keys
-                uint32_t pk[NHW / 2];
-                {
-                    const float4 *m4 = reinterpret_cast<const float4 *>(sMref + mb * NH + hb);
-#pragma unroll
-                    for (int h = 0; h < NHW; h += 4) {
-                        const float4 mr = m4[h >> 2];
-                        const float mm[4] = {mr.x, mr.y, mr.z, mr.w};
-                        float e[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            e[q] = (mm[q] == -INFINITY) ? 0.f : ex2_approx(s[h + q] - mm[q]);
-                            lpart[h + q] += e[q];
-                        }
-                        pk[h >> 1] = pack_bf16x2(e[0], e[1]);
-                        pk[(h >> 1) + 1] = pack_bf16x2(e[2], e[3]);
+                        for (int h = 0; h < NHW; ++h)
+                            nm[h] = -sMref[mb * NH + hb + h];
                     }
+                    // the exponents against the new reference
+                    float sr[NHW];
+                    tmem_ld_cols<NHW>(tl + TM_S0 + sb * NH + hb, sr);
+                    tmem_ld_wait();
+                    exps_of(sr, x);
+                }
+                // P^T row of this key: exp2(s scale - m), 0 for masked keys (a
+                // visible key never meets m = -inf: it would have moved m)
+                uint32_t pk[NHW / 2];
+                if (valid) {
+#pragma unroll
+                    for (int h = 0; h < NHW; h += 2) {
+                        const float e0 = ex2_approx(x[h]), e1 = ex2_approx(x[h + 1]);
+                        lp2[h >> 1] = add_f2(lp2[h >> 1], f2(e0, e1));
+                        pk[h >> 1] = pack_bf16x2(e0, e1);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < NHW / 2; ++h)
+                        pk[h] = 0u;
                 }
                 // P^T buffer sb is free once the PV of tile gt - 2 completed
                 if (gt >= 2)
                     ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1, abort_flag));
                 const uint32_t prow_b = prow + sb * SM::P_STRIDE;
 #pragma unroll
-                for (int cl = 0; cl < NHW / 8; ++cl) {
-                    const int c = hb / 8 + cl;               // 16-byte chunk of the row
-                    uint32_t phys;
-                    if (RB == 128)
-                        phys = c ^ (r & 7);
-                    else if (RB == 64)
-                        phys = c ^ ((r >> 1) & 3);
-                    else
-                        phys = c ^ ((r >> 2) & 1);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_b + phys * 16),
+                for (int cl = 0; cl < NHW / 8; ++cl)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_b + pphys[cl]),
                                  "r"(pk[4 * cl]), "r"(pk[4 * cl + 1]), "r"(pk[4 * cl + 2]), "r"(pk[4 * cl + 3])
                                  : "memory");
-                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
-                if (threadIdx.x == 0)
+                if (trace0)
                     trace_ev(trb, 3, 2, w, i);
             }
+            float lpart[NHW];
+#pragma unroll
+            for (int h = 0; h < NHW; h += 2)
+                f2_split(lp2[h >> 1], lpart[h], lpart[h + 1]);
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
-            if (threadIdx.x == 0)
+            if (trace0)
                 trace_ev(trb, 3, 3, w, nt);
             warp_reduce_heads<NHW, false>(lpart, lane);
             if (head_owner) {
@@ -1004,7 +980,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
-            if (threadIdx.x == 0)
+            if (trace0)
                 trace_ev(trb, 3, 4, w, nt);
         }
     }
@@ -1067,7 +1043,7 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
     ok &= make_map_3d_rows(&mvr, vr, p.Hkv, (long long)p.B * p.Lkv);
     if (!ok)
         return cudaErrorInvalidValue;
-    size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.topk * 8;
+    size_t smem = 1024 + SM::BASE_BYTES + (size_t)p.tsel * 8;
     auto kern = csa_attn_kernel<NH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
@@ -1136,6 +1112,7 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
         return cudaErrorInvalidValue;
     p.pregathered = pregathered;
     p.split = 1;
+    p.tsel = (topk + kSpBN - 1) / kSpBN * kSpBN;
     if (pregathered && (long long)B * Lq * topk * Hkv >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.scale_log2 = scale * 1.4426950408889634f;

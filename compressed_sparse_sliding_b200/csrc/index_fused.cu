@@ -355,53 +355,83 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         mbar_arrive(&bar[11 + db]);
                     }
                     const int j0 = kbase + half * 32;
+                    // the half's 32 scores and order keys first, in straight-line
+                    // code the scheduler can interleave; then the pass's work with
+                    // predicated stores (a branch per score serialises the warp)
+                    float sv[32];
+                    uint32_t kv[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         float s = wv[0] * fmaxf(d[0][c], 0.f);
 #pragma unroll
                         for (int h = 1; h < HI; ++h)
                             s = fmaf(wv[h], fmaxf(d[h][c], 0.f), s);
-                        const int j = j0 + c;
-                        const bool vis = j < nv;
-                        if (ptype == 0) {
-                            const bool in = vis && j >= slot_lo(i);
-                            col[(i * kFxBN + half * 32 + c) * kFxBM] = in ? fx_key(s) : 0u;
-                            ns += in;
-                        } else if (ptype == 1) {
-                            if (mode == FX_OPEN && vis) {
-                                const uint32_t k = fx_key(s);
-                                if (k >= lo) {
-                                    if (k > top_m1) {
-                                        ++ab;
-                                    } else {
-                                        const uint32_t bin = (k - lo) >> sh;
-                                        atomicAdd(hist + (bin >> 1) * kFxBM, 1u << ((bin & 1u) * 16u));
-                                    }
-                                }
+                        sv[c] = s;
+                        kv[c] = fx_key(s);
+                    }
+                    const int nvh = max(0, min(32, nv - j0));     // visible: c < nvh
+                    if (ptype == 0) {
+                        const int clo = max(0, min(32, slot_lo(i) - j0));
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            col[(i * kFxBN + half * 32 + c) * kFxBM] = (c < nvh && c >= clo) ? kv[c] : 0u;
+                        ns += max(0, nvh - clo);
+                    } else if (ptype == 1) {
+                        if (mode == FX_OPEN) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const uint32_t k = kv[c];
+                                const bool inw = c < nvh && k >= lo;
+                                const bool above = k > top_m1;
+                                ab += (inw && above) ? 1 : 0;
+                                const uint32_t bin = (k - lo) >> sh;
+                                if (inw && !above)
+                                    atomicAdd(hist + (bin >> 1) * kFxBM, 1u << ((bin & 1u) * 16u));
                             }
-                        } else if (vis && mode != FX_NONE) {
-                            bool pick = mode == FX_ALL;
-                            if (!pick) {
-                                const uint32_t k = fx_key(s);
-                                if (k > bhi_m1) {
-                                    pick = true;
-                                } else if (k >= blo) {
-                                    if (mode == FX_TIE) {
-                                        pick = taken < need;
-                                        taken += pick;
-                                    } else if (nb < kFxCap) {
-                                        bkey[nb * kFxBM] = k;
-                                        bpk[nb * kFxBM] = (uint32_t)j | ((uint32_t)pos << 16);
-                                        ++nb;
-                                    }
-                                }
-                            }
-                            if (pick && pos < K) {
-                                orow[pos] = j;
+                        }
+                    } else if (mode == FX_ALL) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            if (c < nvh) {
+                                orow[pos + c] = j0 + c;
                                 if (srow)
-                                    srow[pos] = s;
-                                ++pos;
+                                    srow[pos + c] = sv[c];
                             }
+                        }
+                        pos += nvh;
+                    } else if (mode == FX_TIE) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const uint32_t k = kv[c];
+                            const bool v = c < nvh;
+                            const bool tie = v && k >= blo && k <= bhi_m1 && taken < need;
+                            const bool pick = (v && k > bhi_m1) || tie;
+                            taken += tie ? 1 : 0;
+                            if (pick && pos < K) {
+                                orow[pos] = j0 + c;
+                                if (srow)
+                                    srow[pos] = sv[c];
+                            }
+                            pos += pick ? 1 : 0;
+                        }
+                    } else if (mode == FX_BIN) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const uint32_t k = kv[c];
+                            const bool v = c < nvh;
+                            const bool pick = v && k > bhi_m1;
+                            const bool keep = v && k >= blo && k <= bhi_m1 && nb < kFxCap;
+                            if (keep) {
+                                bkey[nb * kFxBM] = k;
+                                bpk[nb * kFxBM] = (uint32_t)(j0 + c) | ((uint32_t)pos << 16);
+                            }
+                            nb += keep ? 1 : 0;
+                            if (pick && pos < K) {
+                                orow[pos] = j0 + c;
+                                if (srow)
+                                    srow[pos] = sv[c];
+                            }
+                            pos += pick ? 1 : 0;
                         }
                     }
                 }

@@ -552,232 +552,6 @@ topk_hist(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
     }
 }
 
-// ------------------------------------------------------------------------
-// Exact top-K for few rows (decode): a cluster of kTcCS CTAs per row, each
-// CTA holding a contiguous chunk of the row's keys in registers.  The K-th
-// key is found by the same narrowing histogram as topk_hist, with each round's
-// histogram summed over the cluster through distributed shared memory (every
-// CTA sums all bins and reaches the same threshold); the selection is then
-// emitted in index order, each CTA placing its entries after those of the
-// lower-ranked CTAs (ties at the threshold go to the lowest indices across the
-// whole row).  Every CTA of a cluster takes the same branches and the same
-// cluster barriers; the last barrier keeps each CTA's shared memory alive
-// until its peers have read it.
-// ------------------------------------------------------------------------
-constexpr int kTcThreads = 256;
-constexpr int kTcCS = 8;
-
-template <int KPT>
-__global__ void __launch_bounds__(kTcThreads)
-topk_cluster(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
-             const int32_t *__restrict__ q_pos, int32_t *__restrict__ idx_out, float *__restrict__ sel_scores)
-{
-    constexpr int NT = kTcThreads;
-    constexpr int PER = kHbBins / NT;   // bins per thread, contiguous
-    __shared__ int hist[kHbBins];       // this CTA's counts of the round
-    __shared__ int tot[3][kHbBins];     // rank 0: the cluster's counts, buffer (round mod 3)
-    __shared__ int s_scan[32];
-    __shared__ int s_sel[3];
-    __shared__ int s_cnt[2];            // this CTA's (greater, equal) counts, read by peers
-
-    const uint32_t rank = cluster_ctarank();
-    const int row = blockIdx.x / kTcCS;
-    const int t = row % Lq;
-    const long long pos = q_pos ? q_pos[row] : t;
-    const int n = visible_entries(pos, m, W, Nc);
-    const int keff = n < K ? n : K;
-    const float *src = scores + (size_t)row * Nc;
-    int32_t *dst = idx_out + (size_t)row * K;
-    float *dsc = sel_scores ? sel_scores + (size_t)row * K : nullptr;
-    const int chunk = (((n + kTcCS - 1) / kTcCS) + 3) & ~3;     // entries per CTA
-    const int c0 = (int)rank * chunk;
-    const int c1 = min(n, c0 + chunk);
-
-    if (keff == n) {  // every visible entry is selected (the same branch in every CTA)
-        for (int i = c0 + threadIdx.x; i < c1; i += NT) {
-            dst[i] = i;
-            if (dsc)
-                dsc[i] = src[i];
-        }
-        if (rank == 0) {
-            for (int i = n + threadIdx.x; i < K; i += NT) {
-                dst[i] = -1;
-                if (dsc)
-                    dsc[i] = -INFINITY;
-            }
-        }
-        return;
-    }
-
-    const int i0 = c0 + threadIdx.x * KPT;
-    const int nv = min(KPT, max(0, c1 - i0));
-    uint32_t key[KPT];
-    if ((Nc & 3) == 0 && nv == KPT) {
-#pragma unroll
-        for (int u = 0; u < KPT; u += 4) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i0 + u));
-            key[u] = order_key(v.x);
-            key[u + 1] = order_key(v.y);
-            key[u + 2] = order_key(v.z);
-            key[u + 3] = order_key(v.w);
-        }
-    } else {
-#pragma unroll
-        for (int u = 0; u < KPT; ++u)
-            key[u] = u < nv ? order_key(__ldg(src + i0 + u)) : 0u;
-    }
-    for (int i = threadIdx.x; i < kHbBins; i += NT) {
-        hist[i] = 0;
-        tot[0][i] = 0;
-        tot[1][i] = 0;
-        tot[2][i] = 0;
-    }
-    // rank 0's totals are zero before any peer adds into them
-    cluster_sync_all();
-
-    uint32_t lo = 0u, hi = 0xFFFFFFFFu;
-    int need = keff;
-    bool whole = false;
-    uint32_t T = lo;
-    const int b0 = (int)threadIdx.x * PER;    // this thread's bins (descending scan order below)
-#pragma unroll 1
-    for (int rnd = 0; lo < hi; ++rnd) {
-        const uint32_t span = hi - lo;
-        const int bits = 32 - __clz(span);
-        const int sh = bits > 11 ? bits - 11 : 0;
-#pragma unroll
-        for (int u = 0; u < KPT; ++u)
-            if (u < nv && key[u] >= lo && key[u] <= hi)
-                atomicAdd(&hist[(key[u] - lo) >> sh], 1);
-        __syncthreads();
-        // add this CTA's counts into rank 0's totals of the round, and clear
-        // them for the next round (each thread its own bins)
-        const uint32_t tr = cluster_addr(&tot[rnd % 3][0], 0);
-#pragma unroll
-        for (int q = 0; q < PER; ++q) {
-            const int c = hist[b0 + q];
-            if (c) {
-                asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(tr + (uint32_t)(b0 + q) * 4u), "r"(c)
-                             : "memory");
-                hist[b0 + q] = 0;
-            }
-        }
-        cluster_sync_all();   // every CTA's counts are in rank 0's totals
-        if (rank == 0) {
-            // the buffer of the previous round: its readers passed the barrier above
-            for (int i = threadIdx.x; i < kHbBins; i += NT)
-                tot[(rnd + 2) % 3][i] = 0;
-        }
-        // this thread's PER bins counted down from the top: bins NB-1-b0-q
-        int v[PER];
-#pragma unroll
-        for (int q = 0; q < PER; ++q)
-            v[q] = cluster_ld(tr + (uint32_t)(kHbBins - 1 - (b0 + q)) * 4u);
-        int mine = 0;
-#pragma unroll
-        for (int q = 0; q < PER; ++q)
-            mine += v[q];
-        const int ex = blk_excl_scan<NT>(mine, s_scan);
-        if (ex < need && ex + mine >= need) {
-            int acc = ex;
-#pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                if (acc + v[q] >= need) {
-                    s_sel[0] = kHbBins - 1 - (b0 + q);
-                    s_sel[1] = acc;
-                    s_sel[2] = v[q];
-                    break;
-                }
-                acc += v[q];
-            }
-        }
-        __syncthreads();
-        const uint32_t bin = (uint32_t)s_sel[0];
-        need -= s_sel[1];
-        const int cnt = s_sel[2];
-        __syncthreads();   // s_sel read before the next round writes it
-        const uint32_t nlo = lo + (bin << sh);
-        const uint32_t nhi = (uint32_t)min((unsigned long long)hi,
-                                           (unsigned long long)nlo + ((1ull << sh) - 1ull));
-        lo = nlo;
-        hi = nhi;
-        T = lo;
-        if (cnt == need) {
-            whole = true;
-            break;
-        }
-    }
-    // this CTA's counts, then every CTA's offsets from its lower-ranked peers
-    int gt = 0, eq = 0;
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-        if (u < nv) {
-            gt += whole ? key[u] >= T : key[u] > T;
-            eq += !whole && key[u] == T;
-        }
-    }
-    const int exs = blk_excl_scan<NT>((gt << 16) | eq, s_scan);
-    if (threadIdx.x == NT - 1) {
-        s_cnt[0] = (exs >> 16) + gt;
-        s_cnt[1] = (exs & 0xffff) + eq;
-    }
-    cluster_sync_all();
-    int gt_before = 0, eq_before_cta = 0;
-    for (uint32_t c = 0; c < rank; ++c) {
-        gt_before += cluster_ld(cluster_addr(&s_cnt[0], c));
-        eq_before_cta += cluster_ld(cluster_addr(&s_cnt[1], c));
-    }
-    // no CTA leaves while a peer may still read its shared memory
-    cluster_sync_all();
-    const int eq_before = eq_before_cta + (exs & 0xffff);       // ties at lower indices in the row
-    const int take_eq = min(eq, max(0, need - eq_before));
-    int out = gt_before + (exs >> 16) + min(eq_before, need);
-    int e_seen = 0;
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-        if (u < nv) {
-            bool pick = whole ? key[u] >= T : key[u] > T;
-            if (!whole && key[u] == T) {
-                pick = e_seen < take_eq;
-                ++e_seen;
-            }
-            if (pick) {
-                dst[out] = i0 + u;
-                if (dsc)
-                    dsc[out] = key_to_score(key[u]);
-                ++out;
-            }
-        }
-    }
-    if (rank == 0) {
-        for (int i = keff + threadIdx.x; i < K; i += NT) {
-            dst[i] = -1;
-            if (dsc)
-                dsc[i] = -INFINITY;
-        }
-    }
-}
-
-template <int KPT>
-static cudaError_t launch_topk_cluster_t(const float *scores, int rows, int Lq, int Nc, int m, int W, int K,
-                                         const int32_t *q_pos, int32_t *idx, float *sel_scores,
-                                         cudaStream_t stream)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)rows * kTcCS, 1, 1);
-    cfg.blockDim = dim3(kTcThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = kTcCS;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, topk_cluster<KPT>, scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores);
-}
-
 cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m, int W, int K,
                               const int32_t *q_pos, int32_t *idx, float *sel_scores,
                               cudaStream_t stream)
@@ -786,17 +560,6 @@ cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m,
     // (512 threads per row measured faster than 128 or 256 on 8192-entry
     // rows); longer rows: the shared-memory radix select.
     const unsigned rows = (unsigned)B * (unsigned)Lq;
-    // few rows (decode): a cluster of CTAs per row keeps every SM busy
-    if (rows <= 1024 && Nc <= kTcCS * kTcThreads * 32) {
-        if (Nc <= kTcCS * kTcThreads * 4)
-            return launch_topk_cluster_t<4>(scores, (int)rows, Lq, Nc, m, W, K, q_pos, idx, sel_scores, stream);
-        if (Nc <= kTcCS * kTcThreads * 8)
-            return launch_topk_cluster_t<8>(scores, (int)rows, Lq, Nc, m, W, K, q_pos, idx, sel_scores, stream);
-        if (Nc <= kTcCS * kTcThreads * 16)
-            return launch_topk_cluster_t<16>(scores, (int)rows, Lq, Nc, m, W, K, q_pos, idx, sel_scores,
-                                             stream);
-        return launch_topk_cluster_t<32>(scores, (int)rows, Lq, Nc, m, W, K, q_pos, idx, sel_scores, stream);
-    }
 #define HYB_TOPK_HIST(NT, KPT)                                                                     \
     do {                                                                                        \
         topk_hist<NT, KPT><<<rows, NT, 0, stream>>>(scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores); \
