@@ -52,6 +52,7 @@ struct SparseParams {
     int pregathered;   // kc / vc hold each token's selected rows in slot order: [B Lq, topk, Hkv, 128]
     int split;         // CTAs (one cluster) sharing each item's key tiles: 1 or 2
     int tsel;          // entries of a decoded selection table: topk rounded up to whole tiles
+    int prefetch;      // compressed caches far larger than L2: pull an item's selected rows into L2 first
     long long n_items;
     float scale_log2;
     const int32_t *q_pos, *kv_pos0, *idx;
@@ -451,6 +452,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int *sSel = sIdx + qb * p.tsel;
             {
                 const long long wstart = k.pos - p.W + 1;
+                // selected slots of this CTA's tiles (the prefetch range)
+                const int pq0 = tile_lo(k.nct + k.nrt) * kSpBN, pq1 = tile_hi(k.nct + k.nrt) * kSpBN;
 #pragma unroll 1
                 for (int q0 = 0; q0 < p.topk; q0 += kSpSelBatch * NPT) {
                     int jv[kSpSelBatch];
@@ -473,6 +476,16 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                  ? ((int)((uint32_t)w / (uint32_t)p.Hkv) * p.topk + q) * p.Hkv + k.kvh
                                                  : (k.b * p.Nc + j) * p.Hkv + k.kvh;
                             sSel[q] = v ? srow : -1;
+                            if (p.prefetch && v && q >= pq0 && q < pq1) {
+                                // the row's K and V lines into L2 now: the copies
+                                // of the item's tiles then wait on L2, not HBM
+                                const __nv_bfloat16 *kr0 = p.kc + (size_t)srow * kSpD;
+                                const __nv_bfloat16 *vr0 = p.vc + (size_t)srow * kSpD;
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0));
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0 + 64));
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0));
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0 + 64));
+                            }
                         }
                     }
                 }
@@ -1113,6 +1126,12 @@ cudaError_t launch_csa_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int Nc, int
     p.pregathered = pregathered;
     p.split = 1;
     p.tsel = (topk + kSpBN - 1) / kSpBN * kSpBN;
+    {
+        // the rows a launch selects are spread over the caches: worth pulling
+        // into L2 ahead of the copies only when the caches are far larger than L2
+        const long long rows = pregathered ? (long long)B * Lq * topk * Hkv : (long long)B * Nc * Hkv;
+        p.prefetch = rows * kSpD * 2 * 2 > (64ll << 20) ? 1 : 0;
+    }
     if (pregathered && (long long)B * Lq * topk * Hkv >= (1ll << 31))
         return cudaErrorInvalidValue;
     p.scale_log2 = scale * 1.4426950408889634f;

@@ -389,6 +389,43 @@ __device__ __forceinline__ int blk_excl_scan(int v, int *warp_tot)
     return r;
 }
 
+// Block-wide max / sum over NT threads (every thread gets the result).
+template <int NT>
+__device__ __forceinline__ uint32_t blk_max_u32(uint32_t v, int *tmp)
+{
+    constexpr int NW = NT / 32;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if ((threadIdx.x & 31) == 0)
+        tmp[threadIdx.x >> 5] = (int)v;
+    __syncthreads();
+    uint32_t r = 0u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+        r = max(r, (uint32_t)tmp[w]);
+    __syncthreads();
+    return r;
+}
+
+template <int NT>
+__device__ __forceinline__ int blk_sum_i32(int v, int *tmp)
+{
+    constexpr int NW = NT / 32;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0)
+        tmp[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int r = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+        r += tmp[w];
+    __syncthreads();
+    return r;
+}
+
 // ------------------------------------------------------------------------
 // Exact top-K, row in registers, histogram select.  Thread t owns entries
 // [t * KPT, (t + 1) * KPT) of its row.  The K-th largest order key is found
@@ -463,6 +500,32 @@ topk_hist(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
     uint32_t lo = 0u, hi = 0xFFFFFFFFu;
 
     int need = keff;
+    // Start from the keys within a factor 16 of the row's largest score (the
+    // 2^25 order keys up to the top key): the K-th largest nearly always lies
+    // there, and bins over that window spread the keys, where over the whole
+    // key range a row's scores share a few exponents and pile into a handful
+    // of bins (their atomics serialise).  Otherwise the rest of the range.
+    {
+        uint32_t kmax = 0u;
+#pragma unroll
+        for (int u = 0; u < KPT; ++u)
+            if (u < nv)
+                kmax = max(kmax, key[u]);
+        kmax = blk_max_u32<NT>(kmax, s_scan);
+        const uint32_t wlo = kmax >= (1u << 25) ? kmax - ((1u << 25) - 1u) : 0u;
+        int cnt = 0;
+#pragma unroll
+        for (int u = 0; u < KPT; ++u)
+            cnt += (u < nv && key[u] >= wlo) ? 1 : 0;
+        cnt = blk_sum_i32<NT>(cnt, s_scan);
+        if (cnt >= need) {
+            lo = wlo;
+            hi = kmax;
+        } else {              // wlo > 0: some visible keys lie below it
+            need -= cnt;
+            hi = wlo - 1u;
+        }
+    }
     bool whole = false;
     uint32_t T = lo;   // the K-th key (or, when whole, the lowest selected key)
 #pragma unroll 1
