@@ -73,14 +73,15 @@ struct SparseSmem {
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
     static constexpr int OFF_P = OFF_V + VS * KV_BYTES;            // 2 buffers
-    static constexpr int OFF_RED = OFF_P + 2 * P_STRIDE;           // [NH][4] floats
-    static constexpr int OFF_MREF = OFF_RED + 4 * NH * 4;          // [2][NH] floats
-    static constexpr int OFF_INV = OFF_MREF + 2 * NH * 4;          // [NH] floats
+    static constexpr int OFF_RED = OFF_P + 2 * P_STRIDE;           // [2 warpgroups][NH][4] floats
+    static constexpr int OFF_MREF = OFF_RED + 2 * 4 * NH * 4;      // [2 warpgroups][2][NH] floats
+    static constexpr int OFF_INV = OFF_MREF + 4 * NH * 4;          // [NH] floats
     static constexpr int OFF_BAR = OFF_INV + NH * 4;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
     static constexpr int OFF_PML = OFF_MISC + 16 * 4;               // split: peer's [max, sum] per head
-    static constexpr int OFF_CMB = OFF_PML + 2 * NH * 4;            // split: [2][NH] combine factors
-    static constexpr int OFF_IDX = OFF_CMB + 2 * NH * 4;            // [2][tsel] decoded selections
+    static constexpr int OFF_CMB = OFF_PML + 2 * NH * 4;            // split / ping-pong: [2][NH] combine factors
+    static constexpr int OFF_PPX = OFF_CMB + 2 * NH * 4;            // ping-pong: [2 warpgroups][max, sum][NH]
+    static constexpr int OFF_IDX = OFF_PPX + 4 * NH * 4;            // [2][tsel] decoded selections
     static constexpr int BASE_BYTES = OFF_IDX;                      // + 2 tsel * 4, tsel = topk rounded up to 128
 };
 
@@ -90,7 +91,8 @@ enum {
     SB_OD = 20, SB_OE = 22, SB_IF = 24, SB_DONE = 26,
     SB_GO = 27,      // split, rank 1: rank 0 can take this item's partial (arrived by rank 0)
     SB_PFULL = 28,   // split, rank 0: rank 1's partial has landed (arrived by rank 1's softmax threads)
-    SB_COUNT = 29
+    SB_SE = 29,      // ping-pong: S^T buffer read into registers (two buffers)
+    SB_COUNT = 31
 };
 
 struct SparseTok {
@@ -210,6 +212,41 @@ __device__ __forceinline__ void sm_sync()
     asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory");
 }
 
+// Named barriers with a run-time id (ping-pong softmax: one per warpgroup,
+// and one over both warpgroups).
+__device__ __forceinline__ void bar_sync_id(uint32_t id, uint32_t n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ bool bar_any_id(uint32_t id, uint32_t n, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ bool bar_all_id(uint32_t id, uint32_t n, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
 // Per-head totals over the 32 lanes of a warp by recursive halving: at each
 // step a lane keeps one half of its values (the upper half where its lane
 // bit is set), receives the partner's copy of that half and combines.  NH
@@ -312,10 +349,23 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float (&v)[N]
 
 // Producer warps: four for up to 32 heads; two for 64 heads, whose softmax
 // threads need up to 255 registers (8 warps in all).
+// Ping-pong softmax for 32-head groups: the two softmax warpgroups take
+// alternate key tiles (all heads of a key each) with their own running maxima,
+// sums and O^T accumulators, combined once per item, so that one tile's
+// softmax overlaps the next one's instead of both warpgroups splitting every
+// tile's heads.
+constexpr bool kSpPingPong = true;
+
 template <int NH>
 struct SpRoles {
-    static constexpr int HS = NH >= 32 ? 2 : 1;       // softmax warpgroups (head halves)
-    static constexpr int NHW = NH / HS;               // heads per softmax thread
+    static constexpr bool PP = kSpPingPong && NH == 32;
+    // ping-pong register split (setmaxnreg): 8 softmax warps up, producer and
+    // MMA warps down; 256 x 144 + 160 x 96 = 52224 <= 416 x 128, the budget
+    // the block launches with
+    static constexpr int PP_SOFTMAX_REGS = 144;
+    static constexpr int PP_OTHER_REGS = 96;
+    static constexpr int HS = NH >= 32 ? 2 : 1;       // softmax warpgroups (head halves, or tile parities)
+    static constexpr int NHW = PP ? NH : NH / HS;     // heads per softmax thread
     static constexpr int SMT = 128 * HS;              // softmax threads
     static constexpr int PW = NH == 64 ? 2 : 4;       // producer warps
     static constexpr int PROD_WARP0 = 4 * HS;
@@ -361,7 +411,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bar[SB_QE + s], 1);
             mbar_init(&bar[SB_SF + s], 1);
             mbar_init(&bar[SB_OE + s], SpRoles<NH>::SMT);
-            mbar_init(&bar[SB_PF + s], SpRoles<NH>::SMT);
+            mbar_init(&bar[SB_PF + s], SpRoles<NH>::PP ? 128 : SpRoles<NH>::SMT);
+            mbar_init(&bar[SB_SE + s], 128);
             mbar_init(&bar[SB_OD + s], 1);
             mbar_init(&bar[SB_IF + s], NPT);
         }
@@ -379,7 +430,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_fence_init();
         misc[1] = 0;
     }
-    if (threadIdx.x < 2 * NH)
+    if (threadIdx.x < 4 * NH)
         sMref[threadIdx.x] = -INFINITY;
     if (warp == SpRoles<NH>::MMA_WARP)
         tmem_alloc(reinterpret_cast<uint32_t *>(&misc[0]), 256);
@@ -403,6 +454,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr int CPT = kSpBN / RPI;            // copies per thread per tile and operand
     constexpr int MMA_WARP = SpRoles<NH>::MMA_WARP;
     if (warp >= SpRoles<NH>::PROD_WARP0 && warp < MMA_WARP) {
+        if constexpr (SpRoles<NH>::PP)
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(SpRoles<NH>::PP_OTHER_REGS));
         // ================================ producer ================================
         // 16 lanes per 256-byte row, two rows per warp instruction.  Within an
         // item no thread leaves early: a failed wait clears `ok`, the copies
@@ -596,6 +649,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 drain_wait(&bar[SB_QF + (q & 1)], (q >> 1) & 1);
         }
     } else if (warp == MMA_WARP) {
+        if constexpr (SpRoles<NH>::PP)
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(SpRoles<NH>::PP_OTHER_REGS));
         // ================================ MMA issue ================================
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_bf16(kSpBN, NH, false, false);
@@ -638,6 +693,72 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++pcnt;
                     return true;
                 };
+                if constexpr (SpRoles<NH>::PP) {
+                    // ping-pong: QK^T runs two tiles ahead of PV, refilling an S^T
+                    // buffer once its warpgroup has read it; PV of tile g goes to
+                    // its parity's O^T accumulator
+                    const uint32_t gt0 = gt;
+                    auto issue_pv_pp = [&](uint32_t g) -> bool {
+                        const uint32_t vs = vc % VS, pb = g & 1;
+                        if (!mbar_wait(&bar[SB_PF + pb], (g >> 1) & 1, abort_flag) ||
+                            !mbar_wait(&bar[SB_VF + vs], (vc / VS) & 1, abort_flag))
+                            return false;
+                        if (g == gt0 && nq >= 2 && !mbar_wait(&bar[SB_OE + ob], ((nq >> 1) - 1) & 1, abort_flag))
+                            return false;
+                        tc_fence_after();
+                        const bool first = g - gt0 < 2;   // this parity's first tile of the item
+#pragma unroll
+                        for (int kk = 0; kk < kSpBN / 16; ++kk) {
+                            const uint64_t da = smem_desc(aV + vs * SM::KV_BYTES + kk * 16 * 128,
+                                                          kSpBN * 128, 1024, 2);
+                            const uint64_t db = smem_desc(aP + pb * SM::P_STRIDE + kk * 16 * RB, 16, 8 * RB,
+                                                          PLAYOUT);
+                            mma_bf16_ss(tmem + TM_O0 + (ob * 2 + pb) * NH, da, db, idesc_pv,
+                                        (first && kk == 0) ? 0u : 1u);
+                        }
+                        mma_commit(&bar[SB_OD + pb]);
+                        mma_commit(&bar[SB_VE + vs]);
+                        trace_ev(trb, 2, 2, w, (int)(g - gt0));
+                        ++vc;
+                        return true;
+                    };
+                    for (int ii = 0; ii < ntl; ++ii, ++gt) {
+                        const uint32_t ks = kc % KS;
+                        if (!mbar_wait(&bar[SB_KF + ks], (kc / KS) & 1, abort_flag) ||
+                            (gt >= 2 && !mbar_wait(&bar[SB_SE + (gt & 1)], ((gt >> 1) - 1) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < kSpD / 16; ++kk) {
+                            const uint64_t da = sw128_desc(aK + ks * SM::KV_BYTES + (kk >> 2) * kSpBN * 128 +
+                                                               (kk & 3) * 32, 16, 1024);
+                            const uint64_t db = sw128_desc(aQ + qb * SM::Q_BYTES + (kk >> 2) * NH * 128 +
+                                                               (kk & 3) * 32, 16, 1024);
+                            mma_bf16_ss(tmem + TM_S0 + (gt & 1) * NH, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&bar[SB_SF + (gt & 1)]);
+                        mma_commit(&bar[SB_KE + ks]);
+                        trace_ev(trb, 2, 1, w, ii);
+                        ++kc;
+                        if (ii == ntl - 1)
+                            mma_commit(&bar[SB_QE + qb]);
+                        if (ii >= 2 && !issue_pv_pp(gt - 2)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    if (ntl == 0)
+                        mma_commit(&bar[SB_QE + qb]);
+                    for (int jj = ntl >= 2 ? ntl - 2 : 0; ok && jj < ntl; ++jj)
+                        ok = issue_pv_pp(gt0 + (uint32_t)jj);
+                    if (!ok)
+                        break;
+                    continue;
+                }
                 for (int ii = 0; ii < ntl; ++ii, ++gt) {
                     const int i = tb + ii;
                     const uint32_t ks = kc % KS;
@@ -676,6 +797,243 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mma_commit(&bar[SB_DONE]);
             drain_wait(&bar[SB_DONE], 0);
+        }
+    } else if constexpr (SpRoles<NH>::PP) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SpRoles<NH>::PP_SOFTMAX_REGS));
+        // ================= ping-pong softmax + epilogue (32-head groups) =================
+        // Warpgroup wg takes the tiles of global parity wg: thread = key lane of
+        // the tile, all NH heads, with its own running maxima (sMref[wg][mb]),
+        // partial sums and O^T accumulator (TMEM O^T[ob][wg]).  An item ends with
+        // the two partial softmaxes combined per head:
+        //   M = max(m0, m1), a_w = 2^(m_w - M), o = (a0 O0 + a1 O1) / (a0 l0 + a1 l1).
+        using HD = SpHeads<NH>;
+        constexpr int SMT = SpRoles<NH>::SMT;
+        constexpr int HH = NH / 2;                     // heads each warpgroup writes out
+        constexpr uint32_t BAR_ALL = 4;                // named barrier over both warpgroups
+        const int wg = warp >> 2;
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;                // key lane (S^T) / d lane (O^T)
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool head_owner = (lane % HD::LPH) == 0;
+        const uint32_t barw = 1u + 2u * (uint32_t)wg;  // this warpgroup's named barrier
+        float *sRedW = sRed + wg * NH * 4;
+        float *sMrefW = sMref + wg * 2 * NH;
+        const float4 *red4W = reinterpret_cast<const float4 *>(sRedW);
+        float *sXch = reinterpret_cast<float *>(smem + SM::OFF_PPX);   // [wg][max | sum][NH]
+        float *sCmb = reinterpret_cast<float *>(smem + SM::OFF_CMB);   // [2][NH]
+        const uint32_t prow = smem_u32(sP) + r * RB;
+        uint32_t pphys[NH / 8];
+#pragma unroll
+        for (int cl = 0; cl < NH / 8; ++cl) {
+            const uint32_t c = (uint32_t)cl;
+            const uint32_t ph = RB == 128 ? (c ^ (r & 7)) : (RB == 64 ? (c ^ ((r >> 1) & 3)) : (c ^ ((r >> 2) & 1)));
+            pphys[cl] = ph * 16u;
+        }
+        const bool trace0 = trb != nullptr && threadIdx.x == 0;
+        const float sl = p.scale_log2;
+        // x[h] = s[h] scale - m[h] against this warpgroup's current reference
+        auto exps_pp = [&](const float (&sr)[NH], float (&x)[NH], const float *mref) {
+#pragma unroll
+            for (int h = 0; h < NH; h += 4) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(mref + h);
+                f2_split(fma_f2(f2(sr[h], sr[h + 1]), f2(sl, sl), f2(-m4.x, -m4.y)), x[h], x[h + 1]);
+                f2_split(fma_f2(f2(sr[h + 2], sr[h + 3]), f2(sl, sl), f2(-m4.z, -m4.w)), x[h + 2], x[h + 3]);
+            }
+        };
+        uint32_t nq = 0, gt = 0, mb = 0;
+        bool ok = true;
+        for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
+            if (!bar_all_id(BAR_ALL, SMT, ok && !*abort_flag))
+                break;
+            const SparseTok k = sparse_tok(p, w);
+            const int nt = k.nct + k.nrt;
+            const int ob = nq & 1;
+            const int *sSel = sIdx + ob * p.tsel;
+            ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_IF + ob], (nq >> 1) & 1, abort_flag));
+            uint64_t lp2[NH / 2];
+#pragma unroll
+            for (int h = 0; h < NH / 2; ++h)
+                lp2[h] = f2(0.f, 0.f);
+            bool first = true;
+            uint32_t glast = 0;
+            for (int i = 0; i < nt; ++i, ++gt) {
+                if ((int)(gt & 1) != wg)
+                    continue;              // the other warpgroup's tile
+                const uint32_t sb = gt & 1;
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_SF + sb], (gt >> 1) & 1, abort_flag));
+                const bool valid = i < k.nct ? sSel[i * kSpBN + r] >= 0
+                                             : k.rlo + (i - k.nct) * kSpBN + r <= k.rhi;
+                tc_fence_after();
+                float x[NH];
+                bool need = first;         // a warpgroup's first tile of an item sets its reference
+                {
+                    float sr[NH];
+                    tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, sr);
+                    tmem_ld_wait();
+                    if (!need)
+                        exps_pp(sr, x, sMrefW + mb * NH);
+                }
+                if (trace0)
+                    trace_ev(trb, 3, 1, w, i);
+                if (!need) {
+                    bool exceed = false;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        exceed |= x[h] > 8.f;
+                    need = bar_any_id(barw, 128, valid && exceed);
+                }
+                if (need) {
+                    float sc[NH];
+                    tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, sc);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+                        sc[h] = valid ? sc[h] * sl : -INFINITY;
+                    warp_reduce_heads<NH, true>(sc, lane);
+                    if (head_owner) {
+#pragma unroll
+                        for (int e = 0; e < HD::VPL; ++e)
+                            sRedW[HD::head(lane, e) * 4 + quad] = sc[e];
+                    }
+                    bar_sync_id(barw, 128);
+                    const float *mold = sMrefW + mb * NH;
+                    bool moved = false;
+                    if (!first) {
+#pragma unroll
+                        for (int h = 0; h < NH; h += 2) {
+                            const float o0 = mold[h], o1 = mold[h + 1];
+                            const float a0 = sp_factor(o0, sp_new_ref(red4W[h], o0));
+                            const float a1 = sp_factor(o1, sp_new_ref(red4W[h + 1], o1));
+                            moved |= (a0 != 1.f) | (a1 != 1.f);
+                            lp2[h >> 1] = fma_f2(lp2[h >> 1], f2(a0, a1), f2(0.f, 0.f));
+                        }
+                    }
+                    if (moved) {
+                        // O^T[ob][wg] holds this warpgroup's earlier PVs of the item;
+                        // the last of them is the PV of tile gt - 2
+                        ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1, abort_flag));
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < NH; c += 16) {
+                            float ov[16];
+                            tmem_ld_cols<16>(tl + TM_O0 + (ob * 2 + wg) * NH + c, ov);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                const float old = mold[c + q];
+                                ov[q] *= sp_factor(old, sp_new_ref(red4W[c + q], old));
+                            }
+                            tmem_st_cols<16>(tl + TM_O0 + (ob * 2 + wg) * NH + c, ov);
+                        }
+                        tmem_st_wait();
+                    }
+                    if (r < NH)
+                        sMrefW[(mb ^ 1) * NH + r] = sp_new_ref(red4W[r], mold[r]);
+                    bar_sync_id(barw, 128);
+                    mb ^= 1;
+                    float sr[NH];
+                    tmem_ld_cols<NH>(tl + TM_S0 + sb * NH, sr);
+                    tmem_ld_wait();
+                    exps_pp(sr, x, sMrefW + mb * NH);
+                }
+                // the scores are in registers: the MMA may refill this S^T buffer
+                tc_fence_before();
+                mbar_arrive(&bar[SB_SE + sb]);
+                uint32_t pk[NH / 2];
+                if (valid) {
+#pragma unroll
+                    for (int h = 0; h < NH; h += 2) {
+                        const float e0 = ex2_approx(x[h]), e1 = ex2_approx(x[h + 1]);
+                        lp2[h >> 1] = add_f2(lp2[h >> 1], f2(e0, e1));
+                        pk[h >> 1] = pack_bf16x2(e0, e1);
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < NH / 2; ++h)
+                        pk[h] = 0u;
+                }
+                // P^T buffer sb is free once the PV of tile gt - 2 completed
+                if (gt >= 2)
+                    ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + sb], ((gt >> 1) - 1) & 1, abort_flag));
+                const uint32_t prow_b = prow + sb * SM::P_STRIDE;
+#pragma unroll
+                for (int cl = 0; cl < NH / 8; ++cl)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow_b + pphys[cl]),
+                                 "r"(pk[4 * cl]), "r"(pk[4 * cl + 1]), "r"(pk[4 * cl + 2]), "r"(pk[4 * cl + 3])
+                                 : "memory");
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar[SB_PF + sb]);
+                if (trace0)
+                    trace_ev(trb, 3, 2, w, i);
+                first = false;
+                glast = gt;
+            }
+            // ---- epilogue: each warpgroup's (max, sum) per head, then the combine ----
+            if (trace0)
+                trace_ev(trb, 3, 3, w, nt);
+            {
+                float lpart[NH];
+#pragma unroll
+                for (int h = 0; h < NH; h += 2)
+                    f2_split(lp2[h >> 1], lpart[h], lpart[h + 1]);
+                warp_reduce_heads<NH, false>(lpart, lane);
+                if (head_owner) {
+#pragma unroll
+                    for (int e = 0; e < HD::VPL; ++e)
+                        sRedW[HD::head(lane, e) * 4 + quad] = lpart[e];
+                }
+            }
+            if (!first) {
+                // this warpgroup's last PV of the item has completed
+                ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OD + wg], (glast >> 1) & 1, abort_flag));
+                tc_fence_after();
+            }
+            bar_sync_id(barw, 128);
+            if (r < NH) {
+                const float4 q4 = red4W[r];
+                sXch[(wg * 2 + 0) * NH + r] = sMrefW[mb * NH + r];
+                sXch[(wg * 2 + 1) * NH + r] = (q4.x + q4.y) + (q4.z + q4.w);
+                sMrefW[(mb ^ 1) * NH + r] = -INFINITY;   // the next item's reference
+            }
+            bar_sync_id(BAR_ALL, SMT);
+            mb ^= 1;
+            float lse_v = -INFINITY;
+            if (wg == 0 && r < NH) {
+                const float m0 = sXch[r], l0 = sXch[NH + r], m1 = sXch[2 * NH + r], l1 = sXch[3 * NH + r];
+                const float M = fmaxf(m0, m1);
+                const float a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M);
+                const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+                const float L = a0 * l0 + a1 * l1;
+                const float inv = L > 0.f ? 1.f / L : 0.f;
+                sCmb[r] = a0 * inv;
+                sCmb[NH + r] = a1 * inv;
+                lse_v = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+            }
+            bar_sync_id(BAR_ALL, SMT);
+            tc_fence_after();
+            float o0[HH], o1[HH];
+            tmem_ld_cols<HH>(tl + TM_O0 + (ob * 2 + 0) * NH + wg * HH, o0);
+            tmem_ld_cols<HH>(tl + TM_O0 + (ob * 2 + 1) * NH + wg * HH, o1);
+            tmem_ld_wait();
+            if (ok) {
+                const size_t obase = (((size_t)k.b * p.Lq + k.t) * p.Hq + (size_t)k.kvh * p.g) * kSpD;
+#pragma unroll
+                for (int h = 0; h < HH; ++h) {
+                    const int hh = wg * HH + h;
+                    const float f0 = sCmb[hh], f1 = sCmb[NH + hh];
+                    // an accumulator a warpgroup did not touch in this item has factor 0
+                    const float v = (f0 != 0.f ? o0[h] * f0 : 0.f) + (f1 != 0.f ? o1[h] * f1 : 0.f);
+                    if (hh < p.g)
+                        p.o[obase + (size_t)hh * kSpD + r] = __float2bfloat16_rn(v);
+                }
+                if (p.lse && wg == 0 && r < p.g)
+                    p.lse[((size_t)k.b * p.Hq + (size_t)k.kvh * p.g + r) * p.Lq + k.t] = lse_v;
+            }
+            tc_fence_before();
+            mbar_arrive(&bar[SB_OE + ob]);
+            if (trace0)
+                trace_ev(trb, 3, 4, w, nt);
         }
     } else {
         // ========================== softmax + epilogue ==========================
@@ -1070,7 +1428,7 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
     const long long slots = (long long)num_sms * per_sm;
     // Few items (decode): two CTAs, one cluster, share each item's key tiles,
     // so that twice as many SMs gather; otherwise one CTA per item.
-    p.split = (p.n_items * 2 <= slots) ? 2 : 1;
+    p.split = (!SpRoles<NH>::PP && p.n_items * 2 <= slots) ? 2 : 1;
     if (p.split == 1) {
         long long grid = slots < p.n_items ? slots : p.n_items;
         if (grid < 1)
