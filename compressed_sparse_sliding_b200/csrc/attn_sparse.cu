@@ -555,9 +555,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int nt = k.nct + k.nrt;
             const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             // source row of copy u of tile i, or -1 (zero-filled)
-            // source row of copy u of selected tile i; an unselected slot reads
-            // row 0 (finite data the softmax masks) rather than a zero fill
-            auto src_of = [&](int i, int u) -> int { return max(sSel[i * kSpBN + u * RPI + rsub], 0); };
+            // source row of copy u of selected tile i, or -1: an unselected slot
+            // is zero-filled without a read (a fixed stand-in row would pile
+            // every early token's empty slots onto one L2 line)
+            auto src_of = [&](int i, int u) -> int { return sSel[i * kSpBN + u * RPI + rsub]; };
             const __nv_bfloat16 *kc8 = p.kc + c8 * 8, *vc8 = p.vc + c8 * 8;   // this thread's chunk
             // K of tile i goes out kSpLead tiles ahead of V of the same tile, so
             // that the next scores need not queue behind a V stage that a PV
@@ -593,8 +594,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             srck[u] = src_of(i, u);
                         const uint32_t dst = smem_u32(sK + ks * SM::KV_BYTES) + dchunk;
 #pragma unroll
-                        for (int u = 0; u < CPT; ++u)
-                            cp_async_16_full(dst + sw128_offset(u * RPI + rsub, c8 & 7), kc8 + (size_t)srck[u] * kSpD);
+                        for (int u = 0; u < CPT; ++u) {
+                            const int sr = srck[u];
+                            cp_async_16(dst + sw128_offset(u * RPI + rsub, c8 & 7), kc8 + (size_t)max(sr, 0) * kSpD,
+                                        sr >= 0 ? 16u : 0u);
+                        }
                         cp_async_mbar_arrive(&bar[SB_KF + ks]);
                         mbar_arrive(&bar[SB_KF + ks]);
                     }
@@ -626,8 +630,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     } else {
                         const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
 #pragma unroll
-                        for (int u = 0; u < CPT; ++u)
-                            cp_async_16_full(dst + sw128_offset(u * RPI + rsub, c8 & 7), vc8 + (size_t)srcv[u] * kSpD);
+                        for (int u = 0; u < CPT; ++u) {
+                            const int sr = srcv[u];
+                            cp_async_16(dst + sw128_offset(u * RPI + rsub, c8 & 7), vc8 + (size_t)max(sr, 0) * kSpD,
+                                        sr >= 0 ? 16u : 0u);
+                        }
                         cp_async_mbar_arrive(&bar[SB_VF + vs]);
                         mbar_arrive(&bar[SB_VF + vs]);
                     }

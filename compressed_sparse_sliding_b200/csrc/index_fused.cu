@@ -319,6 +319,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t *hist = col;                             // [bin / 2] stride kFxBM
         uint32_t *bkey = col + (kFxBins / 2) * kFxBM;     // [slot] stride kFxBM
         uint32_t *bpk = bkey + kFxCap * kFxBM;
+        const uint32_t hist_s = smem_u32(hist), bkey_s = smem_u32(bkey), bpk_s = smem_u32(bpk);
 
         int mode = !valid ? FX_NONE : (nv > K ? FX_OPEN : FX_ALL);
         uint32_t lo = 0, top_m1 = 0xFFFFFFFFu, blo = 0, bhi_m1 = 0;
@@ -361,13 +362,16 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float sv[32];
                     uint32_t kv[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        float s = wv[0] * fmaxf(d[0][c], 0.f);
+                    for (int c = 0; c < 32; c += 2) {
+                        // two keys at a time: sum_h w_h relu(d_h) in packed pairs
+                        uint64_t acc = fma_f2(f2(wv[0], wv[0]), f2(fmaxf(d[0][c], 0.f), fmaxf(d[0][c + 1], 0.f)),
+                                              f2(0.f, 0.f));
 #pragma unroll
                         for (int h = 1; h < HI; ++h)
-                            s = fmaf(wv[h], fmaxf(d[h][c], 0.f), s);
-                        sv[c] = s;
-                        kv[c] = fx_key(s);
+                            acc = fma_f2(f2(wv[h], wv[h]), f2(fmaxf(d[h][c], 0.f), fmaxf(d[h][c + 1], 0.f)), acc);
+                        f2_split(acc, sv[c], sv[c + 1]);
+                        kv[c] = fx_key(sv[c]);
+                        kv[c + 1] = fx_key(sv[c + 1]);
                     }
                     const int nvh = max(0, min(32, nv - j0));     // visible: c < nvh
                     if (ptype == 0) {
@@ -386,7 +390,9 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                 ab += (inw && above) ? 1 : 0;
                                 const uint32_t bin = (k - lo) >> sh;
                                 if (inw && !above)
-                                    atomicAdd(hist + (bin >> 1) * kFxBM, 1u << ((bin & 1u) * 16u));
+                                    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(hist_s + (bin >> 1) * (kFxBM * 4)),
+                                                 "r"(1u << ((bin & 1u) * 16u))
+                                                 : "memory");
                             }
                         }
                     } else if (mode == FX_ALL) {
@@ -422,8 +428,10 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             const bool pick = v && k > bhi_m1;
                             const bool keep = v && k >= blo && k <= bhi_m1 && nb < kFxCap;
                             if (keep) {
-                                bkey[nb * kFxBM] = k;
-                                bpk[nb * kFxBM] = (uint32_t)(j0 + c) | ((uint32_t)pos << 16);
+                                asm volatile("st.shared.u32 [%0], %1;" ::"r"(bkey_s + nb * (kFxBM * 4)), "r"(k) : "memory");
+                                asm volatile("st.shared.u32 [%0], %1;" ::"r"(bpk_s + nb * (kFxBM * 4)),
+                                             "r"((uint32_t)(j0 + c) | ((uint32_t)pos << 16))
+                                             : "memory");
                             }
                             nb += keep ? 1 : 0;
                             if (pick && pos < K) {
