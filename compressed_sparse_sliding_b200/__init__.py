@@ -382,13 +382,14 @@ TRACE_ROLES = {1: "gather", 2: "mma", 3: "softmax"}
 def hyb_trace_attach(buf: Optional[torch.Tensor]) -> None:
     """Attach (or, with None, detach) a device buffer for the per-role timeline
     of CTA 0 of the kernels that record one (see hyb_trace_attach in the C
-    header).  The record count in the buffer's first word is cleared here."""
+    header).  The record counts in the buffer's first four words are cleared
+    here."""
     if buf is None:
         st = _lib.hyb_trace_attach(None, 0)
     else:
         if buf.device.type != "cuda" or not buf.is_contiguous():
             raise ValueError("trace buffer: a contiguous CUDA tensor")
-        buf.view(torch.uint8)[:16].zero_()
+        buf.view(torch.uint8)[:32].zero_()
         st = _lib.hyb_trace_attach(_ptr(buf), buf.numel() * buf.element_size())
     if st != HYB_OK:
         raise HybError(st, "hyb_trace_attach")
@@ -396,15 +397,18 @@ def hyb_trace_attach(buf: Optional[torch.Tensor]) -> None:
 
 def trace_records(buf: torch.Tensor):
     """The records of an attached buffer as a list of dicts (clock, role,
-    event, item, tile), in the order they were appended."""
+    event, item, tile), all roles merged in clock order."""
     words = buf.view(torch.int64).cpu().numpy().view("uint64")
-    n = int(words[0] & 0xFFFFFFFF)
-    cap = (words.size - 2) // 2
+    cap = (words.size - 4) // 8
     out = []
-    for r in range(min(n, cap)):
-        clk, tag = int(words[2 + 2 * r]), int(words[3 + 2 * r])
-        out.append(dict(clock=clk, role=tag >> 56, event=(tag >> 48) & 0xFF,
-                        item=(tag >> 16) & 0xFFFFFFFF, tile=tag & 0xFFFF))
+    for role in range(4):
+        n = min(int(words[role] & 0xFFFFFFFF), cap)
+        base = 4 + 2 * role * cap
+        for r in range(n):
+            clk, tag = int(words[base + 2 * r]), int(words[base + 2 * r + 1])
+            out.append(dict(clock=clk, role=tag >> 56, event=(tag >> 48) & 0xFF,
+                            item=(tag >> 16) & 0xFFFFFFFF, tile=tag & 0xFFFF))
+    out.sort(key=lambda d: d["clock"])
     return out
 
 

@@ -675,9 +675,9 @@ hyb_status hyb_trace_attach(void *buf, size_t bytes)
     unsigned long long *b = static_cast<unsigned long long *>(buf);
     unsigned int cap = 0;
     if (b) {
-        if ((reinterpret_cast<uintptr_t>(buf) & 15u) || bytes < 32)
+        if ((reinterpret_cast<uintptr_t>(buf) & 15u) || bytes < 96)
             return HYB_ERR_INVALID_ARG;
-        const size_t recs = (bytes - 16) / 16;
+        const size_t recs = (bytes / 8 - 4) / 8;   // records per role region
         cap = recs > 0xFFFFFFFFull ? 0xFFFFFFFFu : (unsigned int)recs;
     }
     if (cudaMemcpyToSymbol(g_trace_cap, &cap, sizeof(cap)) != cudaSuccess ||

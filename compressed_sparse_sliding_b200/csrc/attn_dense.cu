@@ -571,6 +571,9 @@ static cudaError_t launch_hca_t(const DenseParams &p, const void *q, const void 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
+    e = check_reg_split(kern, kDnThreads, 256, kDnSoftmaxRegs, kDnOtherRegs);
+    if (e != cudaSuccess)
+        return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDnThreads, smem);
     if (e != cudaSuccess)

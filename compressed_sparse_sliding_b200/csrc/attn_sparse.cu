@@ -67,8 +67,11 @@ struct SparseSmem {
     static constexpr int KV_BYTES = kSpBN * kSpD * 2;
     static constexpr int P_BYTES = kSpBN * NH * 2;
     static constexpr int P_STRIDE = (P_BYTES + 1023) & ~1023;
-    static constexpr int KS = 2;                                   // K ring depth
-    static constexpr int VS = NH == 64 ? 2 : 3;                    // V ring depth
+    // K runs deeper than V: a K stage frees as soon as its scores are taken,
+    // a V stage only after the tile's softmax and PV, and the scores of later
+    // tiles should not wait on a V stage
+    static constexpr int KS = NH == 64 ? 2 : 3;                    // K ring depth
+    static constexpr int VS = 2;                                   // V ring depth
     static constexpr int OFF_Q = 0;                                // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
@@ -131,29 +134,6 @@ __device__ __forceinline__ SparseTok sparse_tok(const SparseParams &p, long long
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)
 {
     asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Barrier among the producer threads (named barrier 2).
-template <int N>
-__device__ __forceinline__ void prod_sync()
-{
-    asm volatile("bar.sync 2, %0;" ::"n"(N) : "memory");
-}
-
-// AND of a predicate over the producer threads (named barrier 2).
-template <int N>
-__device__ __forceinline__ bool prod_all(bool v)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, 2, %2, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "n"(N)
-        : "memory");
-    return r != 0;
 }
 
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2)
@@ -361,7 +341,7 @@ struct SpRoles {
     static constexpr bool PP = kSpPingPong && NH == 32;
     // ping-pong register split (setmaxnreg): 8 softmax warps up, producer and
     // MMA warps down; 256 x 144 + 160 x 96 = 52224 <= 416 x 128, the budget
-    // the block launches with
+    // the block launches with (the launcher checks it against the allocated count)
     static constexpr int PP_SOFTMAX_REGS = 144;
     static constexpr int PP_OTHER_REGS = 96;
     static constexpr int HS = NH >= 32 ? 2 : 1;       // softmax warpgroups (head halves, or tile parities)
@@ -402,6 +382,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
+    uint32_t tn = 0;                                  // this thread's trace records
     constexpr int PW = SpRoles<NH>::PW;
     constexpr int NPT = 32 * PW;                // producer threads
 
@@ -457,31 +438,53 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if constexpr (SpRoles<NH>::PP)
             asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(SpRoles<NH>::PP_OTHER_REGS));
         // ================================ producer ================================
-        // 16 lanes per 256-byte row, two rows per warp instruction.  Within an
-        // item no thread leaves early: a failed wait clears `ok`, the copies
-        // go on (every source row stays in range), and the producers agree
-        // on `ok` once per item before its named barrier.
+        // 16 lanes per 256-byte row, two rows per warp instruction.  Each
+        // producer warp decodes the selection entries of exactly the rows its
+        // own lanes copy, so the warps need no barrier among themselves; the
+        // softmax learns that the whole table is written from an mbarrier.
+        // Within an item no warp leaves early: a failed wait clears `ok` and
+        // the copies go on (every source row stays in range).
         const int pt = threadIdx.x - 32 * SpRoles<NH>::PROD_WARP0;
+        const int pw = pt >> 5;                 // producer warp
         const int c8 = pt & 15;                 // 16-byte chunk of the row
-        const int rsub = pt >> 4;               // rows rsub, rsub + RPI, ...
+        const int rsub = pt >> 4;               // rows rsub, rsub + RPI, ... (2 pw and 2 pw + 1)
         const uint32_t dchunk = (uint32_t)(c8 >> 3) * kSpBN * 128;
         uint32_t kc = 0, vc = 0, nq = 0;
         bool ok = true;
-        // entries q0 + e NPT + pt of item w's selection (-1 past topk); item
-        // w = (b Lq + t) Hkv + KV head, and items number below 2^31
-        auto load_sel = [&](long long w, int q0, int (&jv)[kSpSelBatch]) {
+        // slot of this warp's e-th selection entry, tiles counted from t0s:
+        // rows u RPI + 2 pw + bit of each tile
+        auto slot_of = [&](int t0s, int e) -> int {
+            const int tile = e / (2 * CPT), rem = e - tile * (2 * CPT);
+            return (t0s + tile) * kSpBN + (rem >> 1) * RPI + 2 * pw + (rem & 1);
+        };
+        // this CTA's selected tiles of an item: [s0, s1)
+        auto sel_tiles = [&](const SparseTok &k, int &s0, int &s1) {
+            const int nt = k.nct + k.nrt;
+            s0 = min(tile_lo(nt), k.nct);
+            s1 = min(tile_hi(nt), k.nct);
+        };
+        // this warp's entries e0 + lane + 32 j (of ne) of item w's selection,
+        // -1 past topk; item w = (b Lq + t) Hkv + KV head, below 2^31
+        auto load_sel = [&](long long w, int t0s, int ne, int e0, int (&jv)[kSpSelBatch]) {
             const int32_t *irow = p.idx + (size_t)((uint32_t)w / (uint32_t)p.Hkv) * p.topk;
 #pragma unroll
-            for (int e = 0; e < kSpSelBatch; ++e) {
-                const int q = q0 + e * NPT + pt;
-                jv[e] = q < p.topk ? __ldg(irow + q) : -1;
+            for (int j = 0; j < kSpSelBatch; ++j) {
+                const int e = e0 + lane + 32 * j;
+                const int q = slot_of(t0s, e);
+                jv[j] = (e < ne && q < p.topk) ? __ldg(irow + q) : -1;
             }
+        };
+        auto load_first = [&](long long w, int (&jv)[kSpSelBatch]) {
+            const SparseTok kn = sparse_tok(p, w);
+            int s0, s1;
+            sel_tiles(kn, s0, s1);
+            load_sel(w, s0, (s1 - s0) * 2 * CPT, 0, jv);
         };
         int jnext[kSpSelBatch];
         if (w0 < p.n_items)
-            load_sel(w0, 0, jnext);
+            load_first(w0, jnext);
         for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
-            if (!prod_all<NPT>(ok && !*abort_flag))
+            if (!__all_sync(0xffffffffu, ok && !*abort_flag))
                 break;
             const SparseTok k = sparse_tok(p, w);
             const int qb = nq & 1;
@@ -492,66 +495,72 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ok &= __all_sync(0xffffffffu, mbar_wait(&bar[SB_OE + qb], ((nq >> 1) - 1) & 1, abort_flag));
             }
             if (pt == 0) {
+                trace_ev(trb, tn, 1, 3, w, 0);
                 mbar_arrive_expect_tx(&bar[SB_QF + qb], SM::Q_BYTES);
                 const int qrow = (int)(((long long)k.b * p.Lq + k.t) * p.Hq) + k.kvh * p.g;
                 for (int cb = 0; cb < 2; ++cb)
                     tma_load_2d(sQ + qb * SM::Q_BYTES + cb * NH * 128, &tm_q, &bar[SB_QF + qb], cb * 64,
                                 qrow);
             }
-            // decode the item's selection once into buffer qb: source row of
-            // every slot, or -1 (unselected, invisible or out of range).  A
-            // batch's loads are all in flight together; the first batch was
-            // loaded during the previous item's copies.
+            // decode this warp's part of the item's selection into buffer qb:
+            // source row of every slot, or -1 (unselected, invisible, out of
+            // range or past topk).  A batch's loads are all in flight
+            // together; the first batch was loaded during the previous item.
             int *sSel = sIdx + qb * p.tsel;
             {
                 const long long wstart = k.pos - p.W + 1;
-                // selected slots of this CTA's tiles (the prefetch range)
-                const int pq0 = tile_lo(k.nct + k.nrt) * kSpBN, pq1 = tile_hi(k.nct + k.nrt) * kSpBN;
+                int s0, s1;
+                sel_tiles(k, s0, s1);
+                const int ne = (s1 - s0) * 2 * CPT;
 #pragma unroll 1
-                for (int q0 = 0; q0 < p.topk; q0 += kSpSelBatch * NPT) {
+                for (int e0 = 0; e0 < ne; e0 += 32 * kSpSelBatch) {
                     int jv[kSpSelBatch];
-                    if (q0 == 0) {
+                    if (e0 == 0) {
 #pragma unroll
-                        for (int e = 0; e < kSpSelBatch; ++e)
-                            jv[e] = jnext[e];
+                        for (int j = 0; j < kSpSelBatch; ++j)
+                            jv[j] = jnext[j];
                     } else {
-                        load_sel(w, q0, jv);
+                        load_sel(w, s0, ne, e0, jv);
                     }
 #pragma unroll
-                    for (int e = 0; e < kSpSelBatch; ++e) {
-                        const int q = q0 + e * NPT + pt;
-                        if (q < p.topk) {
-                            const int j = jv[e];
-                            if (j >= p.Nc)
-                                set_error(HYB_ERR_DEVICE_BOUNDS);
-                            const bool v = j >= 0 && j < p.Nc && ((long long)(j + 1) * p.m - 1 < wstart);
-                            const int srow = p.pregathered
-                                                 ? ((int)((uint32_t)w / (uint32_t)p.Hkv) * p.topk + q) * p.Hkv + k.kvh
-                                                 : (k.b * p.Nc + j) * p.Hkv + k.kvh;
-                            sSel[q] = v ? srow : -1;
-                            if (p.prefetch && v && q >= pq0 && q < pq1) {
-                                // the row's K and V lines into L2 now: the copies
-                                // of the item's tiles then wait on L2, not HBM
-                                const __nv_bfloat16 *kr0 = p.kc + (size_t)srow * kSpD;
-                                const __nv_bfloat16 *vr0 = p.vc + (size_t)srow * kSpD;
-                                asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0));
-                                asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0 + 64));
-                                asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0));
-                                asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0 + 64));
+                    for (int j = 0; j < kSpSelBatch; ++j) {
+                        const int e = e0 + lane + 32 * j;
+                        if (e < ne) {
+                            const int q = slot_of(s0, e);
+                            int src = -1;
+                            if (q < p.topk) {
+                                const int jj = jv[j];
+                                if (jj >= p.Nc)
+                                    set_error(HYB_ERR_DEVICE_BOUNDS);
+                                const bool v = jj >= 0 && jj < p.Nc && ((long long)(jj + 1) * p.m - 1 < wstart);
+                                const int srow = p.pregathered
+                                                     ? ((int)((uint32_t)w / (uint32_t)p.Hkv) * p.topk + q) * p.Hkv +
+                                                           k.kvh
+                                                     : (k.b * p.Nc + jj) * p.Hkv + k.kvh;
+                                src = v ? srow : -1;
+                                if (p.prefetch && v) {
+                                    // the row's K and V lines into L2 now: the copies
+                                    // of the item's tiles then wait on L2, not HBM
+                                    const __nv_bfloat16 *kr0 = p.kc + (size_t)srow * kSpD;
+                                    const __nv_bfloat16 *vr0 = p.vc + (size_t)srow * kSpD;
+                                    asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0));
+                                    asm volatile("prefetch.global.L2 [%0];" ::"l"(kr0 + 64));
+                                    asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0));
+                                    asm volatile("prefetch.global.L2 [%0];" ::"l"(vr0 + 64));
+                                }
                             }
+                            sSel[q] = src;
                         }
                     }
                 }
-                // slots past topk in the last selected tile
-                for (int q = p.topk + pt; q < p.tsel; q += NPT)
-                    sSel[q] = -1;
             }
             mbar_arrive(&bar[SB_IF + qb]);      // the softmax reads key validity from it
-            prod_sync<NPT>();
+            __syncwarp();                       // this warp's lanes read each other's entries
+            if (pt == 0)
+                trace_ev(trb, tn, 1, 4, w, 0);
             // the next item's first batch, in flight during this item's copies
-            // (issued after the barrier, which would otherwise wait for it)
             if (w + wstep < p.n_items)
-                load_sel(w + wstep, 0, jnext);
+                load_first(w + wstep, jnext);
             const int nt = k.nct + k.nrt;
             const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             // source row of copy u of tile i, or -1 (zero-filled)
@@ -603,7 +612,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mbar_arrive(&bar[SB_KF + ks]);
                     }
                     if (pt == 0)
-                        trace_ev(trb, 1, 1, w, i);
+                        trace_ev(trb, tn, 1, 1, w, i);
                     ++kc;
                 }
                 if (kSpLead == 0) {
@@ -639,7 +648,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mbar_arrive(&bar[SB_VF + vs]);
                     }
                     if (pt == 0)
-                        trace_ev(trb, 1, 2, w, i - kSpLead);
+                        trace_ev(trb, tn, 1, 2, w, i - kSpLead);
                     ++vc;
                 }
                 if (kSpLead == 1) {
@@ -695,7 +704,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_OD + pb]);
                     mma_commit(&bar[SB_VE + vs]);
-                    trace_ev(trb, 2, 2, w, (int)pcnt);
+                    trace_ev(trb, tn, 2, 2, w, (int)pcnt);
                     ++vc;
                     ++pcnt;
                     return true;
@@ -725,7 +734,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                         mma_commit(&bar[SB_OD + pb]);
                         mma_commit(&bar[SB_VE + vs]);
-                        trace_ev(trb, 2, 2, w, (int)(g - gt0));
+                        trace_ev(trb, tn, 2, 2, w, (int)(g - gt0));
                         ++vc;
                         return true;
                     };
@@ -747,7 +756,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                         mma_commit(&bar[SB_SF + (gt & 1)]);
                         mma_commit(&bar[SB_KE + ks]);
-                        trace_ev(trb, 2, 1, w, ii);
+                        trace_ev(trb, tn, 2, 1, w, ii);
                         ++kc;
                         if (ii == ntl - 1)
                             mma_commit(&bar[SB_QE + qb]);
@@ -784,7 +793,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     mma_commit(&bar[SB_SF + (gt & 1)]);
                     mma_commit(&bar[SB_KE + ks]);
-                    trace_ev(trb, 2, 1, w, i);
+                    trace_ev(trb, tn, 2, 1, w, i);
                     ++kc;
                     if (ii == ntl - 1)
                         mma_commit(&bar[SB_QE + qb]);
@@ -881,7 +890,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         exps_pp(sr, x, sMrefW + mb * NH);
                 }
                 if (trace0)
-                    trace_ev(trb, 3, 1, w, i);
+                    trace_ev(trb, tn, 3, 1, w, i);
                 if (!need) {
                     bool exceed = false;
 #pragma unroll
@@ -972,13 +981,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
                 if (trace0)
-                    trace_ev(trb, 3, 2, w, i);
+                    trace_ev(trb, tn, 3, 2, w, i);
                 first = false;
                 glast = gt;
             }
             // ---- epilogue: each warpgroup's (max, sum) per head, then the combine ----
             if (trace0)
-                trace_ev(trb, 3, 3, w, nt);
+                trace_ev(trb, tn, 3, 3, w, nt);
             {
                 float lpart[NH];
 #pragma unroll
@@ -1040,7 +1049,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
             if (trace0)
-                trace_ev(trb, 3, 4, w, nt);
+                trace_ev(trb, tn, 3, 4, w, nt);
         }
     } else {
         // ========================== softmax + epilogue ==========================
@@ -1138,7 +1147,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         exps_of(sr, x);
                 }
                 if (trace0)
-                    trace_ev(trb, 3, 1, w, i);
+                    trace_ev(trb, tn, 3, 1, w, i);
                 if (!need) {
                     bool exceed = false;
 #pragma unroll
@@ -1238,7 +1247,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_before();
                 mbar_arrive(&bar[SB_PF + sb]);
                 if (trace0)
-                    trace_ev(trb, 3, 2, w, i);
+                    trace_ev(trb, tn, 3, 2, w, i);
             }
             float lpart[NHW];
 #pragma unroll
@@ -1246,7 +1255,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 f2_split(lp2[h >> 1], lpart[h], lpart[h + 1]);
             // ---- epilogue: l[h] = sum over keys; o[h][d] = O^T[d][h] / l[h] ----
             if (trace0)
-                trace_ev(trb, 3, 3, w, nt);
+                trace_ev(trb, tn, 3, 3, w, nt);
             warp_reduce_heads<NHW, false>(lpart, lane);
             if (head_owner) {
 #pragma unroll
@@ -1359,7 +1368,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&bar[SB_OE + ob]);
             if (trace0)
-                trace_ev(trb, 3, 4, w, nt);
+                trace_ev(trb, tn, 3, 4, w, nt);
         }
     }
 
@@ -1426,6 +1435,12 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
+    if constexpr (SpRoles<NH>::PP) {
+        e = check_reg_split(kern, SpRoles<NH>::THREADS, SpRoles<NH>::SMT, SpRoles<NH>::PP_SOFTMAX_REGS,
+                            SpRoles<NH>::PP_OTHER_REGS);
+        if (e != cudaSuccess)
+            return e;
+    }
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, SpRoles<NH>::THREADS, smem);
     if (e != cudaSuccess)

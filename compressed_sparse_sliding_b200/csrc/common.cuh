@@ -49,31 +49,39 @@ __device__ __forceinline__ uint64_t global_ns()
 
 // ---------------------------------------------------------------------------
 // Optional per-role timeline (a debug aid; see hyb_trace_attach).  When a
-// buffer is attached, CTA 0 of a kernel that supports it appends one record
-// per event: word 0 of the buffer counts records, record r occupies words
-// 2 + 2r (the SM clock) and 3 + 2r (role << 56 | event << 48 | item << 16 |
-// tile).  Other CTAs, and every CTA without a buffer, skip the records.
+// buffer is attached, one thread per role of CTA 0 of a kernel that supports
+// it appends a record per event to its role's region: words 0-3 of the buffer
+// count the records of roles 0-3, and role r's region starts at word
+// 4 + 2 r R (R records per region); a record is two words, the SM clock, then
+// role << 56 | event << 48 | item << 16 | tile.  Each tracing thread keeps
+// its count in a register, so an event costs it two stores and no round
+// trip.  Other CTAs, and every CTA without a buffer, skip the records.
 // ---------------------------------------------------------------------------
 __device__ unsigned long long *g_trace_buf = nullptr;
-__device__ unsigned int g_trace_cap = 0;     // records the buffer holds
+__device__ unsigned int g_trace_cap = 0;     // records per role region
 
 __device__ __forceinline__ unsigned long long *trace_buffer()
 {
     return blockIdx.x == 0 && blockIdx.y == 0 ? g_trace_buf : nullptr;
 }
 
-__device__ __forceinline__ void trace_ev(unsigned long long *tb, int role, int ev, long long item, int tile)
+// One event of `role` (0..3) by the role's only tracing thread; tn is that
+// thread's running record count.
+__device__ __forceinline__ void trace_ev(unsigned long long *tb, uint32_t &tn, int role, int ev, long long item,
+                                         int tile)
 {
     if (!tb)
         return;
     const unsigned long long clk = clock64();
-    const unsigned int r = atomicAdd(reinterpret_cast<unsigned int *>(tb), 1u);
-    if (r < g_trace_cap) {
-        tb[2 + 2 * (size_t)r] = clk;
-        tb[3 + 2 * (size_t)r] = ((unsigned long long)role << 56) | ((unsigned long long)ev << 48) |
-                                (((unsigned long long)item & 0xFFFFFFFFull) << 16) |
-                                ((unsigned long long)tile & 0xFFFFull);
+    const size_t cap = g_trace_cap;
+    if (tn < cap) {
+        unsigned long long *rec = tb + 4 + 2 * ((size_t)role * cap + tn);
+        rec[0] = clk;
+        rec[1] = ((unsigned long long)role << 56) | ((unsigned long long)ev << 48) |
+                 (((unsigned long long)item & 0xFFFFFFFFull) << 16) | ((unsigned long long)tile & 0xFFFFull);
     }
+    ++tn;
+    tb[role] = tn;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -553,6 +561,22 @@ static bool make_map(CUtensorMap *map, const void *base, int d, int n1, int n2, 
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// setmaxnreg.inc blocks until the block's register file allows the raise, so
+// a split whose shares add up to more than the block launched with (threads x
+// the kernel's allocated register count) would wait forever.  Launchers of
+// kernels with a register split check it here first and refuse otherwise.
+template <typename Kern>
+static cudaError_t check_reg_split(Kern kern, int threads, int up_threads, int up_regs, int down_regs)
+{
+    cudaFuncAttributes a;
+    const cudaError_t e = cudaFuncGetAttributes(&a, kern);
+    if (e != cudaSuccess)
+        return e;
+    const long long have = (long long)a.numRegs * threads;
+    const long long want = (long long)up_threads * up_regs + (long long)(threads - up_threads) * down_regs;
+    return have >= want ? cudaSuccess : cudaErrorLaunchOutOfResources;
 }
 
 }  // namespace hyb

@@ -31,18 +31,25 @@
 //                  taken during E itself.
 // Order keys are the fp32 scores mapped to uint32 so that larger scores give
 // larger keys (-0.0 folded onto +0.0), as in the two-kernel path.
-// Roles (256 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 4-7 the
-// row epilogue (TMEM lane quadrants 0-3); warps 2-3 idle.  The epilogue
-// decides after each H pass whether another H or the E pass follows; the
-// producer and MMA warps learn it through two shared words and stop after E.
+// Roles (384 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 2-3 idle,
+// and two threads per row for the epilogue: warps 4-7 (TMEM lane quadrants
+// 0-3) take the first half of every pass's key tiles, warps 8-11 the second
+// half, each half with its own TMEM buffer, so that two warps per SM
+// sub-partition hide each other's latencies.  The halves histogram into
+// separate arrays and take the row's decisions together from both; for E,
+// half 1 starts its list where half 0's keys above the bin end (known from
+// half 0's histogram), so that each half writes its part of the ascending
+// list on its own.  The epilogue decides after each H pass whether another H
+// or the E pass follows; the producer and MMA warps learn it through two
+// shared words and stop after E.
 #include "common.cuh"
 
 namespace hyb {
 
-constexpr int kFxThreads = 256;
+constexpr int kFxThreads = 384;
 constexpr int kFxBM = 128;          // query rows per CTA
 constexpr int kFxBN = 64;           // keys per tile
-constexpr int kFxStages = 4;
+constexpr int kFxStages = 3;
 constexpr int kFxSampleTiles = 2;
 constexpr int kFxBins = 128;        // histogram bins per row
 constexpr int kFxCap = 64;          // boundary-bin entries kept per row
@@ -65,15 +72,16 @@ struct FxSmem {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = HI * Q_BYTES;
     static constexpr int OFF_U = OFF_K + kFxStages * K_BYTES;        // union below
-    // pass S: sample keys [slot][row]; later passes: histogram [bin / 2][row]
-    // (two u16 counters per word) followed by the boundary buffer: keys
-    // [slot][row], then (index | list position << 16) [slot][row]
+    // pass S: sample keys [slot][row]; later passes: one histogram per half
+    // [bin / 2][row] (two u16 counters per word), then the boundary buffer:
+    // keys [slot][row], then (index | list position << 16) [slot][row]
     static constexpr int SAMPLE_BYTES = kFxSampleTiles * kFxBN * kFxBM * 4;
     static constexpr int HIST_BYTES = (kFxBins / 2) * kFxBM * 4;
     static constexpr int BND_BYTES = 2 * kFxCap * kFxBM * 4;
-    static constexpr int U_BYTES = SAMPLE_BYTES > HIST_BYTES + BND_BYTES ? SAMPLE_BYTES
-                                                                         : HIST_BYTES + BND_BYTES;
-    static constexpr int OFF_BAR = OFF_U + U_BYTES;
+    static constexpr int U_BYTES = SAMPLE_BYTES > 2 * HIST_BYTES + BND_BYTES ? SAMPLE_BYTES
+                                                                             : 2 * HIST_BYTES + BND_BYTES;
+    static constexpr int OFF_X = OFF_U + U_BYTES;                    // [4][row] counts exchanged by the halves
+    static constexpr int OFF_BAR = OFF_X + 4 * kFxBM * 4;
     static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
     static constexpr int BYTES = OFF_MISC + 16 * 4;
 };
@@ -115,19 +123,25 @@ __device__ __forceinline__ uint32_t fx_last(uint32_t lo, int sh, uint32_t n)
     return e > 0xFFFFFFFFull ? 0xFFFFFFFFu : (uint32_t)e;
 }
 
-// AND of a predicate over the 128 epilogue threads (named barrier 1).
+// AND of a predicate over the 256 epilogue threads (named barrier 1).
 __device__ __forceinline__ bool fx_all(bool v)
 {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, 1, 128, q;\n\t"
+        "bar.red.and.pred p, 1, 256, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)v)
         : "memory");
     return r != 0;
+}
+
+// Barrier over the 256 epilogue threads (named barrier 1).
+__device__ __forceinline__ void fx_sync()
+{
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 // Bounded wait until the shared decision word reaches `p` (or the CTA aborts).
@@ -152,6 +166,21 @@ __device__ __forceinline__ bool fx_wait_decided(volatile int *decided, int p, vo
 // Row modes of the epilogue
 enum { FX_ALL = 0, FX_BIN = 1, FX_TIE = 2, FX_OPEN = 3, FX_NONE = 4 };
 
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void fx_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
 template <int HI, int DI>
 __global__ void __launch_bounds__(kFxThreads, 1)
 index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -165,14 +194,18 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t *sQ = smem + SM::OFF_Q;
     uint8_t *sK = smem + SM::OFF_K;
     uint32_t *sU = reinterpret_cast<uint32_t *>(smem + SM::OFF_U);
+    uint32_t *sX = reinterpret_cast<uint32_t *>(smem + SM::OFF_X);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     volatile int *abort_flag = misc + 1;
     volatile int *decided = misc + 2;      // passes 0 .. *decided are known to exist (or not)
     volatile int *last_pass = misc + 3;    // index of the E pass once known
-    // bars: 0 Q full, 1-4 K full, 5-8 K empty, 9-10 D full, 11-12 D empty, 13 done
+    // bars: 0 Q full, 1.. K full, 1 + S.. K empty, then per half D full, D empty, then done
+    constexpr int S = kFxStages;
+    constexpr int B_KF = 1, B_KE = 1 + S, B_DF = 1 + 2 * S, B_DE = 3 + 2 * S, B_DONE = 5 + 2 * S;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
+    uint32_t tn = 0;                                  // this thread's trace records
 
     // heavy token tiles first, all sequences of one weight class together
     const int ttile = p.n_ttiles - 1 - (int)(blockIdx.x / p.B);
@@ -208,18 +241,22 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     auto slot_lo = [&](int s) -> int { return s == 0 ? 0 : soff[s - 1] + kFxBN; };
     // tiles of pass q: the sample pass has its own tiles, every other pass all visible ones
     auto pass_tiles = [&](int q) -> int { return (has_sel && q == 0) ? kFxSampleTiles : t_vis; };
+    // The two halves of a pass: half 0 takes its first ceil(nt / 2) tiles, half
+    // 1 the rest; tiles go out alternately (u even: half 0, u odd: half 1).
+    auto tile_of = [&](int nt, int u) -> int { return (u & 1) ? (nt + 1) / 2 + (u >> 1) : (u >> 1); };
+    auto tile_start = [&](int q, int tile) -> int { return (has_sel && q == 0) ? soff[tile] : tile * kFxBN; };
 
     if (threadIdx.x == 0) {
         mbar_init(&bar[0], 1);
-        for (int s = 0; s < kFxStages; ++s) {
-            mbar_init(&bar[1 + s], 1);
-            mbar_init(&bar[5 + s], 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bar[B_KF + s], 1);
+            mbar_init(&bar[B_KE + s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[9 + s], 1);
-            mbar_init(&bar[11 + s], 128);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bar[B_DF + h], 1);
+            mbar_init(&bar[B_DE + h], 128);
         }
-        mbar_init(&bar[13], 1);
+        mbar_init(&bar[B_DONE], 1);
         mbar_fence_init();
         misc[1] = 0;
         // with a selection to make: S, H and one more pass (H or E) always run
@@ -246,23 +283,21 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (q > *last_pass)
                     break;
                 const int nt = pass_tiles(q);
-                for (int i = 0; i < nt; ++i) {
-                    const int s = issued % kFxStages;
-                    if (issued >= kFxStages &&
-                        !mbar_wait(&bar[5 + s], ((issued / kFxStages) - 1) & 1, abort_flag)) {
+                for (int u = 0; u < nt; ++u) {
+                    const int s = issued % S;
+                    if (issued >= S && !mbar_wait(&bar[B_KE + s], ((issued / S) - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const int start = (has_sel && q == 0) ? soff[i] : i * kFxBN;
-                    mbar_arrive_expect_tx(&bar[1 + s], SM::K_BYTES);
-                    tma_load_4d(sK + s * SM::K_BYTES, &tm_k, &bar[1 + s], 0, 0, start, b);
-                    trace_ev(trb, 1, 1, q, i);
+                    mbar_arrive_expect_tx(&bar[B_KF + s], SM::K_BYTES);
+                    tma_load_4d(sK + s * SM::K_BYTES, &tm_k, &bar[B_KF + s], 0, 0, tile_start(q, tile_of(nt, u)), b);
+                    trace_ev(trb, tn, 1, 1, q, u);
                     ++issued;
                 }
             }
             drain_wait(&bar[0], 0);
-            for (int i = max(0, issued - kFxStages); i < issued; ++i)
-                drain_wait(&bar[1 + i % kFxStages], (i / kFxStages) & 1);
+            for (int i = max(0, issued - S); i < issued; ++i)
+                drain_wait(&bar[B_KF + i % S], (i / S) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -270,16 +305,17 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
             bool ok = *last_pass < 0 ? true : mbar_wait(&bar[0], 0, abort_flag);
             int g = 0;
+            int nh[2] = {0, 0};     // tiles given to each half so far
             for (int q = 0; ok && q < kFxMaxPasses; ++q) {
                 if (q >= 3 && !fx_wait_decided(decided, q, abort_flag))
                     break;
                 if (q > *last_pass)
                     break;
                 const int nt = pass_tiles(q);
-                for (int i = 0; i < nt; ++i, ++g) {
-                    const int s = g % kFxStages, db = g & 1;
-                    if (!mbar_wait(&bar[1 + s], (g / kFxStages) & 1, abort_flag) ||
-                        (g >= 2 && !mbar_wait(&bar[11 + db], ((g >> 1) - 1) & 1, abort_flag))) {
+                for (int u = 0; u < nt; ++u, ++g) {
+                    const int s = g % S, hx = u & 1;
+                    if (!mbar_wait(&bar[B_KF + s], (g / S) & 1, abort_flag) ||
+                        (nh[hx] >= 1 && !mbar_wait(&bar[B_DE + hx], (nh[hx] - 1) & 1, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -289,19 +325,25 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         for (int kk = 0; kk < DI / 16; ++kk) {
                             const uint64_t da = fx_desc(aQ + h * SM::Q_BYTES + kk * 32, LY::SBO, LY::SWZ);
                             const uint64_t dbk = fx_desc(aK + s * SM::K_BYTES + kk * 32, LY::SBO, LY::SWZ);
-                            mma_bf16_ss(tmem + (db * HI + h) * kFxBN, da, dbk, idesc, kk > 0 ? 1u : 0u);
+                            mma_bf16_ss(tmem + (hx * HI + h) * kFxBN, da, dbk, idesc, kk > 0 ? 1u : 0u);
                         }
                     }
-                    mma_commit(&bar[9 + db]);
-                    mma_commit(&bar[5 + s]);
-                    trace_ev(trb, 2, 1, q, i);
+                    mma_commit(&bar[B_DF + hx]);
+                    mma_commit(&bar[B_KE + s]);
+                    trace_ev(trb, tn, 2, 1, q, u);
+                    ++nh[hx];
                 }
             }
-            mma_commit(&bar[13]);
-            drain_wait(&bar[13], 0);
+            mma_commit(&bar[B_DONE]);
+            drain_wait(&bar[B_DONE], 0);
         }
     } else if (warp >= 4) {
         // ================================ row epilogue ================================
+        // Two threads per row: half 0 (warps 4-7) and half 1 (warps 8-11)
+        // take the first and the second half of every pass's tiles.  Both keep
+        // the row's window state and take the same decisions from the same
+        // shared data; the counts that differ between halves go through sX.
+        const int hx = warp >= 8 ? 1 : 0;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const int t = t0 + row;
@@ -314,55 +356,63 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             wv[h] = valid ? p.wi[((size_t)b * p.Lq + t) * HI + h] : 0.f;
         int32_t *orow = p.idx + ((size_t)b * p.Lq + (valid ? t : 0)) * K;
         float *srow = p.sel ? p.sel + ((size_t)b * p.Lq + (valid ? t : 0)) * K : nullptr;
-        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        uint32_t *col = sU + row;                         // this row's column of the union area
-        uint32_t *hist = col;                             // [bin / 2] stride kFxBM
-        uint32_t *bkey = col + (kFxBins / 2) * kFxBM;     // [slot] stride kFxBM
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(hx * HI * kFxBN);
+        uint32_t *col = sU + row;                                    // this row's column of the union area
+        uint32_t *hist0 = col;                                       // half 0: [bin / 2] stride kFxBM
+        uint32_t *hist1 = col + (kFxBins / 2) * kFxBM;               // half 1
+        uint32_t *histx = hx ? hist1 : hist0;
+        uint32_t *bkey = col + kFxBins * kFxBM;                      // [slot] stride kFxBM
         uint32_t *bpk = bkey + kFxCap * kFxBM;
-        const uint32_t hist_s = smem_u32(hist), bkey_s = smem_u32(bkey), bpk_s = smem_u32(bpk);
+        const uint32_t hist_s = smem_u32(histx), bkey_s = smem_u32(bkey), bpk_s = smem_u32(bpk);
+        uint32_t *xs = sX + row;                                     // [4][kFxBM]: ns per half, ab per half
 
         int mode = !valid ? FX_NONE : (nv > K ? FX_OPEN : FX_ALL);
         uint32_t lo = 0, top_m1 = 0xFFFFFFFFu, blo = 0, bhi_m1 = 0;
         int sh = 25, need = 0, a_cnt = 0;
-        int ab = 0, ns = 0, pos = 0, taken = 0, nb = 0;
+        int ab = 0, ns = 0, pos = 0, taken = 0, quota = 0, nb = 0, nbin = 0;
         bool ok = true, emitted = false;
-        int g = 0;
+        int nd = 0;              // this half's tiles so far (D barrier phases)
         // index of the E pass as this thread knows it (every epilogue thread
         // takes the same decisions from the same barrier votes)
         int lastp = has_sel ? 0x7fffffff : (t_vis > 0 ? 0 : -1);
+        const bool tracer = threadIdx.x == 128;
         for (int q = 0; q < kFxMaxPasses; ++q) {
             if (q > lastp)
                 break;
             const int ptype = (has_sel && q == 0) ? 0 : (q == lastp ? 2 : 1);   // S / H / E
             const int nt = pass_tiles(q);
-            for (int i = 0; i < nt; ++i, ++g) {
-                const int db = g & 1;
+            const int ta = (nt + 1) / 2;
+            const int nmine = hx ? nt - ta : ta;
+            if (ptype == 2 && mode == FX_ALL && hx == 1)
+                pos = min(nv, ta * kFxBN);          // every visible key of half 0 comes first
+            for (int i = 0; i < nmine; ++i, ++nd) {
                 if (ok)
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bar[9 + db], (g >> 1) & 1, abort_flag));
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_DF + hx], nd & 1, abort_flag));
                 if (!ok)
                     continue;
                 tc_fence_after();
-                const int kbase = ptype == 0 ? soff[i] : i * kFxBN;
+                const int tile = hx ? ta + i : i;
+                const int kbase = tile_start(q, tile);
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float d[HI][32];
+                for (int ch = 0; ch < kFxBN / 16; ++ch) {
+                    float d[HI][16];
 #pragma unroll
                     for (int h = 0; h < HI; ++h)
-                        tmem_ld32(tl + (db * HI + h) * kFxBN + half * 32, d[h]);
+                        fx_ld16(tl + h * kFxBN + ch * 16, d[h]);
                     tmem_ld_wait();
-                    if (half == 1) {
-                        // both halves are in registers: the MMA may refill this buffer
+                    if (ch == kFxBN / 16 - 1) {
+                        // the whole tile is read: the MMA may refill this half's buffer
                         tc_fence_before();
-                        mbar_arrive(&bar[11 + db]);
+                        mbar_arrive(&bar[B_DE + hx]);
                     }
-                    const int j0 = kbase + half * 32;
-                    // the half's 32 scores and order keys first, in straight-line
+                    const int j0 = kbase + ch * 16;
+                    // the chunk's 16 scores and order keys first, in straight-line
                     // code the scheduler can interleave; then the pass's work with
                     // predicated stores (a branch per score serialises the warp)
-                    float sv[32];
-                    uint32_t kv[32];
+                    float sv[16];
+                    uint32_t kv[16];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
+                    for (int c = 0; c < 16; c += 2) {
                         // two keys at a time: sum_h w_h relu(d_h) in packed pairs
                         uint64_t acc = fma_f2(f2(wv[0], wv[0]), f2(fmaxf(d[0][c], 0.f), fmaxf(d[0][c + 1], 0.f)),
                                               f2(0.f, 0.f));
@@ -373,17 +423,17 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         kv[c] = fx_key(sv[c]);
                         kv[c + 1] = fx_key(sv[c + 1]);
                     }
-                    const int nvh = max(0, min(32, nv - j0));     // visible: c < nvh
+                    const int nvh = max(0, min(16, nv - j0));     // visible: c < nvh
                     if (ptype == 0) {
-                        const int clo = max(0, min(32, slot_lo(i) - j0));
+                        const int clo = max(0, min(16, slot_lo(tile) - j0));
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            col[(i * kFxBN + half * 32 + c) * kFxBM] = (c < nvh && c >= clo) ? kv[c] : 0u;
+                        for (int c = 0; c < 16; ++c)
+                            col[(tile * kFxBN + ch * 16 + c) * kFxBM] = (c < nvh && c >= clo) ? kv[c] : 0u;
                         ns += max(0, nvh - clo);
                     } else if (ptype == 1) {
                         if (mode == FX_OPEN) {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
+                            for (int c = 0; c < 16; ++c) {
                                 const uint32_t k = kv[c];
                                 const bool inw = c < nvh && k >= lo;
                                 const bool above = k > top_m1;
@@ -397,7 +447,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     } else if (mode == FX_ALL) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < 16; ++c) {
                             if (c < nvh) {
                                 orow[pos + c] = j0 + c;
                                 if (srow)
@@ -407,10 +457,10 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         pos += nvh;
                     } else if (mode == FX_TIE) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < 16; ++c) {
                             const uint32_t k = kv[c];
                             const bool v = c < nvh;
-                            const bool tie = v && k >= blo && k <= bhi_m1 && taken < need;
+                            const bool tie = v && k >= blo && k <= bhi_m1 && taken < quota;
                             const bool pick = (v && k > bhi_m1) || tie;
                             taken += tie ? 1 : 0;
                             if (pick && pos < K) {
@@ -422,7 +472,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     } else if (mode == FX_BIN) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
+                        for (int c = 0; c < 16; ++c) {
                             const uint32_t k = kv[c];
                             const bool v = c < nvh;
                             const bool pick = v && k > bhi_m1;
@@ -443,12 +493,12 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         }
                     }
                 }
-                if (threadIdx.x == 128)
-                    trace_ev(trb, 3, 1, q, i);
+                if (tracer)
+                    trace_ev(trb, tn, 3, 1, q, tile);
             }
             // ------------------------------ end of pass q ------------------------------
             if (!fx_all(ok)) {
-                if (threadIdx.x == 128) {
+                if (tracer) {
                     *abort_flag = 1;
                     *last_pass = -1;
                     __threadfence_block();
@@ -465,7 +515,10 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // sample key of rank klo, a rank that the row's K-th largest key
                 // reaches with a wide margin; its 96 lower bins span up to the
                 // sample maximum, the 32 upper bins leave room above it
+                xs[hx * kFxBM] = (uint32_t)ns;
+                fx_sync();
                 if (mode == FX_OPEN) {
+                    ns = (int)(xs[0] + xs[kFxBM]);
                     uint32_t kmax = 0;
                     for (int u = 0; u < kFxSampleTiles * kFxBN; ++u)
                         kmax = max(kmax, col[u * kFxBM]);
@@ -494,29 +547,38 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     top_m1 = fx_last(lo, sh, kFxBins);
                 }
-                // the sample area becomes the histogram: clear this row's column
+                // every sample read is done: the area becomes the two histograms
+                fx_sync();
 #pragma unroll 4
                 for (int w = 0; w < kFxBins / 2; ++w)
-                    hist[w * kFxBM] = 0u;
+                    histx[w * kFxBM] = 0u;
             } else {
-                // after H: find the bin holding the K-th largest key
+                // after H: find the bin holding the K-th largest key from both
+                // halves' histograms (u16 pairs: the sums stay below 2^16)
+                xs[(2 + hx) * kFxBM] = (uint32_t)ab;
+                fx_sync();
                 if (mode == FX_OPEN) {
-                    int cum = ab, bstar = -1, cnt = 0;
-                    for (int w = kFxBins / 2 - 1; w >= 0; --w) {
-                        const uint32_t v = hist[w * kFxBM];
-                        hist[w * kFxBM] = 0u;
-                        if (bstar >= 0)
-                            continue;
+                    const int ab0 = (int)xs[2 * kFxBM];
+                    ab = ab0 + (int)xs[3 * kFxBM];
+                    int cum = ab, cum0 = ab0, bstar = -1, cnt = 0, cnt0 = 0;
+                    for (int w = kFxBins / 2 - 1; w >= 0 && bstar < 0; --w) {
+                        const uint32_t v0 = hist0[w * kFxBM];
+                        const uint32_t v = v0 + hist1[w * kFxBM];
                         const int c_hi = (int)(v >> 16), c_lo = (int)(v & 0xFFFFu);
+                        const int c0_hi = (int)(v0 >> 16), c0_lo = (int)(v0 & 0xFFFFu);
                         if (cum + c_hi >= K) {
                             bstar = 2 * w + 1;
                             cnt = c_hi;
+                            cnt0 = c0_hi;
                         } else if (cum + c_hi + c_lo >= K) {
                             cum += c_hi;
+                            cum0 += c0_hi;
                             bstar = 2 * w;
                             cnt = c_lo;
+                            cnt0 = c0_lo;
                         } else {
                             cum += c_hi + c_lo;
+                            cum0 += c0_hi + c0_lo;
                         }
                     }
                     if (ab >= K) {
@@ -535,6 +597,14 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             bhi_m1 = fx_last(bl, sh, 1);
                             a_cnt = cum;
                             need = K - cum;
+                            // half 1 writes after half 0's keys above the bin, and
+                            // keeps its bin entries after half 0's; of a tie, half 0
+                            // takes the first ones
+                            const int q0 = min(need, cnt0);
+                            pos = hx ? cum0 + (sh == 0 ? q0 : 0) : 0;
+                            nb = hx ? cnt0 : 0;
+                            nbin = cnt;
+                            quota = hx ? need - q0 : q0;
                         } else {
                             // too many keys share the bin: narrow to it
                             lo = bl;
@@ -544,12 +614,15 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     top_m1 = fx_last(lo, sh, kFxBins);
                     ab = 0;
                 }
+                // every histogram read is done before either half clears its own
                 const bool all_set = fx_all(mode != FX_OPEN);
+#pragma unroll 4
+                for (int w = 0; w < kFxBins / 2; ++w)
+                    histx[w * kFxBM] = 0u;
                 if (all_set)
                     lastp = q + 1;
-                if (threadIdx.x == 128)
-                    trace_ev(trb, 3, 2, q, all_set ? 1 : 0);
-                if (threadIdx.x == 128) {
+                if (tracer) {
+                    trace_ev(trb, tn, 3, 2, q, all_set ? 1 : 0);
                     if (all_set) {
                         *last_pass = q + 1;       // the next pass emits
                         __threadfence_block();
@@ -562,15 +635,17 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         // ---- boundary bin: take the `need` largest (lower index first), merge ----
-        if (threadIdx.x == 128)
-            trace_ev(trb, 3, 3, lastp, nb);
-        if (emitted && mode == FX_BIN) {
+        // Half 0 merges once both halves' list writes and bin entries are done.
+        fx_sync();
+        if (tracer)
+            trace_ev(trb, tn, 3, 3, lastp, nbin);
+        if (hx == 0 && emitted && mode == FX_BIN) {
             // largest key T in [blo, bhi_m1] with #(key >= T) >= need
             uint32_t lo_b = blo, hi_b = bhi_m1;
             while (lo_b < hi_b) {
                 const uint32_t mid = lo_b + ((hi_b - lo_b) >> 1) + 1u;
                 int cnt = 0;
-                for (int e = 0; e < nb; ++e)
+                for (int e = 0; e < nbin; ++e)
                     cnt += bkey[e * kFxBM] >= mid;
                 if (cnt >= need)
                     lo_b = mid;
@@ -579,7 +654,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             const uint32_t T = lo_b;
             int gt = 0, eq = 0;
-            for (int e = 0; e < nb; ++e) {
+            for (int e = 0; e < nbin; ++e) {
                 const uint32_t k = bkey[e * kFxBM];
                 gt += k > T;
                 eq += k == T;
@@ -588,7 +663,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // chosen entries in reverse list order: the m-th chosen one goes to
             // its above-count + m - 1; the above entries after it move right by m
             int m = need, hi_end = a_cnt, eq_back = 0;
-            for (int e = nb - 1; e >= 0 && m > 0; --e) {
+            for (int e = nbin - 1; e >= 0 && m > 0; --e) {
                 const uint32_t k = bkey[e * kFxBM];
                 bool ch = k > T;
                 if (k == T) {
@@ -631,12 +706,14 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 hi_end = abf;
                 --m;
             }
-            pos = K;
         }
-        if (threadIdx.x == 128)
-            trace_ev(trb, 3, 4, lastp, mode);
-        if ((emitted || lastp < 0) && mode != FX_NONE) {
-            for (int u = pos; u < K; ++u) {
+        if (hx == 0 && valid && mode == FX_OPEN && !emitted && lastp >= 0 && !*abort_flag)
+            set_error(HYB_ERR_DEVICE_BOUNDS);   // the window never settled within the pass limit
+        if (tracer)
+            trace_ev(trb, tn, 3, 4, lastp, mode);
+        // a row with at most K visible keys lists all of them, then -1
+        if (hx == 0 && (emitted || lastp < 0) && mode == FX_ALL) {
+            for (int u = nv; u < K; ++u) {
                 orow[u] = -1;
                 if (srow)
                     srow[u] = -INFINITY;

@@ -308,16 +308,19 @@ hyb_status hyb_set_wait_limit_ns(unsigned long long ns);
 
 /* Debug aid (the pages have no counterpart): a per-role timeline of one CTA.
  * Attaches a caller-owned device buffer of `bytes` bytes (16-byte aligned,
- * >= 32) for the kernels launched afterwards on the current device; NULL
- * detaches.  CTA 0 of a kernel that supports it (the CSA attention kernel)
- * then appends a record per event: the first 8-byte word counts records (set
- * it to 0 before the launch), record r is two words at 8 * (2 + 2r) bytes --
- * the SM clock, then role << 56 | event << 48 | item << 16 | tile.  Records
- * past the buffer are dropped (the count still grows).  Roles and events of
- * the CSA attention kernel: 1 gather (1 K tile issued, 2 V tile issued),
- * 2 MMA (1 QK^T issued, 2 PV issued), 3 softmax warpgroup 0 (1 scores read,
- * 2 P written, 3 item epilogue begun, 4 item done).  Tracing serialises a
- * little work of CTA 0 only; detach it before timing anything. */
+ * >= 96) for the kernels launched afterwards on the current device; NULL
+ * detaches.  One thread per role of CTA 0 of a kernel that supports it (the
+ * CSA attention kernel, the fused indexer) then appends a record per event to
+ * its role's region.  Layout, in 8-byte words: words 0-3 count the records of
+ * roles 0-3 (zero them before the launch); with R = (bytes / 8 - 4) / 8,
+ * role r's records start at word 4 + 2 r R, each two words -- the SM clock,
+ * then role << 56 | event << 48 | item << 16 | tile.  Records past R are
+ * dropped (the count still grows).  Roles and events of the CSA attention
+ * kernel: 1 gather (1 K tile issued, 2 V tile issued, 3 item begun, 4 item's
+ * selection decoded), 2 MMA (1 QK^T issued, 2 PV issued), 3 softmax
+ * warpgroup 0 (1 scores read, 2 P written, 3 item epilogue begun, 4 item
+ * done).  A record costs the tracing thread two stores; detach the buffer
+ * before timing anything. */
 hyb_status hyb_trace_attach(void *buf, size_t bytes);
 
 /* Measurement kernel (the pages have no counterpart): the rate at which the

@@ -42,22 +42,30 @@ def test_csa_attention_timeline(hb):
     rec = hb.trace_records(buf)
     assert rec, "no records"
     items = sorted({r["item"] for r in rec})
+    # each role's region in append order: its clocks never go backwards
+    words = buf.cpu().numpy().view("uint64")
+    cap = (words.size - 4) // 8
     for role in (1, 2, 3):
-        clk = [r["clock"] for r in rec if r["role"] == role]
-        assert clk and np.all(np.diff(clk) >= 0), f"role {role}: clocks out of order"
+        n = int(words[role])
+        assert 0 < n <= cap, f"role {role}: {n} records"
+        base = 4 + 2 * role * cap
+        clk = words[base:base + 2 * n:2].astype(np.int64)
+        tags = words[base + 1:base + 2 * n:2]
+        assert np.all((tags >> 56) == role)
+        assert np.all(np.diff(clk) >= 0), f"role {role}: clocks out of order"
     # every item of CTA 0: K and V gathered, QK^T and PV issued for each of its
     # key tiles (2 selected tiles of 128 + the window); the softmax events come
     # from one thread of the first softmax warpgroup, which (for 32-head groups)
     # takes every other tile
     for it in items:
         ev = {(r["role"], r["event"]) for r in rec if r["item"] == it}
-        assert {(1, 1), (1, 2), (2, 1), (2, 2), (3, 3), (3, 4)} <= ev
+        assert {(1, 1), (1, 2), (1, 3), (1, 4), (2, 1), (2, 2), (3, 3), (3, 4)} <= ev
         n_qk = sum(1 for r in rec if r["item"] == it and r["role"] == 2 and r["event"] == 1)
         n_pv = sum(1 for r in rec if r["item"] == it and r["role"] == 2 and r["event"] == 2)
         n_p = sum(1 for r in rec if r["item"] == it and r["role"] == 3 and r["event"] == 2)
         assert n_qk == n_pv == 3 and 1 <= n_p <= n_qk
     # detached: nothing more is appended
-    n0 = int(buf[0].item())
+    n0 = buf[:4].clone()
     hb.hyb_attn_fwd(p, q, kc[0], kc[1], idx, kv[0], kv[1])
     torch.cuda.synchronize()
-    assert int(buf[0].item()) == n0
+    assert torch.equal(buf[:4], n0)
