@@ -471,7 +471,11 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int j = 0; j < kSpSelBatch; ++j) {
                 const int e = e0 + lane + 32 * j;
                 const int q = slot_of(t0s, e);
-                jv[j] = (e < ne && q < p.topk) ? __ldg(irow + q) : -1;
+                // volatile: issued here, not sunk to the first use an item later
+                int v = -1;
+                if (e < ne && q < p.topk)
+                    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(irow + q));
+                jv[j] = v;
             }
         };
         auto load_first = [&](long long w, int (&jv)[kSpSelBatch]) {
@@ -481,11 +485,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             load_sel(w, s0, (s1 - s0) * 2 * CPT, 0, jv);
         };
         int jnext[kSpSelBatch];
-        if (w0 < p.n_items)
-            load_first(w0, jnext);
-        for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
-            if (!__all_sync(0xffffffffu, ok && !*abort_flag))
-                break;
+        uint32_t nql = 0;                       // items whose Q tile was sent for
+        // An item's prologue: its Q tile, its selection decoded into buffer
+        // nq & 1 (the first batch of entries already in jnext), and the next
+        // item's first batch sent for.  It runs during the previous item's
+        // copies, right after that item's last K tile, so that the gather
+        // does not pause between items.
+        auto prologue = [&](long long w, uint32_t nq) {
             const SparseTok k = sparse_tok(p, w);
             const int qb = nq & 1;
             if (nq >= 2) {
@@ -502,6 +508,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tma_load_2d(sQ + qb * SM::Q_BYTES + cb * NH * 128, &tm_q, &bar[SB_QF + qb], cb * 64,
                                 qrow);
             }
+            nql = nq + 1;
             // decode this warp's part of the item's selection into buffer qb:
             // source row of every slot, or -1 (unselected, invisible, out of
             // range or past topk).  A batch's loads are all in flight
@@ -558,9 +565,18 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             __syncwarp();                       // this warp's lanes read each other's entries
             if (pt == 0)
                 trace_ev(trb, tn, 1, 4, w, 0);
-            // the next item's first batch, in flight during this item's copies
             if (w + wstep < p.n_items)
                 load_first(w + wstep, jnext);
+        };
+        if (w0 < p.n_items) {
+            load_first(w0, jnext);
+            prologue(w0, 0);
+        }
+        for (long long w = w0; w < p.n_items; w += wstep, ++nq) {
+            if (!__all_sync(0xffffffffu, ok && !*abort_flag))
+                break;
+            const SparseTok k = sparse_tok(p, w);
+            const int *sSel = sIdx + (nq & 1) * p.tsel;
             const int nt = k.nct + k.nrt;
             const int tb = tile_lo(nt), ntl = tile_hi(nt) - tb;   // this CTA's tiles
             // source row of copy u of tile i, or -1 (zero-filled)
@@ -572,11 +588,12 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // K of tile i goes out kSpLead tiles ahead of V of the same tile, so
             // that the next scores need not queue behind a V stage that a PV
             // still holds.  A tile's source rows are read into registers
-            // before its copies (each copy is a compiler barrier).
-            int srcv[CPT];
+            // before its copies (each copy is a compiler barrier), for K and
+            // again for V.
             for (int ii = 0; ii < ntl + kSpLead; ++ii) {
                 const int i = tb + ii;
-                int srck[CPT];
+                if (ii == ntl && w + wstep < p.n_items)
+                    prologue(w + wstep, nq + 1);
                 if (ii < ntl) {
                     const uint32_t ks = kc % KS;
                     if (kc >= KS)
@@ -594,10 +611,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         } else {
                             mbar_arrive(&bar[SB_KF + ks]);
                         }
-#pragma unroll
-                        for (int u = 0; u < CPT; ++u)
-                            srck[u] = -1;
                     } else {
+                        int srck[CPT];
 #pragma unroll
                         for (int u = 0; u < CPT; ++u)
                             srck[u] = src_of(i, u);
@@ -614,11 +629,6 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (pt == 0)
                         trace_ev(trb, tn, 1, 1, w, i);
                     ++kc;
-                }
-                if (kSpLead == 0) {
-#pragma unroll
-                    for (int u = 0; u < CPT; ++u)
-                        srcv[u] = srck[u];
                 }
                 if (ii >= kSpLead) {
                     const int iv = i - kSpLead;
@@ -637,6 +647,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             mbar_arrive(&bar[SB_VF + vs]);
                         }
                     } else {
+                        int srcv[CPT];
+#pragma unroll
+                        for (int u = 0; u < CPT; ++u)
+                            srcv[u] = src_of(iv, u);
                         const uint32_t dst = smem_u32(sV + vs * SM::KV_BYTES) + dchunk;
 #pragma unroll
                         for (int u = 0; u < CPT; ++u) {
@@ -651,17 +665,14 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         trace_ev(trb, tn, 1, 2, w, i - kSpLead);
                     ++vc;
                 }
-                if (kSpLead == 1) {
-#pragma unroll
-                    for (int u = 0; u < CPT; ++u)
-                        srcv[u] = srck[u];
-                }
             }
         }
         // unwinding: every copy issued by this thread has landed
         cp_async_wait_group<0>();
         if (pt == 0) {
-            for (uint32_t q = (nq > 2 ? nq - 2 : 0); q < nq; ++q)
+            // the Q tiles of the last two items whose prologue ran (one may be
+            // an item the loop did not reach)
+            for (uint32_t q = (nql > 2 ? nql - 2 : 0); q < nql; ++q)
                 drain_wait(&bar[SB_QF + (q & 1)], (q >> 1) & 1);
         }
     } else if (warp == MMA_WARP) {
