@@ -106,11 +106,16 @@ struct SparseTok {
 
 __device__ __forceinline__ SparseTok sparse_tok(const SparseParams &p, long long w)
 {
+    // items number below 2^31 (checked at launch): 32-bit divisions, which
+    // cost a fraction of 64-bit ones, and none for the common single KV head
+    // or single sequence
     SparseTok k;
-    k.kvh = (int)(w % p.Hkv);
-    const long long bt = w / p.Hkv;
-    k.b = (int)(bt / p.Lq);
-    k.t = (int)(bt % p.Lq);
+    const uint32_t wu = (uint32_t)w, hkv = (uint32_t)p.Hkv, lq = (uint32_t)p.Lq;
+    const uint32_t bt = hkv == 1u ? wu : wu / hkv;
+    k.kvh = (int)(wu - bt * hkv);
+    const uint32_t bb = p.B == 1 ? 0u : bt / lq;
+    k.b = (int)bb;
+    k.t = (int)(bt - bb * lq);
     k.pos = p.q_pos ? p.q_pos[bt] : k.t;
     k.kv0 = p.kv_pos0 ? p.kv_pos0[k.b] : 0;
     k.nct = (p.topk + kSpBN - 1) / kSpBN;

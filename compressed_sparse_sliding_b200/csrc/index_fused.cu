@@ -42,6 +42,8 @@
 // list on its own.  The epilogue decides after each H pass whether another H
 // or the E pass follows; the producer and MMA warps learn it through two
 // shared words and stop after E.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace hyb {
@@ -53,6 +55,7 @@ constexpr int kFxStages = 3;
 constexpr int kFxSampleTiles = 2;
 constexpr int kFxBins = 128;        // histogram bins per row
 constexpr int kFxCap = 64;          // boundary-bin entries kept per row
+constexpr int kFxStage = 64;        // list entries staged per row (E pass) before a flush
 constexpr int kFxMaxPasses = 16;    // S + H rounds + E, far above what the window moves need
 constexpr int kFxMaxNc = 65535;     // index and list position share one 32-bit word
 
@@ -76,7 +79,8 @@ struct FxSmem {
     // [bin / 2][row] (two u16 counters per word), then the boundary buffer:
     // keys [slot][row], then (index | list position << 16) [slot][row]
     static constexpr int SAMPLE_BYTES = kFxSampleTiles * kFxBN * kFxBM * 4;
-    static constexpr int HIST_BYTES = (kFxBins / 2) * kFxBM * 4;
+    static constexpr int HIST_WORDS = kFxBins / 2 + 1;                // + bin 128: keys above the window
+    static constexpr int HIST_BYTES = HIST_WORDS * kFxBM * 4;
     static constexpr int BND_BYTES = 2 * kFxCap * kFxBM * 4;
     static constexpr int U_BYTES = SAMPLE_BYTES > 2 * HIST_BYTES + BND_BYTES ? SAMPLE_BYTES
                                                                              : 2 * HIST_BYTES + BND_BYTES;
@@ -358,10 +362,11 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float *srow = p.sel ? p.sel + ((size_t)b * p.Lq + (valid ? t : 0)) * K : nullptr;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(hx * HI * kFxBN);
         uint32_t *col = sU + row;                                    // this row's column of the union area
+        constexpr int HW = SM::HIST_WORDS;
         uint32_t *hist0 = col;                                       // half 0: [bin / 2] stride kFxBM
-        uint32_t *hist1 = col + (kFxBins / 2) * kFxBM;               // half 1
+        uint32_t *hist1 = col + HW * kFxBM;                          // half 1
         uint32_t *histx = hx ? hist1 : hist0;
-        uint32_t *bkey = col + kFxBins * kFxBM;                      // [slot] stride kFxBM
+        uint32_t *bkey = col + 2 * HW * kFxBM;                       // [slot] stride kFxBM
         uint32_t *bpk = bkey + kFxCap * kFxBM;
         const uint32_t hist_s = smem_u32(histx), bkey_s = smem_u32(bkey), bpk_s = smem_u32(bpk);
         uint32_t *xs = sX + row;                                     // [4][kFxBM]: ns per half, ab per half
@@ -370,6 +375,54 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t lo = 0, top_m1 = 0xFFFFFFFFu, blo = 0, bhi_m1 = 0;
         int sh = 25, need = 0, a_cnt = 0;
         int ab = 0, ns = 0, pos = 0, taken = 0, quota = 0, nb = 0, nbin = 0;
+        // E pass: list entries are staged in this half's histogram area
+        // ([slot][row], kFxStage slots) and flushed by the warp, one row at a
+        // time with consecutive lanes on consecutive entries; fb is the list
+        // position of the row's first staged entry, sc the staged count
+        int fb = 0, sc = 0;
+        // staging rows of 65 words: a lane's own slots and a row's consecutive
+        // slots both fall in distinct banks
+        constexpr int SROW = kFxStage + 1;
+        static_assert(SROW * kFxBM <= SM::HIST_WORDS * kFxBM, "staging fits a histogram area");
+        const uint32_t stage_base = smem_u32(hx ? sU + SM::HIST_WORDS * kFxBM : sU);
+        const uint32_t stage_s = stage_base + (uint32_t)(row * SROW * 4);
+        auto flush = [&]() {
+            __syncwarp();                  // every lane's staged entries are visible
+            // eight rows at a time: their shuffles, then their staged-entry
+            // loads, then their stores, so that the latencies overlap
+#pragma unroll 1
+            for (int r0 = 0; r0 < 32; r0 += 8) {
+                int n[8], base[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    n[u] = __shfl_sync(0xffffffffu, sc, r0 + u);
+                    base[u] = __shfl_sync(0xffffffffu, fb, r0 + u);
+                }
+                uint32_t v0[8], v1[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t a0 = stage_base + (uint32_t)(((quad * 32 + r0 + u) * SROW + lane) * 4);
+                    v0[u] = 0u;
+                    v1[u] = 0u;
+                    if (lane < n[u])
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v0[u]) : "r"(a0));
+                    if (lane + 32 < n[u])
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v1[u]) : "r"(a0 + 128u));
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int rrow = quad * 32 + r0 + u;
+                    int32_t *dst = p.idx + ((size_t)b * p.Lq + (size_t)min(t0 + rrow, p.Lq - 1)) * K + base[u];
+                    if (lane < n[u])
+                        dst[lane] = (int32_t)v0[u];
+                    if (lane + 32 < n[u])
+                        dst[lane + 32] = (int32_t)v1[u];
+                }
+            }
+            fb += sc;
+            sc = 0;
+            __syncwarp();                  // read before any lane stages again
+        };
         bool ok = true, emitted = false;
         int nd = 0;              // this half's tiles so far (D barrier phases)
         // index of the E pass as this thread knows it (every epilogue thread
@@ -385,6 +438,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int nmine = hx ? nt - ta : ta;
             if (ptype == 2 && mode == FX_ALL && hx == 1)
                 pos = min(nv, ta * kFxBN);          // every visible key of half 0 comes first
+            if (ptype == 2)
+                fb = pos;
             for (int i = 0; i < nmine; ++i, ++nd) {
                 if (ok)
                     ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_DF + hx], nd & 1, abort_flag));
@@ -395,6 +450,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int kbase = tile_start(q, tile);
 #pragma unroll 1
                 for (int ch = 0; ch < kFxBN / 16; ++ch) {
+                    if (ptype == 2 && __any_sync(0xffffffffu, sc > kFxStage - 16))
+                        flush();
                     float d[HI][16];
 #pragma unroll
                     for (int h = 0; h < HI; ++h)
@@ -424,74 +481,90 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         kv[c + 1] = fx_key(sv[c + 1]);
                     }
                     const int nvh = max(0, min(16, nv - j0));     // visible: c < nvh
-                    if (ptype == 0) {
-                        const int clo = max(0, min(16, slot_lo(tile) - j0));
+                    // the pass's work, in a variant without per-key visibility
+                    // tests for the (common) chunks that are visible throughout
+                    auto work = [&](auto full_tag) {
+                        constexpr bool FULL = decltype(full_tag)::value;
+                        if (ptype == 0) {
+                            const int clo = max(0, min(16, slot_lo(tile) - j0));
 #pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            col[(tile * kFxBN + ch * 16 + c) * kFxBM] = (c < nvh && c >= clo) ? kv[c] : 0u;
-                        ns += max(0, nvh - clo);
-                    } else if (ptype == 1) {
-                        if (mode == FX_OPEN) {
+                            for (int c = 0; c < 16; ++c)
+                                col[(tile * kFxBN + ch * 16 + c) * kFxBM] = (c < nvh && c >= clo) ? kv[c] : 0u;
+                            ns += max(0, nvh - clo);
+                        } else if (ptype == 1) {
+                            if (mode == FX_OPEN) {
+                                // bin 128 collects the keys above the window (when the
+                                // window reaches the top key, none are)
 #pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const uint32_t k = kv[c];
-                                const bool inw = c < nvh && k >= lo;
-                                const bool above = k > top_m1;
-                                ab += (inw && above) ? 1 : 0;
-                                const uint32_t bin = (k - lo) >> sh;
-                                if (inw && !above)
-                                    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(hist_s + (bin >> 1) * (kFxBM * 4)),
-                                                 "r"(1u << ((bin & 1u) * 16u))
-                                                 : "memory");
+                                for (int c = 0; c < 16; ++c) {
+                                    const uint32_t k = kv[c];
+                                    const uint32_t bin = min((k - lo) >> sh, (uint32_t)kFxBins);
+                                    if ((FULL || c < nvh) && k >= lo)
+                                        asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(hist_s + (bin >> 1) * (kFxBM * 4)),
+                                                     "r"(1u << ((bin & 1u) * 16u))
+                                                     : "memory");
+                                }
                             }
-                        }
-                    } else if (mode == FX_ALL) {
+                        } else if (mode != FX_NONE) {
+                            // E: this chunk's list entries as a mask, in index order
+                            uint32_t pm = 0;
+                            if (mode == FX_ALL) {
+                                pm = FULL ? 0xFFFFu : ((1u << nvh) - 1u);
+                            } else if (mode == FX_TIE) {
+                                uint32_t tm = 0;
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            if (c < nvh) {
-                                orow[pos + c] = j0 + c;
-                                if (srow)
-                                    srow[pos + c] = sv[c];
+                                for (int c = 0; c < 16; ++c) {
+                                    const uint32_t k = kv[c];
+                                    const bool v = FULL || c < nvh;
+                                    pm |= (uint32_t)(v && k > bhi_m1) << c;
+                                    tm |= (uint32_t)(v && k >= blo && k <= bhi_m1) << c;
+                                }
+                                // the first ties in index order, up to this half's quota
+                                while (tm != 0u && taken < quota) {
+                                    const uint32_t lowb = tm & (0u - tm);
+                                    pm |= lowb;
+                                    tm ^= lowb;
+                                    ++taken;
+                                }
+                            } else {   // FX_BIN
+#pragma unroll
+                                for (int c = 0; c < 16; ++c) {
+                                    const uint32_t k = kv[c];
+                                    const bool v = FULL || c < nvh;
+                                    const bool keep = v && k >= blo && k <= bhi_m1 && nb < kFxCap;
+                                    if (keep) {
+                                        // with the list position it would take: the row's
+                                        // entries so far and this chunk's before it
+                                        asm volatile("st.shared.u32 [%0], %1;" ::"r"(bkey_s + nb * (kFxBM * 4)), "r"(k) : "memory");
+                                        asm volatile("st.shared.u32 [%0], %1;" ::"r"(bpk_s + nb * (kFxBM * 4)),
+                                                     "r"((uint32_t)(j0 + c) | ((uint32_t)(pos + __popc(pm)) << 16))
+                                                     : "memory");
+                                    }
+                                    nb += keep ? 1 : 0;
+                                    pm |= (uint32_t)(v && k > bhi_m1) << c;
+                                }
                             }
-                        }
-                        pos += nvh;
-                    } else if (mode == FX_TIE) {
+                            if (srow) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const uint32_t k = kv[c];
-                            const bool v = c < nvh;
-                            const bool tie = v && k >= blo && k <= bhi_m1 && taken < quota;
-                            const bool pick = (v && k > bhi_m1) || tie;
-                            taken += tie ? 1 : 0;
-                            if (pick && pos < K) {
-                                orow[pos] = j0 + c;
-                                if (srow)
-                                    srow[pos] = sv[c];
+                                for (int c = 0; c < 16; ++c)
+                                    if ((pm >> c) & 1u)
+                                        srow[pos + __popc(pm & ((1u << c) - 1u))] = sv[c];
                             }
-                            pos += pick ? 1 : 0;
-                        }
-                    } else if (mode == FX_BIN) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            const uint32_t k = kv[c];
-                            const bool v = c < nvh;
-                            const bool pick = v && k > bhi_m1;
-                            const bool keep = v && k >= blo && k <= bhi_m1 && nb < kFxCap;
-                            if (keep) {
-                                asm volatile("st.shared.u32 [%0], %1;" ::"r"(bkey_s + nb * (kFxBM * 4)), "r"(k) : "memory");
-                                asm volatile("st.shared.u32 [%0], %1;" ::"r"(bpk_s + nb * (kFxBM * 4)),
-                                             "r"((uint32_t)(j0 + c) | ((uint32_t)pos << 16))
+                            pos += __popc(pm);
+                            uint32_t m = pm;
+                            while (m != 0u) {
+                                const int c = __ffs(m) - 1;
+                                m &= m - 1u;
+                                asm volatile("st.shared.u32 [%0], %1;" ::"r"(stage_s + sc * 4), "r"((uint32_t)(j0 + c))
                                              : "memory");
+                                ++sc;
                             }
-                            nb += keep ? 1 : 0;
-                            if (pick && pos < K) {
-                                orow[pos] = j0 + c;
-                                if (srow)
-                                    srow[pos] = sv[c];
-                            }
-                            pos += pick ? 1 : 0;
                         }
-                    }
+                    };
+                    if (nvh == 16)
+                        work(std::true_type{});
+                    else
+                        work(std::false_type{});
                 }
                 if (tracer)
                     trace_ev(trb, tn, 3, 1, q, tile);
@@ -507,6 +580,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 break;
             }
             if (ptype == 2) {
+                flush();
                 emitted = true;
                 break;
             }
@@ -517,7 +591,8 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // sample maximum, the 32 upper bins leave room above it
                 xs[hx * kFxBM] = (uint32_t)ns;
                 fx_sync();
-                if (mode == FX_OPEN) {
+                // half 0 derives the window, half 1 takes it from sX
+                if (mode == FX_OPEN && hx == 0) {
                     ns = (int)(xs[0] + xs[kFxBM]);
                     uint32_t kmax = 0;
                     for (int u = 0; u < kFxSampleTiles * kFxBN; ++u)
@@ -545,21 +620,26 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         lo = 0;
                         sh = 25;
                     }
-                    top_m1 = fx_last(lo, sh, kFxBins);
+                    xs[2 * kFxBM] = lo;
+                    xs[3 * kFxBM] = (uint32_t)sh;
                 }
                 // every sample read is done: the area becomes the two histograms
                 fx_sync();
+                if (mode == FX_OPEN) {
+                    lo = xs[2 * kFxBM];
+                    sh = (int)xs[3 * kFxBM];
+                    top_m1 = fx_last(lo, sh, kFxBins);
+                }
 #pragma unroll 4
-                for (int w = 0; w < kFxBins / 2; ++w)
+                for (int w = 0; w < HW; ++w)
                     histx[w * kFxBM] = 0u;
             } else {
                 // after H: find the bin holding the K-th largest key from both
                 // halves' histograms (u16 pairs: the sums stay below 2^16)
-                xs[(2 + hx) * kFxBM] = (uint32_t)ab;
                 fx_sync();
                 if (mode == FX_OPEN) {
-                    const int ab0 = (int)xs[2 * kFxBM];
-                    ab = ab0 + (int)xs[3 * kFxBM];
+                    const int ab0 = (int)(hist0[(HW - 1) * kFxBM] & 0xFFFFu);
+                    ab = ab0 + (int)(hist1[(HW - 1) * kFxBM] & 0xFFFFu);
                     int cum = ab, cum0 = ab0, bstar = -1, cnt = 0, cnt0 = 0;
                     for (int w = kFxBins / 2 - 1; w >= 0 && bstar < 0; --w) {
                         const uint32_t v0 = hist0[w * kFxBM];
@@ -617,7 +697,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // every histogram read is done before either half clears its own
                 const bool all_set = fx_all(mode != FX_OPEN);
 #pragma unroll 4
-                for (int w = 0; w < kFxBins / 2; ++w)
+                for (int w = 0; w < HW; ++w)
                     histx[w * kFxBM] = 0u;
                 if (all_set)
                     lastp = q + 1;
@@ -635,76 +715,116 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         // ---- boundary bin: take the `need` largest (lower index first), merge ----
-        // Half 0 merges once both halves' list writes and bin entries are done.
+        // Once both halves' lists and bin entries are written: half 0 picks the
+        // row's threshold T inside the bin and compacts the chosen entries
+        // (index order, with their list positions) to the front of the bin
+        // buffer; then one warp per row rewrites the row's list with the
+        // chosen entries in place, lanes on consecutive positions.
         fx_sync();
         if (tracer)
             trace_ev(trb, tn, 3, 3, lastp, nbin);
-        if (hx == 0 && emitted && mode == FX_BIN) {
-            // largest key T in [blo, bhi_m1] with #(key >= T) >= need
-            uint32_t lo_b = blo, hi_b = bhi_m1;
-            while (lo_b < hi_b) {
-                const uint32_t mid = lo_b + ((hi_b - lo_b) >> 1) + 1u;
-                int cnt = 0;
+        const bool merging = emitted && mode == FX_BIN;
+        if (hx == 0) {
+            if (merging) {
+                // largest key T in [blo, bhi_m1] with #(key >= T) >= need
+                uint32_t lo_b = blo, hi_b = bhi_m1;
+                while (lo_b < hi_b) {
+                    const uint32_t mid = lo_b + ((hi_b - lo_b) >> 1) + 1u;
+                    int cnt = 0;
+                    for (int e = 0; e < nbin; ++e)
+                        cnt += bkey[e * kFxBM] >= mid;
+                    if (cnt >= need)
+                        lo_b = mid;
+                    else
+                        hi_b = mid - 1u;
+                }
+                const uint32_t T = lo_b;
+                int gt = 0;
                 for (int e = 0; e < nbin; ++e)
-                    cnt += bkey[e * kFxBM] >= mid;
-                if (cnt >= need)
-                    lo_b = mid;
-                else
-                    hi_b = mid - 1u;
-            }
-            const uint32_t T = lo_b;
-            int gt = 0, eq = 0;
-            for (int e = 0; e < nbin; ++e) {
-                const uint32_t k = bkey[e * kFxBM];
-                gt += k > T;
-                eq += k == T;
-            }
-            const int take_eq = need - gt;
-            // chosen entries in reverse list order: the m-th chosen one goes to
-            // its above-count + m - 1; the above entries after it move right by m
-            int m = need, hi_end = a_cnt, eq_back = 0;
-            for (int e = nbin - 1; e >= 0 && m > 0; --e) {
-                const uint32_t k = bkey[e * kFxBM];
-                bool ch = k > T;
-                if (k == T) {
-                    ch = (eq - 1 - eq_back) < take_eq;
-                    ++eq_back;
-                }
-                if (!ch)
-                    continue;
-                const uint32_t pk = bpk[e * kFxBM];
-                const int j = (int)(pk & 0xFFFFu), abf = (int)(pk >> 16);
-                if (abf > hi_end || abf + m > K) {   // cannot happen: E recomputes H's scores exactly
-                    set_error(HYB_ERR_DEVICE_BOUNDS);
-                    break;
-                }
-                int qq = hi_end - 1;
-                for (; qq - 7 >= abf; qq -= 8) {
-                    int32_t v[8];
-                    float sv[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        v[u] = orow[qq - u];
-                        if (srow)
-                            sv[u] = srow[qq - u];
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        orow[qq - u + m] = v[u];
-                        if (srow)
-                            srow[qq - u + m] = sv[u];
+                    gt += bkey[e * kFxBM] > T;
+                int eq_left = need - gt;          // entries equal to T taken, lower index first
+                int w = 0;
+                for (int e = 0; e < nbin; ++e) {
+                    const uint32_t k = bkey[e * kFxBM];
+                    const bool ch = k > T || (k == T && eq_left > 0);
+                    eq_left -= (k == T && ch) ? 1 : 0;
+                    if (ch) {
+                        bpk[w * kFxBM] = bpk[e * kFxBM];
+                        bkey[w * kFxBM] = k;
+                        ++w;
                     }
                 }
-                for (; qq >= abf; --qq) {
-                    orow[qq + m] = orow[qq];
-                    if (srow)
-                        srow[qq + m] = srow[qq];
+            }
+            // rows to merge: above count and chosen count
+            sX[row] = merging ? (uint32_t)a_cnt : 0xFFFFFFFFu;
+            sX[kFxBM + row] = merging ? (uint32_t)need : 0u;
+        }
+        fx_sync();
+        {
+            // One warp per row (epilogue warp ew takes rows ew, ew + 8, ...):
+            // output position i holds the chosen entry m when i = f_m (its list
+            // position plus m), else the above entry i - #(f_m < i).  Every
+            // lane gathers its outputs of a block of 512 positions into
+            // registers before any lane writes; blocks go from the top, so no
+            // write lands on an entry a later block still reads.
+            const int et = (hx * 4 + quad) * 32 + lane;
+            const int ew = et >> 5;                        // epilogue warp 0..7
+            for (int list = 0; list < (p.sel ? 2 : 1); ++list) {
+#pragma unroll 1
+                for (int r = ew; r < kFxBM; r += 8) {
+                    const uint32_t ac = sX[r];
+                    if (ac == 0xFFFFFFFFu)
+                        continue;
+                    const int nch = (int)sX[kFxBM + r];
+                    // the row's chosen entries in registers: lane l holds numbers
+                    // l and l + 32 (f = list position + number; f is strictly
+                    // increasing, absent entries have f = ~0)
+                    uint32_t f_lo = 0xFFFFFFFFu, f_hi = 0xFFFFFFFFu, j_lo = 0u, j_hi = 0u;
+                    auto chosen_of = [&](int m, uint32_t &f, uint32_t &jv) {
+                        const uint32_t pk = sU[(2 * HW + kFxCap + m) * kFxBM + r];     // bpk[m] of row r
+                        f = (pk >> 16) + (uint32_t)m;
+                        jv = list == 0 ? (pk & 0xFFFFu) : __float_as_uint(fx_score(sU[(2 * HW + m) * kFxBM + r]));
+                    };
+                    if (lane < nch)
+                        chosen_of(lane, f_lo, j_lo);
+                    if (lane + 32 < nch)
+                        chosen_of(lane + 32, f_hi, j_hi);
+                    const size_t grow = (size_t)b * p.Lq + (size_t)(t0 + r);
+                    uint32_t *L = list == 0 ? reinterpret_cast<uint32_t *>(p.idx + grow * K)
+                                            : reinterpret_cast<uint32_t *>(p.sel + grow * K);
+#pragma unroll 1
+                    for (int i0 = (K - 1) / 512 * 512; i0 >= 0; i0 -= 512) {
+                        // chosen entries placed before position i0
+                        int c = __popc(__ballot_sync(0xffffffffu, f_lo < (uint32_t)i0)) +
+                                __popc(__ballot_sync(0xffffffffu, f_hi < (uint32_t)i0));
+                        uint32_t v[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            // the window of 32 positions from w0: which hold chosen entries
+                            const uint32_t w0 = (uint32_t)(i0 + 32 * j);
+                            const uint32_t bl = f_lo - w0 < 32u ? 1u << (f_lo - w0) : 0u;
+                            const uint32_t bh = f_hi - w0 < 32u ? 1u << (f_hi - w0) : 0u;
+                            const uint32_t mask = __reduce_or_sync(0xffffffffu, bl | bh);
+                            const int i = (int)w0 + lane;
+                            const int before = c + __popc(mask & ((1u << lane) - 1u));
+                            const uint32_t ca = __shfl_sync(0xffffffffu, j_lo, before & 31);
+                            const uint32_t cb = __shfl_sync(0xffffffffu, j_hi, before & 31);
+                            if ((mask >> lane) & 1u)
+                                v[j] = before < 32 ? ca : cb;
+                            else
+                                v[j] = i < K ? L[i - before] : 0u;
+                            c += __popc(mask);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int i = i0 + lane + 32 * j;
+                            if (i < K)
+                                L[i] = v[j];
+                        }
+                        __syncwarp();
+                    }
                 }
-                orow[abf + m - 1] = j;
-                if (srow)
-                    srow[abf + m - 1] = fx_score(k);
-                hi_end = abf;
-                --m;
             }
         }
         if (hx == 0 && valid && mode == FX_OPEN && !emitted && lastp >= 0 && !*abort_flag)
