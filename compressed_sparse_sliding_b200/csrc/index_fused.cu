@@ -31,9 +31,9 @@
 //                  taken during E itself.
 // Order keys are the fp32 scores mapped to uint32 so that larger scores give
 // larger keys (-0.0 folded onto +0.0), as in the two-kernel path.
-// Roles (384 threads): warp 0 TMA producer, warp 1 TMEM + MMA, warps 2-3 idle,
-// and two threads per row for the epilogue: warps 4-7 (TMEM lane quadrants
-// 0-3) take the first half of every pass's key tiles, warps 8-11 the second
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM + MMA, and two
+// threads per row for the epilogue: warps 2-5 (TMEM lane quadrants 2, 3, 0,
+// 1) take the first half of every pass's key tiles, warps 6-9 the second
 // half, each half with its own TMEM buffer, so that two warps per SM
 // sub-partition hide each other's latencies.  The halves histogram into
 // separate arrays and take the row's decisions together from both; for E,
@@ -48,7 +48,7 @@
 
 namespace hyb {
 
-constexpr int kFxThreads = 384;
+constexpr int kFxThreads = 320;
 constexpr int kFxBM = 128;          // query rows per CTA
 constexpr int kFxBN = 64;           // keys per tile
 constexpr int kFxStages = 3;
@@ -341,13 +341,13 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_commit(&bar[B_DONE]);
             drain_wait(&bar[B_DONE], 0);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         // ================================ row epilogue ================================
-        // Two threads per row: half 0 (warps 4-7) and half 1 (warps 8-11)
+        // Two threads per row: half 0 (warps 2-5) and half 1 (warps 6-9)
         // take the first and the second half of every pass's tiles.  Both keep
         // the row's window state and take the same decisions from the same
         // shared data; the counts that differ between halves go through sX.
-        const int hx = warp >= 8 ? 1 : 0;
+        const int hx = warp >= 6 ? 1 : 0;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const int t = t0 + row;
@@ -428,7 +428,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // index of the E pass as this thread knows it (every epilogue thread
         // takes the same decisions from the same barrier votes)
         int lastp = has_sel ? 0x7fffffff : (t_vis > 0 ? 0 : -1);
-        const bool tracer = threadIdx.x == 128;
+        const bool tracer = threadIdx.x == 64;
         for (int q = 0; q < kFxMaxPasses; ++q) {
             if (q > lastp)
                 break;
@@ -767,7 +767,7 @@ index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // lane gathers its outputs of a block of 512 positions into
             // registers before any lane writes; blocks go from the top, so no
             // write lands on an entry a later block still reads.
-            const int et = (hx * 4 + quad) * 32 + lane;
+            const int et = (warp - 2) * 32 + lane;
             const int ew = et >> 5;                        // epilogue warp 0..7
             for (int list = 0; list < (p.sel ? 2 : 1); ++list) {
 #pragma unroll 1
