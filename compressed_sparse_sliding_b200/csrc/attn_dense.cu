@@ -172,6 +172,8 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     volatile int *abort_flag = misc + 1;
+    unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
+    uint32_t tn = 0;                                  // this thread's trace records
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -237,6 +239,7 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_4d(sK + ks * SM::KV_BYTES + cb * kDnBN * 128, comp ? &tm_kc : &tm_kr,
                                     &bar[DB_KF + ks], cb * 64, kvh, row0, it.b);
+                    trace_ev(trb, tn, 1, 1, w, i);
                     ++kc;
                     const uint32_t vs = vc % kDnVStages;
                     if (vc >= kDnVStages &&
@@ -248,6 +251,7 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_4d(sV + vs * SM::KV_BYTES + cb * kDnBN * 128, comp ? &tm_vc : &tm_vr,
                                     &bar[DB_VF + vs], cb * 64, kvh, row0, it.b);
+                    trace_ev(trb, tn, 1, 2, w, i);
                     ++vc;
                 }
             }
@@ -323,6 +327,7 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                             (first_pv[x] && kk == 0) ? 0u : 1u);
                             }
                             first_pv[x] = false;
+                            trace_ev(trb, tn, 2, 2 + 2 * x, w, i - 1);
                         }
                         if (act_cur[x]) {
 #pragma unroll
@@ -335,6 +340,7 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 mma_bf16_ss(tmem + TM_S[x], da, db, idesc_qk, kk > 0 ? 1u : 0u);
                             }
                             mma_commit(&bar[DB_SF + x]);
+                            trace_ev(trb, tn, 2, 1 + 2 * x, w, i);
                         }
                     }
                     if (!ok)
@@ -379,6 +385,9 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t tS = tl + TM_S[x];
         const uint32_t tO = tl + TM_O[x];
+        // the first thread of each softmax warpgroup traces: role 3 (tile A), role 0 (tile B)
+        const bool tracer = (threadIdx.x & 127) == 0;
+        const int trole = x == 0 ? 3 : 0;
         uint32_t scnt = 0, ocnt = 0;
         bool ok = true;
         for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
@@ -420,6 +429,8 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c = 0; c < kDnBN / 32; ++c)
                     tmem_ld32(tS + c * 32, *reinterpret_cast<float(*)[32]>(&sv[c * 32]));
                 tmem_ld_wait();
+                if (tracer)
+                    trace_ev(trb, tn, trole, 1, w, i);
                 if (!full) {
 #pragma unroll
                     for (int c = 0; c < kDnBN; ++c)
@@ -495,11 +506,15 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bar[DB_PF + x]);
+                if (tracer)
+                    trace_ev(trb, tn, trole, 2, w, i);
                 any = true;
             }
             if (!ok)
                 break;
             // epilogue
+            if (tracer)
+                trace_ev(trb, tn, trole, 3, w, nt);
             if (any) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&bar[DB_OF + x], ocnt & 1, abort_flag))) {
                     ok = false;
@@ -539,6 +554,8 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
             tc_fence_before();
             mbar_arrive(&bar[DB_OE + x]);
+            if (tracer)
+                trace_ev(trb, tn, trole, 4, w, nt);
         }
     }
 

@@ -310,7 +310,7 @@ hyb_status hyb_set_wait_limit_ns(unsigned long long ns);
  * Attaches a caller-owned device buffer of `bytes` bytes (16-byte aligned,
  * >= 96) for the kernels launched afterwards on the current device; NULL
  * detaches.  One thread per role of CTA 0 of a kernel that supports it (the
- * CSA attention kernel, the fused indexer) then appends a record per event to
+ * CSA and HCA attention kernels, the fused indexer) then appends a record per event to
  * its role's region.  Layout, in 8-byte words: words 0-3 count the records of
  * roles 0-3 (zero them before the launch); with R = (bytes / 8 - 4) / 8,
  * role r's records start at word 4 + 2 r R, each two words -- the SM clock,
@@ -319,8 +319,11 @@ hyb_status hyb_set_wait_limit_ns(unsigned long long ns);
  * kernel: 1 gather (1 K tile issued, 2 V tile issued, 3 item begun, 4 item's
  * selection decoded), 2 MMA (1 QK^T issued, 2 PV issued), 3 softmax
  * warpgroup 0 (1 scores read, 2 P written, 3 item epilogue begun, 4 item
- * done).  A record costs the tracing thread two stores; detach the buffer
- * before timing anything. */
+ * done).  The HCA attention kernel: 1 K / V loads (1 K tile, 2 V tile), 2 MMA
+ * (1 QK^T of tile A, 2 PV of tile A, 3 QK^T of tile B, 4 PV of tile B), 3 and
+ * 0 the softmax of query tiles A and B (1 scores read, 2 P written, 3 item
+ * epilogue begun, 4 item done).  A record costs the tracing thread two stores;
+ * detach the buffer before timing anything. */
 hyb_status hyb_trace_attach(void *buf, size_t bytes);
 
 /* Measurement kernel (the pages have no counterpart): the rate at which the
