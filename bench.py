@@ -794,6 +794,13 @@ def run_micro(args):
     for stages in range(2, 7):
         ms = best_ms(lambda: hb.hyb_probe_l2_gather(table, rows, stages, sink, stream), 10)
         gather[str(stages)] = round(sms * rows * 256 / (ms / 1e3) / 1e9, 1)
+    # the same rows by the tensor memory accelerator's four-row gather
+    sink_t = torch.zeros(257, dtype=torch.int32, device=dev)
+    gather_tma = {}
+    for stages in range(2, 7):
+        ms = best_ms(lambda: hb.hyb_probe_l2_gather_tma(table, rows, stages, sink_t, stream), 10)
+        gather_tma[str(stages)] = round(sms * rows * 256 / (ms / 1e3) / 1e9, 1)
+    misplaced = int(sink_t[256].item())
     n = 8192
     x = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
     y = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
@@ -804,10 +811,13 @@ def run_micro(args):
             "l2_gather_GBps_by_stages": gather, "l2_gather_GBps": max(gather.values()),
             "l2_gather_B_per_clk_per_sm": round(max(gather.values()) * 1e9 / sms /
                                                (((clocks or {}).get("sm_mhz") or 1965.0) * 1e6), 1),
+            "l2_gather_tma_GBps_by_stages": gather_tma, "l2_gather_tma_GBps": max(gather_tma.values()),
+            "l2_gather_tma_misplaced_chunks": misplaced,
             "bf16_gemm_TFLOPs": round(gemm, 1), "sms": sms,
             "how": "HBM: 1 GiB bf16 copy (read + write bytes); L2 gather: random 256-byte rows of a 4 MB "
                    "table into 32 KB shared-memory stages with 16-byte cp.async, one CTA per SM, "
-                   f"{rows} rows per SM (hyb_probe_l2_gather); GEMM: torch.matmul bf16 {n}^3; "
+                   f"{rows} rows per SM (hyb_probe_l2_gather), and with tile::gather4 TMA copies, one "
+                   f"warp per SM (hyb_probe_l2_gather_tma); GEMM: torch.matmul bf16 {n}^3; "
                    "best of 10 with CUDA events",
             "clocks": clocks}
 

@@ -106,6 +106,8 @@ try:
     _lib.hyb_trace_attach.restype = _I
     _lib.hyb_probe_l2_gather.argtypes = [_P, ctypes.c_longlong, ctypes.c_longlong, _I, _P, _P]
     _lib.hyb_probe_l2_gather.restype = _I
+    _lib.hyb_probe_l2_gather_tma.argtypes = [_P, ctypes.c_longlong, ctypes.c_longlong, _I, _P, _P]
+    _lib.hyb_probe_l2_gather_tma.restype = _I
 except AttributeError as exc:   # a library built from older sources
     raise ImportError(f"{LIB_PATH} lacks an entry point ({exc}); rebuild: {_BUILD_HINT}") from exc
 
@@ -166,15 +168,22 @@ def hyb_hca_compress(x: torch.Tensor, w: torch.Tensor, m: int, out: Optional[tor
 
 
 def hyb_csa_index_topk(p: HybProblem, qi, wi, kic, idx=None, sel_scores=None, ws=None,
-                       stream=None):
-    """Top-K entry indices [B, Lq, topk] int32 (ascending, -1 padded)."""
+                       stream=None, ws_bytes: Optional[int] = None):
+    """Top-K entry indices [B, Lq, topk] int32 (ascending, -1 padded).
+    ws_bytes: the workspace bytes to declare (default: all of ws, which is
+    allocated at hyb_workspace_size(p) when absent or short); 0 passes none,
+    which runs the one-kernel path on the shapes it takes."""
     if idx is None:
         idx = torch.empty((p.B, p.Lq, p.topk), dtype=torch.int32, device=qi.device)
-    need = hyb_workspace_size(p)
-    if ws is None or ws.numel() < need:
-        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=qi.device)
+    if ws_bytes == 0:
+        ws = None
+    else:
+        need = hyb_workspace_size(p)
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=qi.device)
+        ws_bytes = ws.numel() if ws_bytes is None else min(int(ws_bytes), ws.numel())
     st = _lib.hyb_csa_index_topk(ctypes.byref(p), _ptr(qi), _ptr(wi), _ptr(kic), _ptr(idx),
-                                 _ptr(sel_scores), _ptr(ws), ws.numel(), _stream(stream))
+                                 _ptr(sel_scores), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "hyb_csa_index_topk")
     return idx
 
@@ -419,6 +428,18 @@ def hyb_probe_l2_gather(table: torch.Tensor, rows_per_sm: int, stages: int, sink
                                   int(stages), _ptr(sink), _stream(stream))
     if st != HYB_OK:
         raise HybError(st, "hyb_probe_l2_gather")
+
+
+def hyb_probe_l2_gather_tma(table: torch.Tensor, rows_per_sm: int, stages: int, sink: torch.Tensor,
+                            stream=None) -> None:
+    """The same probe with tile::gather4 copies; sink holds 257 words, sink[256]
+    counting misplaced 16-byte chunks (see the C header)."""
+    if sink.numel() * sink.element_size() < 257 * 4:
+        raise ValueError("sink must hold 257 uint32 words")
+    st = _lib.hyb_probe_l2_gather_tma(_ptr(table), table.numel() * table.element_size(), int(rows_per_sm),
+                                      int(stages), _ptr(sink), _stream(stream))
+    if st != HYB_OK:
+        raise HybError(st, "hyb_probe_l2_gather_tma")
 
 
 def hyb_set_wait_limit_ns(ns: int) -> None:

@@ -139,11 +139,28 @@ static cudaError_t index_topk_into(const hyb_problem *p, const void *qi, const f
                              sel_scores, stream);
 }
 
-// Stage 2 in one kernel (scores recomputed on chip, no score rows stored) for
-// the shapes it takes; the two-kernel path above for the others.
-static bool index_topk_fused_path(const hyb_problem *p)
+// Bytes of the two-kernel path's score rows (B * Lq * Nc fp32), 256-byte rounded.
+static size_t index_scores_bytes(const hyb_problem *p)
 {
-    return index_fused_supported(p->Lq, p->Hi, p->di, p->Nc, p->topk);
+    const size_t scores = (size_t)p->B * p->Lq * p->Nc * sizeof(float);
+    return (scores + 255) & ~(size_t)255;
+}
+
+// Stage 2 in one kernel (scores recomputed on chip, no score rows stored), or
+// the two-kernel path above.  Where both take the shape, the two kernels
+// finish first as long as the score rows stay small (measured on one B200 at
+// L = 1024 to 16384 with up to 256 MB of rows: 0.034 against 0.089 ms at
+// L = 1024, 0.28 against 0.44 ms at L = 16384; at L = 32768, 1 GB of rows,
+// the two are within 5% and the one kernel stores nothing), so they run when
+// the rows take at most kIndexScoresMaxBytes and `ws_avail` bytes hold them.
+constexpr size_t kIndexScoresMaxBytes = (size_t)256 << 20;
+
+static bool index_topk_fused_path(const hyb_problem *p, size_t ws_avail)
+{
+    if (!index_fused_supported(p->Lq, p->Hi, p->di, p->Nc, p->topk))
+        return false;
+    const size_t need = index_scores_bytes(p);
+    return need > kIndexScoresMaxBytes || ws_avail < need;
 }
 
 static float softmax_scale(const hyb_problem *p)
@@ -231,10 +248,12 @@ extern "C" {
 
 size_t hyb_workspace_size(const hyb_problem *p)
 {
-    if (!p || p->topk <= 0 || index_topk_fused_path(p))
+    if (!p || p->topk <= 0 || p->B <= 0 || p->Lq <= 0 || p->Nc <= 0)
         return 0;
-    size_t scores = (size_t)p->B * p->Lq * p->Nc * sizeof(float);
-    return (scores + 255) & ~(size_t)255;
+    // an unlimited workspace picks the path the shape runs fastest on
+    if (index_topk_fused_path(p, ~(size_t)0))
+        return 0;
+    return index_scores_bytes(p);
 }
 
 hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m, const float *w,
@@ -260,11 +279,11 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
         return st;
     if (!qi || !wi || !kic || !idx || !aligned16(qi) || !aligned16(kic))
         return HYB_ERR_INVALID_ARG;
-    if (index_topk_fused_path(p))
+    const size_t avail = ws && !(reinterpret_cast<uintptr_t>(ws) & 255u) ? ws_bytes : 0;
+    if (index_topk_fused_path(p, avail))
         return cuda_status(launch_index_topk_fused(qi, wi, kic, idx, sel_scores, p->B, p->Lq, p->Hi, p->di,
                                                    p->Nc, p->m, p->W, p->topk, p->q_pos, stream));
-    const size_t need = hyb_workspace_size(p);
-    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    if (avail < index_scores_bytes(p))
         return HYB_ERR_WORKSPACE;
     return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, static_cast<float *>(ws),
                                        stream));
@@ -462,7 +481,7 @@ hyb_status hyb_csa_index_topk_fp4(const hyb_problem *p, const void *qi, const fl
                                           num_sms_current());
     if (e != cudaSuccess)
         return cuda_status(e);
-    if (index_topk_fused_path(p))
+    if (index_topk_fused_path(p, hyb_workspace_size(p)))
         return cuda_status(launch_index_topk_fused(qi, wi, kic, idx, sel_scores, p->B, p->Lq, p->Hi, p->di,
                                                    p->Nc, p->m, p->W, p->topk, p->q_pos, stream));
     return cuda_status(index_topk_into(p, qi, wi, kic, idx, sel_scores, scores, stream));

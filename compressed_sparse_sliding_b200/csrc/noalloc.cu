@@ -59,8 +59,9 @@ extern "C" hyb_status hyb_csa_index_topk_noalloc(const hyb_problem *p, const voi
         return st;
     if (!qi || !wi || !kic || !idx || !aligned16(qi) || !aligned16(kic))
         return HYB_ERR_INVALID_ARG;
-    // shapes whose selection runs in one kernel need no scratch at all
-    if (index_topk_fused_path(p))
+    // the two-kernel path on the fixed scratch where it is the faster one and
+    // the rows fit; otherwise the one kernel, which needs no scratch at all
+    if (index_topk_fused_path(p, kNoallocScratchBytes))
         return cuda_status(launch_index_topk_fused(qi, wi, kic, idx, sel_scores, p->B, p->Lq, p->Hi, p->di,
                                                    p->Nc, p->m, p->W, p->topk, p->q_pos, stream));
     const size_t need = (size_t)p->B * p->Lq * p->Nc * sizeof(float);

@@ -75,11 +75,14 @@ typedef struct hyb_problem {
     const int32_t *kv_pos0;  /* [B] position of raw row 0, or NULL (0)        */
 } hyb_problem;
 
-/* Bytes of device workspace hyb_csa_index_topk / hyb_fused_fwd need for `p`:
- * 0 for HCA, and 0 for CSA problems whose selection runs in one kernel
- * (Lq >= 64 query rows per sequence, Hi <= 4, Nc <= 65535: the scores are
- * recomputed on chip and never stored); otherwise B * Lq * Nc fp32 score rows.
- * A nonzero workspace must be 256-byte aligned; with 0, ws may be NULL. */
+/* Bytes of device workspace for the fastest path of hyb_csa_index_topk /
+ * hyb_fused_fwd on `p`: 0 for HCA; for CSA, B * Lq * Nc fp32 score rows
+ * (256-byte rounded), except 0 where the selection runs in one kernel that
+ * recomputes the scores on chip and stores none: problems of Lq >= 64 query
+ * rows per sequence, Hi <= 4, di 32 or 64, Nc <= 65535 and topk <= 2048 whose
+ * score rows would exceed 256 MiB.  Such one-kernel problems with smaller
+ * rows also run without the workspace (ws NULL or too small), in the one
+ * kernel, only more slowly.  A workspace must be 256-byte aligned. */
 size_t hyb_workspace_size(const hyb_problem *p);
 
 /* Stage 1, block_merge (CSDN code page, section 1):
@@ -99,11 +102,13 @@ hyb_status hyb_hca_compress(const void *x, int B, int L, int H, int dx, int m,
  * padded when fewer than K are visible.  sel_scores (nullable) receives the
  * fp32 score of each idx slot (-inf for padding).
  * qi: [B, Lq, Hi, di] bf16; wi: [B, Lq, Hi] fp32; kic: [B, Nc, di] bf16;
- * idx: [B, Lq, topk] int32; ws: workspace of >= hyb_workspace_size(p) bytes.
- * Problems of 64 or more query rows per sequence (Hi <= 4, Nc <= 65535) are
- * scored and selected in one kernel that keeps only per-row histograms on
- * chip; decode-shaped problems (few query rows) score into the workspace and
- * select from it. */
+ * idx: [B, Lq, topk] int32; ws: workspace of hyb_workspace_size(p) bytes.
+ * Two paths: score rows written to the workspace by a tensor-core kernel,
+ * then one CTA per row selecting from them; or one kernel that scores and
+ * selects on chip with only per-row histograms (the one-kernel shapes of
+ * hyb_workspace_size).  The two kernels run when the workspace holds the
+ * score rows and they take at most 256 MiB; the one kernel otherwise.  Both
+ * give the same selection.  HYB_ERR_WORKSPACE when neither can run. */
 hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float *wi,
                               const void *kic, int32_t *idx, float *sel_scores,
                               void *ws, size_t ws_bytes, cudaStream_t stream);
@@ -337,6 +342,17 @@ hyb_status hyb_trace_attach(void *buf, size_t bytes);
  * (rows_per_sm is rounded down to a multiple of 128). */
 hyb_status hyb_probe_l2_gather(const void *table, long long table_bytes, long long rows_per_sm,
                                int stages, unsigned int *sink, cudaStream_t stream);
+
+/* The same measurement with the tensor memory accelerator's row gather
+ * (cp.async.bulk.tensor tile::gather4, four rows per copy, one warp per CTA):
+ * rows land in 128-byte-swizzled stages and each stage's completion is counted
+ * in bytes on an mbarrier.  sink: device array of 257 uint32; sink[0..255]
+ * receive a checksum and sink[256] the number of 16-byte chunks of each CTA's
+ * last stage that are not where the 128-byte swizzle places them (added to
+ * what it holds; 0 when the layout is the one the CSA attention reads).  The
+ * table must hold fewer than 2^31 rows; other arguments as above. */
+hyb_status hyb_probe_l2_gather_tma(const void *table, long long table_bytes, long long rows_per_sm,
+                                   int stages, unsigned int *sink, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

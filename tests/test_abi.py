@@ -54,16 +54,19 @@ def test_host_side_argument_checks(lib):
     assert hb._lib.hyb_attn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, None,
                                 None) == hb.HYB_ERR_UNSUPPORTED
     # workspace: none when the selection runs in one kernel (64 or more query
-    # rows per sequence, at most 4 indexer heads, Nc <= 65535) ...
-    p = hb.problem(B=2, Lq=100, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=2, di=32, Nc=25)
+    # rows per sequence, at most 4 indexer heads, Nc <= 65535) and the score
+    # rows would take more than 256 MiB ...
+    p = hb.problem(B=2, Lq=2048, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=2, di=32, Nc=65535)
     assert hb.hyb_workspace_size(p) == 0
-    p.Lq = 2048
-    p.Nc = 65535
+    p = hb.problem(B=1, Lq=32768, Lkv=32768, Hq=32, Hkv=1, d=128, m=4, W=128, topk=512, Hi=4, di=64,
+                   Nc=8192)
     assert hb.hyb_workspace_size(p) == 0
-    # ... otherwise the scores of every (query row, entry) pair, fp32, 256-byte rounded
-    for lq, hi, nc in ((63, 2, 25), (100, 5, 25), (100, 2, 65536)):
-        p = hb.problem(B=2, Lq=lq, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=hi, di=32, Nc=nc)
-        assert hb.hyb_workspace_size(p) == (2 * lq * nc * 4 + 255) // 256 * 256
+    # ... otherwise the scores of every (query row, entry) pair, fp32, 256-byte rounded:
+    # shapes the one kernel does not take, and smaller ones, which the two kernels finish first
+    for lq, hi, nc in ((63, 2, 25), (100, 5, 25), (100, 2, 65536), (100, 2, 25), (16384, 4, 4096)):
+        p = hb.problem(B=2 if lq < 16384 else 1, Lq=lq, Lkv=100, Hq=4, Hkv=1, d=64, m=4, W=8, topk=8, Hi=hi,
+                       di=32, Nc=nc)
+        assert hb.hyb_workspace_size(p) == (p.B * lq * nc * 4 + 255) // 256 * 256
     p.topk = 0
     assert hb.hyb_workspace_size(p) == 0
     # missing workspace is reported as such
@@ -71,6 +74,13 @@ def test_host_side_argument_checks(lib):
     buf = ctypes.c_void_p(256)
     st = hb._lib.hyb_csa_index_topk(ctypes.byref(p), buf, buf, buf, buf, None, None, 0, None)
     assert st == hb.HYB_ERR_WORKSPACE
+    # the gather probes: null buffers, too few rows, stage counts outside 2..6
+    for fn in (hb._lib.hyb_probe_l2_gather, hb._lib.hyb_probe_l2_gather_tma):
+        assert fn(None, 1 << 20, 1024, 3, buf, None) == hb.HYB_ERR_INVALID_ARG
+        assert fn(buf, 1 << 20, 1024, 3, None, None) == hb.HYB_ERR_INVALID_ARG
+        assert fn(buf, 1 << 20, 64, 3, buf, None) == hb.HYB_ERR_INVALID_ARG
+        assert fn(buf, 1 << 20, 1024, 7, buf, None) == hb.HYB_ERR_INVALID_ARG
+        assert fn(buf, 1 << 20, 1024, 1, buf, None) == hb.HYB_ERR_INVALID_ARG
 
 
 def test_decode_append_argument_checks(lib):
@@ -117,10 +127,10 @@ def test_fp4_argument_checks(lib):
     # prefill: the whole caches are dequantized
     p = hb.problem(B=1, Lq=64, Lkv=64, Hq=4, Hkv=1, d=64, m=4, W=8, topk=4, Hi=2, di=32, Nc=16)
     attn = 2 * ((16 * 64 * 2 + 255) // 256 * 256)
-    index = (16 * 32 * 2 + 255) // 256 * 256    # keys dequantized once; no score rows (one-kernel selection)
-    assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
-    p.Hi = 5                                     # selection from stored score rows
+    # keys dequantized once, plus the score rows (small problems select from stored rows)
     index = (64 * 16 * 4 + 255) // 256 * 256 + (16 * 32 * 2 + 255) // 256 * 256
+    assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
+    p.Hi = 5                                     # a shape only the two-kernel path takes: the same
     assert hb.hyb_fp4_workspace_size(p) == max(attn, index)
     p.Hi = 2
     assert hb._lib.hyb_attn_fwd_fp4(ctypes.byref(p), *([buf] * 10), None, 0, None) == hb.HYB_ERR_WORKSPACE

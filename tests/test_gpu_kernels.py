@@ -50,7 +50,7 @@ def test_block_merge_matches_oracle(hb, B, L, H, dx, m):
 
 # ------------------------------------------------------------ indexer + top-K
 def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, pool=0, neg_w=False,
-                ramp=False):
+                ramp=False, one_kernel=False):
     g = torch.Generator().manual_seed(seed)
     qi = _randn_bf16(g, (B, Lq, Hi, di))
     wi = torch.rand((B, Lq, Hi), generator=g)
@@ -71,7 +71,9 @@ def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, p
     p = hb.problem(B=B, Lq=Lq, Lkv=max(W, 1), Hq=4, Hkv=1, d=64, m=m, W=W, topk=K, Hi=Hi, di=di,
                    Nc=Nc, q_pos=None if qp is None else qp.cuda())
     sel_scores = torch.empty((B, Lq, K), dtype=torch.float32, device="cuda")
-    idx = hb.hyb_csa_index_topk(p, qi.cuda(), wi.cuda(), kic.cuda(), sel_scores=sel_scores)
+    # one_kernel: no workspace, so shapes the one-kernel selection takes run there
+    idx = hb.hyb_csa_index_topk(p, qi.cuda(), wi.cuda(), kic.cuda(), sel_scores=sel_scores,
+                                ws_bytes=0 if one_kernel else None)
     torch.cuda.synchronize()
     assert hb.hyb_get_device_status() == hb.HYB_OK
     sc, nv = oracle.index_scores(bits(qi), wi.numpy(), bits(kic), m, W,
@@ -93,15 +95,18 @@ def _index_case(hb, B, Lq, Hi, di, Nc, m, W, K, q_pos=None, seed=0, rows=None, p
     return exact
 
 
-def test_index_topk_tiny_workload_shape(hb):
+@pytest.mark.parametrize("one_kernel", [False, True])
+def test_index_topk_tiny_workload_shape(hb, one_kernel):
     # the tiny CSA workload: L=1024, 2 indexer heads of dim 32, m=4, W=128, K=16
-    exact = _index_case(hb, 1, 1024, 2, 32, 256, 4, 128, 16, seed=1)
+    # (its 1 MB of score rows go to the two-kernel path unless no workspace is given)
+    exact = _index_case(hb, 1, 1024, 2, 32, 256, 4, 128, 16, seed=1, one_kernel=one_kernel)
     assert exact.mean() > 0.95
 
 
-def test_index_topk_ragged_and_small_K(hb):
-    _index_case(hb, 2, 333, 4, 64, 83, 4, 8, 5, seed=2)
-    _index_case(hb, 1, 200, 3, 32, 66, 3, 0, 64, seed=3)   # W = 0, K > n_vis for early rows
+@pytest.mark.parametrize("one_kernel", [False, True])
+def test_index_topk_ragged_and_small_K(hb, one_kernel):
+    _index_case(hb, 2, 333, 4, 64, 83, 4, 8, 5, seed=2, one_kernel=one_kernel)
+    _index_case(hb, 1, 200, 3, 32, 66, 3, 0, 64, seed=3, one_kernel=one_kernel)   # W = 0, K > n_vis early
 
 
 def test_index_topk_decode_positions(hb):
@@ -138,8 +143,9 @@ def test_index_topk_exact_ties_and_row_lengths(hb, Nc, pool):
         assert exact.all()   # exact ties are compared index for index
 
 
+@pytest.mark.parametrize("one_kernel", [False, True])
 @pytest.mark.parametrize("Nc,pool", [(3000, 0), (3000, 16), (8192, 0), (12000, 16)])
-def test_index_topk_many_rows(hb, Nc, pool):
+def test_index_topk_many_rows(hb, Nc, pool, one_kernel):
     # 1500 query rows at spread positions: the narrow per-row selection CTAs
     B, Lq, m, W, K = 3, 500, 4, 128, 300
     L = Nc * m + W
@@ -148,7 +154,7 @@ def test_index_topk_many_rows(hb, Nc, pool):
     pos[0, :4] = [L - 1, W + K * m + 3, W + K * m - 5, 0]
     rows = [0, 1, 2, 3] + sorted(rng.choice(B * Lq, size=40, replace=False).tolist())
     exact = _index_case(hb, B, Lq, 4, 64, Nc, m, W, K, q_pos=pos, seed=Nc + 7 * pool, pool=pool,
-                        rows=rows)
+                        rows=rows, one_kernel=one_kernel)
     if pool:
         assert exact.all()
 
@@ -156,27 +162,27 @@ def test_index_topk_many_rows(hb, Nc, pool):
 @pytest.mark.parametrize("case", ["ramp", "signed", "two_values", "random_pos", "all_visible", "k1",
                                   "short_rows"])
 def test_index_topk_selection_paths(hb, case):
-    # prefill-shaped problems select in one kernel that recomputes the scores
-    # pass by pass and moves or narrows a per-row key window until the K-th
+    # prefill-shaped problems given no workspace select in one kernel that
+    # recomputes the scores pass by pass and moves or narrows a per-row key window until the K-th
     # score is pinned; each case drives one of its paths
     rng = np.random.default_rng(len(case))
     if case == "ramp":          # the K-th score lies above every sampled score
-        _index_case(hb, 1, 700, 4, 64, 3000, 4, 128, 300, seed=11, ramp=True)
+        _index_case(hb, 1, 700, 4, 64, 3000, 4, 128, 300, seed=11, ramp=True, one_kernel=True)
     elif case == "signed":      # negative scores (order keys below +0)
-        _index_case(hb, 2, 400, 3, 64, 2500, 4, 64, 200, seed=12, neg_w=True)
+        _index_case(hb, 2, 400, 3, 64, 2500, 4, 64, 200, seed=12, neg_w=True, one_kernel=True)
     elif case == "two_values":  # two distinct keys: the threshold bin is one exact score
-        exact = _index_case(hb, 1, 520, 4, 32, 2000, 4, 128, 100, seed=13, pool=2)
+        exact = _index_case(hb, 1, 520, 4, 32, 2000, 4, 128, 100, seed=13, pool=2, one_kernel=True)
         assert exact.all()
     elif case == "random_pos":  # rows of one tile with very different visible counts
         L = 4000 * 4 + 128
         pos = rng.integers(0, L, size=(2, 300)).astype(np.int32)
-        _index_case(hb, 2, 300, 4, 64, 4000, 4, 128, 256, q_pos=pos, seed=14)
+        _index_case(hb, 2, 300, 4, 64, 4000, 4, 128, 256, q_pos=pos, seed=14, one_kernel=True)
     elif case == "all_visible":  # K >= every row's visible count
-        _index_case(hb, 1, 777, 2, 64, 190, 4, 16, 200, seed=15)
+        _index_case(hb, 1, 777, 2, 64, 190, 4, 16, 200, seed=15, one_kernel=True)
     elif case == "k1":
-        _index_case(hb, 1, 300, 4, 64, 500, 4, 32, 1, seed=16)
+        _index_case(hb, 1, 300, 4, 64, 500, 4, 32, 1, seed=16, one_kernel=True)
     else:                       # rows shorter than one sampled tile
-        _index_case(hb, 1, 200, 2, 32, 60, 2, 64, 7, seed=17)
+        _index_case(hb, 1, 200, 2, 32, 60, 2, 64, 7, seed=17, one_kernel=True)
 
 
 # ----------------------------------------------------------------- attention
@@ -342,3 +348,21 @@ def test_out_of_range_index_is_reported_not_read(hb, d):
     hb.hyb_attn_fwd(p, q, kc, kc, idx.cuda(), k, k)
     assert hb.hyb_get_device_status() == hb.HYB_ERR_DEVICE_BOUNDS
     assert hb.hyb_get_device_status() == hb.HYB_OK  # read clears it
+
+
+# ------------------------------------------------------------ gather probes
+@pytest.mark.parametrize("stages", [2, 6])
+def test_l2_gather_probes_land_rows_where_the_attention_reads_them(hb, stages):
+    """Both measurement probes run to completion; the tile::gather4 form puts
+    every 16-byte chunk of its last stage where the 128-byte swizzle of the
+    attention's K / V tiles expects it (sink[256] counts misplaced chunks)."""
+    dev = torch.device("cuda")
+    table = torch.randint(0, 1 << 30, ((1 << 20) // 4,), dtype=torch.int32, device=dev)
+    sink = torch.zeros(257, dtype=torch.int32, device=dev)
+    hb.hyb_probe_l2_gather(table, 128 * 8, stages, sink)
+    sink.zero_()
+    hb.hyb_probe_l2_gather_tma(table, 128 * 8, stages, sink)
+    torch.cuda.synchronize()
+    assert hb.hyb_get_device_status() == 0
+    assert int(sink[256].item()) == 0
+    assert int(sink[:256].abs().sum().item()) != 0   # the copied words reached the checksum

@@ -49,9 +49,10 @@ def _index_case(hb):
     qi = _randn(g, (B, Lq, Hi, di))
     wi = torch.rand((B, Lq, Hi), generator=g).cuda()
     kic = _randn(g, (B, Nc, di))
-    # m = 1, W = 0: row t sees t + 1 entries, so most rows select (all passes run)
+    # m = 1, W = 0: row t sees t + 1 entries, so most rows select (all passes run);
+    # no workspace, so the selection runs in the one kernel
     p = hb.problem(B=B, Lq=Lq, Lkv=Lq, Hq=4, Hkv=1, d=64, m=1, W=0, topk=K, Hi=Hi, di=di, Nc=Nc)
-    return lambda: hb.hyb_csa_index_topk(p, qi, wi, kic)
+    return lambda: hb.hyb_csa_index_topk(p, qi, wi, kic, ws_bytes=0)
 
 
 @pytest.mark.parametrize("case", ["csa_attention", "csa_attention_decode_split", "index_topk"])
