@@ -7,6 +7,8 @@
 // the Hi accumulators of its row, forms the weighted ReLU sum and stores the
 // visible part of the tile into the token's score row.  Queries (one TMA box
 // per head) stay in shared memory; key tiles stream through a 4-stage ring.
+// Indexer dims 64 (rows of 128 bytes, 128-byte swizzle) and 32 (64-byte rows
+// and swizzle): the MMA takes di / 16 steps of K = 16.
 // When a score row is a multiple of 16 bytes the epilogue stages each 128 x 32
 // block of scores in shared memory (128-byte swizzle) and one thread writes it
 // with a TMA tensor store, so the rows leave as whole 128-byte lines instead of
@@ -24,7 +26,7 @@ constexpr int kIxThreads = 256;
 constexpr int kIxBM = 128;        // query tokens per CTA
 constexpr int kIxBN = 64;         // keys per tile
 constexpr int kIxStages = 4;
-constexpr int kIxDi = 64;         // indexer dim handled here
+constexpr int kIxDi = 64;         // indexer dim of the decode form
 constexpr int kIxChunkTiles = 32; // key tiles per CTA (2048 entries)
 
 struct IndexParams {
@@ -36,10 +38,10 @@ struct IndexParams {
     float *scores;                // [B * Lq, Nc]
 };
 
-template <int HI>
+template <int HI, int DI>
 struct IxSmem {
-    static constexpr int Q_BYTES = kIxBM * kIxDi * 2;     // one head
-    static constexpr int K_BYTES = kIxBN * kIxDi * 2;
+    static constexpr int Q_BYTES = kIxBM * DI * 2;        // one head
+    static constexpr int K_BYTES = kIxBN * DI * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = HI * Q_BYTES;
     static constexpr int OFF_BAR = OFF_K + kIxStages * K_BYTES;
@@ -59,12 +61,27 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-template <int HI>
+// Shared-memory matrix descriptor of a K-major operand whose rows are DI bf16
+// (128- or 64-byte swizzle; 8-row groups DI * 16 bytes apart).
+template <int DI>
+__device__ __forceinline__ uint64_t ix_desc(uint32_t saddr)
+{
+    static_assert(DI == 64 || DI == 32, "indexer dim 64 or 32");
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                               // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(((DI * 16) >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)(DI == 64 ? 2u : 4u) << 61;            // 128- or 64-byte swizzle
+    return d;
+}
+
+template <int HI, int DI>
 __global__ void __launch_bounds__(kIxThreads, 1)
 index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_s, const IndexParams p)
 {
-    using SM = IxSmem<HI>;
+    using SM = IxSmem<HI, DI>;
     extern __shared__ __align__(1024) uint8_t ix_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(ix_smem_raw) + 1023) &
                                                 ~(uintptr_t)1023);
@@ -157,9 +174,9 @@ index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
                 for (int h = 0; h < HI; ++h) {
 #pragma unroll
-                    for (int kk = 0; kk < kIxDi / 16; ++kk) {
-                        const uint64_t da = sw128_desc(aQ + h * SM::Q_BYTES + kk * 32, 16, 1024);
-                        const uint64_t dbk = sw128_desc(aK + s * SM::K_BYTES + kk * 32, 16, 1024);
+                    for (int kk = 0; kk < DI / 16; ++kk) {
+                        const uint64_t da = ix_desc<DI>(aQ + h * SM::Q_BYTES + kk * 32);
+                        const uint64_t dbk = ix_desc<DI>(aK + s * SM::K_BYTES + kk * 32);
                         mma_bf16_ss(tmem + (db * HI + h) * kIxBN, da, dbk, idesc, kk > 0 ? 1u : 0u);
                     }
                 }
@@ -274,16 +291,33 @@ index_scores_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-template <int HI>
+// 4-D map over a [n3][n2][n1][DI] bf16 tensor with a (DI, 1, box_rows, 1) box,
+// 128-byte swizzle for DI = 64 and 64-byte swizzle for DI = 32.
+template <int DI>
+static bool ix_map(CUtensorMap *map, const void *base, int n1, int n2, int n3, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[4] = {(cuuint64_t)DI, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+    cuuint64_t strides[3] = {(cuuint64_t)DI * 2, (cuuint64_t)DI * 2 * n1, (cuuint64_t)DI * 2 * n1 * n2};
+    cuuint32_t box[4] = {(cuuint32_t)DI, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, DI == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HI, int DI>
 static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const void *kic,
                                      cudaStream_t stream)
 {
-    using SM = IxSmem<HI>;
+    using SM = IxSmem<HI, DI>;
     CUtensorMap mq, mk;
-    // qi [B, Lq, Hi, 64] as (64, Hi, Lq, B) with a (64, 1, 128, 1) box
-    bool ok = make_map(&mq, qi, kIxDi, HI, p.Lq, p.B, 1, kIxBM);
-    // kic [B, Nc, 64] as (64, 1, Nc, B) with a (64, 1, 64, 1) box
-    ok &= make_map(&mk, kic, kIxDi, 1, p.Nc, p.B, 1, kIxBN);
+    // qi [B, Lq, Hi, DI] as (DI, Hi, Lq, B) with a (DI, 1, 128, 1) box
+    bool ok = ix_map<DI>(&mq, qi, HI, p.Lq, p.B, kIxBM);
+    // kic [B, Nc, DI] as (DI, 1, Nc, B) with a (DI, 1, 64, 1) box
+    ok &= ix_map<DI>(&mk, kic, 1, p.Nc, p.B, kIxBN);
     if (!ok)
         return cudaErrorInvalidValue;
     // scores [B, Lq, Nc] fp32 as (Nc, Lq, B) with a (32, 128, 1) box, 128-byte
@@ -304,7 +338,7 @@ static cudaError_t launch_index_tc_t(const IndexParams &p, const void *qi, const
     size_t smem = 1024 + SM::BYTES;
     if (smem < 120 * 1024)
         smem = 120 * 1024;  // one CTA per SM: each holds all 512 TMEM columns
-    auto kern = index_scores_tc<HI>;
+    auto kern = index_scores_tc<HI, DI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -617,15 +651,18 @@ cudaError_t launch_index_dec_fp4(const void *qi, const float *wi, const uint8_t 
                             stream);
 }
 
-// Prefill indexer scores on tensor cores (di = 64, Hi <= 4).  Returns
-// cudaErrorNotSupported for other shapes (the caller uses the CUDA-core path).
+// Indexer scores on tensor cores: prefill (di 64 or 32, Hi <= 4) and decode
+// (di 64).  Returns cudaErrorNotSupported for other shapes (the caller uses
+// the CUDA-core path).
 cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *kic, float *scores,
                                    int B, int Lq, int Hi, int di, int Nc, int m, int W,
                                    const int32_t *q_pos, cudaStream_t stream)
 {
-    if (di != kIxDi || Hi < 1)
+    if ((di != 64 && di != 32) || Hi < 1)
         return cudaErrorNotSupported;
     if (Lq < 64) {
+        if (di != kIxDi)
+            return cudaErrorNotSupported;
         // decode: one tile of keys per MMA, the query's heads in N
         if (Hi > kDcN)
             return cudaErrorNotSupported;
@@ -649,11 +686,19 @@ cudaError_t launch_index_scores_tc(const void *qi, const float *wi, const void *
     p.scores = scores;
     // the tensor store needs 16-byte row strides and a 16-byte aligned base
     p.tma_store = (Nc % 4 == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) ? 1 : 0;
+    if (di == 32) {
+        switch (Hi) {
+        case 1: return launch_index_tc_t<1, 32>(p, qi, kic, stream);
+        case 2: return launch_index_tc_t<2, 32>(p, qi, kic, stream);
+        case 3: return launch_index_tc_t<3, 32>(p, qi, kic, stream);
+        default: return launch_index_tc_t<4, 32>(p, qi, kic, stream);
+        }
+    }
     switch (Hi) {
-    case 1: return launch_index_tc_t<1>(p, qi, kic, stream);
-    case 2: return launch_index_tc_t<2>(p, qi, kic, stream);
-    case 3: return launch_index_tc_t<3>(p, qi, kic, stream);
-    default: return launch_index_tc_t<4>(p, qi, kic, stream);
+    case 1: return launch_index_tc_t<1, 64>(p, qi, kic, stream);
+    case 2: return launch_index_tc_t<2, 64>(p, qi, kic, stream);
+    case 3: return launch_index_tc_t<3, 64>(p, qi, kic, stream);
+    default: return launch_index_tc_t<4, 64>(p, qi, kic, stream);
     }
 }
 
