@@ -45,6 +45,12 @@ namespace hyb {
 constexpr int kSpBN = 128;       // keys per tile (the M of S^T)
 constexpr int kSpSelBatch = 8;   // selection entries a producer thread loads at once
 constexpr int kSpLead = 1;       // tiles by which the K copies run ahead of the V copies
+// The next item's prologue runs before this item's K copy of tile
+// ntl - kSpPrologueAhead (of ntl tiles).  On the CSA prefill 2 measured best:
+// 1.795 ms against 1.870 (0, after the last K tile), 2.18 (1), 1.85 (3),
+// 2.10 (4), 2.26 (5), and against forms that ran it at the first ring wait
+// that would block (1.95 to 2.3 ms).
+constexpr int kSpPrologueAhead = 2;
 constexpr int kSpD = 128;        // head dim handled by this kernel
 
 struct SparseParams {
@@ -494,8 +500,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // An item's prologue: its Q tile, its selection decoded into buffer
         // nq & 1 (the first batch of entries already in jnext), and the next
         // item's first batch sent for.  It runs during the previous item's
-        // copies, right after that item's last K tile, so that the gather
-        // does not pause between items.
+        // copies (before its K tile ntl - kSpPrologueAhead), so that the
+        // gather does not pause between items.
         auto prologue = [&](long long w, uint32_t nq) {
             const SparseTok k = sparse_tok(p, w);
             const int qb = nq & 1;
@@ -597,7 +603,7 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // again for V.
             for (int ii = 0; ii < ntl + kSpLead; ++ii) {
                 const int i = tb + ii;
-                if (ii == ntl && w + wstep < p.n_items)
+                if (ii == max(ntl - kSpPrologueAhead, 0) && w + wstep < p.n_items)
                     prologue(w + wstep, nq + 1);
                 if (ii < ntl) {
                     const uint32_t ks = kc % KS;
