@@ -43,7 +43,6 @@
 namespace hyb {
 
 constexpr int kSpBN = 128;       // keys per tile (the M of S^T)
-constexpr int kSpSelBatch = 8;   // selection entries a producer thread loads at once
 constexpr int kSpLead = 1;       // tiles by which the K copies run ahead of the V copies
 // The next item's prologue runs before this item's K copy of tile
 // ntl - kSpPrologueAhead (of ntl tiles).  On the CSA prefill 2 measured best:
@@ -362,6 +361,10 @@ struct SpRoles {
     static constexpr int PROD_WARP0 = 4 * HS;
     static constexpr int MMA_WARP = PROD_WARP0 + PW;
     static constexpr int THREADS = 32 * (MMA_WARP + 1);
+    // selection entries a producer thread loads at once: 4 covers a 512-entry
+    // selection over four warps in one batch (CSA prefill: 1.756 ms against
+    // 1.793 with 8); 8 for the two-warp decode form (25.6 against 27.6 us)
+    static constexpr int SEL_BATCH = NH == 64 ? 8 : 4;
 };
 
 template <int NH>
@@ -476,10 +479,10 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         // this warp's entries e0 + lane + 32 j (of ne) of item w's selection,
         // -1 past topk; item w = (b Lq + t) Hkv + KV head, below 2^31
-        auto load_sel = [&](long long w, int t0s, int ne, int e0, int (&jv)[kSpSelBatch]) {
+        auto load_sel = [&](long long w, int t0s, int ne, int e0, int (&jv)[SpRoles<NH>::SEL_BATCH]) {
             const int32_t *irow = p.idx + (size_t)((uint32_t)w / (uint32_t)p.Hkv) * p.topk;
 #pragma unroll
-            for (int j = 0; j < kSpSelBatch; ++j) {
+            for (int j = 0; j < SpRoles<NH>::SEL_BATCH; ++j) {
                 const int e = e0 + lane + 32 * j;
                 const int q = slot_of(t0s, e);
                 // volatile: issued here, not sunk to the first use an item later
@@ -489,13 +492,13 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 jv[j] = v;
             }
         };
-        auto load_first = [&](long long w, int (&jv)[kSpSelBatch]) {
+        auto load_first = [&](long long w, int (&jv)[SpRoles<NH>::SEL_BATCH]) {
             const SparseTok kn = sparse_tok(p, w);
             int s0, s1;
             sel_tiles(kn, s0, s1);
             load_sel(w, s0, (s1 - s0) * 2 * CPT, 0, jv);
         };
-        int jnext[kSpSelBatch];
+        int jnext[SpRoles<NH>::SEL_BATCH];
         uint32_t nql = 0;                       // items whose Q tile was sent for
         // An item's prologue: its Q tile, its selection decoded into buffer
         // nq & 1 (the first batch of entries already in jnext), and the next
@@ -531,17 +534,17 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 sel_tiles(k, s0, s1);
                 const int ne = (s1 - s0) * 2 * CPT;
 #pragma unroll 1
-                for (int e0 = 0; e0 < ne; e0 += 32 * kSpSelBatch) {
-                    int jv[kSpSelBatch];
+                for (int e0 = 0; e0 < ne; e0 += 32 * SpRoles<NH>::SEL_BATCH) {
+                    int jv[SpRoles<NH>::SEL_BATCH];
                     if (e0 == 0) {
 #pragma unroll
-                        for (int j = 0; j < kSpSelBatch; ++j)
+                        for (int j = 0; j < SpRoles<NH>::SEL_BATCH; ++j)
                             jv[j] = jnext[j];
                     } else {
                         load_sel(w, s0, ne, e0, jv);
                     }
 #pragma unroll
-                    for (int j = 0; j < kSpSelBatch; ++j) {
+                    for (int j = 0; j < SpRoles<NH>::SEL_BATCH; ++j) {
                         const int e = e0 + lane + 32 * j;
                         if (e < ne) {
                             const int q = slot_of(s0, e);
