@@ -11,11 +11,11 @@ bit-identically (the entry the step's append closes is not yet visible to
 the query), so its rows follow that rule exactly and the attention output is
 compared on every row whose selection is not a near tie.  In prefill the GPU's
 indexer reads the GPU's own compressed keys, which may differ from the
-oracle's in about one element in 10^4 by one bf16 ulp; a prefill row whose
-selection then differs must still be a valid top-K of the oracle's scores
-within 1e-3 relative, at most 2% of sampled rows may be such rows, and the
-attention output is compared on the other rows (the attention kernel itself is
-checked with identical indices elsewhere)."""
+oracle's in about one element in 10^4 by one bf16 ulp (the caches themselves
+are checked against the oracle's within the block_merge bound), so the oracle
+scores those same keys: every sampled row is then bit-exact except near ties,
+and the attention output is compared on every sampled row against the
+oracle's attention over the GPU's (checked) selection."""
 import numpy as np
 import pytest
 import torch
@@ -64,20 +64,6 @@ def sample_positions(w, n_random=40, seed=0):
     rng = np.random.default_rng(seed)
     pts |= set(rng.integers(0, L, n_random).tolist())
     return sorted(p for p in pts if 0 <= p < L)
-
-
-def _valid_topk_rows(idx_gpu, scores, nvis, K, rel):
-    for r in range(len(nvis)):
-        n = nvis[r]
-        sel = idx_gpu[r][idx_gpu[r] >= 0]
-        assert len(sel) == min(K, n) and np.all(np.diff(sel) > 0) and (len(sel) == 0 or sel.max() < n)
-        if n <= K:
-            continue
-        kth = np.sort(scores[r, :n])[::-1][K - 1]
-        tol = rel * abs(kth) + 1e-30
-        assert scores[r, sel].min() >= kth - tol
-        rest = np.setdiff1d(np.arange(n), sel)
-        assert scores[r, rest].max() <= kth + tol
 
 
 @pytest.mark.parametrize("no", [1, 2, 3, 4, 5])
@@ -155,17 +141,16 @@ def test_workload_end_to_end(hb, no):
     qsel = torch.as_tensor(pos, device="cuda")
     q_sub = bits(inp["q"][:, qsel].contiguous())
     o_sub = o[:, qsel].reshape(w.B * S, w.Hq, w.d)
-    keep = np.ones(w.B * S, dtype=bool)
-    idx_ref = None
+    idx_sel = None
     if w.topk:
         qi_sub = bits(inp["qi"][:, qsel].contiguous())
         wi_sub = inp["wi"][:, qsel].contiguous().cpu().numpy()
-        sc, nv = oracle.index_scores(qi_sub, wi_sub, kic_ref, w.m, w.W, q_pos=q_pos)
+        # the GPU's own compressed indexer keys (checked above): both sides
+        # rank identical keys, so rows are bit-exact except near ties
+        sc, nv = oracle.index_scores(qi_sub, wi_sub, bits(out["kic"]), w.m, w.W, q_pos=q_pos)
         idx_ref = oracle.topk(sc, nv, w.topk)
         gidx = out["idx"][:, qsel].reshape(w.B * S, w.topk).cpu().numpy()
-        keep = np.all(gidx == idx_ref, axis=1)
-        _valid_topk_rows(gidx, sc, nv, w.topk, 1e-3)
-        assert keep.mean() >= 0.98, f"{(~keep).sum()} of {len(keep)} rows select differently"
-        idx_ref = idx_ref.reshape(w.B, S, w.topk)
-    ref = oracle.hybrid_attention(q_sub, kc_ref, vc_ref, idx_ref, k_b, v_b, w.m, w.W, q_pos=q_pos)
-    check_output(o_sub[torch.from_numpy(keep).cuda()], ref["o"][keep])
+        check_topk(gidx, idx_ref, sc, nv, w.topk)
+        idx_sel = gidx.reshape(w.B, S, w.topk)
+    ref = oracle.hybrid_attention(q_sub, kc_ref, vc_ref, idx_sel, k_b, v_b, w.m, w.W, q_pos=q_pos)
+    check_output(o_sub, ref["o"])
