@@ -123,9 +123,11 @@ hyb_status hyb_csa_index_topk(const hyb_problem *p, const void *qi, const float 
  * needs no workspace.  Meant for callers that may not allocate device memory
  * themselves: an engine whose memory planner owns every buffer, or a decode
  * loop where cudaMalloc / cudaFree would synchronise the device.
- *   - B * Lq * Nc * 4 bytes must fit in HYB_NOALLOC_SCRATCH_BYTES, otherwise
- *     the call returns HYB_ERR_UNSUPPORTED and launches nothing (the decode
- *     shape 64 x 16384 entries uses 4 MiB).
+ *   - Problems the one-kernel selection takes (see hyb_workspace_size) run
+ *     there when their B * Lq * Nc * 4 bytes of score rows exceed
+ *     HYB_NOALLOC_SCRATCH_BYTES; any other problem must fit its rows in it,
+ *     otherwise the call returns HYB_ERR_UNSUPPORTED and launches nothing
+ *     (the decode shape 64 x 16384 entries uses 4 MiB).
  *   - Every GPU that loads the library holds the array until the process
  *     exits.  The first call on a device looks up the array's address with
  *     that device current; make that first call before any stream capture.
