@@ -26,6 +26,7 @@ constexpr int kIxThreads = 256;
 constexpr int kIxBM = 128;        // query tokens per CTA
 constexpr int kIxBN = 64;         // keys per tile
 constexpr int kIxStages = 4;
+static_assert(kIxStages == 4, "the prefill score kernel's barrier map (1-4 K full, 5-8 K empty) is written for four stages");
 constexpr int kIxDi = 64;         // indexer dim of the decode form
 constexpr int kIxChunkTiles = 32; // key tiles per CTA (2048 entries)
 
@@ -367,6 +368,7 @@ constexpr int kDcAhead = 8;      // 4-bit form: tiles of codes in flight per con
 constexpr int kDcBM = 128;       // keys per tile
 constexpr int kDcN = 16;         // padded indexer heads
 constexpr int kDcStages = 4;
+static_assert(kDcStages == 4, "the decode score kernel's barrier map (1-4 K full, 5-8 K empty) is written for four stages");
 constexpr int kDcChunk = 16;     // key tiles per CTA
 
 struct DecIndexParams {
