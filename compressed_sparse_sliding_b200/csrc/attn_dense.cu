@@ -40,6 +40,7 @@ constexpr int kDnBM = 128;
 constexpr int kDnBN = 128;
 constexpr int kDnKStages = 2;
 constexpr int kDnVStages = 2;
+static_assert(kDnKStages == 2 && kDnVStages == 2, "the barrier slots (DB_KF .. DB_VE) hold two stages each");
 
 struct DenseParams {
     int B, L, Lkv, Hq, Hkv, g, Nc, m, W;

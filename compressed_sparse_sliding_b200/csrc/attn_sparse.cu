@@ -79,6 +79,7 @@ struct SparseSmem {
     // tiles should not wait on a V stage
     static constexpr int KS = NH == 64 ? 2 : 3;                    // K ring depth
     static constexpr int VS = 2;                                   // V ring depth
+    static_assert(KS <= 3 && VS <= 3, "the barrier slots SB_KF .. SB_VE hold three stages each");
     static constexpr int OFF_Q = 0;                                // 2 buffers
     static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
