@@ -230,7 +230,8 @@ class Step:
                                     dw=self.dwk, ws=self.bws, stream=stream)
             hb.hyb_hca_compress_bwd(inp["v"], inp["wv"], w.m, self.grads["dvc"], dx=self.grads["dv_raw"],
                                     dw=self.dwv, ws=self.bws, stream=stream)
-            launches += 5
+            # dense problems with d = 128: three tensor-core launches, else one
+            launches += 4 + (3 if (w.topk == 0 and w.d == 128) else 1)
             ev[4].record(stream)
             self.launches = launches
             return
@@ -593,15 +594,22 @@ def run_gpu(args, rank, world):
     peaks = load_peaks()
     att_ms = statistics.mean(att)
     hbm_bound = w.is_decode or w.no == 2
+    bwd_tc = train and w.topk == 0 and w.d == 128
     if train:
-        # the attention backward on CUDA cores: 10 d FLOP per (query head, key)
-        # (the scores again, dP, dq, dk, dv); peak = 148 SMs x 128 fp32 lanes x
-        # 2 FLOP x the clock measured during the run
+        # the attention backward: 10 d FLOP per (query head, key) (the scores
+        # again, dP, dq, dk, dv).  Dense problems with d = 128 run on the tensor
+        # cores (bf16 peak); the others on CUDA cores, whose peak is 148 SMs x
+        # 128 fp32 lanes x 2 FLOP x the clock measured during the run
         bwd_ms = statistics.mean(back)
-        mhz = (clocks or {}).get("sm_mhz") or 1965.0
-        peak = round(148 * 128 * 2 * mhz * 1e6 / 1e12, 1)
         achieved = 2.5 * counts["attn_flop"] / (bwd_ms / 1e3) / 1e12
-        roof = {"bound": "alu", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+        if bwd_tc:
+            peak = peaks["bf16_tflops"]
+            bound = "tensor"
+        else:
+            mhz = (clocks or {}).get("sm_mhz") or 1965.0
+            peak = round(148 * 128 * 2 * mhz * 1e6 / 1e12, 1)
+            bound = "alu"
+        roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4)}
     elif hbm_bound:
         achieved = counts["attn_bytes"] / (att_ms / 1e3) / 1e9
@@ -619,9 +627,11 @@ def run_gpu(args, rank, world):
     if fp4:
         kname = "hyb_attn_fwd_fp4 (fp4_gather_kernel + csa_attn_kernel)"
     if train:
-        kname = "attn_bwd_kernel"
+        kname = ("bwd_delta_kernel + attn_bwd_kv_kernel + attn_bwd_q_kernel" if bwd_tc
+                 else "attn_bwd_kernel")
     roof["kernel"] = kname
-    roof["peak_source"] = "derived (unit counts x measured clock)" if train else peaks["source"]
+    roof["peak_source"] = ("derived (unit counts x measured clock)" if train and not bwd_tc
+                           else peaks["source"])
     roof["traffic"] = kernel_traffic(kname, w.no)
     stages = {("append_ms" if w.is_decode else "compress_ms"): round(statistics.mean(comp), 4),
               "index_topk_ms": round(statistics.mean(idx), 4),

@@ -549,6 +549,11 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
         return HYB_ERR_INVALID_ARG;
     if (p->Lkv <= 0)
         return HYB_ERR_INVALID_ARG;
+    const float scale = softmax_scale(p);
+    if (attn_bwd_tc_ok(idx != nullptr, p->d, p->q_pos, p->kv_pos0, p->Lq, p->Lkv, p->Nc, p->m, p->W))
+        return cuda_status(launch_attn_bwd_tc(p->B, p->Lq, p->Hq, p->Hkv, p->Nc, p->m, p->W, scale, q, kc, vc,
+                                              k_raw, v_raw, o, lse, dout, dq, dkc, dvc, dk_raw, dv_raw, stream,
+                                              num_sms_current()));
     const size_t ck = (size_t)p->B * p->Nc * p->Hkv * p->d * sizeof(float);
     const size_t rk = (size_t)p->B * p->Lkv * p->Hkv * p->d * sizeof(float);
     cudaError_t e = cudaSuccess;
@@ -575,7 +580,7 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
     b.m = p->m;
     b.W = p->W;
     b.topk = idx ? p->topk : 0;
-    b.scale = softmax_scale(p);
+    b.scale = scale;
     b.q_pos = p->q_pos;
     b.kv_pos0 = p->kv_pos0;
     b.idx = idx;

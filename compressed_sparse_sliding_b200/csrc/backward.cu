@@ -220,9 +220,46 @@ cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
 }
 
 // ---------------------------------------------------------------- block_merge
+// sP[i][lane] = softmax over positions i of w[i, c] for the CTA's channel
+// c = 32 blockIdx.x + lane, computed by all eight warps (warp w takes
+// positions w, w + 8, ...); sRed: 8 x 32 floats of scratch.
+__device__ __forceinline__ void bm_softmax_weights(const float *__restrict__ w, int D, int m, float *sP,
+                                                   float *sRed)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + lane;
+    float mx = -INFINITY;
+    for (int i = warp; i < m; i += 8)
+        mx = fmaxf(mx, w[(size_t)i * D + c]);
+    sRed[warp * 32 + lane] = mx;
+    __syncthreads();
+    mx = sRed[lane];
+    for (int k = 1; k < 8; ++k)
+        mx = fmaxf(mx, sRed[k * 32 + lane]);
+    __syncthreads();
+    float den = 0.f;
+    for (int i = warp; i < m; i += 8) {
+        const float e = expf(w[(size_t)i * D + c] - mx);
+        sP[i * 32 + lane] = e;
+        den += e;
+    }
+    sRed[warp * 32 + lane] = den;
+    __syncthreads();
+    den = 0.f;
+    for (int k = 0; k < 8; ++k)
+        den += sRed[k * 32 + lane];
+    const float inv = 1.f / den;
+    for (int i = warp; i < m; i += 8)
+        sP[i * 32 + lane] *= inv;
+    __syncthreads();
+}
+
 // grid (dx / 32, row groups of rpc rows); warp w of the CTA takes rows w,
-// w + 8, ... of its group; lane = channel.  G partials in shared memory [m][32].
-__global__ void __launch_bounds__(256)
+// w + 8, ... of its group; lane = channel.  Positions go 16 at a time: the
+// 16 rows' x and dx values are loaded together, dx written back, and the G
+// terms kept in registers over the warp's rows, then added to the CTA's G
+// partials in shared memory [m][32] (one atomic per position and lane).
+__global__ void __launch_bounds__(256, 2)
 block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
                        const float *__restrict__ dc, float *__restrict__ dx, float *__restrict__ G,
                        int B, int L, int H, int D, int m, int rpc)
@@ -230,61 +267,75 @@ block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restr
     extern __shared__ float bm_smem[];
     float *sP = bm_smem;                  // [m][32] softmax weights of the CTA's channels
     float *sG = bm_smem + m * 32;         // [m][32] G partials
+    float *sRed = sG + m * 32;            // [8][32]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int c = blockIdx.x * 32 + lane;
     const int Nc = L / m;
     const long long rows = (long long)B * Nc * H;
-    if (warp == 0) {
-        float mx = -INFINITY;
-        for (int i = 0; i < m; ++i)
-            mx = fmaxf(mx, w[(size_t)i * D + c]);
-        float den = 0.f;
-        for (int i = 0; i < m; ++i)
-            den += expf(w[(size_t)i * D + c] - mx);
-        for (int i = 0; i < m; ++i)
-            sP[i * 32 + lane] = expf(w[(size_t)i * D + c] - mx) / den;
-    }
     for (int e = threadIdx.x; e < m * 32; e += 256)
         sG[e] = 0.f;
-    __syncthreads();
+    bm_softmax_weights(w, D, m, sP, sRed);
     const long long r0 = (long long)blockIdx.y * rpc;
-    for (long long r = r0 + warp; r < r0 + rpc && r < rows; r += 8) {
-        const int h = (int)(r % H);
-        const long long bj = r / H;
-        const int b = (int)(bj / Nc), j = (int)(bj % Nc);
-        const float g = dc[((size_t)bj * H + h) * D + c];
-        const size_t xrow0 = (((size_t)b * L + (size_t)j * m) * H + h) * D + c;
-        for (int i = 0; i < m; ++i) {
-            const size_t at = xrow0 + (size_t)i * H * D;
-            dx[at] += sP[i * 32 + lane] * g;
-            atomicAdd(&sG[i * 32 + lane], g * __bfloat162float(x[at]));
+    const size_t istride = (size_t)H * D;
+    for (int i0 = 0; i0 < m; i0 += 16) {
+        float gacc[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            gacc[k] = 0.f;
+        for (long long r = r0 + warp; r < r0 + rpc && r < rows; r += 8) {
+            const int h = (int)(r % H);
+            const long long bj = r / H;
+            const int b = (int)(bj / Nc), j = (int)(bj % Nc);
+            const float g = dc[((size_t)bj * H + h) * D + c];
+            const size_t xrow0 = (((size_t)b * L + (size_t)j * m + i0) * H + h) * D + c;
+            float xv[16], dv[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                if (i0 + k < m) {
+                    xv[k] = __bfloat162float(x[xrow0 + k * istride]);
+                    dv[k] = dx[xrow0 + k * istride];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                if (i0 + k < m) {
+                    dx[xrow0 + k * istride] = dv[k] + sP[(i0 + k) * 32 + lane] * g;
+                    gacc[k] += g * xv[k];
+                }
+            }
         }
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if (i0 + k < m)
+                atomicAdd(&sG[(i0 + k) * 32 + lane], gacc[k]);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < m * 32; e += 256)
         atomicAdd(&G[(size_t)(e / 32) * D + blockIdx.x * 32 + (e % 32)], sG[e]);
 }
 
-// dw[i, c] = P[i, c] (G[i, c] - sum_k P[k, c] G[k, c]); thread per channel.
-__global__ void block_merge_dw_kernel(const float *__restrict__ w, const float *__restrict__ G,
-                                      float *__restrict__ dw, int D, int m)
+// dw[i, c] = P[i, c] (G[i, c] - sum_k P[k, c] G[k, c]); a CTA per 32 channels,
+// warp w takes positions w, w + 8, ...
+__global__ void __launch_bounds__(256)
+block_merge_dw_kernel(const float *__restrict__ w, const float *__restrict__ G, float *__restrict__ dw, int D,
+                      int m)
 {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= D)
-        return;
-    float mx = -INFINITY;
-    for (int i = 0; i < m; ++i)
-        mx = fmaxf(mx, w[(size_t)i * D + c]);
-    float den = 0.f;
-    for (int i = 0; i < m; ++i)
-        den += expf(w[(size_t)i * D + c] - mx);
+    extern __shared__ float bm_smem[];
+    float *sP = bm_smem;          // [m][32]
+    float *sRed = sP + m * 32;    // [8][32]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + lane;
+    bm_softmax_weights(w, D, m, sP, sRed);
     float pg = 0.f;
-    for (int i = 0; i < m; ++i)
-        pg += expf(w[(size_t)i * D + c] - mx) / den * G[(size_t)i * D + c];
-    for (int i = 0; i < m; ++i) {
-        const float pi = expf(w[(size_t)i * D + c] - mx) / den;
-        dw[(size_t)i * D + c] = pi * (G[(size_t)i * D + c] - pg);
-    }
+    for (int i = warp; i < m; i += 8)
+        pg += sP[i * 32 + lane] * G[(size_t)i * D + c];
+    sRed[warp * 32 + lane] = pg;
+    __syncthreads();
+    pg = 0.f;
+    for (int k = 0; k < 8; ++k)
+        pg += sRed[k * 32 + lane];
+    for (int i = warp; i < m; i += 8)
+        dw[(size_t)i * D + c] = sP[i * 32 + lane] * (G[(size_t)i * D + c] - pg);
 }
 
 // G: m * D floats of workspace, zeroed by the caller.
@@ -298,15 +349,19 @@ cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, in
         while ((rows + rpc - 1) / rpc > 65535)
             rpc += 8;
         const long long groups = (rows + rpc - 1) / rpc;
-        const size_t smem = (size_t)2 * m * 32 * sizeof(float);
+        const size_t smem = ((size_t)2 * m * 32 + 8 * 32) * sizeof(float);   // 66 KB at m = 256
+        cudaError_t e = cudaFuncSetAttribute(block_merge_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess)
+            return e;
         dim3 grid(D / 32, (unsigned)groups);
         block_merge_bwd_kernel<<<grid, 256, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x), w, dc, dx,
                                                             G, B, L, H, D, m, (int)rpc);
-        cudaError_t e = cudaGetLastError();
+        e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
     }
-    block_merge_dw_kernel<<<(D + 127) / 128, 128, 0, stream>>>(w, G, dw, D, m);
+    block_merge_dw_kernel<<<D / 32, 256, ((size_t)m * 32 + 8 * 32) * sizeof(float), stream>>>(w, G, dw, D, m);
     return cudaGetLastError();
 }
 

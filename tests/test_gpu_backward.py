@@ -45,6 +45,11 @@ def _close(name, got, ref, rmax, rmean):
     (1, 300, 32, 1, 128, 4, 64, 40),    # CSA, MQA, d = 128
     (2, 200, 4, 4, 128, 16, 32, 0),     # HCA, MHA
     (1, 90, 16, 1, 128, 4, 128, 6),     # L < W: window only for every query
+    # dense, d = 128: the tensor-core kernels (key-tile and query-tile passes)
+    (1, 300, 8, 2, 128, 4, 128, 0),     # GQA, 75 entries, ragged last tiles
+    (1, 700, 4, 1, 128, 2, 160, 0),     # MQA, 350 entries (3 key tiles), W > 128
+    (2, 260, 2, 2, 128, 8, 0, 0),       # no window: early rows see nothing
+    (1, 1100, 2, 1, 128, 4, 128, 0),    # 275 entries: several compressed chunks
 ])
 def test_attention_gradients_match_oracle(hb, B, L, Hq, Hkv, d, m, W, K):
     g = torch.Generator().manual_seed(100 + L + K)
