@@ -63,7 +63,8 @@ cudaError_t launch_hybrid_attn(int B, int Lq, int Lkv, int Hq, int Hkv, int d, i
 cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream);
 cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream);
 cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, int m, const float *w,
-                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream);
+                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream,
+                                   int num_sms);
 cudaError_t launch_gated_combine(const void *o1, const void *o2, const void *o3, const float *gate,
                                  void *o, long long rows, int d, cudaStream_t stream, int num_sms);
 
@@ -625,7 +626,7 @@ hyb_status hyb_hca_compress_bwd(const void *x, int B, int L, int H, int dx, int 
     cudaError_t e = cudaMemsetAsync(G, 0, (size_t)m * dx * sizeof(float), stream);
     if (e != cudaSuccess)
         return cuda_status(e);
-    return cuda_status(launch_block_merge_bwd(x, B, L, H, dx, m, w, dc, dx_acc, dw, G, stream));
+    return cuda_status(launch_block_merge_bwd(x, B, L, H, dx, m, w, dc, dx_acc, dw, G, stream, num_sms_current()));
 }
 
 size_t hyb_gated_workspace_size(const hyb_problem *p)

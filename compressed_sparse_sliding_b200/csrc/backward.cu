@@ -254,11 +254,49 @@ __device__ __forceinline__ void bm_softmax_weights(const float *__restrict__ w, 
     __syncthreads();
 }
 
-// grid (dx / 32, row groups of rpc rows); warp w of the CTA takes rows w,
-// w + 8, ... of its group; lane = channel.  Positions go 16 at a time: the
-// 16 rows' x and dx values are loaded together, dx written back, and the G
-// terms kept in registers over the warp's rows, then added to the CTA's G
-// partials in shared memory [m][32] (one atomic per position and lane).
+// grid (dx / 32, row groups of rpc rows, about two CTAs per SM in all); warp
+// w of the CTA takes rows w, w + 8, ... of its group; lane = channel.
+// Positions go 16 at a time and rows two at a time: the two rows' 32 x and
+// dx values are loaded together, dx written back, and the G terms kept in
+// registers over the warp's rows, then added to the CTA's G partials in
+// shared memory [m][32] (one atomic per position and lane).
+__device__ __forceinline__ void bm_rows16(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dc,
+                                          float *__restrict__ dx, const float *sP, int L, int H, int D, int m,
+                                          int Nc, long long r, int i0, int c, float (&gacc)[16], bool two)
+{
+    const int lane = threadIdx.x & 31;
+    const size_t istride = (size_t)H * D;
+    size_t x0[2];
+    float g[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const long long rr = r + 8 * q;
+        const int h = (int)(rr % H);
+        const long long bj = rr / H;
+        const int b = (int)(bj / Nc), j = (int)(bj % Nc);
+        const bool on = q == 0 || two;
+        g[q] = on ? dc[((size_t)bj * H + h) * D + c] : 0.f;
+        x0[q] = (((size_t)b * L + (size_t)j * m + i0) * H + h) * D + c;
+    }
+    float xv[2][16], dv[2][16];
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if ((q == 0 || two) && i0 + k < m) {
+                xv[q][k] = __bfloat162float(x[x0[q] + k * istride]);
+                dv[q][k] = dx[x0[q] + k * istride];
+            }
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            if ((q == 0 || two) && i0 + k < m) {
+                dx[x0[q] + k * istride] = dv[q][k] + sP[(i0 + k) * 32 + lane] * g[q];
+                gacc[k] += g[q] * xv[q][k];
+            }
+}
+
 __global__ void __launch_bounds__(256, 2)
 block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
                        const float *__restrict__ dc, float *__restrict__ dx, float *__restrict__ G,
@@ -276,34 +314,14 @@ block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restr
         sG[e] = 0.f;
     bm_softmax_weights(w, D, m, sP, sRed);
     const long long r0 = (long long)blockIdx.y * rpc;
-    const size_t istride = (size_t)H * D;
+    const long long rend = min(r0 + rpc, rows);
     for (int i0 = 0; i0 < m; i0 += 16) {
         float gacc[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
             gacc[k] = 0.f;
-        for (long long r = r0 + warp; r < r0 + rpc && r < rows; r += 8) {
-            const int h = (int)(r % H);
-            const long long bj = r / H;
-            const int b = (int)(bj / Nc), j = (int)(bj % Nc);
-            const float g = dc[((size_t)bj * H + h) * D + c];
-            const size_t xrow0 = (((size_t)b * L + (size_t)j * m + i0) * H + h) * D + c;
-            float xv[16], dv[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                if (i0 + k < m) {
-                    xv[k] = __bfloat162float(x[xrow0 + k * istride]);
-                    dv[k] = dx[xrow0 + k * istride];
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                if (i0 + k < m) {
-                    dx[xrow0 + k * istride] = dv[k] + sP[(i0 + k) * 32 + lane] * g;
-                    gacc[k] += g * xv[k];
-                }
-            }
-        }
+        for (long long r = r0 + warp; r < rend; r += 16)
+            bm_rows16(x, dc, dx, sP, L, H, D, m, Nc, r, i0, c, gacc, r + 8 < rend);
 #pragma unroll
         for (int k = 0; k < 16; ++k)
             if (i0 + k < m)
@@ -312,6 +330,119 @@ block_merge_bwd_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restr
     __syncthreads();
     for (int e = threadIdx.x; e < m * 32; e += 256)
         atomicAdd(&G[(size_t)(e / 32) * D + blockIdx.x * 32 + (e % 32)], sG[e]);
+}
+
+constexpr int kBmHeads = 8;   // heads of one position in flight per thread
+
+// Whole-block form (dx / 8 dividing 256, P, G and one block's dc in shared
+// memory): a work unit is one compression block (b, j) and a share of its m
+// positions; thread t takes channels 8 (t % CG) .. + 7 (CG = dx / 8) and
+// positions t / CG, + 256 / CG, ...; for each position it runs over the H
+// heads, so CG consecutive threads read 16 contiguous bytes each of x and 32
+// of dx (one 256- / 512-byte run at dx = 128).  Each thread owns its
+// (position, channel) G partials in shared memory; the CTA adds them to G
+// with vector reductions at the end.  Persistent: one CTA per SM.
+__global__ void __launch_bounds__(256, 1)
+block_merge_bwd_blocks_kernel(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
+                              const float *__restrict__ dc, float *__restrict__ dx, float *__restrict__ G,
+                              int B, int L, int H, int D, int m, int splits)
+{
+    extern __shared__ float bm_smem[];
+    float *sP = bm_smem;            // [m][D]
+    float *sG = sP + m * D;         // [m][D]
+    float *sDc = sG + m * D;        // [H][D]
+    const int CG = D / 8, PL = 256 / CG;
+    const int cg = threadIdx.x % CG, il = threadIdx.x / CG;
+    const int c0 = cg * 8;
+    const int Nc = L / m;
+    for (int c = threadIdx.x; c < D; c += 256) {
+        float mx = -INFINITY;
+        for (int i = 0; i < m; ++i)
+            mx = fmaxf(mx, w[(size_t)i * D + c]);
+        float den = 0.f;
+        for (int i = 0; i < m; ++i) {
+            const float e = expf(w[(size_t)i * D + c] - mx);
+            sP[i * D + c] = e;
+            den += e;
+        }
+        const float inv = 1.f / den;
+        for (int i = 0; i < m; ++i)
+            sP[i * D + c] *= inv;
+    }
+    for (int e = threadIdx.x; e < m * D; e += 256)
+        sG[e] = 0.f;
+    const int kpos = (m + PL - 1) / PL;               // positions per thread and block
+    const int kper = (kpos + splits - 1) / splits;    // of them per work unit
+    const long long units = (long long)B * Nc * splits;
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const long long bj = u / splits;
+        const int part = (int)(u % splits);
+        __syncthreads();   // the previous unit's sDc reads are done (and sP / sG are set)
+        for (int e = threadIdx.x * 4; e < H * D; e += 1024)
+            *reinterpret_cast<float4 *>(&sDc[e]) = *reinterpret_cast<const float4 *>(&dc[(size_t)bj * H * D + e]);
+        __syncthreads();
+        const int b = (int)(bj / Nc), j = (int)(bj % Nc);
+        for (int k = part * kper; k < min(kpos, (part + 1) * kper); ++k) {
+            const int i = il + PL * k;
+            if (i >= m)
+                break;
+            float pv[8], ga[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                pv[e] = sP[i * D + c0 + e];
+                ga[e] = 0.f;
+            }
+            const size_t base = ((size_t)b * L + (size_t)j * m + i) * H * D + c0;
+            for (int h0 = 0; h0 < H; h0 += kBmHeads) {
+                uint4 xr[kBmHeads];
+                float4 d0[kBmHeads], d1[kBmHeads];
+#pragma unroll
+                for (int q = 0; q < kBmHeads; ++q) {
+                    if (h0 + q < H) {
+                        const size_t at = base + (size_t)(h0 + q) * D;
+                        xr[q] = *reinterpret_cast<const uint4 *>(x + at);
+                        d0[q] = *reinterpret_cast<const float4 *>(dx + at);
+                        d1[q] = *reinterpret_cast<const float4 *>(dx + at + 4);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kBmHeads; ++q) {
+                    if (h0 + q < H) {
+                        const size_t at = base + (size_t)(h0 + q) * D;
+                        const float *g = &sDc[(h0 + q) * D + c0];
+                        const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+                        float xv[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[e]));
+                            xv[2 * e] = f.x;
+                            xv[2 * e + 1] = f.y;
+                        }
+                        float gv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            gv[e] = g[e];
+                            ga[e] += gv[e] * xv[e];
+                        }
+                        *reinterpret_cast<float4 *>(dx + at) =
+                            make_float4(d0[q].x + pv[0] * gv[0], d0[q].y + pv[1] * gv[1], d0[q].z + pv[2] * gv[2],
+                                        d0[q].w + pv[3] * gv[3]);
+                        *reinterpret_cast<float4 *>(dx + at + 4) =
+                            make_float4(d1[q].x + pv[4] * gv[4], d1[q].y + pv[5] * gv[5], d1[q].z + pv[6] * gv[6],
+                                        d1[q].w + pv[7] * gv[7]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                sG[i * D + c0 + e] += ga[e];
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x * 4; e < m * D; e += 1024)
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(G + e), "f"(sG[e]), "f"(sG[e + 1]),
+                     "f"(sG[e + 2]), "f"(sG[e + 3])
+                     : "memory");
 }
 
 // dw[i, c] = P[i, c] (G[i, c] - sum_k P[k, c] G[k, c]); a CTA per 32 channels,
@@ -340,14 +471,42 @@ block_merge_dw_kernel(const float *__restrict__ w, const float *__restrict__ G, 
 
 // G: m * D floats of workspace, zeroed by the caller.
 cudaError_t launch_block_merge_bwd(const void *x, int B, int L, int H, int D, int m, const float *w,
-                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream)
+                                   const float *dc, float *dx, float *dw, float *G, cudaStream_t stream,
+                                   int num_sms)
 {
     const long long rows = (long long)B * (L / m) * H;
-    if (rows > 0) {
-        // one row per warp where the grid allows, more rows per CTA beyond
-        long long rpc = 8;
+    const size_t bsmem = ((size_t)2 * m * D + (size_t)H * D) * sizeof(float);
+    const bool al16 = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dx) |
+                        reinterpret_cast<uintptr_t>(dc)) & 15u) == 0;
+    if (rows > 0 && al16 && D % 8 == 0 && 256 % (D / 8) == 0 && bsmem <= 200 * 1024) {
+        // whole-block form: about two work units per SM
+        const long long blocks = (long long)B * (L / m);
+        const int PL = 256 / (D / 8);
+        const int kpos = (m + PL - 1) / PL;
+        int splits = (int)((2LL * num_sms + blocks - 1) / blocks);
+        if (splits > kpos)
+            splits = kpos;
+        if (splits < 1)
+            splits = 1;
+        cudaError_t e = cudaFuncSetAttribute(block_merge_bwd_blocks_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem);
+        if (e != cudaSuccess)
+            return e;
+        const long long units = blocks * splits;
+        const int grid = (int)(units < num_sms ? units : num_sms);
+        block_merge_bwd_blocks_kernel<<<grid, 256, bsmem, stream>>>(static_cast<const __nv_bfloat16 *>(x), w, dc,
+                                                                    dx, G, B, L, H, D, m, splits);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    } else if (rows > 0) {
+        // rows per CTA: a multiple of 16 (two per warp and pass) giving about two
+        // CTAs per SM over all channel blocks, within the grid's y limit
+        const long long cblocks = D / 32;
+        long long rpc = (rows * cblocks + 2LL * num_sms - 1) / (2LL * num_sms);
+        rpc = (rpc + 15) / 16 * 16;
         while ((rows + rpc - 1) / rpc > 65535)
-            rpc += 8;
+            rpc += 16;
         const long long groups = (rows + rpc - 1) / rpc;
         const size_t smem = ((size_t)2 * m * 32 + 8 * 32) * sizeof(float);   // 66 KB at m = 256
         cudaError_t e = cudaFuncSetAttribute(block_merge_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -25,6 +25,13 @@
 // bf16(x - hi)), so the products carry ~16 bits of the fp32 values (one bf16
 // term alone would leave ~2^-9 relative error in every gradient).
 //
+// Timeline (hyb_trace_attach, CTA 0): the dK / dV kernel records roles 1
+// (producer: 1 K / V issued, 2 a unit's Q / dO issued and its columns stored),
+// 2 (MMA: 1 S^T and dP^T issued, 2 dV issued, 3 dK issued) and 3 (thread 0:
+// 1 S^T seen, 2 P written, 3 dS written, 4 epilogue start, 5 epilogue end);
+// the dQ kernel records role 0 (thread 0: 1 S seen, 3 dS written, 4 / 5 its
+// epilogue), so one attached buffer holds both kernels' timelines.
+//
 // Roles (320 threads): warps 0-3 and 4-7 are two warpgroups that each own
 // 64 of the 128 columns of S / dP (thread = TMEM lane = tile row), warp 8 is
 // the TMA producer, lane 0 of warp 9 issues every tcgen05.mma.  TMEM: S
@@ -58,9 +65,9 @@ struct BtParams {
     float *dkr, *dvr;   // [B, L, Hkv, 128], stored
 };
 
-// smem layout shared by both kernels: four 32 KB tiles (1024-aligned) and,
-// for the kv kernel, two more (the Q / dO ring), then per-stage lse / D
-// columns and the barriers.
+// smem layout shared by both kernels: six 32 KB tiles (1024-aligned), the
+// barriers, the kv kernel's per-stage lse / D columns and a 2 KB staging
+// area per softmax warp for coalesced gradient stores.
 struct BtSmem {
     static constexpr int OFF_T0 = 0;                 // kv: K     q: Q
     static constexpr int OFF_T1 = kBtTile;           // kv: V     q: dO
@@ -68,10 +75,11 @@ struct BtSmem {
     static constexpr int OFF_T3 = 3 * kBtTile;       // kv: dO[0] q: V[0]
     static constexpr int OFF_T4 = 4 * kBtTile;       // kv: Q[1]  q: K[1]
     static constexpr int OFF_T5 = 5 * kBtTile;       // kv: dO[1] q: V[1]
-    static constexpr int OFF_COL = 6 * kBtTile;      // kv: lse2[2][128], D[2][128]
-    static constexpr int OFF_BAR = OFF_COL + 4 * 128 * 4;
+    static constexpr int OFF_BAR = 6 * kBtTile;
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
-    static constexpr int BYTES = OFF_MISC + 16 * 4;
+    static constexpr int OFF_COL = OFF_MISC + 16 * 4;   // kv: lse2[2][128], D[2][128]
+    static constexpr int OFF_STAGE = OFF_COL + 4 * 128 * 4;   // 8 warps x 32 rows x 16 fp32
+    static constexpr int BYTES = OFF_STAGE + 8 * 32 * 16 * 4;
 };
 
 enum {
@@ -86,6 +94,41 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                  : "memory");
 }
 
+// Staged store of this warp's 32 rows x 16 consecutive fp32 columns: the
+// thread's v[0..15] (times f) go to a 2 KB area of shared memory (16-byte
+// chunks swizzled so that neither pass has bank conflicts), then every lane
+// moves one 16-byte chunk per pass, so a store instruction covers eight rows'
+// 64-byte segments instead of 32 rows' 16 bytes.  dst: the thread's row at
+// these columns, or nullptr (row not written); red: add instead of store.
+__device__ __forceinline__ void store_rows16(float *stage, const float *v, float *dst, float f, bool red)
+{
+    const int lane = threadIdx.x & 31;
+    float4 *st4 = reinterpret_cast<float4 *>(stage);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        st4[lane * 4 + (c ^ ((lane >> 1) & 3))] =
+            make_float4(v[4 * c] * f, v[4 * c + 1] * f, v[4 * c + 2] * f, v[4 * c + 3] * f);
+    __syncwarp();
+    const unsigned long long mine = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), c = lane & 3;
+        const float4 x = st4[r * 4 + (c ^ ((r >> 1) & 3))];
+        float *d = reinterpret_cast<float *>(__shfl_sync(0xffffffffu, mine, r));
+        if (d) {
+            if (red)
+                red_add_v4(d + 4 * c, x.x, x.y, x.z, x.w);
+            else
+                *reinterpret_cast<float4 *>(d + 4 * c) = x;
+        }
+    }
+    __syncwarp();
+}
+
+// P and dS enter the MMAs as bf16 hi terms only (kBtLo false) or as hi + lo
+// pairs (true): see the header.
+constexpr bool kBtLo = false;
+
 // Writes 32 fp32 values x[0..31] as a chunk of hi / lo bf16 pairs at TMEM
 // column taddr: hi pairs (x[2i], x[2i+1]) in columns 0-15, lo pairs in 16-31.
 __device__ __forceinline__ void tmem_st_hi_lo32(uint32_t taddr, const float *x)
@@ -94,12 +137,15 @@ __device__ __forceinline__ void tmem_st_hi_lo32(uint32_t taddr, const float *x)
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        const float2 hf = __bfloat1622float2(h);
         hi[i] = *reinterpret_cast<const uint32_t *>(&h);
-        lo[i] = pack_bf16x2(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+        if (kBtLo) {
+            const float2 hf = __bfloat1622float2(h);
+            lo[i] = pack_bf16x2(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+        }
     }
     tmem_st16(taddr, hi);
-    tmem_st16(taddr + 16, lo);
+    if (kBtLo)
+        tmem_st16(taddr + 16, lo);
 }
 
 // 64 consecutive fp32 TMEM columns of this thread's lane.
@@ -117,7 +163,7 @@ __device__ __forceinline__ void mma_hi_lo(uint32_t d_tmem, uint32_t a_tmem, uint
                                           bool first)
 {
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
+    for (int part = 0; part < (kBtLo ? 2 : 1); ++part) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t db = sw128_desc(b_saddr + kk * 16 * 128, 128 * 128, 1024);
@@ -228,9 +274,12 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     static_assert(SM::OFF_T4 - SM::OFF_T2 == 2 * kBtTile && SM::OFF_T5 - SM::OFF_T3 == 2 * kBtTile, "stage stride");
     float *sLse2 = reinterpret_cast<float *>(smem + SM::OFF_COL);         // [2][128]
     float *sDel = sLse2 + 2 * 128;                                        // [2][128]
+    float *const sStage = reinterpret_cast<float *>(smem + SM::OFF_STAGE) + (threadIdx.x >> 5) * 512;
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     volatile int *abort_flag = misc + 1;
+    unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
+    uint32_t tn = 0;                                  // this thread's trace records
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -284,16 +333,28 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 it.row0, it.b);
                 }
             }
+            if (lane == 0)
+                trace_ev(trb, tn, 1, 1, w, 0);
             ++nk;
             for (int u = it.u0; u < it.u1; ++u) {
                 const uint32_t s = qc & 1;
+                const int tq = it.tq0 + 128 * (u / p.g);
+                const int h = it.kvh * p.g + u % p.g;
+                // the unit's 128 columns, four per lane, loaded together before the
+                // stage wait: lse in base-2 units (+inf: no keys, or past L) and D
+                const size_t rowbase = ((size_t)it.b * p.Hq + h) * p.L;
+                float lv[4], dv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int t = min(tq + lane * 4 + k, p.L - 1);
+                    lv[k] = p.lse[rowbase + t];
+                    dv[k] = p.dq[(((size_t)it.b * p.L + t) * p.Hq + h) * 128];
+                }
                 if (qc >= 2 &&
                     !__all_sync(0xffffffffu, mbar_wait(&bar[BT_QE + s], ((qc >> 1) - 1) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
-                const int tq = it.tq0 + 128 * (u / p.g);
-                const int h = it.kvh * p.g + u % p.g;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bar[BT_QF + s], 2 * kBtTile);
                     for (int cb = 0; cb < 2; ++cb) {
@@ -301,22 +362,16 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         tma_load_4d(sDO0 + s * 2 * kBtTile + cb * 128 * 128, &tm_do, &bar[BT_QF + s], cb * 64, h, tq, it.b);
                     }
                 }
-                // the unit's 128 columns: lse in base-2 units (+inf: no keys, or past L) and D
-                const size_t rowbase = ((size_t)it.b * p.Hq + h) * p.L;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int c = lane * 4 + k;
-                    const int t = tq + c;
-                    float l2 = INFINITY, dl = 0.f;
-                    if (t < p.L) {
-                        const float l = p.lse[rowbase + t];
-                        l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-                        dl = p.dq[(((size_t)it.b * p.L + t) * p.Hq + h) * 128];
-                    }
-                    sLse2[s * 128 + c] = l2;
-                    sDel[s * 128 + c] = dl;
+                    const bool in = tq + c < p.L;
+                    sLse2[s * 128 + c] = !in || lv[k] == -INFINITY ? INFINITY : lv[k] * 1.4426950408889634f;
+                    sDel[s * 128 + c] = in ? dv[k] : 0.f;
                 }
                 mbar_arrive(&bar[BT_QF + s]);
+                if (lane == 0)
+                    trace_ev(trb, tn, 1, 2, w, u);
                 ++qc;
             }
         }
@@ -355,6 +410,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     mma_commit(&bar[BT_SF]);
                     mma_nt(tmem + TM_DP, aV, aDO0 + s * 2 * kBtTile, id_nt);     // dP^T = V dO^T
                     mma_commit(&bar[BT_DPF]);
+                    trace_ev(trb, tn, 2, 1, w, u);
                     if (!mbar_wait(&bar[BT_PF], qc & 1, abort_flag)) {
                         ok = false;
                         break;
@@ -365,6 +421,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     tc_fence_after();
                     mma_hi_lo(tmem + TM_DV, tmem + TM_S, aDO0 + s * 2 * kBtTile, id_mn, u == it.u0);    // dV += P^T dO
+                    trace_ev(trb, tn, 2, 2, w, u);
                     if (!mbar_wait(&bar[BT_DSF], qc & 1, abort_flag)) {
                         ok = false;
                         break;
@@ -372,6 +429,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_fence_after();
                     mma_hi_lo(tmem + TM_DK, tmem + TM_DP, aQ0 + s * 2 * kBtTile, id_mn, u == it.u0);    // dK += dS^T Q
                     mma_commit(&bar[BT_QE + s]);
+                    trace_ev(trb, tn, 2, 3, w, u);
                     ++qc;
                 }
                 if (!ok)
@@ -389,6 +447,7 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int quad = warp & 3;
         const int row = quad * 32 + lane;    // key row of the tile
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool tracer = threadIdx.x == 0;
         uint32_t nk = 0, qc = 0;
         bool ok = true;
         for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
@@ -419,6 +478,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     break;
                 }
                 tc_fence_after();
+                if (tracer)
+                    trace_ev(trb, tn, 3, 1, w, u);
                 float x[64];
                 tmem_ld64(tl + TM_S + 64 * wg, x);
                 const float4 *cl = reinterpret_cast<const float4 *>(sLse2 + s * 128 + 64 * wg);
@@ -438,6 +499,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bar[BT_PF]);
+                if (tracer)
+                    trace_ev(trb, tn, 3, 2, w, u);
                 if (!__all_sync(0xffffffffu, mbar_wait(&bar[BT_DPF], qc & 1, abort_flag))) {
                     ok = false;
                     break;
@@ -461,6 +524,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bar[BT_DSF]);
+                if (tracer)
+                    trace_ev(trb, tn, 3, 3, w, u);
                 ++qc;
             }
             if (!ok)
@@ -471,6 +536,8 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 break;
             }
             tc_fence_after();
+            if (tracer)
+                trace_ev(trb, tn, 3, 4, w, 0);
             float *dv_row, *dk_row;
             if (it.comp) {
                 const size_t at = (((size_t)it.b * p.Nc + kr) * p.Hkv + it.kvh) * 128 + 64 * wg;
@@ -483,23 +550,19 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
 #pragma unroll 1
             for (int part = 0; part < 2; ++part) {
+                // this half's 64 columns of dV, then of dK
                 float z[64];
                 tmem_ld64(tl + (part ? TM_DK : TM_DV) + 64 * wg, z);
                 const float f = part ? p.scale : 1.f;
-                float *dst = part ? dk_row : dv_row;
-                if (valid) {
+                float *dst = valid ? (part ? dk_row : dv_row) : nullptr;
 #pragma unroll
-                    for (int j = 0; j < 64; j += 4) {
-                        if (it.comp)
-                            red_add_v4(dst + j, z[j] * f, z[j + 1] * f, z[j + 2] * f, z[j + 3] * f);
-                        else
-                            *reinterpret_cast<float4 *>(dst + j) =
-                                make_float4(z[j] * f, z[j + 1] * f, z[j + 2] * f, z[j + 3] * f);
-                    }
-                }
+                for (int k = 0; k < 4; ++k)
+                    store_rows16(sStage, &z[16 * k], dst ? dst + 16 * k : nullptr, f, it.comp);
             }
             tc_fence_before();
             mbar_arrive(&bar[BT_OE]);
+            if (tracer)
+                trace_ev(trb, tn, 3, 5, w, 0);
             ++nk;
         }
     }
@@ -556,12 +619,15 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                                 ~(uintptr_t)1023);
     uint8_t *sQ = smem + SM::OFF_T0;
     uint8_t *sDO = smem + SM::OFF_T1;
+    float *const sStage = reinterpret_cast<float *>(smem + SM::OFF_STAGE) + (threadIdx.x >> 5) * 512;
     // stage s of the K / V ring: T2 / T3 + 2 s tiles
     uint8_t *const sK0 = smem + SM::OFF_T2;
     uint8_t *const sV0 = smem + SM::OFF_T3;
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + SM::OFF_BAR);
     int *misc = reinterpret_cast<int *>(smem + SM::OFF_MISC);
     volatile int *abort_flag = misc + 1;
+    unsigned long long *const trb = trace_buffer();   // timeline of CTA 0, when attached
+    uint32_t tn = 0;                                  // this thread's trace records
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -691,6 +757,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int quad = warp & 3;
         const int row = quad * 32 + lane;    // query row of the tile
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool tracer = threadIdx.x == 0;
         uint32_t ni = 0, kc = 0;
         bool ok = true;
         for (long long w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
@@ -736,6 +803,8 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     break;
                 }
                 tc_fence_after();
+                if (tracer)
+                    trace_ev(trb, tn, 0, 1, w, i);
                 float x[64];
                 tmem_ld64(tl + TM_S + 64 * wg, x);
 #pragma unroll
@@ -759,6 +828,8 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bar[BT_DSF]);
+                if (tracer)
+                    trace_ev(trb, tn, 0, 3, w, i);
                 ++kc;
             }
             if (!ok)
@@ -768,16 +839,17 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 break;
             }
             tc_fence_after();
+            if (tracer)
+                trace_ev(trb, tn, 0, 4, w, 0);
             float z[64];
             tmem_ld64(tl + TM_DQ + 64 * wg, z);
-            if (valid_row) {
 #pragma unroll
-                for (int j = 0; j < 64; j += 4)
-                    *reinterpret_cast<float4 *>(dq_row + j) =
-                        make_float4(z[j] * p.scale, z[j + 1] * p.scale, z[j + 2] * p.scale, z[j + 3] * p.scale);
-            }
+            for (int k = 0; k < 4; ++k)
+                store_rows16(sStage, &z[16 * k], valid_row ? dq_row + 16 * k : nullptr, p.scale, false);
             tc_fence_before();
             mbar_arrive(&bar[BT_OE]);
+            if (tracer)
+                trace_ev(trb, tn, 0, 5, w, 0);
             ++ni;
         }
     }
