@@ -21,9 +21,12 @@
 //   3. attn_bwd_q_kernel: one item per (query tile, head); per key tile S = Q K^T
 //      and dP = dO V^T, then dQ += dS K with dS from TMEM; dq stored once per
 //      row.
-// P and dS enter the MMAs as two bf16 terms each (hi = bf16(x), lo =
-// bf16(x - hi)), so the products carry ~16 bits of the fp32 values (one bf16
-// term alone would leave ~2^-9 relative error in every gradient).
+// P and dS enter the MMAs as bf16 (fp32 accumulation), like the forward's P:
+// rounding them leaves ~2^-9 relative error per term, which keeps the
+// gradients well inside the backward parity bounds (measured: worst case 0.41
+// of the max-abs and 0.38 of the mean-abs bound).  kBtLo = true adds a second
+// bf16 term lo = bf16(x - hi) per value (twice the P / dS MMAs and
+// conversions) for ~16-bit operands.
 //
 // Timeline (hyb_trace_attach, CTA 0): the dK / dV kernel records roles 1
 // (producer: 1 K / V issued, 2 a unit's Q / dO issued and its columns stored),
@@ -32,12 +35,16 @@
 // the dQ kernel records role 0 (thread 0: 1 S seen, 3 dS written, 4 / 5 its
 // epilogue), so one attached buffer holds both kernels' timelines.
 //
+// Gradient rows leave through a 2 KB staging area per softmax warp (16
+// columns x 32 rows, 64-byte swizzle), so one store instruction writes eight
+// rows' 64-byte segments.
+//
 // Roles (320 threads): warps 0-3 and 4-7 are two warpgroups that each own
 // 64 of the 128 columns of S / dP (thread = TMEM lane = tile row), warp 8 is
 // the TMA producer, lane 0 of warp 9 issues every tcgen05.mma.  TMEM: S
 // (columns 0-127), dP (128-255), and the accumulators (dV 256-383 and dK
 // 384-511, or dQ 256-383).  P (or dS) overwrites the columns it came from in
-// 32-column chunks, hi pairs then lo pairs:
+// 32-column chunks, hi pairs then (with kBtLo) lo pairs:
 //     element c (0..127) -> hi column 32 (c / 32) + (c % 32) / 2, lo column + 16,
 // so K-step kk of an MMA reads columns 32 (kk / 2) + 8 (kk % 2) (+ 16 for lo),
 // and a chunk is written as soon as its 32 values are final.
@@ -146,6 +153,18 @@ __device__ __forceinline__ void tmem_st_hi_lo32(uint32_t taddr, const float *x)
     tmem_st16(taddr, hi);
     if (kBtLo)
         tmem_st16(taddr + 16, lo);
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane, raw.
+__device__ __forceinline__ void tmem_ld16u(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
 }
 
 // 64 consecutive fp32 TMEM columns of this thread's lane.
@@ -506,18 +525,25 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     break;
                 }
                 tc_fence_after();
+                // dS = P (dP - D) with P read back from TMEM (the bf16 values the
+                // dV MMA uses), so P does not stay in registers across the wait
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     float y[32];
+                    uint32_t pk[16];
                     tmem_ld32(tl + TM_DP + 64 * wg + 32 * c, y);
+                    tmem_ld16u(tl + TM_S + 64 * wg + 32 * c, pk);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         const float4 d4 = cd[(32 * c + j) >> 2];
-                        y[j] = x[32 * c + j] * (y[j] - d4.x);
-                        y[j + 1] = x[32 * c + j + 1] * (y[j + 1] - d4.y);
-                        y[j + 2] = x[32 * c + j + 2] * (y[j + 2] - d4.z);
-                        y[j + 3] = x[32 * c + j + 3] * (y[j + 3] - d4.w);
+                        const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[j >> 1]));
+                        const float2 p1 =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[(j >> 1) + 1]));
+                        y[j] = p0.x * (y[j] - d4.x);
+                        y[j + 1] = p0.y * (y[j + 1] - d4.y);
+                        y[j + 2] = p1.x * (y[j + 2] - d4.z);
+                        y[j + 3] = p1.y * (y[j + 3] - d4.w);
                     }
                     tmem_st_hi_lo32(tl + TM_DP + 64 * wg + 32 * c, y);
                 }

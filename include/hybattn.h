@@ -231,7 +231,12 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
  * dq = scale sum_j dS_j k_j, dk_j += scale dS_j q, dv_j += P_j dout.
  * Outputs fp32, caller-owned, overwritten: dq [B, Lq, Hq, d]; dkc, dvc
  * [B, Nc, Hkv, d]; dk_raw, dv_raw [B, Lkv, Hkv, d] (the window path only:
- * the path through the compression is hyb_hca_compress_bwd's). */
+ * the path through the compression is hyb_hca_compress_bwd's).  Dense
+ * prefill problems (idx NULL, d = 128, q_pos and kv_pos0 NULL, Lq == Lkv) run
+ * on the tensor cores: a pass over key tiles for dk / dv and one over query
+ * tiles for dq, with P and dS rounded to bf16 as MMA operands (fp32
+ * accumulation); dq's memory holds dout.o of each row while the call runs.
+ * Every other problem runs an fp32 CUDA-core kernel. */
 hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
                         const int32_t *idx, const void *k_raw, const void *v_raw, const void *o,
                         const float *lse, const void *dout, float *dq, float *dkc, float *dvc,
@@ -243,7 +248,10 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
  * heads (P = softmax over positions of w, per channel).  dc [B, L/m, H, dx]
  * fp32; x bf16 as the forward; dx a multiple of 32, m <= 256.  ws: device
  * workspace of hyb_hca_compress_bwd_workspace_size(dx, m) bytes, 256-byte
- * aligned. */
+ * aligned.  With x, dc and dx_acc 16-byte aligned and the softmax weights,
+ * the G partials and one block of dc fitting in shared memory, one pass
+ * walks whole compression blocks (contiguous rows of every head); otherwise
+ * a pass per 32 channels. */
 size_t hyb_hca_compress_bwd_workspace_size(int dx, int m);
 hyb_status hyb_hca_compress_bwd(const void *x, int B, int L, int H, int dx, int m, const float *w,
                                 const float *dc, float *dx_acc, float *dw, void *ws, size_t ws_bytes,
