@@ -162,6 +162,8 @@ hca_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_vr, const DenseParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     using SM = DenseSmem<D>;
     constexpr int NCB = D / 64;
     extern __shared__ __align__(1024) uint8_t dn_smem_raw[];
@@ -603,8 +605,7 @@ static cudaError_t launch_hca_t(const DenseParams &p, const void *q, const void 
         grid = p.n_items;
     if (grid < 1)
         return cudaSuccess;
-    kern<<<(unsigned)grid, kDnThreads, smem, stream>>>(mq, mkc, mvc, mkr, mvr, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kDnThreads), smem, stream, mq, mkc, mvc, mkr, mvr, p);
 }
 
 // Prefill HCA: idx == NULL, positions 0..L-1, raw rows 0..L-1.

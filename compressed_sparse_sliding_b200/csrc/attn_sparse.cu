@@ -376,6 +376,8 @@ csa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_vr, const SparseParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     using SM = SparseSmem<NH>;
     constexpr int KS = SM::KS;
     constexpr int VS = SM::VS;
@@ -1483,15 +1485,17 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
         long long grid = slots < p.n_items ? slots : p.n_items;
         if (grid < 1)
             return cudaSuccess;
-        kern<<<(unsigned)grid, SpRoles<NH>::THREADS, smem, stream>>>(mq, mkc, mvc, mkr, mvr, p);
-        return cudaGetLastError();
+        return launch_pdl(kern, dim3((unsigned)grid), dim3(SpRoles<NH>::THREADS), smem, stream, mq, mkc, mvc, mkr,
+                          mvr, p);
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 2;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(SpRoles<NH>::THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1506,6 +1510,7 @@ static cudaError_t launch_csa_t(SparseParams p, const void *q, const void *kc, c
         return cudaErrorLaunchOutOfResources;
     const long long clusters = max_clusters < p.n_items ? max_clusters : p.n_items;
     cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, mq, mkc, mvc, mkr, mvr, p);
 }
 

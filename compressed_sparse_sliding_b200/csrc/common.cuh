@@ -154,6 +154,45 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel of the forward chain (compression,
+// indexer, top-K, attention, decode append) is launched with programmatic
+// stream serialization and starts with pdl_wait(), which returns once the
+// previous kernel in the stream has completed and its writes are visible (at
+// once for a normal launch), then pdl_trigger(), which lets the next kernel's
+// blocks launch while this one runs its last blocks: they sit in their own
+// pdl_wait() instead of paying the launch gap afterwards.  Nothing touches
+// global memory before pdl_wait(), so stream order holds exactly.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// kern<<<grid, block, smem, stream>>>(args...) as a programmatic dependent
+// launch (see pdl_wait).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters: rank, full-cluster barrier, distributed shared memory
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank()

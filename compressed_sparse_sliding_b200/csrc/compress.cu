@@ -178,6 +178,8 @@ __global__ void __launch_bounds__(kMergeThreads)
 block_merge_regs(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ w,
                  __nv_bfloat16 *__restrict__ out, int B, int L, int H, int dx, int m, int S)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     extern __shared__ __align__(16) float sm_rg[];
     const int tid = threadIdx.x;
     const int ipc = kMergeThreads / S;
@@ -395,10 +397,9 @@ static cudaError_t launch_merge_regs(const void *x, int B, int L, int H, int dx,
     long long grid = (long long)num_sms * per_sm;
     if (grid > ntiles)
         grid = ntiles;
-    block_merge_regs<NPOS><<<(unsigned)grid, kMergeThreads, smem, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), w, static_cast<__nv_bfloat16 *>(out), B, L, H, dx, m,
-        S);
-    return cudaGetLastError();
+    return launch_pdl(block_merge_regs<NPOS>, dim3((unsigned)grid), dim3(kMergeThreads), smem, stream,
+                      static_cast<const __nv_bfloat16 *>(x), w, static_cast<__nv_bfloat16 *>(out), B, L, H, dx,
+                      m, S);
 }
 
 // Launch helper: picks the position split S and a persistent grid.

@@ -53,6 +53,8 @@ __device__ __forceinline__ uint32_t ap_fp4_code(float x, float mn, float sc)
 __global__ void __launch_bounds__(kApThreads)
 decode_append_fp4_kernel(const AppendParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     const int b = blockIdx.x;
     const long long t = p.t_new[b];
     if (t < 0) {
@@ -172,6 +174,8 @@ decode_append_fp4_kernel(const AppendParams p)
 __global__ void __launch_bounds__(kApThreads)
 decode_append_kernel(const AppendParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     const int b = blockIdx.x;
     const long long t = p.t_new[b];
     if (t < 0) {
@@ -252,10 +256,8 @@ cudaError_t launch_decode_append(const AppendParams &p, cudaStream_t stream)
     if (p.B <= 0)
         return cudaSuccess;
     if (p.kcq)
-        decode_append_fp4_kernel<<<p.B, kApThreads, 0, stream>>>(p);
-    else
-        decode_append_kernel<<<p.B, kApThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_pdl(decode_append_fp4_kernel, dim3(p.B), dim3(kApThreads), 0, stream, p);
+    return launch_pdl(decode_append_kernel, dim3(p.B), dim3(kApThreads), 0, stream, p);
 }
 
 }  // namespace hyb

@@ -190,6 +190,8 @@ __global__ void __launch_bounds__(kFxThreads, 1)
 index_topk_fused(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const FusedIndexParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     using SM = FxSmem<HI, DI>;
     using LY = FxLayout<DI>;
     extern __shared__ __align__(1024) uint8_t fx_smem_raw[];
@@ -886,8 +888,7 @@ static cudaError_t launch_fx_t(const FusedIndexParams &p, const void *qi, const 
     if (e != cudaSuccess)
         return e;
     const unsigned grid = (unsigned)p.n_ttiles * (unsigned)p.B;
-    kern<<<grid, kFxThreads, smem, stream>>>(mq, mk, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kFxThreads), smem, stream, mq, mk, p);
 }
 
 // Shapes the fused kernel takes: query tiles of many rows (not the decode

@@ -397,6 +397,8 @@ __global__ void __launch_bounds__(DecRoles<Q4>::THREADS, 1)
 index_scores_dec(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const DecIndexParams p)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     using RL = DecRoles<Q4>;
     constexpr int Q_BYTES = RL::Q_BYTES;
     constexpr int K_BYTES = RL::K_BYTES;
@@ -630,14 +632,19 @@ static cudaError_t launch_index_dec(const void *qi, const float *wi, const void 
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
-        index_scores_dec<true><<<grid, DecRoles<true>::THREADS, smem, stream>>>(mq, mk, p);
+        e = launch_pdl(index_scores_dec<true>, dim3(grid), dim3(DecRoles<true>::THREADS), smem, stream, mq, mk, p);
+        if (e != cudaSuccess)
+            return e;
     } else {
         const size_t smem = DecRoles<false>::SMEM;
         cudaError_t e = cudaFuncSetAttribute(index_scores_dec<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return e;
-        index_scores_dec<false><<<grid, DecRoles<false>::THREADS, smem, stream>>>(mq, mk, p);
+        e = launch_pdl(index_scores_dec<false>, dim3(grid), dim3(DecRoles<false>::THREADS), smem, stream, mq, mk,
+                       p);
+        if (e != cudaSuccess)
+            return e;
     }
     return cudaGetLastError();
 }

@@ -453,6 +453,8 @@ topk_hist(const float *__restrict__ scores, int Lq, int Nc, int m, int W, int K,
           const int32_t *__restrict__ q_pos, int32_t *__restrict__ idx_out,
           float *__restrict__ sel_scores)
 {
+    pdl_wait();      // launched as a programmatic dependent: the previous kernel's writes
+    pdl_trigger();   // are visible from here on; the next kernel may start its launch
     constexpr int PER = kHbBins / NT;          // bins per thread in the descending scan
     static_assert(PER >= 1 && kHbBins % NT == 0, "");
     __shared__ int hist[2][kHbBins];
@@ -625,8 +627,8 @@ cudaError_t launch_topk_radix(const float *scores, int B, int Lq, int Nc, int m,
     const unsigned rows = (unsigned)B * (unsigned)Lq;
 #define HYB_TOPK_HIST(NT, KPT)                                                                     \
     do {                                                                                        \
-        topk_hist<NT, KPT><<<rows, NT, 0, stream>>>(scores, Lq, Nc, m, W, K, q_pos, idx, sel_scores); \
-        return cudaGetLastError();                                                              \
+        return launch_pdl(topk_hist<NT, KPT>, dim3(rows), dim3(NT), 0, stream, scores, Lq, Nc, m, W, K,  \
+                          q_pos, idx, sel_scores);                                              \
     } while (0)
     if (Nc <= 512 * 8)
         HYB_TOPK_HIST(512, 8);
