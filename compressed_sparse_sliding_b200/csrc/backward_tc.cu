@@ -177,31 +177,37 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64])
 
 // 2 x 8 MMAs: D (+)= A_hi B + A_lo B, A in TMEM at column a_tmem (hi / lo
 // chunks above), B a 128-row tile in shared memory read MN-major (rows = K
-// index).
-__device__ __forceinline__ void mma_hi_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_saddr, uint32_t idesc,
+// index).  b_desc0: the tile's descriptor (LBO 16 KB, SBO 1 KB); the K steps
+// advance its address field by 16 rows (2 KB) each, computed once per call so
+// that the issuing thread spends a 64-bit add per MMA.
+__device__ __forceinline__ void mma_hi_lo(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc0, uint32_t idesc,
                                           bool first)
 {
 #pragma unroll
     for (int part = 0; part < (kBtLo ? 2 : 1); ++part) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t db = sw128_desc(b_saddr + kk * 16 * 128, 128 * 128, 1024);
-            mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * part, db, idesc,
-                        (first && part == 0 && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * part, b_desc0 + (uint64_t)(kk * 128),
+                        idesc, (first && part == 0 && kk == 0) ? 0u : 1u);
     }
 }
 
-// 8 MMAs: D = A B^T over K = 128, both 128-row tiles K-major in shared memory.
-__device__ __forceinline__ void mma_nt(uint32_t d_tmem, uint32_t a_saddr, uint32_t b_saddr, uint32_t idesc)
+// 8 MMAs: D = A B^T over K = 128, both 128-row tiles K-major in shared memory
+// (descriptors of the tiles' starts; K step kk moves 32 bytes inside the
+// swizzle atom, and the second 64-channel half starts 16 KB on).
+__device__ __forceinline__ void mma_nt(uint32_t d_tmem, uint64_t a_desc0, uint64_t b_desc0, uint32_t idesc)
 {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-        mma_bf16_ss(d_tmem, sw128_desc(a_saddr + off, 16, 1024), sw128_desc(b_saddr + off, 16, 1024), idesc,
-                    kk > 0 ? 1u : 0u);
+        const uint64_t off = (uint64_t)(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4);
+        mma_bf16_ss(d_tmem, a_desc0 + off, b_desc0 + off, idesc, kk > 0 ? 1u : 0u);
     }
 }
+
+// Descriptors of a 128-row bf16 tile at shared address a: K-major (A or B of
+// mma_nt) and MN-major (B of mma_hi_lo).
+__device__ __forceinline__ uint64_t tile_desc_k(uint32_t a) { return sw128_desc(a, 16, 1024); }
+__device__ __forceinline__ uint64_t tile_desc_mn(uint32_t a) { return sw128_desc(a, 128 * 128, 1024); }
 
 // ------------------------------------------------------------------ launch 1
 // D of row r = (b, t, h): sum_c dO[r, c] o[r, c] (fp32 over the bf16 values),
@@ -425,9 +431,9 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    mma_nt(tmem + TM_S, aK, aQ0 + s * 2 * kBtTile, id_nt);       // S^T = K Q^T
+                    mma_nt(tmem + TM_S, tile_desc_k(aK), tile_desc_k(aQ0 + s * 2 * kBtTile), id_nt);       // S^T = K Q^T
                     mma_commit(&bar[BT_SF]);
-                    mma_nt(tmem + TM_DP, aV, aDO0 + s * 2 * kBtTile, id_nt);     // dP^T = V dO^T
+                    mma_nt(tmem + TM_DP, tile_desc_k(aV), tile_desc_k(aDO0 + s * 2 * kBtTile), id_nt);     // dP^T = V dO^T
                     mma_commit(&bar[BT_DPF]);
                     trace_ev(trb, tn, 2, 1, w, u);
                     if (!mbar_wait(&bar[BT_PF], qc & 1, abort_flag)) {
@@ -439,14 +445,14 @@ attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    mma_hi_lo(tmem + TM_DV, tmem + TM_S, aDO0 + s * 2 * kBtTile, id_mn, u == it.u0);    // dV += P^T dO
+                    mma_hi_lo(tmem + TM_DV, tmem + TM_S, tile_desc_mn(aDO0 + s * 2 * kBtTile), id_mn, u == it.u0);    // dV += P^T dO
                     trace_ev(trb, tn, 2, 2, w, u);
                     if (!mbar_wait(&bar[BT_DSF], qc & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    mma_hi_lo(tmem + TM_DK, tmem + TM_DP, aQ0 + s * 2 * kBtTile, id_mn, u == it.u0);    // dK += dS^T Q
+                    mma_hi_lo(tmem + TM_DK, tmem + TM_DP, tile_desc_mn(aQ0 + s * 2 * kBtTile), id_mn, u == it.u0);    // dK += dS^T Q
                     mma_commit(&bar[BT_QE + s]);
                     trace_ev(trb, tn, 2, 3, w, u);
                     ++qc;
@@ -750,9 +756,9 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         break;
                     }
                     tc_fence_after();
-                    mma_nt(tmem + TM_S, aQ, aK0 + s * 2 * kBtTile, id_nt);       // S = Q K^T
+                    mma_nt(tmem + TM_S, tile_desc_k(aQ), tile_desc_k(aK0 + s * 2 * kBtTile), id_nt);       // S = Q K^T
                     mma_commit(&bar[BT_SF]);
-                    mma_nt(tmem + TM_DP, aDO, aV0 + s * 2 * kBtTile, id_nt);     // dP = dO V^T
+                    mma_nt(tmem + TM_DP, tile_desc_k(aDO), tile_desc_k(aV0 + s * 2 * kBtTile), id_nt);     // dP = dO V^T
                     mma_commit(&bar[BT_DPF]);
                     if (i == nt - 1)
                         mma_commit(&bar[BT_QE]);
@@ -765,7 +771,7 @@ attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         break;
                     }
                     tc_fence_after();
-                    mma_hi_lo(tmem + TM_DQ, tmem + TM_S, aK0 + s * 2 * kBtTile, id_mn, i == 0);   // dQ += dS K
+                    mma_hi_lo(tmem + TM_DQ, tmem + TM_S, tile_desc_mn(aK0 + s * 2 * kBtTile), id_mn, i == 0);   // dQ += dS K
                     mma_commit(&bar[BT_KVE + s]);
                     ++kc;
                 }

@@ -109,3 +109,61 @@ def test_hca_attention_timeline(hb):
         assert ev.count((1, 1)) == ev.count((1, 2)) >= 1
         for role, qk, pv in ((3, (2, 1), (2, 2)), (0, (2, 3), (2, 4))):
             assert ev.count(qk) == ev.count(pv) == ev.count((role, 1)) == ev.count((role, 2)) >= 1
+
+
+def test_attention_backward_timeline(hb):
+    # tensor-core backward of a dense problem: the key-tile pass records roles
+    # 1-3 (producer, MMA, softmax thread 0), the query-tile pass role 0
+    g = torch.Generator().manual_seed(79)
+    B, L, Hq, Hkv, d, m, W = 1, 600, 2, 1, 128, 4, 128
+    Nc = L // m
+    q = torch.randn((B, L, Hq, d), generator=g).to(torch.bfloat16).cuda()
+    kv = [torch.randn((B, L, Hkv, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
+    kc = [torch.randn((B, Nc, Hkv, d), generator=g).to(torch.bfloat16).cuda() for _ in range(2)]
+    dout = torch.randn((B, L, Hq, d), generator=g).to(torch.bfloat16).cuda()
+    p = hb.problem(B=B, Lq=L, Lkv=L, Hq=Hq, Hkv=Hkv, d=d, m=m, W=W, Nc=Nc)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device="cuda")
+    o = hb.hyb_attn_fwd(p, q, kc[0], kc[1], None, kv[0], kv[1], lse=lse)
+    ref = hb.hyb_attn_bwd(p, q, kc[0], kc[1], None, kv[0], kv[1], o, lse, dout)
+    buf = torch.zeros(1 << 20, dtype=torch.int64, device="cuda")
+    hb.hyb_trace_attach(buf)
+    try:
+        got = hb.hyb_attn_bwd(p, q, kc[0], kc[1], None, kv[0], kv[1], o, lse, dout)
+        torch.cuda.synchronize()
+    finally:
+        hb.hyb_trace_attach(None)
+    assert hb.hyb_get_device_status() == hb.HYB_OK
+    for name in ("dq", "dk_raw", "dv_raw"):
+        assert torch.equal(got[name], ref[name]), name
+    # dkc / dvc take reductions from several blocks: equal up to their order
+    for name in ("dkc", "dvc"):
+        assert torch.allclose(got[name], ref[name], rtol=1e-5, atol=1e-5), name
+    rec = hb.trace_records(buf)
+    words = buf.cpu().numpy().view("uint64")
+    cap = (words.size - 4) // 8
+    for role in (0, 1, 2, 3):
+        n = int(words[role])
+        assert 0 < n <= cap, f"role {role}: {n} records"
+        base = 4 + 2 * role * cap
+        clk = words[base:base + 2 * n:2].astype(np.int64)
+        assert np.all((words[base + 1:base + 2 * n:2] >> 56) == role)
+        assert np.all(np.diff(clk) >= 0), f"role {role}: clocks out of order"
+    kv_items = sorted({r["item"] for r in rec if r["role"] in (1, 2, 3)})
+    for it in kv_items:
+        ev = [(r["role"], r["event"], r["tile"]) for r in rec if r["item"] == it]
+        units = sorted({u for role, e, u in ev if role == 2 and e == 1})
+        assert units, f"item {it}: no unit issued"
+        for u in units:
+            # per unit: columns staged, S^T / dP^T, dV and dK issued; P and dS written
+            for key in ((1, 2), (2, 1), (2, 2), (2, 3), (3, 1), (3, 2), (3, 3)):
+                assert (key[0], key[1], u) in ev, f"item {it} unit {u}: event {key} missing"
+        # one epilogue per item, after its last dS
+        ep = [r["clock"] for r in rec if r["item"] == it and r["role"] == 3 and r["event"] == 4]
+        last_ds = max(r["clock"] for r in rec if r["item"] == it and r["role"] == 3 and r["event"] == 3)
+        assert len(ep) == 1 and ep[0] >= last_ds
+    # the query-tile pass: every S seen is followed by its dS, and each item
+    # closes with one epilogue
+    q_rec = [r for r in rec if r["role"] == 0]
+    for it in sorted({r["item"] for r in q_rec}):
+        ev = [r["event"] for r in q_rec if r["item"] == it]
+        assert ev.count(1) == ev.count(3) >= 1 and ev.count(4) == ev.count(5) == 1
