@@ -60,8 +60,8 @@ struct BtParams {
     int nqt;            // ceil(L / 128): query tiles (q kernel)
     int nkt_c;          // ceil(Nc / 128): compressed key tiles
     int nkt_r;          // ceil(L / 128) raw key tiles, 0 without a window
-    int chunk;          // units per compressed item
-    int max_chunks;     // items of compressed key tile 0
+    int chunk_qt;       // query tiles per compressed item (chunk c: tiles c chunk_qt ..)
+    int max_chunks;     // ceil(nqt / chunk_qt)
     int nqw;            // query tiles per raw key tile
     long long n_comp_items, n_items;
     float scale, scale_log2;
@@ -243,28 +243,33 @@ struct BtKvItem {
     bool comp;
 };
 
-// Items: first every (b, kvh, compressed key tile, chunk), chunks innermost
-// (a chunk past the tile's units is empty), then every (b, kvh, raw key tile).
+// Items: first every (b, kvh, chunk, compressed key tile), key tiles
+// innermost: a chunk is the same run of 128-aligned query tiles for every key
+// tile (the part each one sees), so the key tiles of a chunk run side by side
+// and read the same Q / dO tiles through L2; an empty part is an empty item.
+// Then every (b, kvh, raw key tile).
 __device__ __forceinline__ BtKvItem bt_kv_item(const BtParams &p, long long w)
 {
     // item counts and positions fit in 32 bits (the launcher checks)
     BtKvItem it;
     if (w < p.n_comp_items) {
         unsigned wu = (unsigned)w;
-        const int chunk = (int)(wu % (unsigned)p.max_chunks);
-        wu /= (unsigned)p.max_chunks;
         const int kt = (int)(wu % (unsigned)p.nkt_c);
         wu /= (unsigned)p.nkt_c;
+        const int chunk = (int)(wu % (unsigned)p.max_chunks);
+        wu /= (unsigned)p.max_chunks;
         it.kvh = (int)(wu % (unsigned)p.Hkv);
         it.b = (int)(wu / (unsigned)p.Hkv);
         it.comp = true;
         it.row0 = kt * 128;
         // the first query that sees entry row0: (row0 + 1) m - 1 < t - W + 1
         const int tmin = (it.row0 + 1) * p.m - 1 + p.W;
-        const int units = tmin < p.L ? ((p.L - tmin + 127) / 128) * p.g : 0;
-        it.tq0 = tmin;
-        it.u0 = min(chunk * p.chunk, units);
-        it.u1 = min(it.u0 + p.chunk, units);
+        const int qt_first = tmin < p.L ? tmin / 128 : p.nqt;
+        const int qa = max(qt_first, chunk * p.chunk_qt);
+        const int qb = min(p.nqt, (chunk + 1) * p.chunk_qt);
+        it.tq0 = qa * 128;
+        it.u0 = 0;
+        it.u1 = qb > qa ? (qb - qa) * p.g : 0;
     } else {
         unsigned wu = (unsigned)(w - p.n_comp_items);
         const int kt = (int)(wu % (unsigned)p.nkt_r);
@@ -935,11 +940,13 @@ static cudaError_t launch_attn_bwd_tc(int B, int L, int Hq, int Hkv, int Nc, int
         total_cu += u;
     }
     total_cu *= (long long)B * Hkv;
-    long long chunk = (total_cu + 2LL * num_sms - 1) / (2LL * num_sms);
+    // about four compressed items per SM (they are the long ones), at least
+    // four units each
+    long long chunk = (total_cu + 4LL * num_sms - 1) / (4LL * num_sms);
     if (chunk < 4)
         chunk = 4;
-    p.chunk = (int)chunk;
-    p.max_chunks = units0 > 0 ? (int)((units0 + chunk - 1) / chunk) : 0;
+    p.chunk_qt = (int)((chunk + p.g - 1) / p.g);
+    p.max_chunks = (p.nqt + p.chunk_qt - 1) / p.chunk_qt;
     p.n_comp_items = units0 > 0 ? (long long)B * Hkv * p.nkt_c * p.max_chunks : 0;
     p.n_items = p.n_comp_items + (long long)B * Hkv * p.nkt_r;
     const long long n_q_items = (long long)p.nqt * B * Hq;
