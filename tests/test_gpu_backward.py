@@ -53,6 +53,8 @@ def _close(name, got, ref, rmax, rmean):
     (1, 700, 4, 1, 128, 2, 160, 0),     # MQA, 350 entries (3 key tiles), W > 128
     (2, 260, 2, 2, 128, 8, 0, 0),       # no window: early rows see nothing
     (1, 1100, 2, 1, 128, 4, 128, 0),    # 275 entries: several compressed chunks
+    (1, 260, 2, 1, 128, 1, 0, 0),       # m = 1, no window: plain causal attention, all through entries
+    (1, 520, 16, 2, 128, 128, 128, 0),  # eight query heads per KV head, 4 entries of 128 tokens
 ])
 def test_attention_gradients_match_oracle(hb, B, L, Hq, Hkv, d, m, W, K):
     g = torch.Generator().manual_seed(100 + L + K)
