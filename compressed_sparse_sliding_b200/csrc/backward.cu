@@ -12,7 +12,8 @@
 // without a head (groups of fewer than eight) only take part in the sums.  Keys go
 // four at a time: each warp adds its heads' dk / dv parts into shared
 // memory, then the CTA adds the keys' sums to the fp32 gradients with one
-// atomic per element.  CUDA cores throughout: a correct first form.
+// vector reduction per four channels (the form for problems the tensor-core
+// passes do not take: CSA selections, d = 64, decode positions).
 //
 // block_merge, c_j = sum_i P[i] x_{jm+i} with P = softmax over i of w (per
 // channel):  dx_{jm+i} += P[i] dc_j  (each raw row belongs to one block, so
@@ -94,8 +95,8 @@ attn_bwd_kernel(const BwdParams p)
         lse[e] = on ? p.lse[((size_t)b * p.Hq + (size_t)kvh * p.g + h) * p.Lq + t] : -INFINITY;
     }
 
-    __shared__ float sdk[kBwKeys][kBwWarps][128];
-    __shared__ float sdv[kBwKeys][kBwWarps][128];
+    __shared__ __align__(16) float sdk[kBwKeys][kBwWarps][128];
+    __shared__ __align__(16) float sdv[kBwKeys][kBwWarps][128];
     __shared__ long long srow[kBwKeys];     // source row of each key (-1: none)
     __shared__ int scomp[kBwKeys];          // compressed (1) or raw (0)
     const int total = ncomp + nwin;
@@ -166,19 +167,28 @@ attn_bwd_kernel(const BwdParams p)
             }
         }
         __syncthreads();
-        // thread -> (key, channel) sums over the warps, one atomic each
-        for (int e = threadIdx.x; e < kBwKeys * d; e += 32 * kBwWarps) {
-            const int u = e / d, c = e % d;
+        // thread -> (key, four channels) sums over the warps, one vector
+        // reduction each for dk and dv
+        for (int e = threadIdx.x; e < kBwKeys * d / 4; e += 32 * kBwWarps) {
+            const int u = e / (d / 4), c = (e % (d / 4)) * 4;
             const long long r = srow[u];
             if (r < 0)
                 continue;
-            float sk = 0.f, sv = 0.f;
+            float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
             for (int w = 0; w < nw; ++w) {
-                sk += sdk[u][w][c];
-                sv += sdv[u][w][c];
+                const float4 a = *reinterpret_cast<const float4 *>(&sdk[u][w][c]);
+                const float4 b = *reinterpret_cast<const float4 *>(&sdv[u][w][c]);
+                sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+                sv.x += b.x; sv.y += b.y; sv.z += b.z; sv.w += b.w;
             }
-            atomicAdd((scomp[u] ? p.dkc : p.dkr) + r * d + c, sk * p.scale);
-            atomicAdd((scomp[u] ? p.dvc : p.dvr) + r * d + c, sv);
+            float *dk = (scomp[u] ? p.dkc : p.dkr) + r * d + c;
+            float *dv = (scomp[u] ? p.dvc : p.dvr) + r * d + c;
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dk), "f"(sk.x * p.scale),
+                         "f"(sk.y * p.scale), "f"(sk.z * p.scale), "f"(sk.w * p.scale)
+                         : "memory");
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dv), "f"(sv.x), "f"(sv.y),
+                         "f"(sv.z), "f"(sv.w)
+                         : "memory");
         }
         __syncthreads();
     }
