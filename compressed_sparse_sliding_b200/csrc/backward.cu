@@ -28,7 +28,7 @@
 namespace hyb {
 
 constexpr int kBwWarps = 8;
-constexpr int kBwKeys = 4;      // keys per shared-memory round (2 x 16 KB of partials)
+// Keys per shared-memory round: NK (4 or 8), partials 2 x NK x 4 KB in dynamic shared memory.
 
 struct BwdParams {
     int B, Lq, Lkv, Hq, Hkv, g, d, Nc, m, W, topk;
@@ -47,7 +47,7 @@ __device__ __forceinline__ float bw_warp_sum(float v)
     return v;
 }
 
-template <int CPL, int HPW>
+template <int CPL, int HPW, int NK>
 __global__ void __launch_bounds__(32 * kBwWarps)
 attn_bwd_kernel(const BwdParams p)
 {
@@ -95,14 +95,15 @@ attn_bwd_kernel(const BwdParams p)
         lse[e] = on ? p.lse[((size_t)b * p.Hq + (size_t)kvh * p.g + h) * p.Lq + t] : -INFINITY;
     }
 
-    __shared__ __align__(16) float sdk[kBwKeys][kBwWarps][128];
-    __shared__ __align__(16) float sdv[kBwKeys][kBwWarps][128];
-    __shared__ long long srow[kBwKeys];     // source row of each key (-1: none)
-    __shared__ int scomp[kBwKeys];          // compressed (1) or raw (0)
+    extern __shared__ __align__(16) float bw_partials[];
+    float(*sdk)[kBwWarps][128] = reinterpret_cast<float(*)[kBwWarps][128]>(bw_partials);   // [NK][warps][128]
+    float(*sdv)[kBwWarps][128] = reinterpret_cast<float(*)[kBwWarps][128]>(bw_partials + NK * kBwWarps * 128);
+    __shared__ long long srow[NK];     // source row of each key (-1: none)
+    __shared__ int scomp[NK];          // compressed (1) or raw (0)
     const int total = ncomp + nwin;
     const int nw = p.g < kBwWarps ? p.g : kBwWarps;   // warps holding a head
-    for (int k0 = 0; k0 < total; k0 += kBwKeys) {
-        if (threadIdx.x < kBwKeys) {
+    for (int k0 = 0; k0 < total; k0 += NK) {
+        if (threadIdx.x < NK) {
             const int kk = k0 + threadIdx.x;
             long long r = -1;
             int comp = 0;
@@ -121,7 +122,7 @@ attn_bwd_kernel(const BwdParams p)
         }
         __syncthreads();
 #pragma unroll 1
-        for (int u = 0; u < kBwKeys && warp < nw; ++u) {
+        for (int u = 0; u < NK && warp < nw; ++u) {
             const long long r = srow[u];
             float dkp[CPL], dvp[CPL];
 #pragma unroll
@@ -169,7 +170,7 @@ attn_bwd_kernel(const BwdParams p)
         __syncthreads();
         // thread -> (key, four channels) sums over the warps, one vector
         // reduction each for dk and dv
-        for (int e = threadIdx.x; e < kBwKeys * d / 4; e += 32 * kBwWarps) {
+        for (int e = threadIdx.x; e < NK * d / 4; e += 32 * kBwWarps) {
             const int u = e / (d / 4), c = (e % (d / 4)) * 4;
             const long long r = srow[u];
             if (r < 0)
@@ -204,19 +205,33 @@ attn_bwd_kernel(const BwdParams p)
     }
 }
 
+// One launch with NK keys per round (dynamic shared memory for the partials).
+template <int CPL, int HPW, int NK>
+static cudaError_t launch_attn_bwd_k(const BwdParams &p, long long items, cudaStream_t stream)
+{
+    const size_t smem = (size_t)2 * NK * kBwWarps * 128 * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<CPL, HPW, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    attn_bwd_kernel<CPL, HPW, NK><<<(unsigned)items, 32 * kBwWarps, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// Heads per warp by group width; groups wider than 16 take eight keys per
+// round (half the block barriers, and every thread busy in the reduction),
+// the narrower ones four (more blocks per SM).
 template <int CPL>
 static cudaError_t launch_attn_bwd_c(const BwdParams &p, long long items, cudaStream_t stream)
 {
     const int hpw = (p.g + kBwWarps - 1) / kBwWarps;
     if (hpw <= 1)
-        attn_bwd_kernel<CPL, 1><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
-    else if (hpw <= 2)
-        attn_bwd_kernel<CPL, 2><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
-    else if (hpw <= 4)
-        attn_bwd_kernel<CPL, 4><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
-    else
-        attn_bwd_kernel<CPL, 8><<<(unsigned)items, 32 * kBwWarps, 0, stream>>>(p);
-    return cudaGetLastError();
+        return launch_attn_bwd_k<CPL, 1, 4>(p, items, stream);
+    if (hpw <= 2)
+        return launch_attn_bwd_k<CPL, 2, 4>(p, items, stream);
+    if (hpw <= 4)
+        return launch_attn_bwd_k<CPL, 4, 8>(p, items, stream);
+    return launch_attn_bwd_k<CPL, 8, 8>(p, items, stream);
 }
 
 cudaError_t launch_attn_bwd(const BwdParams &p, cudaStream_t stream)
