@@ -10,8 +10,8 @@
 // One CTA per (token, KV head): warp w holds heads w, w + 8, ... of the group
 // (q, dO and the dq accumulators in registers; lane = d/32 channels); warps
 // without a head (groups of fewer than eight) only take part in the sums.  Keys go
-// four at a time: each warp adds its heads' dk / dv parts into shared
-// memory, then the CTA adds the keys' sums to the fp32 gradients with one
+// four or eight at a time (NK): each warp adds its heads' dk / dv parts into
+// shared memory, then the CTA adds the keys' sums to the fp32 gradients with one
 // vector reduction per four channels (the form for problems the tensor-core
 // passes do not take: CSA selections, d = 64, decode positions).
 //
