@@ -230,8 +230,10 @@ class Step:
                                     dw=self.dwk, ws=self.bws, stream=stream)
             hb.hyb_hca_compress_bwd(inp["v"], inp["wv"], w.m, self.grads["dvc"], dx=self.grads["dv_raw"],
                                     dw=self.dwv, ws=self.bws, stream=stream)
-            # dense problems with d = 128: three tensor-core launches, else one
-            launches += 4 + (3 if (w.topk == 0 and w.d == 128) else 1)
+            # dense problems with d = 128: three tensor-core launches; CSA with
+            # d = 128: those three for the window keys plus the CUDA-core one
+            # for the selected entries; else the CUDA-core one alone
+            launches += 4 + (3 if (w.topk == 0 and w.d == 128) else (4 if w.d == 128 else 1))
             ev[4].record(stream)
             self.launches = launches
             return
@@ -628,6 +630,7 @@ def run_gpu(args, rank, world):
         kname = "hyb_attn_fwd_fp4 (fp4_gather_kernel + csa_attn_kernel)"
     if train:
         kname = ("bwd_delta_kernel + attn_bwd_kv_kernel + attn_bwd_q_kernel" if bwd_tc
+                 else "attn_bwd_kernel (selected entries) + tensor-core window passes" if w.d == 128
                  else "attn_bwd_kernel")
     roof["kernel"] = kname
     roof["peak_source"] = ("derived (unit counts x measured clock)" if train and not bwd_tc

@@ -555,21 +555,31 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
         return cuda_status(launch_attn_bwd_tc(p->B, p->Lq, p->Hq, p->Hkv, p->Nc, p->m, p->W, scale, q, kc, vc,
                                               k_raw, v_raw, o, lse, dout, dq, dkc, dvc, dk_raw, dv_raw, stream,
                                               num_sms_current()));
-    const size_t ck = (size_t)p->B * p->Nc * p->Hkv * p->d * sizeof(float);
-    const size_t rk = (size_t)p->B * p->Lkv * p->Hkv * p->d * sizeof(float);
+    // CSA prefill with a window and d = 128: the tensor-core passes take the
+    // window keys (they zero dkc / dvc, store dk_raw / dv_raw and write dq's
+    // window part), then the CUDA-core pass adds the selected entries' part
+    const bool split = idx && attn_bwd_tc_window_ok(p->d, p->q_pos, p->kv_pos0, p->Lq, p->Lkv, p->W);
     cudaError_t e = cudaSuccess;
-    if (ck) {
-        e = cudaMemsetAsync(dkc, 0, ck, stream);
+    if (split) {
+        e = launch_attn_bwd_tc(p->B, p->Lq, p->Hq, p->Hkv, p->Nc, p->m, p->W, scale, q, kc, vc, k_raw, v_raw, o,
+                               lse, dout, dq, dkc, dvc, dk_raw, dv_raw, stream, num_sms_current(), true);
+    } else {
+        const size_t ck = (size_t)p->B * p->Nc * p->Hkv * p->d * sizeof(float);
+        const size_t rk = (size_t)p->B * p->Lkv * p->Hkv * p->d * sizeof(float);
+        if (ck) {
+            e = cudaMemsetAsync(dkc, 0, ck, stream);
+            if (e == cudaSuccess)
+                e = cudaMemsetAsync(dvc, 0, ck, stream);
+        }
         if (e == cudaSuccess)
-            e = cudaMemsetAsync(dvc, 0, ck, stream);
+            e = cudaMemsetAsync(dk_raw, 0, rk, stream);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(dv_raw, 0, rk, stream);
     }
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(dk_raw, 0, rk, stream);
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(dv_raw, 0, rk, stream);
     if (e != cudaSuccess)
         return cuda_status(e);
     BwdParams b;
+    b.comp_only = split ? 1 : 0;
     b.B = p->B;
     b.Lq = p->Lq;
     b.Lkv = p->Lkv;

@@ -32,6 +32,8 @@ constexpr int kBwWarps = 8;
 
 struct BwdParams {
     int B, Lq, Lkv, Hq, Hkv, g, d, Nc, m, W, topk;
+    int comp_only;     // 1: the window keys are another pass's (the tensor-core one): skip them
+                       // here and add this pass's part to dq instead of storing it
     float scale;
     const int32_t *q_pos, *kv_pos0, *idx;
     const __nv_bfloat16 *q, *kc, *vc, *kr, *vr, *o, *dout;
@@ -69,7 +71,7 @@ attn_bwd_kernel(const BwdParams p)
     long long hi = pos - kv0;
     if (hi > p.Lkv - 1)
         hi = p.Lkv - 1;
-    const int nwin = (p.W > 0 && hi >= lo) ? (int)(hi - lo + 1) : 0;
+    const int nwin = (!p.comp_only && p.W > 0 && hi >= lo) ? (int)(hi - lo + 1) : 0;
     const long long wstart = pos - p.W + 1;
     int nvis = 0;
     if (wstart > 0)
@@ -201,7 +203,7 @@ attn_bwd_kernel(const BwdParams p)
         const size_t row = ((size_t)bt * p.Hq + (size_t)kvh * p.g + h) * d + lane * CPL;
 #pragma unroll
         for (int c = 0; c < CPL; ++c)
-            p.dq[row + c] = dqv[e][c] * p.scale;
+            p.dq[row + c] = p.comp_only ? p.dq[row + c] + dqv[e][c] * p.scale : dqv[e][c] * p.scale;
     }
 }
 

@@ -63,6 +63,7 @@ struct BtParams {
     int chunk_qt;       // query tiles per compressed item (chunk c: tiles c chunk_qt ..)
     int max_chunks;     // ceil(nqt / chunk_qt)
     int nqw;            // query tiles per raw key tile
+    int win_only;       // 1: raw (window) keys only -- the selected entries of a CSA problem are another pass's
     long long n_comp_items, n_items;
     float scale, scale_log2;
     const float *lse;               // [B, Hq, L], natural log
@@ -638,7 +639,7 @@ __device__ __forceinline__ BtQItem bt_q_item(const BtParams &p, long long w)
     it.b = (int)(r / (unsigned)p.Hq);
     it.h = (int)(r % (unsigned)p.Hq);
     const int tmax = min(it.t0 + 127, p.L - 1);
-    it.nct = (bt_visible(tmax, p.m, p.W, p.Nc) + 127) / 128;
+    it.nct = p.win_only ? 0 : (bt_visible(tmax, p.m, p.W, p.Nc) + 127) / 128;
     it.rlo = max(0, it.t0 - p.W + 1);
     it.nrt = p.W > 0 ? (tmax - it.rlo + 128) / 128 : 0;
     return it;
@@ -909,13 +910,21 @@ static bool attn_bwd_tc_ok(bool has_idx, int d, const int32_t *q_pos, const int3
            (long long)Lq + W < (1LL << 30) && ((long long)Nc + 128) * m + W < (1LL << 30);
 }
 
+// CSA prefill problems with d = 128 and a window: the tensor-core passes take
+// the window keys (win_only), the CUDA-core pass the selected entries.
+static bool attn_bwd_tc_window_ok(int d, const int32_t *q_pos, const int32_t *kv_pos0, int Lq, int Lkv, int W)
+{
+    return d == 128 && !q_pos && !kv_pos0 && Lq == Lkv && Lq > 0 && W > 0 && (long long)Lq + W < (1LL << 30);
+}
+
 // Zeroes dkc / dvc (reduced into), and dk_raw / dv_raw without a window (no
-// raw item stores them), then runs the three launches.
+// raw item stores them), then runs the three launches.  win_only: raw keys
+// only (no compressed item, no compressed tile in the dq pass).
 static cudaError_t launch_attn_bwd_tc(int B, int L, int Hq, int Hkv, int Nc, int m, int W, float scale,
                                       const void *q, const void *kc, const void *vc, const void *kr,
                                       const void *vr, const void *o, const float *lse, const void *dout,
                                       float *dq, float *dkc, float *dvc, float *dkr, float *dvr,
-                                      cudaStream_t stream, int num_sms)
+                                      cudaStream_t stream, int num_sms, bool win_only = false)
 {
     BtParams p;
     p.B = B;
@@ -927,7 +936,8 @@ static cudaError_t launch_attn_bwd_tc(int B, int L, int Hq, int Hkv, int Nc, int
     p.m = m;
     p.W = W;
     p.nqt = (L + 127) / 128;
-    p.nkt_c = Nc > 0 ? (Nc + 127) / 128 : 0;
+    p.win_only = win_only ? 1 : 0;
+    p.nkt_c = (Nc > 0 && !win_only) ? (Nc + 127) / 128 : 0;
     p.nkt_r = W > 0 ? (L + 127) / 128 : 0;
     p.nqw = (127 + W + 127) / 128;
     // compressed units (query tile, head) per key tile; key tile 0 has the most

@@ -236,7 +236,9 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
  * on the tensor cores: a pass over key tiles for dk / dv and one over query
  * tiles for dq, with P and dS rounded to bf16 as MMA operands (fp32
  * accumulation); dq's memory holds dout.o of each row while the call runs.
- * Every other problem runs an fp32 CUDA-core kernel. */
+ * CSA prefill problems with d = 128 and a window split: those passes take the
+ * window keys, an fp32 CUDA-core kernel the selected entries (adding into
+ * dq).  Every other problem runs the CUDA-core kernel alone. */
 hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, const void *vc,
                         const int32_t *idx, const void *k_raw, const void *v_raw, const void *o,
                         const float *lse, const void *dout, float *dq, float *dkc, float *dvc,
