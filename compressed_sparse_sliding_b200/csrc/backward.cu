@@ -49,6 +49,62 @@ __device__ __forceinline__ float bw_warp_sum(float v)
     return v;
 }
 
+
+// The 2 HPW per-lane partial dot products of a key (q_e . k and dO_e . v over
+// this lane's CPL channels, e < HPW) summed over the warp: a halving butterfly
+// (each step a lane keeps the half of its values named by its lane bit and adds
+// the partner's copy of it: 2 HPW - 1 shuffles) leaves each lane one value's
+// partial over its group, plain steps finish the sums, and 2 HPW shuffles hand
+// every total to every lane -- against 5 shuffles per value one by one.
+template <int HPW, int CPL>
+__device__ __forceinline__ void bw_multi_sum_impl(const float (&qv)[HPW][CPL], const float (&dov)[HPW][CPL],
+                                                  const float (&kv)[CPL], const float (&vv)[CPL],
+                                                  float (&out)[2 * HPW])
+{
+    constexpr int NV = 2 * HPW;
+    const int lane = threadIdx.x & 31;
+    float v[NV];
+#pragma unroll
+    for (int e = 0; e < HPW; ++e) {
+        float a = 0.f, b = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            a = fmaf(qv[e][c], kv[c], a);
+            b = fmaf(dov[e][c], vv[c], b);
+        }
+        v[e] = a;
+        v[HPW + e] = b;
+    }
+    // halving steps over lane bits 4, 3, ...: after them v[0] holds value
+    // idx(lane) = the lane's top log2(NV) bits read as a binary number
+    int off = 16;
+#pragma unroll
+    for (int n = NV; n > 1; n >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float t = v[0];
+#pragma unroll
+    for (; off > 0; off >>= 1)
+        t += __shfl_xor_sync(0xffffffffu, t, off);
+    // value j sits in the lanes whose top bits spell j
+    constexpr int LOGNV = NV == 2 ? 1 : NV == 4 ? 2 : NV == 8 ? 3 : 4;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        int src = 0;
+#pragma unroll
+        for (int bit = 0; bit < LOGNV; ++bit)
+            if (j & (1 << (LOGNV - 1 - bit)))
+                src |= 16 >> bit;
+        out[j] = __shfl_sync(0xffffffffu, t, src);
+    }
+}
+
 template <int CPL, int HPW, int NK>
 __global__ void __launch_bounds__(32 * kBwWarps)
 attn_bwd_kernel(const BwdParams p)
@@ -141,18 +197,14 @@ attn_bwd_kernel(const BwdParams p)
                     kv[c] = __bfloat162float(kp[c]);
                     vv[c] = __bfloat162float(vp[c]);
                 }
+                // the warp's 2 HPW dot products (scores, then dP) reduced together
+                float sums[2 * HPW];
+                bw_multi_sum_impl<HPW, CPL>(qv, dov, kv, vv, sums);
 #pragma unroll
                 for (int e = 0; e < HPW; ++e) {
                     if (warp + kBwWarps * e >= p.g)
                         continue;
-                    float s = 0.f, dp = 0.f;
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) {
-                        s = fmaf(qv[e][c], kv[c], s);
-                        dp = fmaf(dov[e][c], vv[c], dp);
-                    }
-                    s = bw_warp_sum(s);
-                    dp = bw_warp_sum(dp);
+                    const float s = sums[e], dp = sums[HPW + e];
                     const float pr = expf(s * p.scale - lse[e]);
                     const float ds = pr * (dp - Dh[e]);
 #pragma unroll
