@@ -135,6 +135,7 @@ attn_bwd_kernel(const BwdParams p)
     const int ncomp = p.idx ? p.topk : nvis;
 
     // this warp's heads: h = warp + kBwWarps * e
+    const float scale_log2 = p.scale * 1.4426950408889634f;
     float qv[HPW][CPL], dov[HPW][CPL], dqv[HPW][CPL], lse[HPW], Dh[HPW];
 #pragma unroll
     for (int e = 0; e < HPW; ++e) {
@@ -150,7 +151,9 @@ attn_bwd_kernel(const BwdParams p)
             dqv[e][c] = 0.f;
         }
         Dh[e] = bw_warp_sum(od);
-        lse[e] = on ? p.lse[((size_t)b * p.Hq + (size_t)kvh * p.g + h) * p.Lq + t] : -INFINITY;
+        // the row's lse in base-2 units (+inf for a row without keys: P = 0)
+        const float l = on ? p.lse[((size_t)b * p.Hq + (size_t)kvh * p.g + h) * p.Lq + t] : -INFINITY;
+        lse[e] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
     }
 
     extern __shared__ __align__(16) float bw_partials[];
@@ -205,7 +208,7 @@ attn_bwd_kernel(const BwdParams p)
                     if (warp + kBwWarps * e >= p.g)
                         continue;
                     const float s = sums[e], dp = sums[HPW + e];
-                    const float pr = expf(s * p.scale - lse[e]);
+                    const float pr = ex2_approx(fmaf(s, scale_log2, -lse[e]));
                     const float ds = pr * (dp - Dh[e]);
 #pragma unroll
                     for (int c = 0; c < CPL; ++c) {
