@@ -550,6 +550,11 @@ hyb_status hyb_attn_bwd(const hyb_problem *p, const void *q, const void *kc, con
         return HYB_ERR_INVALID_ARG;
     if (p->Lkv <= 0)
         return HYB_ERR_INVALID_ARG;
+    // every kernel of the pass moves whole 16-byte pieces of these rows
+    if (!aligned16(q) || !aligned16(k_raw) || !aligned16(v_raw) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk_raw) || !aligned16(dv_raw) ||
+        (p->Nc > 0 && (!aligned16(kc) || !aligned16(vc) || !aligned16(dkc) || !aligned16(dvc))))
+        return HYB_ERR_INVALID_ARG;
     const float scale = softmax_scale(p);
     if (attn_bwd_tc_ok(idx != nullptr, p->d, p->q_pos, p->kv_pos0, p->Lq, p->Lkv, p->Nc, p->m, p->W))
         return cuda_status(launch_attn_bwd_tc(p->B, p->Lq, p->Hq, p->Hkv, p->Nc, p->m, p->W, scale, q, kc, vc,

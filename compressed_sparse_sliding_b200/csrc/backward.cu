@@ -194,11 +194,26 @@ attn_bwd_kernel(const BwdParams p)
             if (r >= 0) {
                 const __nv_bfloat16 *kp = (scomp[u] ? p.kc : p.kr) + r * d + lane * CPL;
                 const __nv_bfloat16 *vp = (scomp[u] ? p.vc : p.vr) + r * d + lane * CPL;
+                // this lane's CPL channels of the key and value rows in one load each
+                // (rows are 256-byte aligned; CPL = 4 or 2 bf16 = 8 or 4 bytes)
                 float kv[CPL], vv[CPL];
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) {
-                    kv[c] = __bfloat162float(kp[c]);
-                    vv[c] = __bfloat162float(vp[c]);
+                static_assert(CPL == 2 || CPL == 4, "lane channel counts of d = 64 and 128");
+                if constexpr (CPL == 4) {
+                    const uint2 ka = *reinterpret_cast<const uint2 *>(kp);
+                    const uint2 va = *reinterpret_cast<const uint2 *>(vp);
+                    const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ka.x));
+                    const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ka.y));
+                    const float2 v0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&va.x));
+                    const float2 v1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&va.y));
+                    kv[0] = k0.x; kv[1] = k0.y; kv[2] = k1.x; kv[3] = k1.y;
+                    vv[0] = v0.x; vv[1] = v0.y; vv[2] = v1.x; vv[3] = v1.y;
+                } else {
+                    const uint32_t ka = *reinterpret_cast<const uint32_t *>(kp);
+                    const uint32_t va = *reinterpret_cast<const uint32_t *>(vp);
+                    const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ka));
+                    const float2 v0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&va));
+                    kv[0] = k0.x; kv[1] = k0.y;
+                    vv[0] = v0.x; vv[1] = v0.y;
                 }
                 // the warp's 2 HPW dot products (scores, then dP) reduced together
                 float sums[2 * HPW];

@@ -229,6 +229,7 @@ hyb_status hyb_gated_fwd(const hyb_problem *p, const void *q, const void *kc, co
  * that call's outputs, dout [B, Lq, Hq, d] bf16.  Per query row with key set
  * S: P_j = exp(scale q.k_j - lse), dS_j = P_j (dout.v_j - dout.o),
  * dq = scale sum_j dS_j k_j, dk_j += scale dS_j q, dv_j += P_j dout.
+ * Every pointer 16-byte aligned (else HYB_ERR_INVALID_ARG, nothing launched).
  * Outputs fp32, caller-owned, overwritten: dq [B, Lq, Hq, d]; dkc, dvc
  * [B, Nc, Hkv, d]; dk_raw, dv_raw [B, Lkv, Hkv, d] (the window path only:
  * the path through the compression is hyb_hca_compress_bwd's).  Dense

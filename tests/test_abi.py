@@ -154,3 +154,18 @@ def test_backward_argument_checks(lib):
                                         None) == hb.HYB_ERR_UNSUPPORTED
     assert hb._lib.hyb_hca_compress_bwd(buf, 1, 8, 1, 64, 4, buf, buf, buf, buf, buf, 512,
                                         None) == hb.HYB_ERR_WORKSPACE
+
+
+def test_backward_rejects_misaligned_rows(lib):
+    # the backward's kernels move 16-byte pieces of every row: a pointer off
+    # that grid is refused on the host, before anything is launched
+    import compressed_sparse_sliding_b200 as hb
+    p = hb.problem(B=1, Lq=256, Lkv=256, Hq=2, Hkv=1, d=128, m=4, W=128, Nc=64)
+    ok, bad = ctypes.c_void_p(256), ctypes.c_void_p(256 + 8)
+    args = [ok] * 15   # q kc vc idx k v o lse dout dq dkc dvc dk dv stream
+    args[3] = None     # dense: no selection
+    args[14] = None    # default stream
+    for i in (0, 1, 4, 6, 8, 9, 10, 12):
+        a = list(args)
+        a[i] = bad
+        assert hb._lib.hyb_attn_bwd(ctypes.byref(p), *a) == hb.HYB_ERR_INVALID_ARG, i
