@@ -106,7 +106,9 @@ __device__ __forceinline__ void bw_multi_sum_impl(const float (&qv)[HPW][CPL], c
 }
 
 template <int CPL, int HPW, int NK>
-__global__ void __launch_bounds__(32 * kBwWarps)
+// Four heads per warp (32-head groups): capped for three blocks per SM, which
+// measured faster than two blocks with no spill
+__global__ void __launch_bounds__(32 * kBwWarps, HPW == 4 ? 3 : 1)
 attn_bwd_kernel(const BwdParams p)
 {
     // item = (b, t, KV head)
